@@ -1,0 +1,189 @@
+/*
+ * rmm.h — C ABI of librmm, a B200 (sm_100a) implementation of Reduced Matrix
+ * Multiplication (RMM).
+ *
+ * Source page: "Reduced Matrix Multiplication: Input-Adaptive Matrix-Product
+ * Reduction for LLM Inference" (technical summary; section names are those of
+ * its Spanish edition).  RMM replaces a product Y = AB (A the activation, B a
+ * weight or intermediate representation; Metodología) by A[:,I] B[I,:], where
+ * I holds the k = ceil(rho d) contraction indices with the largest activation
+ * column norms s_j = ||A[:,j]||_2 (Metodología › Mecanismo Central,
+ * Estrategia de Selección).  It applies to linear projections XW, to QK^T
+ * along head_dim and to PV along the token dimension (Metodología › Alcance
+ * de Aplicación).
+ *
+ * Conventions shared by every entry point
+ *  - Every data pointer is a caller-owned DEVICE pointer on the current CUDA
+ *    device; the library never allocates, frees or retains memory.  Scratch
+ *    space ("workspace") is passed in by the caller; its size comes from the
+ *    matching *_workspace_size query.  A NULL workspace with ws_bytes == 0 is
+ *    allowed when the query returns 0.
+ *  - Matrices are row-major with an explicit leading dimension in ELEMENTS
+ *    (ld >= number of columns).  Indices are int32.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *    enqueued asynchronously on it; no call synchronises unless stated.
+ *  - Every call validates its arguments on the host before launching and
+ *    returns an rmm_status; on failure nothing was launched and
+ *    rmm_last_error() gives a message (per host thread).
+ *  - Errors found on the device (an index outside [0, d), a bounded wait that
+ *    ran out) are recorded in a per-device error word and reported by
+ *    rmm_device_error(), which synchronises the stream.  Kernels never trap.
+ *  - dtype codes: RMM_F32 (fp32) or RMM_BF16 (bf16 stored as 16-bit words).
+ *    bf16 products accumulate in fp32.
+ */
+#ifndef RMM_H_
+#define RMM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RMM_API __attribute__((visibility("default")))
+#else
+#define RMM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rmm_status {
+  RMM_OK = 0,
+  RMM_ERR_INVALID_ARG = 1,   /* null pointer, bad size, rho outside (0,1], k outside [1,d] */
+  RMM_ERR_UNSUPPORTED = 2,   /* dtype, alignment or shape the kernels do not take */
+  RMM_ERR_WORKSPACE = 3,     /* workspace missing or smaller than the query's size */
+  RMM_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+  RMM_ERR_DEVICE = 5         /* rmm_device_error() found a device-side error */
+} rmm_status;
+
+typedef enum rmm_dtype { RMM_F32 = 0, RMM_BF16 = 1 } rmm_dtype;
+
+/* Device-side error codes stored in the error word (0 = none). */
+#define RMM_DEVERR_BAD_INDEX 1u        /* an index outside [0, d) was read; its row/column was zero-filled */
+#define RMM_DEVERR_TIMEOUT_BASE 0x100u /* + site: a bounded wait ran out and the kernel returned early */
+
+/* ABI version of this header (incremented on any incompatible change). */
+#define RMM_ABI_VERSION 1
+RMM_API int rmm_abi_version(void);
+
+/* Message describing the last failing call on this host thread ("" if none).
+ * The pointer stays valid until the next rmm_* call on this thread. */
+RMM_API const char* rmm_last_error(void);
+
+/* k = ceil(rho * d) (Metodología › Estrategia de Selección), computed in fp64
+ * with a guard of 1e-9*d against representation error (0.3*10 gives 3) and
+ * clamped to [1, d].  Returns -1 when rho is not in (0, 1] or d < 1. */
+RMM_API int64_t rmm_k_from_rho(double rho, int64_t d);
+
+/* Synchronises `stream`, then reads the current device's error word into
+ * *code (may be NULL); clears it when `clear` != 0.  Returns RMM_ERR_DEVICE
+ * when the word was non-zero, RMM_ERR_CUDA if the sync failed. */
+RMM_API rmm_status rmm_device_error(void* stream, int clear, unsigned* code);
+
+/* ------------------------------------------------------------------ score
+ * Column scores of `batch` activation matrices (Metodología › Estrategia de
+ * Selección): ss[b*ld_ss + j] = sum_i A_b[i,j]^2, with A_b = A + b*batch_stride
+ * (elements) an [M x d] row-major matrix of leading dimension lda.  Squares
+ * are exact in fp32; the sum is an fp32 tree in a fixed order, so results are
+ * deterministic for a given shape.  With sqrt_out != 0 the output is
+ * s_j = sqrt(ss_j) instead (the page's norm; ranking is identical, but the
+ * square root can merge distinct scores, so rmm_topk should be given ss).
+ * Layout: lda >= d; for the vectorised path A and lda*elt must be 16-byte
+ * aligned (otherwise a scalar path runs).  Workspace: rmm_score_workspace_size
+ * bytes (fp32 partial sums of the row splits; 0 when one split suffices).
+ * M == 0 gives all-zero scores. */
+RMM_API size_t rmm_score_workspace_size(int dtype, int64_t batch, int64_t M, int64_t d);
+RMM_API rmm_status rmm_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t d,
+                     int64_t lda, int64_t batch_stride, float* ss, int64_t ld_ss,
+                     int sqrt_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ top-k
+ * For each of `batch` score rows (row b at scores + b*ld_s, length d), writes
+ * the k indices with the largest scores to idx + b*ld_idx, in ascending index
+ * order; equal scores are taken lowest index first (Metodología › Estrategia
+ * de Selección keeps the top-k; the tie rule and the order are this library's
+ * reading).  Scores must be finite; -0.0 ranks equal to +0.0.  The selection
+ * is an exact radix select on the fp32 bit patterns, so the index set is the
+ * unique one defined by that rule.  1 <= k <= d, ld_idx >= k, ld_s >= d.  */
+RMM_API rmm_status rmm_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k,
+                    int32_t* idx, int64_t ld_idx, void* stream);
+
+/* ------------------------------------------------------------------ compaction
+ * A_I[i, r] = A[i, idx[r]] for r < k (Metodología › Mecanismo Central: the
+ * reduced operand A_{:,I}).  A is [M x d] (lda), A_I is [M x k] (ld_ai >= k).
+ * Columns k..ld_ai-1 of A_I are not written.  Indices outside [0, d) are
+ * replaced by zero and flagged in the device error word. */
+RMM_API rmm_status rmm_compact(const void* A, int dtype, int64_t M, int64_t d, int64_t lda,
+                       const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai, void* stream);
+
+/* ------------------------------------------------------------------ row gather
+ * B_I[r, :] = B[idx[r], :] for r < k (Metodología › Mecanismo Central: the
+ * reduced operand B_{I,:}).  B is [d x N] (ldb), B_I is [k x N] (ld_bi).
+ * Rows are copied whole with 16-byte accesses: B, B_I and the row pitches in
+ * bytes must be 16-byte aligned (RMM_ERR_UNSUPPORTED otherwise).  Indices outside [0, d) give a zero row
+ * and are flagged in the device error word. */
+RMM_API rmm_status rmm_gather_rows(const void* B, int dtype, int64_t d, int64_t N, int64_t ldb,
+                                   const int32_t* idx, int64_t k, void* B_I, int64_t ld_bi, void* stream);
+
+/* ------------------------------------------------------------------ reduced GEMM
+ * Y = A_I · B[idx, :]  (Metodología › Mecanismo Central), where A_I is the
+ * compacted [M x k] activation (ld_ai), B the full [d x N] row-major operand
+ * (ldb >= N) whose rows idx[0..k) are the kept contraction indices, and Y is
+ * [M x N] (ldy >= N) written as out_dtype (RMM_BF16 or RMM_F32).
+ *  - dtype RMM_BF16: B's kept rows are first copied into workspace (a
+ *    streaming row gather), then a persistent tcgen05 tensor-core kernel
+ *    computes the product with fp32 accumulation in tensor memory.  Requires
+ *    16-byte aligned A_I, B, Y, and ld_ai, ldb multiples of 8
+ *    (RMM_ERR_UNSUPPORTED otherwise).  B must be finite.
+ *  - dtype RMM_F32: fp32 FMA kernel (A_I, B fp32; Y fp32 only); no workspace.
+ * Workspace: rmm_gemm_workspace_size(dtype, N, k) bytes, 256-byte aligned.
+ * Out-of-range indices contribute zero and are flagged.  k >= 1. */
+RMM_API size_t rmm_gemm_workspace_size(int dtype, int64_t N, int64_t k);
+RMM_API rmm_status rmm_gemm(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb,
+                            const int32_t* idx, int64_t d, int64_t M, int64_t N, int64_t k,
+                            int dtype, void* Y, int out_dtype, int64_t ldy,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ whole path
+ * The method end to end on one product: ss = score(A); I = topk(ss, k) with
+ * k = rmm_k_from_rho(rho, d); A_I = compact(A, I); B_I = gather_rows(B, I);
+ * Y = A_I · B_I.
+ * A is [M x d] (lda), B is [d x N] (ldb), Y is [M x N] (ldy).  idx_out (k
+ * int32, may be NULL) and ss_out (d floats, may be NULL) receive the
+ * intermediate index set and scores.  Workspace: rmm_matmul_workspace_size
+ * bytes, 256-byte aligned pointer. */
+RMM_API size_t rmm_matmul_workspace_size(int dtype, int64_t M, int64_t d, int64_t N, double rho);
+RMM_API rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t ldb,
+                      int64_t M, int64_t d, int64_t N, double rho, int dtype,
+                      void* Y, int out_dtype, int64_t ldy, int32_t* idx_out, float* ss_out,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------ reduced attention
+ * Causal attention with both reductions of Metodología › Alcance de
+ * Aplicación, for Q [B, Hq, S, D] and K, V [B, Hkv, S, D] bf16, contiguous
+ * row-major (Hq a multiple of Hkv; q-head h reads kv-head h*Hkv/Hq):
+ *   1. per (b, h): ssq = column scores of Q_bh over its S tokens;
+ *      I_d = top k_d = ceil(rho_d*D) head_dim indices (lowest index on ties);
+ *   2. logits S_ij = scale * sum_{c in I_d} Q[i,c] K[j,c] for j <= i
+ *      (scale <= 0 selects 1/sqrt(D), the unreduced temperature);
+ *      lse_i = logsumexp_{j<=i} S_ij;  P_ij = exp(S_ij - lse_i);
+ *   3. token scores t_j = sum_{i>=j} P_ij^2 (squared column norms of P);
+ *      I_t = top k_t = ceil(rho_t*S) tokens;
+ *   4. O_i = sum_{j in I_t, j<=i} P_ij V[j,:]  (P not renormalised; a query
+ *      with no kept token in its window gets a zero row).
+ * O is [B, Hq, S, D] written as out_dtype.  Optional outputs (may be NULL):
+ * idx_d [B*Hq, k_d], idx_t [B*Hq, k_t], lse [B*Hq, S], tscore [B*Hq, S].
+ * Requires D in {64, 128} and S >= 1. Workspace: rmm_attention_workspace_size. */
+RMM_API size_t rmm_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D,
+                                    double rho_d, double rho_t);
+RMM_API rmm_status rmm_attention(const void* Q, const void* K, const void* V,
+                         int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D,
+                         double rho_d, double rho_t, float scale,
+                         void* O, int out_dtype, int32_t* idx_d, int32_t* idx_t,
+                         float* lse, float* tscore, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RMM_H_ */

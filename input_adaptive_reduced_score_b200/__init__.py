@@ -1,0 +1,276 @@
+"""Python binding of librmm (Reduced Matrix Multiplication on B200, sm_100a).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``librmm.so`` behind the C ABI declared in ``include/rmm.h``.  PyTorch is used
+for device memory and streams.  There is no fallback: importing this package
+without the built library raises, and every call whose status is not RMM_OK
+raises ``RMMError``.
+
+The functions keep the C names (``rmm_score``, ``rmm_topk``, ``rmm_compact``,
+``rmm_gemm``, ``rmm_matmul``, ``rmm_attention`` ...) and take torch tensors;
+``lib`` is the raw ctypes handle for pointer-level calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+__all__ = [
+    "lib", "LIB_PATH", "RMMError", "RMM_F32", "RMM_BF16", "rmm_abi_version", "rmm_k_from_rho",
+    "rmm_device_error", "rmm_score", "rmm_score_workspace_size", "rmm_topk", "rmm_compact", "rmm_gather_rows",
+    "rmm_gemm", "rmm_gemm_workspace_size",
+    "rmm_matmul", "rmm_matmul_workspace_size", "rmm_attention", "rmm_attention_workspace_size",
+    "exported_symbols", "declared_symbols",
+]
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+ROOT_DIR = os.path.dirname(PKG_DIR)
+LIB_PATH = os.path.join(PKG_DIR, "librmm.so")
+HEADER_PATH = os.path.join(ROOT_DIR, "include", "rmm.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"librmm.so not built ({LIB_PATH}); run: python -m input_adaptive_reduced_score_b200.build")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+RMM_F32, RMM_BF16 = 0, 1
+_STATUS = {0: "RMM_OK", 1: "RMM_ERR_INVALID_ARG", 2: "RMM_ERR_UNSUPPORTED", 3: "RMM_ERR_WORKSPACE",
+           4: "RMM_ERR_CUDA", 5: "RMM_ERR_DEVICE"}
+
+c_i64, c_int, c_sz, c_dbl, c_flt, c_vp = (ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_double,
+                                          ctypes.c_float, ctypes.c_void_p)
+
+
+def _sig(name, res, *args):
+    f = getattr(lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_sig("rmm_abi_version", c_int)
+_sig("rmm_last_error", ctypes.c_char_p)
+_sig("rmm_k_from_rho", c_i64, c_dbl, c_i64)
+_sig("rmm_device_error", c_int, c_vp, c_int, ctypes.POINTER(ctypes.c_uint))
+_sig("rmm_score_workspace_size", c_sz, c_int, c_i64, c_i64, c_i64)
+_sig("rmm_score", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_int, c_vp, c_sz, c_vp)
+_sig("rmm_topk", c_int, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp)
+_sig("rmm_compact", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp)
+_sig("rmm_gather_rows", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp)
+_sig("rmm_gemm_workspace_size", c_sz, c_int, c_i64, c_i64)
+_sig("rmm_gemm", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_int, c_vp, c_int, c_i64, c_vp,
+     c_sz, c_vp)
+_sig("rmm_matmul_workspace_size", c_sz, c_int, c_i64, c_i64, c_i64, c_dbl)
+_sig("rmm_matmul", c_int, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_dbl, c_int, c_vp, c_int, c_i64, c_vp, c_vp,
+     c_vp, c_sz, c_vp)
+_sig("rmm_attention_workspace_size", c_sz, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl)
+_sig("rmm_attention", c_int, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl, c_flt, c_vp, c_int,
+     c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp)
+
+
+class RMMError(RuntimeError):
+    def __init__(self, status, where):
+        msg = lib.rmm_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _check(status, where):
+    if status != 0:
+        raise RMMError(status, where)
+
+
+def declared_symbols():
+    """Function names declared with RMM_API in include/rmm.h."""
+    with open(HEADER_PATH) as f:
+        return sorted(set(re.findall(r"^RMM_API\s+[\w\s\*]+?\b(rmm_\w+)\s*\(", f.read(), re.M)))
+
+
+def exported_symbols():
+    return [s for s in declared_symbols() if hasattr(lib, s)]
+
+
+# ------------------------------------------------------------------ helpers
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return RMM_BF16
+    if t.dtype == torch.float32:
+        return RMM_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return c_vp(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t):
+    return c_vp(0 if t is None else t.data_ptr())
+
+
+def _row_major(t: torch.Tensor, name: str):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D row-major tensor (unit column stride)")
+    return t.stride(0)
+
+
+def _workspace(nbytes: int, device, ws):
+    if nbytes == 0:
+        return None, 0
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise ValueError(f"workspace too small: need {nbytes} bytes")
+        return ws, ws.numel() * ws.element_size()
+    return torch.empty(nbytes, dtype=torch.uint8, device=device), nbytes
+
+
+# ------------------------------------------------------------------ API
+
+def rmm_abi_version() -> int:
+    return lib.rmm_abi_version()
+
+
+def rmm_k_from_rho(rho: float, d: int) -> int:
+    return lib.rmm_k_from_rho(float(rho), int(d))
+
+
+def rmm_device_error(stream=None, clear: bool = True) -> int:
+    """Synchronise the stream and return the device error word (0 = none)."""
+    code = ctypes.c_uint(0)
+    st = lib.rmm_device_error(_stream_ptr(stream), int(clear), ctypes.byref(code))
+    if st not in (0, 5):
+        _check(st, "rmm_device_error")
+    return code.value
+
+
+def rmm_score_workspace_size(dtype: int, batch: int, M: int, d: int) -> int:
+    return lib.rmm_score_workspace_size(dtype, batch, M, d)
+
+
+def rmm_score(A: torch.Tensor, out: torch.Tensor = None, sqrt_out: bool = False, ws=None, stream=None):
+    """Column scores ss_j = sum_i A[i,j]^2 of A [M x d] or a batch A [b x M x d]."""
+    batched = A.dim() == 3
+    A3 = A if batched else A.unsqueeze(0)
+    if A3.stride(2) != 1:
+        raise ValueError("A must have unit column stride")
+    b, M, d = A3.shape
+    dt = _dtype_code(A3)
+    if out is None:
+        out = torch.empty((b, d), dtype=torch.float32, device=A.device)
+    out2 = out if out.dim() == 2 else out.view(1, -1)
+    wsb = lib.rmm_score_workspace_size(dt, b, M, d)
+    w, wn = _workspace(wsb, A.device, ws)
+    _check(lib.rmm_score(_ptr(A3), dt, b, M, d, A3.stride(1), A3.stride(0) if b > 1 else 0, _ptr(out2),
+                         out2.stride(0), int(sqrt_out), _ptr(w), wn, _stream_ptr(stream)), "rmm_score")
+    return out if batched or out.dim() == 1 else out2[0]
+
+
+def rmm_topk(scores: torch.Tensor, k: int, out: torch.Tensor = None, stream=None):
+    """Ascending top-k indices (int32) per row of scores [d] or [b x d]."""
+    s2 = scores if scores.dim() == 2 else scores.view(1, -1)
+    if s2.dtype != torch.float32 or s2.stride(1) != 1:
+        raise ValueError("scores must be fp32 with unit stride")
+    b, d = s2.shape
+    if out is None:
+        out = torch.empty((b, k), dtype=torch.int32, device=scores.device)
+    o2 = out if out.dim() == 2 else out.view(1, -1)
+    _check(lib.rmm_topk(_ptr(s2), b, d, s2.stride(0), k, _ptr(o2), o2.stride(0), _stream_ptr(stream)), "rmm_topk")
+    return out if scores.dim() == 2 else o2[0]
+
+
+def rmm_compact(A: torch.Tensor, idx: torch.Tensor, out: torch.Tensor = None, stream=None):
+    """A_I[:, r] = A[:, idx[r]] for A [M x d]."""
+    lda = _row_major(A, "A")
+    M, d = A.shape
+    k = idx.numel()
+    if out is None:
+        ld = (k + 7) // 8 * 8
+        out = torch.empty((M, ld), dtype=A.dtype, device=A.device)[:, :k]
+    _check(lib.rmm_compact(_ptr(A), _dtype_code(A), M, d, lda, _ptr(idx), k, _ptr(out), out.stride(0),
+                           _stream_ptr(stream)), "rmm_compact")
+    return out
+
+
+def rmm_gather_rows(B: torch.Tensor, idx: torch.Tensor, out: torch.Tensor = None, stream=None):
+    """B_I[r, :] = B[idx[r], :] for B [d x N]."""
+    ldb = _row_major(B, "B")
+    d, N = B.shape
+    k = idx.numel()
+    if out is None:
+        ld = (N + 7) // 8 * 8
+        out = torch.empty((k, ld), dtype=B.dtype, device=B.device)[:, :N]
+    _check(lib.rmm_gather_rows(_ptr(B), _dtype_code(B), d, N, ldb, _ptr(idx), k, _ptr(out), out.stride(0),
+                               _stream_ptr(stream)), "rmm_gather_rows")
+    return out
+
+
+def rmm_gemm_workspace_size(dtype: int, N: int, k: int) -> int:
+    return lib.rmm_gemm_workspace_size(dtype, N, k)
+
+
+def rmm_gemm(A_I: torch.Tensor, B: torch.Tensor, idx: torch.Tensor, out: torch.Tensor = None,
+             out_dtype=None, ws=None, stream=None):
+    """Y = A_I · B[idx, :], A_I [M x k] (compacted), B [d x N]."""
+    ld_ai = _row_major(A_I, "A_I")
+    ldb = _row_major(B, "B")
+    M, k = A_I.shape
+    d, N = B.shape
+    if idx.numel() != k:
+        raise ValueError("idx must hold k indices")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or A_I.dtype, device=A_I.device)
+    ldy = _row_major(out, "Y")
+    dt = _dtype_code(A_I)
+    w, wn = _workspace(lib.rmm_gemm_workspace_size(dt, N, k), A_I.device, ws)
+    _check(lib.rmm_gemm(_ptr(A_I), ld_ai, _ptr(B), ldb, _ptr(idx), d, M, N, k, dt, _ptr(out),
+                        _dtype_code(out), ldy, _ptr(w), wn, _stream_ptr(stream)), "rmm_gemm")
+    return out
+
+
+def rmm_matmul_workspace_size(dtype: int, M: int, d: int, N: int, rho: float) -> int:
+    return lib.rmm_matmul_workspace_size(dtype, M, d, N, float(rho))
+
+
+def rmm_matmul(A: torch.Tensor, B: torch.Tensor, rho: float, out: torch.Tensor = None, out_dtype=None,
+               idx_out: torch.Tensor = None, ss_out: torch.Tensor = None, ws=None, stream=None):
+    """The whole path: score -> top-k -> compaction -> reduced GEMM."""
+    lda = _row_major(A, "A")
+    ldb = _row_major(B, "B")
+    M, d = A.shape
+    N = B.shape[1]
+    dt = _dtype_code(A)
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or A.dtype, device=A.device)
+    ldy = _row_major(out, "Y")
+    wsb = lib.rmm_matmul_workspace_size(dt, M, d, N, float(rho))
+    w, wn = _workspace(wsb, A.device, ws)
+    _check(lib.rmm_matmul(_ptr(A), lda, _ptr(B), ldb, M, d, N, float(rho), dt, _ptr(out), _dtype_code(out), ldy,
+                          _ptr(idx_out), _ptr(ss_out), _ptr(w), wn, _stream_ptr(stream)), "rmm_matmul")
+    return out
+
+
+def rmm_attention_workspace_size(B, Hq, Hkv, S, D, rho_d, rho_t) -> int:
+    return lib.rmm_attention_workspace_size(B, Hq, Hkv, S, D, float(rho_d), float(rho_t))
+
+
+def rmm_attention(Q, K, V, rho_d: float, rho_t: float, scale: float = 0.0, out=None, out_dtype=None,
+                  idx_d=None, idx_t=None, lse=None, tscore=None, ws=None, stream=None):
+    """Reduced causal attention; Q [B,Hq,S,D], K/V [B,Hkv,S,D] bf16 contiguous."""
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V")):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{n} must be a contiguous 4-D bf16 tensor")
+    B, Hq, S, D = Q.shape
+    Hkv = K.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, S, D), dtype=out_dtype or torch.bfloat16, device=Q.device)
+    wsb = lib.rmm_attention_workspace_size(B, Hq, Hkv, S, D, float(rho_d), float(rho_t))
+    w, wn = _workspace(wsb, Q.device, ws)
+    _check(lib.rmm_attention(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, S, D, float(rho_d), float(rho_t), float(scale),
+                             _ptr(out), _dtype_code(out), _ptr(idx_d), _ptr(idx_t), _ptr(lse), _ptr(tscore),
+                             _ptr(w), wn, _stream_ptr(stream)), "rmm_attention")
+    return out

@@ -1,0 +1,351 @@
+// rmm_api.cu — the extern "C" entry points of librmm (declared in rmm.h):
+// argument validation, workspace carving, launches, error reporting.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "../../include/rmm.h"
+#include "rmm_internal.h"
+
+namespace rmm {
+
+namespace {
+thread_local std::string g_last_error;
+
+// Per-device error word written by kernels (RMM_DEVERR_* codes).
+__device__ unsigned g_device_error_word;
+}  // namespace
+
+void set_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
+void clear_error() { g_last_error.clear(); }
+
+unsigned* device_error_word() {
+  static std::mutex mu;
+  static unsigned* cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    set_error("no current CUDA device");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_device_error_word);
+    if (e != cudaSuccess) {
+      set_error("cudaGetSymbolAddress(error word): %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    cache[dev] = static_cast<unsigned*>(p);
+  }
+  return cache[dev];
+}
+
+int device_sm_count() {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace rmm
+
+using namespace rmm;
+
+namespace {
+
+rmm_status fail(rmm_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  set_error("%s", buf);
+  return s;
+}
+
+rmm_status from_cuda(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return RMM_OK;
+  return fail(RMM_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+size_t elt_size(int dtype) { return dtype == RMM_BF16 ? 2 : 4; }
+
+bool valid_dtype(int dtype) { return dtype == RMM_F32 || dtype == RMM_BF16; }
+
+constexpr int64_t kIntMax = 0x7FFFFFFFLL;
+
+int64_t k_from_rho_impl(double rho, int64_t d) {
+  if (!(rho > 0.0 && rho <= 1.0) || d < 1) return -1;
+  const double x = rho * static_cast<double>(d) - 1e-9 * static_cast<double>(d);
+  int64_t k = static_cast<int64_t>(std::ceil(x));
+  if (k < 1) k = 1;
+  if (k > d) k = d;
+  return k;
+}
+
+int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+extern "C" size_t rmm_gemm_workspace_size(int dtype, int64_t N, int64_t k);
+namespace {
+
+struct MatmulWs {
+  size_t ss, idx, score, ai, bi, total;
+  int64_t k, ld_ai;
+};
+
+MatmulWs matmul_ws(int dtype, int64_t M, int64_t d, int64_t N, double rho) {
+  MatmulWs w{};
+  w.k = k_from_rho_impl(rho, d);
+  if (w.k < 1) return w;
+  w.ld_ai = round_up(w.k, 8);
+  size_t off = 0;
+  w.ss = off;
+  off += align_up(static_cast<size_t>(d) * 4, kWsAlign);
+  w.idx = off;
+  off += align_up(static_cast<size_t>(w.k) * 4, kWsAlign);
+  w.score = off;
+  off += score_workspace_bytes(dtype, 1, M, d);
+  w.ai = off;
+  off += align_up(static_cast<size_t>(M) * w.ld_ai * elt_size(dtype), kWsAlign);
+  w.bi = off;
+  off += rmm_gemm_workspace_size(dtype, N, w.k);
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rmm_abi_version(void) { return RMM_ABI_VERSION; }
+
+const char* rmm_last_error(void) { return g_last_error.c_str(); }
+
+int64_t rmm_k_from_rho(double rho, int64_t d) { return k_from_rho_impl(rho, d); }
+
+rmm_status rmm_device_error(void* stream, int clear, unsigned* code) {
+  clear_error();
+  unsigned* w = device_error_word();
+  if (!w) return RMM_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return from_cuda(e, "rmm_device_error: stream sync");
+  unsigned v = 0;
+  e = cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return from_cuda(e, "rmm_device_error: read");
+  if (clear && v) {
+    e = cudaMemset(w, 0, sizeof(unsigned));
+    if (e != cudaSuccess) return from_cuda(e, "rmm_device_error: clear");
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return from_cuda(e, "rmm_device_error: clear sync");
+  }
+  if (code) *code = v;
+  if (v) return fail(RMM_ERR_DEVICE, "device error word = 0x%x", v);
+  return RMM_OK;
+}
+
+size_t rmm_score_workspace_size(int dtype, int64_t batch, int64_t M, int64_t d) {
+  if (!valid_dtype(dtype) || batch < 1 || M < 0 || d < 1) return 0;
+  return score_workspace_bytes(dtype, batch, M, d);
+}
+
+rmm_status rmm_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
+                     int64_t batch_stride, float* ss, int64_t ld_ss, int sqrt_out, void* ws, size_t ws_bytes,
+                     void* stream) {
+  clear_error();
+  if (!valid_dtype(dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_score: dtype %d", dtype);
+  if (batch < 1 || batch > 65535 || M < 0 || d < 1 || lda < d || ld_ss < d)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_score: bad sizes (batch %lld M %lld d %lld lda %lld ld_ss %lld)",
+                (long long)batch, (long long)M, (long long)d, (long long)lda, (long long)ld_ss);
+  if (batch > 1 && batch_stride < M * lda)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_score: batch_stride smaller than one matrix");
+  if (!ss || (M > 0 && !A)) return fail(RMM_ERR_INVALID_ARG, "rmm_score: null pointer");
+  const size_t need = score_workspace_bytes(dtype, batch, M, d);
+  if (need && (!ws || ws_bytes < need))
+    return fail(RMM_ERR_WORKSPACE, "rmm_score: workspace %zu < %zu bytes", ws_bytes, need);
+  if (M == 0) {
+    for (int64_t b = 0; b < batch; ++b) {
+      cudaError_t e = cudaMemsetAsync(ss + b * ld_ss, 0, d * sizeof(float), static_cast<cudaStream_t>(stream));
+      if (e != cudaSuccess) return from_cuda(e, "rmm_score: memset");
+    }
+    return RMM_OK;
+  }
+  return from_cuda(launch_score(A, dtype, batch, M, d, lda, batch_stride, ss, ld_ss, sqrt_out, ws,
+                                static_cast<cudaStream_t>(stream)),
+                   "rmm_score: launch");
+}
+
+rmm_status rmm_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k, int32_t* idx,
+                    int64_t ld_idx, void* stream) {
+  clear_error();
+  if (!scores || !idx) return fail(RMM_ERR_INVALID_ARG, "rmm_topk: null pointer");
+  if (batch < 1 || batch > kIntMax || d < 1 || d > kIntMax || ld_s < d)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_topk: bad sizes");
+  if (k < 1 || k > d) return fail(RMM_ERR_INVALID_ARG, "rmm_topk: k = %lld outside [1, %lld]", (long long)k, (long long)d);
+  if (ld_idx < k) return fail(RMM_ERR_INVALID_ARG, "rmm_topk: ld_idx < k");
+  return from_cuda(launch_topk(scores, batch, d, ld_s, k, idx, ld_idx, static_cast<cudaStream_t>(stream)),
+                   "rmm_topk: launch");
+}
+
+rmm_status rmm_compact(const void* A, int dtype, int64_t M, int64_t d, int64_t lda, const int32_t* idx, int64_t k,
+                       void* A_I, int64_t ld_ai, void* stream) {
+  clear_error();
+  if (!valid_dtype(dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_compact: dtype %d", dtype);
+  if (M < 0 || d < 1 || lda < d || k < 1 || k > d || ld_ai < k)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_compact: bad sizes");
+  if (M > 0 && (!A || !idx || !A_I)) return fail(RMM_ERR_INVALID_ARG, "rmm_compact: null pointer");
+  unsigned* err = device_error_word();
+  if (!err) return RMM_ERR_CUDA;
+  return from_cuda(launch_compact(A, dtype, M, d, lda, idx, k, A_I, ld_ai, err, static_cast<cudaStream_t>(stream)),
+                   "rmm_compact: launch");
+}
+
+size_t rmm_gemm_workspace_size(int dtype, int64_t N, int64_t k) {
+  if (dtype != RMM_BF16 || N < 1 || k < 1) return 0;
+  return align_up(static_cast<size_t>(k) * static_cast<size_t>(round_up(N, 8)) * 2, kWsAlign);
+}
+
+rmm_status rmm_gather_rows(const void* B, int dtype, int64_t d, int64_t N, int64_t ldb, const int32_t* idx, int64_t k,
+                           void* B_I, int64_t ld_bi, void* stream) {
+  clear_error();
+  if (!valid_dtype(dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_gather_rows: dtype %d", dtype);
+  if (d < 1 || N < 0 || ldb < N || k < 1 || ld_bi < N)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_gather_rows: bad sizes");
+  if (N == 0) return RMM_OK;
+  if (!B || !idx || !B_I) return fail(RMM_ERR_INVALID_ARG, "rmm_gather_rows: null pointer");
+  const int64_t e = static_cast<int64_t>(elt_size(dtype));
+  if (!aligned16(B) || !aligned16(B_I) || (ldb * e) % 16 || (ld_bi * e) % 16)
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_gather_rows: needs 16-byte aligned bases and row pitches");
+  unsigned* err = device_error_word();
+  if (!err) return RMM_ERR_CUDA;
+  return from_cuda(launch_gather_rows(B, d, N * e, ldb * e, idx, k, B_I, ld_bi * e, err,
+                                      static_cast<cudaStream_t>(stream)),
+                   "rmm_gather_rows: launch");
+}
+
+rmm_status rmm_gemm(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, const int32_t* idx, int64_t d,
+                    int64_t M, int64_t N, int64_t k, int dtype, void* Y, int out_dtype, int64_t ldy, void* ws,
+                    size_t ws_bytes, void* stream) {
+  clear_error();
+  if (!valid_dtype(dtype) || !valid_dtype(out_dtype))
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm: dtype %d / out dtype %d", dtype, out_dtype);
+  if (M < 0 || N < 0 || d < 1 || k < 1 || k > d || ld_ai < k || ldb < N || ldy < N || M > kIntMax ||
+      N > kIntMax || d > kIntMax)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_gemm: bad sizes");
+  if (M == 0 || N == 0) return RMM_OK;
+  if (!A_I || !B || !idx || !Y) return fail(RMM_ERR_INVALID_ARG, "rmm_gemm: null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == RMM_F32) {
+    if (out_dtype != RMM_F32) return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm: fp32 inputs need fp32 output");
+    unsigned* err = device_error_word();
+    if (!err) return RMM_ERR_CUDA;
+    return from_cuda(launch_gemm_f32_simt(static_cast<const float*>(A_I), ld_ai, static_cast<const float*>(B), ldb,
+                                          idx, d, M, N, k, static_cast<float*>(Y), ldy, err, s),
+                     "rmm_gemm(f32): launch");
+  }
+  if (!aligned16(A_I) || !aligned16(B) || !aligned16(Y) || ld_ai % 8 || ldb % 8)
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm(bf16): needs 16-byte aligned A_I/B/Y, ld_ai and ldb multiples of 8");
+  if (((M + 127) / 128) * ((N + 255) / 256) > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm: too many tiles");
+  const size_t need = rmm_gemm_workspace_size(dtype, N, k);
+  if (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
+    return fail(RMM_ERR_WORKSPACE, "rmm_gemm: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes, need);
+  unsigned* err = device_error_word();
+  if (!err) return RMM_ERR_CUDA;
+  const int64_t ld_bi = round_up(N, 8);
+  cudaError_t e = launch_gather_rows(B, d, N * 2, ldb * 2, idx, k, ws, ld_bi * 2, err, s);
+  if (e != cudaSuccess) return from_cuda(e, "rmm_gemm: row gather launch");
+  e = launch_gemm_bf16_tc(A_I, ld_ai, ws, ld_bi, M, N, k, Y, out_dtype, ldy, err, s);
+  if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+  return from_cuda(e, "rmm_gemm(bf16): launch");
+}
+
+size_t rmm_matmul_workspace_size(int dtype, int64_t M, int64_t d, int64_t N, double rho) {
+  if (!valid_dtype(dtype) || M < 0 || d < 1 || N < 0) return 0;
+  const MatmulWs w = matmul_ws(dtype, M, d, N, rho);
+  return w.k < 1 ? 0 : w.total;
+}
+
+rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t M, int64_t d, int64_t N,
+                      double rho, int dtype, void* Y, int out_dtype, int64_t ldy, int32_t* idx_out, float* ss_out,
+                      void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (!valid_dtype(dtype) || !valid_dtype(out_dtype))
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul: dtype %d / out dtype %d", dtype, out_dtype);
+  const int64_t k = k_from_rho_impl(rho, d);
+  if (k < 1) return fail(RMM_ERR_INVALID_ARG, "rmm_matmul: rho %g outside (0,1] or d < 1", rho);
+  if (M < 0 || N < 0 || lda < d || ldb < N || ldy < N) return fail(RMM_ERR_INVALID_ARG, "rmm_matmul: bad sizes");
+  if (!A || !B || !Y) return fail(RMM_ERR_INVALID_ARG, "rmm_matmul: null pointer");
+  const MatmulWs w = matmul_ws(dtype, M, d, N, rho);
+  if (!ws || ws_bytes < w.total || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
+    return fail(RMM_ERR_WORKSPACE, "rmm_matmul: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes,
+                w.total);
+  char* base = static_cast<char*>(ws);
+  float* ss = ss_out ? ss_out : reinterpret_cast<float*>(base + w.ss);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+  void* score_ws = base + w.score;
+  void* ai = base + w.ai;
+  rmm_status st = rmm_score(A, dtype, 1, M, d, lda, 0, ss, d, 0, score_ws, score_workspace_bytes(dtype, 1, M, d), stream);
+  if (st != RMM_OK) return st;
+  st = rmm_topk(ss, 1, d, d, k, idx, k, stream);
+  if (st != RMM_OK) return st;
+  st = rmm_compact(A, dtype, M, d, lda, idx, k, ai, w.ld_ai, stream);
+  if (st != RMM_OK) return st;
+  return rmm_gemm(ai, w.ld_ai, B, ldb, idx, d, M, N, k, dtype, Y, out_dtype, ldy, base + w.bi, w.total - w.bi,
+                  stream);
+}
+
+size_t rmm_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D, double rho_d,
+                                    double rho_t) {
+  const int64_t kd = k_from_rho_impl(rho_d, D), kt = k_from_rho_impl(rho_t, S);
+  if (kd < 1 || kt < 1 || B < 1 || Hq < 1 || Hkv < 1) return 0;
+  return attention_workspace_bytes(B, Hq, Hkv, S, D, kd, kt);
+}
+
+rmm_status rmm_attention(const void* Q, const void* K, const void* V, int64_t B, int64_t Hq, int64_t Hkv, int64_t S,
+                         int64_t D, double rho_d, double rho_t, float scale, void* O, int out_dtype, int32_t* idx_d,
+                         int32_t* idx_t, float* lse, float* tscore, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (!valid_dtype(out_dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_attention: out dtype %d", out_dtype);
+  if (!Q || !K || !V || !O) return fail(RMM_ERR_INVALID_ARG, "rmm_attention: null pointer");
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || S < 1 || S > (1LL << 24) || B * Hq > 65535)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_attention: bad sizes");
+  if (D != 64 && D != 128) return fail(RMM_ERR_UNSUPPORTED, "rmm_attention: head_dim %lld (64 or 128 only)", (long long)D);
+  const int64_t kd = k_from_rho_impl(rho_d, D), kt = k_from_rho_impl(rho_t, S);
+  if (kd < 1 || kt < 1) return fail(RMM_ERR_INVALID_ARG, "rmm_attention: rho outside (0,1]");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_attention: tensors must be 16-byte aligned");
+  const size_t need = attention_workspace_bytes(B, Hq, Hkv, S, D, kd, kt);
+  if (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
+    return fail(RMM_ERR_WORKSPACE, "rmm_attention: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes,
+                need);
+  unsigned* err = device_error_word();
+  if (!err) return RMM_ERR_CUDA;
+  if (!(scale > 0.f)) scale = 1.0f / std::sqrt(static_cast<float>(D));
+  const cudaError_t e = launch_attention(Q, K, V, B, Hq, Hkv, S, D, kd, kt, scale, O, out_dtype, idx_d, idx_t, lse,
+                                         tscore, ws, err, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return fail(RMM_ERR_UNSUPPORTED, "rmm_attention: %s", g_last_error.c_str());
+  return from_cuda(e, "rmm_attention: launch");
+}
+
+}  // extern "C"

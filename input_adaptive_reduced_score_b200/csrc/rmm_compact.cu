@@ -1,0 +1,133 @@
+// rmm_compact.cu — the reduced operands of A_{:,I} B_{I,:} (Reduced Matrix
+// Multiplication technical summary, Metodología › Mecanismo Central):
+//   compact_kernel      A_I[:, r] = A[:, I_r]   (column gather of the activation)
+//   gather_rows_kernel  B_I[r, :] = B[I_r, :]   (row gather of the weight)
+//
+// HBM-bound gather.  Each thread produces 8 consecutive output columns of one
+// row (one 16-byte store for bf16): it reads 8 indices, gathers the 8 source
+// elements through the read-only cache (the kept indices are increasing, so a
+// warp's 256 gathers cover a short run of the source row and reuse its
+// sectors), and writes them with one vector store.  A 256-thread CTA covers
+// 2048 output columns of one row.
+#include <cuda_bf16.h>
+
+#include "rmm_device.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+constexpr int kCompactThreads = 256;
+constexpr int kPerThread = 8;
+constexpr int64_t kColsPerCta = kCompactThreads * kPerThread;
+
+template <typename T>
+__global__ void __launch_bounds__(kCompactThreads) compact_kernel(const T* __restrict__ A, int64_t M, int64_t d,
+                                                                  int64_t lda, const int32_t* __restrict__ idx,
+                                                                  int64_t k, T* __restrict__ AI, int64_t ld_ai,
+                                                                  int64_t chunks, bool vec_ok, unsigned* err) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) / chunks;
+  const int64_t chunk = static_cast<int64_t>(blockIdx.x) % chunks;
+  const int64_t c0 = chunk * kColsPerCta + static_cast<int64_t>(threadIdx.x) * kPerThread;
+  if (row >= M || c0 >= k) return;
+  const T* a = A + row * lda;
+  T* o = AI + row * ld_ai + c0;
+  alignas(16) T v[kPerThread];
+  bool bad = false;
+#pragma unroll
+  for (int e = 0; e < kPerThread; ++e) {
+    v[e] = T(0.f);
+    if (c0 + e < k) {
+      const int32_t j = __ldg(idx + c0 + e);
+      if (j >= 0 && j < d) {
+        v[e] = __ldg(a + j);
+      } else {
+        bad = true;
+      }
+    }
+  }
+  if (bad) record_error(err, kDevErrBadIndex);
+  if (vec_ok && c0 + kPerThread <= k) {
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(v);
+    } else {
+      reinterpret_cast<float4*>(o)[0] = *reinterpret_cast<const float4*>(&v[0]);
+      reinterpret_cast<float4*>(o)[1] = *reinterpret_cast<const float4*>(&v[4]);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPerThread; ++e)
+      if (c0 + e < k) o[e] = v[e];
+  }
+}
+
+// One CTA per kept row: the row I_r of B is copied whole with 16-byte loads and
+// stores, four in flight per thread (rows are contiguous, so this is a pure
+// streaming copy); a row length that is not a multiple of 16 bytes ends with
+// 2-byte copies.  Out-of-range indices produce a zero row and are flagged.
+constexpr int kGatherThreads = 256;
+
+__global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint4* __restrict__ B, int64_t d,
+                                                                       int64_t vecs, int64_t tail_halves,
+                                                                       int64_t ldb_vec, const int32_t* __restrict__ idx,
+                                                                       int64_t k, uint4* __restrict__ BI,
+                                                                       int64_t ldbi_vec, unsigned* err) {
+  const int64_t r = blockIdx.x;
+  if (r >= k) return;
+  const int32_t j = __ldg(idx + r);
+  uint4* dst = BI + r * ldbi_vec;
+  if (j < 0 || j >= d) {
+    if (threadIdx.x == 0) record_error(err, kDevErrBadIndex);
+    for (int64_t v = threadIdx.x; v < vecs; v += kGatherThreads) dst[v] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x < tail_halves) reinterpret_cast<uint16_t*>(dst + vecs)[threadIdx.x] = 0;
+    return;
+  }
+  const uint4* src = B + static_cast<int64_t>(j) * ldb_vec;
+  if (threadIdx.x < tail_halves)  // bytes past the last whole 16-byte vector of the row
+    reinterpret_cast<uint16_t*>(dst + vecs)[threadIdx.x] = reinterpret_cast<const uint16_t*>(src + vecs)[threadIdx.x];
+  int64_t v = threadIdx.x;
+  for (; v + 3 * kGatherThreads < vecs; v += 4 * kGatherThreads) {
+    const uint4 a0 = __ldcs(src + v);
+    const uint4 a1 = __ldcs(src + v + kGatherThreads);
+    const uint4 a2 = __ldcs(src + v + 2 * kGatherThreads);
+    const uint4 a3 = __ldcs(src + v + 3 * kGatherThreads);
+    dst[v] = a0;
+    dst[v + kGatherThreads] = a1;
+    dst[v + 2 * kGatherThreads] = a2;
+    dst[v + 3 * kGatherThreads] = a3;
+  }
+  for (; v < vecs; v += kGatherThreads) dst[v] = __ldcs(src + v);
+}
+
+}  // namespace
+
+cudaError_t launch_gather_rows(const void* B, int64_t d, int64_t row_bytes, int64_t ldb_bytes, const int32_t* idx,
+                               int64_t k, void* B_I, int64_t ldbi_bytes, unsigned* err, cudaStream_t stream) {
+  if (k == 0 || row_bytes == 0) return cudaSuccess;
+  if (k > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  gather_rows_kernel<<<static_cast<unsigned>(k), kGatherThreads, 0, stream>>>(
+      static_cast<const uint4*>(B), d, row_bytes / 16, (row_bytes % 16) / 2, ldb_bytes / 16, idx, k,
+      static_cast<uint4*>(B_I), ldbi_bytes / 16, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64_t lda, const int32_t* idx,
+                           int64_t k, void* A_I, int64_t ld_ai, unsigned* err, cudaStream_t stream) {
+  if (M == 0) return cudaSuccess;
+  const int64_t chunks = (k + kColsPerCta - 1) / kColsPerCta;
+  const int64_t blocks = M * chunks;
+  const size_t elt = dtype == 1 ? 2 : 4;
+  const bool vec_ok = reinterpret_cast<uintptr_t>(A_I) % 16 == 0 && (ld_ai * elt) % 16 == 0;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  if (dtype == 1) {
+    compact_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kCompactThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(A), M, d, lda, idx, k, static_cast<__nv_bfloat16*>(A_I), ld_ai, chunks,
+        vec_ok, err);
+  } else {
+    compact_kernel<float><<<static_cast<unsigned>(blocks), kCompactThreads, 0, stream>>>(
+        static_cast<const float*>(A), M, d, lda, idx, k, static_cast<float*>(A_I), ld_ai, chunks, vec_ok, err);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace rmm

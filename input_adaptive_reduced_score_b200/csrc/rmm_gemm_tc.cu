@@ -1,0 +1,344 @@
+// rmm_gemm_tc.cu — the reduced product Y = A_I · B_I on the 5th-generation
+// tensor cores, where A_I = A[:, I] and B_I = B[I, :] are the compacted
+// operands (Reduced Matrix Multiplication technical summary, Metodología ›
+// Mecanismo Central: compute A_{:,I} B_{I,:} instead of AB).
+//
+// Persistent, warp-specialised kernel, one CTA per SM, 128 x 256 output tiles,
+// 64-deep K blocks, 4-stage shared-memory ring, fp32 accumulators in tensor
+// memory (two 256-column buffers, so the epilogue of one tile overlaps the
+// main loop of the next).
+//   warp 0     producer (one lane): per k-block, one TMA load of the A_I tile
+//              (128 rows x 64, K-major) and four of the B_I tile (64 rows x 64
+//              columns each, MN-major), all with 128-byte swizzle; rows and
+//              columns past M, N or k read as zero.
+//   warp 1     TMEM allocation; one thread issues tcgen05.mma (M=128, N=256,
+//              K=16 per instruction, four per k-block) and tcgen05.commit to
+//              release stages and publish finished accumulators.
+//   warps 2-9  epilogue: two warps per TMEM lane quarter, each draining 128
+//              of the 256 columns with tcgen05.ld, converting, and storing rows
+//              of Y with 16-byte stores.
+// All waits are bounded (rmm_device.cuh); on a timeout the kernel records an
+// error, drains its own copies and MMAs, frees TMEM and returns.
+//
+// Why B_I is gathered beforehand rather than inside this kernel: gathering
+// the k rows of B per k-block with tile::gather4 (64 four-row TMA gathers per
+// stage) or with 16-byte cp.async was measured on B200 at about 2.2 TB/s of
+// operand delivery, an order of magnitude short of what the tensor cores
+// consume; the streaming row copy plus large-box TMA tiles is faster overall.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "rmm_device.cuh"
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_STAGE = BM * BK * 2;   // 16 KB
+constexpr int B_STAGE = BK * BN * 2;   // 32 KB
+constexpr int B_CHUNK = BK * 128;      // one 64-column chunk of a B stage: 8 KB
+constexpr int MMA_WARP = 1;
+constexpr int EPI_WARP0 = 2;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + BAR_BYTES + 1024;
+constexpr unsigned long long kDrainNs = 100000000ull;  // 100 ms
+
+static_assert(BK == 64 && BN == 256, "stage layout assumes 64 x 256 B stages");
+
+struct Bars {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t accfull[2];
+  uint64_t accempty[2];
+  uint64_t drain;
+  uint32_t tmem_slot;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= BAR_BYTES, "barrier block");
+
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kDrainNs) return false;
+  }
+  return true;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, int M,
+                        int N, int K, void* __restrict__ Y, int out_f32, int64_t ldy, int y_vec_ok, unsigned* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+  const uint32_t base = smem_u32(smem);
+  Bars* bars = reinterpret_cast<Bars*>(smem + STAGES * (A_STAGE + B_STAGE));
+  volatile int* abort_flag = &bars->abort_flag;
+  auto sA = [&](uint32_t s) { return base + s * A_STAGE; };
+  auto sB = [&](uint32_t s) { return base + STAGES * A_STAGE + s * B_STAGE; };
+  auto full = [&](uint32_t s) { return smem_u32(&bars->full[s]); };
+  auto empty = [&](uint32_t s) { return smem_u32(&bars->empty[s]); };
+  auto accfull = [&](uint32_t b) { return smem_u32(&bars->accfull[b]); };
+  auto accempty = [&](uint32_t b) { return smem_u32(&bars->accempty[b]); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_m = (M + BM - 1) / BM, num_n = (N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int nk = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full(s), 1);   // producer: arrive + expected transaction bytes
+      mbar_init(empty(s), 1);  // tcgen05.commit
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accfull(b), 1);           // tcgen05.commit
+      mbar_init(accempty(b), EPI_WARPS);  // one arrive per epilogue warp
+    }
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_u32(&bars->tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int m_blk = tile % num_m, n_blk = tile / num_m;
+        const int n0 = n_blk * BN;
+        const int live_chunks = min(4, (N - n0 + 63) / 64);
+        const uint32_t stage_bytes = A_STAGE + static_cast<uint32_t>(live_chunks) * B_CHUNK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, err, 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full(stage), stage_bytes);
+          tma_load_2d(sA(stage), &tmap_a, full(stage), kb * BK, m_blk * BM);
+          for (int c = 0; c < live_chunks; ++c)
+            tma_load_2d(sB(stage) + c * B_CHUNK, &tmap_b, full(stage), n0 + c * 64, kb * BK);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // the copies this thread issued must land before the CTA may exit
+      uint32_t st = stage, ph = phase;
+      const uint32_t n = issued < STAGES ? issued : STAGES;
+      for (uint32_t j = 0; j < n; ++j) {
+        if (st == 0) {
+          st = STAGES - 1;
+          ph ^= 1u;
+        } else {
+          --st;
+        }
+        wait_drain(full(st), ph);
+      }
+    }
+    __syncwarp();
+  } else if (warp == MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, /*a_mn=*/false, /*b_mn=*/true);
+    uint32_t stage = 0, phase = 0;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+      const uint32_t b = it & 1, acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(accempty(b), acc_phase ^ 1u, abort_flag, err, 2)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + b * BN;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(full(stage), phase, abort_flag, err, 3)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sA(stage) + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sB(stage) + kk * 16 * 128, B_CHUNK, 1024);
+            mma_f16_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(empty(stage));
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(accfull(b));
+      __syncwarp();
+    }
+    if (lane == 0) {
+      mma_commit(smem_u32(&bars->drain));
+      wait_drain(smem_u32(&bars->drain), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int qtr = warp & 3;                 // TMEM lanes 32*qtr ... 32*qtr+31
+    const int half = (warp - EPI_WARP0) / 4;  // columns [128*half, 128*half + 128)
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const uint32_t b = it & 1, acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(accfull(b), acc_phase, abort_flag, err, 4)) break;
+      tc_fence_after();
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      const int row = m_blk * BM + qtr * 32 + lane;
+      const uint32_t taddr = tmem_base + b * BN + half * 128 + (static_cast<uint32_t>(qtr * 32) << 16);
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(taddr + cc * 32, v);
+        tmem_wait_ld();
+        const int col0 = n_blk * BN + half * 128 + cc * 32;
+        if (row < M && col0 < N) {
+          if (out_f32) {
+            float* y = static_cast<float*>(Y) + static_cast<int64_t>(row) * ldy + col0;
+            if (y_vec_ok && col0 + 32 <= N) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                reinterpret_cast<float4*>(y)[i] =
+                    make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (col0 + e < N) y[e] = __uint_as_float(v[e]);
+            }
+          } else {
+            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y) + static_cast<int64_t>(row) * ldy + col0;
+            if (y_vec_ok && col0 + 32 <= N) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+                w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+                w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+                w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+                reinterpret_cast<uint4*>(y)[i] = w;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (col0 + e < N) y[e] = __float2bfloat16_rn(__uint_as_float(v[e]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accempty(b));
+    }
+  }
+
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool configure_kernel_once() {
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(gemm_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+// 2-D bf16 tensor map over a row-major [rows x cols] matrix (pitch in elements).
+bool encode_2d(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int64_t pitch, uint32_t box_cols,
+               uint32_t box_rows, const char* what) {
+  EncodeTiledFn encode = encode_fn();
+  if (!encode) {
+    set_error("rmm_gemm: cuTensorMapEncodeTiled entry point unavailable");
+    return false;
+  }
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(pitch) * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride, box,
+                            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("rmm_gemm: cuTensorMapEncodeTiled(%s) failed (CUresult %d)", what, static_cast<int>(r));
+    return false;
+  }
+  return true;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I, int64_t ld_bi, int64_t M, int64_t N,
+                                int64_t k, void* Y, int out_dtype, int64_t ldy, unsigned* err, cudaStream_t stream) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  CUtensorMap tmap_a, tmap_b;
+  if (!encode_2d(&tmap_a, A_I, k, M, ld_ai, BK, BM, "A_I")) return cudaErrorInvalidValue;
+  if (!encode_2d(&tmap_b, B_I, N, k, ld_bi, 64, BK, "B_I")) return cudaErrorInvalidValue;
+  if (!configure_kernel_once()) {
+    set_error("rmm_gemm: cannot raise the dynamic shared-memory limit to %d bytes", SMEM_BYTES);
+    return cudaErrorInvalidValue;
+  }
+  const int sms = device_sm_count();
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  const int out_f32 = out_dtype == 0 ? 1 : 0;
+  const size_t oelt = out_f32 ? 4 : 2;
+  const int y_vec_ok = (reinterpret_cast<uintptr_t>(Y) % 16 == 0) && ((ldy * oelt) % 16 == 0);
+  gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmap_a, tmap_b, static_cast<int>(M),
+                                                              static_cast<int>(N), static_cast<int>(k), Y, out_f32,
+                                                              ldy, y_vec_ok, err);
+  return cudaGetLastError();
+}
+
+}  // namespace rmm

@@ -1,0 +1,74 @@
+// rmm_internal.h — host-side declarations shared by the librmm translation
+// units (launchers, error reporting, device queries).  Not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace rmm {
+
+// Thread-local error message for rmm_last_error().
+void set_error(const char* fmt, ...);
+void clear_error();
+
+// Device address of the current device's error word (nullptr on failure;
+// the message is set).
+unsigned* device_error_word();
+
+// Streaming multiprocessor count of the current device (0 on failure).
+int device_sm_count();
+
+constexpr size_t kWsAlign = 256;
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- score (rmm_score.cu)
+struct ScorePlan {
+  int vec;          // elements per 16-byte vector
+  int col_threads;  // threads across columns in a CTA (power of two <= 64)
+  int row_groups;   // 256 / col_threads
+  int64_t strips;   // column strips
+  int64_t splits;   // row splits
+  int64_t rows_per_split;
+};
+ScorePlan score_plan(int dtype, int64_t batch, int64_t M, int64_t d);
+size_t score_workspace_bytes(int dtype, int64_t batch, int64_t M, int64_t d);
+cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
+                         int64_t batch_stride, float* ss, int64_t ld_ss, int sqrt_out, void* ws,
+                         cudaStream_t stream);
+
+// ---- top-k (rmm_topk.cu)
+cudaError_t launch_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k,
+                        int32_t* idx, int64_t ld_idx, cudaStream_t stream);
+
+// ---- compaction (rmm_compact.cu)
+cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64_t lda,
+                           const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai, unsigned* err,
+                           cudaStream_t stream);
+
+// Row gather B_I[r, :] = B[idx[r], :]; bases and pitches 16-byte aligned,
+// row_bytes even (checked by the caller).
+cudaError_t launch_gather_rows(const void* B, int64_t d, int64_t row_bytes, int64_t ldb_bytes, const int32_t* idx,
+                               int64_t k, void* B_I, int64_t ldbi_bytes, unsigned* err, cudaStream_t stream);
+
+// ---- reduced GEMM (rmm_gemm_tc.cu, rmm_gemm_simt.cu)
+// Returns cudaSuccess or an error; on a driver error in tensor-map encoding
+// the message is set and cudaErrorInvalidValue returned.
+// Dense tcgen05 GEMM on the compacted operands: Y = A_I [M x k] · B_I [k x N].
+cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I, int64_t ld_bi, int64_t M,
+                                int64_t N, int64_t k, void* Y, int out_dtype, int64_t ldy, unsigned* err,
+                                cudaStream_t stream);
+cudaError_t launch_gemm_f32_simt(const float* A_I, int64_t ld_ai, const float* B, int64_t ldb,
+                                 const int32_t* idx, int64_t d, int64_t M, int64_t N, int64_t k,
+                                 float* Y, int64_t ldy, unsigned* err, cudaStream_t stream);
+
+// ---- reduced attention (rmm_attention.cu)
+size_t attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D, int64_t kd,
+                                 int64_t kt);
+cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_t B, int64_t Hq,
+                             int64_t Hkv, int64_t S, int64_t D, int64_t kd, int64_t kt, float scale,
+                             void* O, int out_dtype, int32_t* idx_d, int32_t* idx_t, float* lse,
+                             float* tscore, void* ws, unsigned* err, cudaStream_t stream);
+
+}  // namespace rmm

@@ -1,0 +1,210 @@
+// rmm_score.cu — column scores ss_j = sum_i A[i,j]^2 (Reduced Matrix
+// Multiplication technical summary, Metodología › Estrategia de Selección:
+// s_j = ||A[:,j]||_2; the square keeps the ranking).
+//
+// HBM-bound design: each thread owns one 16-byte column vector (8 bf16 or 4
+// fp32 columns) and walks rows with 16-byte loads, so a warp reads 512
+// contiguous bytes of a row.  A 256-thread CTA is col_threads wide and
+// row_groups tall; CTAs tile (column strip, row split, batch).  Squares of bf16
+// values are exact in fp32 and accumulate with one rounding per row (fma).
+// Row groups combine by a fixed pairwise tree in shared memory; row splits are
+// combined by a second kernel in a fixed blocked order.  No atomics, so the
+// result depends only on the shape.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "rmm_internal.h"
+
+namespace rmm {
+namespace {
+
+constexpr int kScoreThreads = 256;
+constexpr int64_t kTargetCtas = 2368;  // 16 x 148: enough 256-thread CTAs to cover HBM latency
+constexpr int64_t kMinRowsPerSplit = 32;
+constexpr int64_t kMaxSplits = 64;
+
+template <typename T>
+struct Lanes;
+template <>
+struct Lanes<__nv_bfloat16> {
+  static constexpr int kVec = 8;
+  __device__ static void load(const __nv_bfloat16* p, float (&x)[8]) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  __device__ static float scalar(const __nv_bfloat16* p) { return __bfloat162float(p[0]); }
+};
+template <>
+struct Lanes<float> {
+  static constexpr int kVec = 4;
+  __device__ static void load(const float* p, float (&x)[4]) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    x[0] = v.x;
+    x[1] = v.y;
+    x[2] = v.z;
+    x[3] = v.w;
+  }
+  __device__ static float scalar(const float* p) { return __ldg(p); }
+};
+
+// Grid: x = column strip, y = row split, z = batch.
+template <typename T>
+__global__ void __launch_bounds__(kScoreThreads) score_partial_kernel(
+    const T* __restrict__ A, int64_t M, int64_t d, int64_t lda, int64_t batch_stride, int col_threads,
+    int64_t rows_per_split, bool vec_ok, float* __restrict__ out, int64_t out_batch_stride,
+    int64_t out_split_stride, int sqrt_out) {
+  constexpr int V = Lanes<T>::kVec;
+  __shared__ float red[kScoreThreads * V];
+  const int tx = threadIdx.x % col_threads;
+  const int ty = threadIdx.x / col_threads;
+  const int row_groups = kScoreThreads / col_threads;
+  const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * col_threads + tx) * V;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(M, r0 + rows_per_split);
+  const T* Ab = A + static_cast<int64_t>(blockIdx.z) * batch_stride;
+
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+
+  if (col0 < d) {
+    if (vec_ok && col0 + V <= d) {
+      int64_t r = r0 + ty;
+      // four independent 16-byte loads in flight per thread
+      for (; r + 3 * row_groups < r1; r += 4 * row_groups) {
+        float x0[V], x1[V], x2[V], x3[V];
+        Lanes<T>::load(Ab + r * lda + col0, x0);
+        Lanes<T>::load(Ab + (r + row_groups) * lda + col0, x1);
+        Lanes<T>::load(Ab + (r + 2 * row_groups) * lda + col0, x2);
+        Lanes<T>::load(Ab + (r + 3 * row_groups) * lda + col0, x3);
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          acc[e] = fmaf(x0[e], x0[e], acc[e]);
+          acc[e] = fmaf(x1[e], x1[e], acc[e]);
+          acc[e] = fmaf(x2[e], x2[e], acc[e]);
+          acc[e] = fmaf(x3[e], x3[e], acc[e]);
+        }
+      }
+      for (; r < r1; r += row_groups) {
+        float x0[V];
+        Lanes<T>::load(Ab + r * lda + col0, x0);
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] = fmaf(x0[e], x0[e], acc[e]);
+      }
+    } else {
+      for (int64_t r = r0 + ty; r < r1; r += row_groups) {
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          if (col0 + e < d) {
+            const float x = Lanes<T>::scalar(Ab + r * lda + col0 + e);
+            acc[e] = fmaf(x, x, acc[e]);
+          }
+        }
+      }
+    }
+  }
+
+  // pairwise tree over the row groups (fixed order)
+#pragma unroll
+  for (int e = 0; e < V; ++e) red[(ty * col_threads + tx) * V + e] = acc[e];
+  __syncthreads();
+  for (int s = row_groups / 2; s >= 1; s >>= 1) {
+    if (ty < s) {
+#pragma unroll
+      for (int e = 0; e < V; ++e) red[(ty * col_threads + tx) * V + e] += red[((ty + s) * col_threads + tx) * V + e];
+    }
+    __syncthreads();
+  }
+  if (ty == 0) {
+    float* o = out + static_cast<int64_t>(blockIdx.z) * out_batch_stride +
+               static_cast<int64_t>(blockIdx.y) * out_split_stride;
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      if (col0 + e < d) {
+        const float v = red[tx * V + e];
+        o[col0 + e] = sqrt_out ? sqrtf(v) : v;
+      }
+    }
+  }
+}
+
+// Sum the row-split partials of one column: blocks of 8 sequentially, then
+// the block sums sequentially (fixed order).  Grid: x = column blocks, y = batch.
+__global__ void score_finalize_kernel(const float* __restrict__ partial, int64_t d, int64_t splits,
+                                      float* __restrict__ ss, int64_t ld_ss, int sqrt_out) {
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (j >= d) return;
+  const float* p = partial + static_cast<int64_t>(blockIdx.y) * splits * d + j;
+  float total = 0.f;
+  for (int64_t s0 = 0; s0 < splits; s0 += 8) {
+    float blk = 0.f;
+    const int64_t s1 = min(splits, s0 + 8);
+    for (int64_t s = s0; s < s1; ++s) blk += p[s * d];
+    total += blk;
+  }
+  ss[static_cast<int64_t>(blockIdx.y) * ld_ss + j] = sqrt_out ? sqrtf(total) : total;
+}
+
+}  // namespace
+
+ScorePlan score_plan(int dtype, int64_t batch, int64_t M, int64_t d) {
+  ScorePlan p{};
+  p.vec = dtype == 1 ? 8 : 4;
+  const int64_t vecs = (d + p.vec - 1) / p.vec;
+  int ct = 1;
+  while (ct < 64 && ct < vecs) ct <<= 1;
+  p.col_threads = ct;
+  p.row_groups = kScoreThreads / ct;
+  p.strips = (vecs + ct - 1) / ct;
+  const int64_t base = std::max<int64_t>(1, p.strips * batch);
+  int64_t splits = (kTargetCtas + base - 1) / base;
+  splits = std::min(splits, std::max<int64_t>(1, (M + kMinRowsPerSplit - 1) / kMinRowsPerSplit));
+  splits = std::max<int64_t>(1, std::min(splits, kMaxSplits));
+  const int64_t rps = std::max<int64_t>(1, (M + splits - 1) / splits);
+  p.rows_per_split = rps;
+  p.splits = M > 0 ? (M + rps - 1) / rps : 1;
+  return p;
+}
+
+size_t score_workspace_bytes(int dtype, int64_t batch, int64_t M, int64_t d) {
+  const ScorePlan p = score_plan(dtype, batch, M, d);
+  if (p.splits <= 1) return 0;
+  return align_up(static_cast<size_t>(batch) * p.splits * d * sizeof(float), kWsAlign);
+}
+
+cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
+                         int64_t batch_stride, float* ss, int64_t ld_ss, int sqrt_out, void* ws,
+                         cudaStream_t stream) {
+  const ScorePlan p = score_plan(dtype, batch, M, d);
+  const size_t elt = dtype == 1 ? 2 : 4;
+  const bool vec_ok = (reinterpret_cast<uintptr_t>(A) % 16 == 0) && ((lda * elt) % 16 == 0) &&
+                      (batch == 1 || (batch_stride * elt) % 16 == 0);
+  const dim3 grid(static_cast<unsigned>(p.strips), static_cast<unsigned>(p.splits), static_cast<unsigned>(batch));
+  const bool direct = p.splits <= 1;
+  float* out = direct ? ss : static_cast<float*>(ws);
+  const int64_t out_bs = direct ? ld_ss : p.splits * d;
+  const int64_t out_ss = direct ? 0 : d;
+  const int sq = direct ? sqrt_out : 0;
+  if (dtype == 1) {
+    score_partial_kernel<__nv_bfloat16><<<grid, kScoreThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(A), M, d, lda, batch_stride, p.col_threads, p.rows_per_split, vec_ok, out,
+        out_bs, out_ss, sq);
+  } else {
+    score_partial_kernel<float><<<grid, kScoreThreads, 0, stream>>>(static_cast<const float*>(A), M, d, lda,
+                                                                    batch_stride, p.col_threads, p.rows_per_split,
+                                                                    vec_ok, out, out_bs, out_ss, sq);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || direct) return e;
+  const dim3 g2(static_cast<unsigned>((d + 255) / 256), static_cast<unsigned>(batch));
+  score_finalize_kernel<<<g2, 256, 0, stream>>>(static_cast<const float*>(ws), d, p.splits, ss, ld_ss, sqrt_out);
+  return cudaGetLastError();
+}
+
+}  // namespace rmm

