@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the reduced-matrix-multiplication hot path on B200.
+
+One step = the whole path on one batch of the MLP up/gate projection
+workload (X [4096 x 4096] bf16 activation with per-channel lognormal scale
+and 1% outlier channels, W [4096 x 14336] bf16 ~ N(0, 0.02^2), rho = 0.5):
+column scores -> top-k -> compaction of X -> row gather of W -> tcgen05
+reduced GEMM, every stage a librmm kernel called through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rmm|reference]
+
+Prints one JSON line (rank 0).  `value` is the effective throughput
+2*M*N*k / step time in TFLOP/s over all ranks (weak scaling: each rank runs
+its own batch, no data-path collective).  Timing: K steps between a barrier
+and a device synchronisation; each step is bracketed by CUDA events on the
+launching stream and the step times are summed; a 256 MiB buffer is written
+between steps (L2 flush) outside the event intervals; the max over ranks is
+reported.  `--impl reference` times the fp64 CPU oracle on a bounded sample of
+the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import faulthandler
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+faulthandler.enable()
+
+METRIC = "reduced-GEMM effective TFLOP/s & speedup vs dense bf16 at rho=0.5; % roofline"
+WORKLOAD = "MLP up/gate projection: X[4096x4096] bf16 (lognormal channel scale, 1% outliers x20) · W[4096x14336] bf16 N(0,0.02^2), rho=0.5"
+M, D, N, RHO = 4096, 4096, 14336, 0.5
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SOURCES = ["input_adaptive_reduced_score_b200/csrc/rmm_gemm_tc.cu",
+                "input_adaptive_reduced_score_b200/csrc/rmm_device.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rmm_gemm_tc_mlp_up_traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+def k_of(rho, d):
+    import math
+    return min(max(math.ceil(rho * d - 1e-9 * d), 1), d)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {k: float(j[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sources_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def traffic_per_launch():
+    """DRAM bytes per GEMM launch from the committed ncu capture, or None when
+    the kernel sources changed since it was taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        if t.get("sources_sha256") != sources_sha(GEMM_SOURCES):
+            return None
+        return float(t["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only)."""
+    NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+             0x1: "gpu_idle"}
+
+    @staticmethod
+    def _handle(nv, props):
+        """NVML handle of the torch device: by UUID, else by a formatted PCI bus id string."""
+        uuid = str(getattr(props, "uuid", "") or "")
+        if uuid:
+            try:
+                return nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                pass
+        bus_id = f"{int(props.pci_domain_id):08x}:{int(props.pci_bus_id):02x}:{int(props.pci_device_id):02x}.0"
+        return nv.nvmlDeviceGetHandleByPciBusId(bus_id)
+
+    def __init__(self, props):
+        self.samples, self.reasons, self.max_mhz, self.err = [], 0, None, None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(pynvml, props)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - reported, not fatal
+            self.nv, self.err = None, repr(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                fn = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                self.reasons |= fn(self.h)
+            except Exception as e:
+                self.err = repr(e)
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        names = sorted(n for bit, n in self.NAMES.items() if self.reasons & bit)
+        med = statistics.median(self.samples) if self.samples else None
+        out = {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+        if self.err:
+            out["error"] = self.err
+        return out
+
+    def rejected(self):
+        s = self.summary()
+        bad = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"} & set(s["reasons"])
+        stuck = (s["sm_mhz"] is not None and self.max_mhz and s["sm_mhz"] < 0.5 * self.max_mhz
+                 and not s["reasons"])
+        return bool(bad) or bool(stuck)
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample_step(oracle, Xf, Wf, rows, k):
+    """One bounded sample of the workload through the fp64 oracle: scores and
+    top-k over the sampled rows' activation, reduced product of those rows."""
+    A = Xf[rows]
+    ss = oracle.column_sq_norms(A)
+    idx = oracle.topk_indices(ss, k)
+    Y = oracle.reduced_matmul(A, Wf, idx)
+    return Y
+
+
+def cpu_oracle_inputs():
+    import workloads
+    import oracle
+    X = workloads.llm_activation_bf16(1, M, D)
+    Wb = workloads.weight_bf16(1, D, N)
+    return oracle, oracle.decode(X, "bf16"), oracle.decode(Wb, "bf16")
+
+
+def time_cpu_oracle(target_s=15.0):
+    """CPU baseline: the oracle as it stands on the host cores; the row count
+    of the sample is sized to about `target_s` seconds of work."""
+    oracle, Xf, Wf = cpu_oracle_inputs()
+    k = k_of(RHO, D)
+    t0 = time.perf_counter()
+    oracle_sample_step(oracle, Xf, Wf, list(range(32)), k)
+    t32 = time.perf_counter() - t0
+    rows_n = int(max(32, min(M, 32 * target_s / max(t32, 1e-3))) // 32 * 32)
+    rows = list(range(rows_n))
+    t0 = time.perf_counter()
+    oracle_sample_step(oracle, Xf, Wf, rows, k)
+    t = time.perf_counter() - t0
+    tflops = 2.0 * rows_n * N * k / t / 1e12
+    return {"value": tflops, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle on the first {rows_n} of {M} rows (scores, top-k and reduced product of "
+                      f"the sampled rows), {t:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle, timed step by step on bounded samples."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    oracle, Xf, Wf = cpu_oracle_inputs()
+    k = k_of(RHO, D)
+    t0 = time.perf_counter()
+    oracle_sample_step(oracle, Xf, Wf, list(range(16)), k)
+    t16 = time.perf_counter() - t0
+    budget = 150.0 / (args.steps + args.warmup)
+    rows_n = int(max(8, min(M, 16 * budget / max(t16, 1e-3))) // 8 * 8)
+    for i in range(args.warmup):
+        oracle_sample_step(oracle, Xf, Wf, list(range(rows_n)), k)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        r0 = (i * rows_n) % (M - rows_n + 1)
+        oracle_sample_step(oracle, Xf, Wf, list(range(r0, r0 + rows_n)), k)
+    t = time.perf_counter() - t0
+    value = 2.0 * rows_n * N * k * args.steps / t / 1e12
+    cores = cpu_threads()
+    sample = f"each step: fp64 oracle on {rows_n} of {M} rows (scores, top-k, reduced product)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "M": M, "d": D, "N": N, "rho": RHO, "k": k},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def aggregate(local_ms, local_flops, world):
+    """Max of step-time totals and sum of flops over ranks (no-op at world 1)."""
+    import torch
+    if world == 1:
+        return local_ms, local_flops
+    import torch.distributed as dist
+    t = torch.tensor([local_ms], dtype=torch.float64)
+    f = torch.tensor([local_flops], dtype=torch.float64)
+    if dist.get_backend() == "nccl":
+        t, f = t.cuda(), f.cuda()
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(f, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(f.item())
+
+
+def run_rmm(args):
+    import numpy as np
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    import input_adaptive_reduced_score_b200 as R
+    import workloads
+    from tests.helpers import bf16_tensor
+
+    dev = torch.device("cuda", local_rank)
+    k = R.rmm_k_from_rho(RHO, D)
+    X = bf16_tensor(workloads.llm_activation_bf16(1 + 101 * rank, M, D), dev)
+    Wt = bf16_tensor(workloads.weight_bf16(1, D, N), dev)
+    ss = torch.empty(D, dtype=torch.float32, device=dev)
+    idx = torch.empty(k, dtype=torch.int32, device=dev)
+    AI = torch.empty((M, (k + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)[:, :k]
+    BI = torch.empty((k, N), dtype=torch.bfloat16, device=dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    sws_n = R.rmm_score_workspace_size(R.RMM_BF16, 1, M, D)
+    sws = torch.empty(max(sws_n, 256), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    stages = ["score", "topk", "compact", "gather", "gemm"]
+    launches_per_step = (2 if sws_n else 1) + 4
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        R.rmm_score(X, out=ss, ws=sws)
+        if ev is not None:
+            ev[1].record(stream)
+        R.rmm_topk(ss, k, out=idx)
+        if ev is not None:
+            ev[2].record(stream)
+        R.rmm_compact(X, idx, out=AI)
+        if ev is not None:
+            ev[3].record(stream)
+        R.rmm_gather_rows(Wt, idx, out=BI)
+        if ev is not None:
+            ev[4].record(stream)
+        R.rmm_gemm_compacted(AI, BI, out=Y)
+        if ev is not None:
+            ev[5].record(stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def timed(fn, steps, nev):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        for i in range(steps):
+            flush.zero_()
+            fn(evs[i])
+        torch.cuda.synchronize(dev)
+        barrier()
+        return [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nev - 1)] for i in range(steps)]
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during warm-up")
+
+    remeasured = False
+    for attempt in range(2):
+        with ClockSampler(torch.cuda.get_device_properties(dev)) as clk:
+            per = timed(step, args.steps, 6)
+        if not clk.rejected():
+            break
+        remeasured = True
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the timed steps")
+    step_ms = [sum(p) for p in per]
+    stage_ms = {s: statistics.mean(p[j] for p in per) for j, s in enumerate(stages)}
+    local_ms = sum(step_ms)
+    flops_step = 2.0 * M * N * k
+    tot_ms, tot_flops = aggregate(local_ms, flops_step * args.steps, world)
+    value = tot_flops / (tot_ms * 1e-3) / 1e12
+
+    # dense cuBLAS bf16 at the same shape, same flush protocol
+    def dense(ev):
+        ev[0].record(stream)
+        torch.matmul(X, Wt, out=Y)
+        ev[1].record(stream)
+    for _ in range(3):
+        torch.matmul(X, Wt, out=Y)
+    dense_ms = statistics.mean(p[0] for p in timed(dense, min(args.steps, 100), 2))
+
+    # end to end through the public API: pinned host X in, pinned host Y out
+    Xh = X.cpu().pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty_like(X)
+    mws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, M, D, N, RHO), dtype=torch.uint8, device=dev)
+
+    def e2e(ev):
+        ev[0].record(stream)
+        Xd.copy_(Xh, non_blocking=True)
+        R.rmm_matmul(Xd, Wt, RHO, out=Y, ws=mws)
+        Yh.copy_(Y, non_blocking=True)
+        ev[1].record(stream)
+    for _ in range(3):
+        e2e([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    e2e_ms = [p[0] for p in timed(e2e, args.e2e_steps, 2)]
+    e2e_tot, e2e_flops = aggregate(sum(e2e_ms), flops_step * len(e2e_ms), world)
+    e2e_value = e2e_flops / (e2e_tot * 1e-3) / 1e12
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the dense / end-to-end runs")
+
+    peaks, peak_src = load_peaks()
+    gemm_ms = stage_ms["gemm"]
+    achieved = flops_step / (gemm_ms * 1e-3) / 1e12
+    traffic = traffic_per_launch()
+    hbm = peaks["hbm_gbs"]
+    kbytes = {"score": 2.0 * M * D, "topk": 4.0 * D + 4.0 * k, "compact": 2.0 * M * D + 2.0 * M * k,
+              "gather": 4.0 * k * N}
+    kernels = {}
+    for s in stages:
+        us = stage_ms[s] * 1e3
+        if s == "gemm":
+            kernels[s] = {"us": us, "TFLOP/s": achieved}
+        else:
+            gbs = kbytes[s] / (stage_ms[s] * 1e-3) / 1e9
+            kernels[s] = {"us": us, "GB/s": gbs, "frac_hbm": gbs / hbm}
+    path_ms = statistics.mean(step_ms)
+    min_bytes = 2.0 * M * D + 2.0 * k * N + 2.0 * M * N
+    path_roof_ms = max(flops_step / (peaks["bf16_tflops"] * 1e12), min_bytes / (hbm * 1e9)) * 1e3
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Philox inputs of the workload's shape and distribution)",
+            "config": {"workload": WORKLOAD, "M": M, "d": D, "N": N, "rho": RHO, "k": k,
+                       "l2": "256 MiB buffer written between steps, outside the timed intervals",
+                       "parallelism": f"independent batch per GPU x{world}"},
+            "speedup_vs_dense": dense_ms / path_ms, "dense_ms": dense_ms,
+            "dense_tflops": 2.0 * M * N * D / (dense_ms * 1e-3) / 1e12,
+            "dense_equivalent_tflops": 2.0 * M * N * D / (path_ms * 1e-3) / 1e12,
+            "path_roofline_frac": path_roof_ms / path_ms,
+            "roofline": {"kernel": "gemm_bf16_tc_kernel", "bound": "tensor", "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": traffic, "peak_source": f"{peak_src} (burst bf16)"},
+            "kernels": kernels,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(X.numel() * 2),
+                    "d2h_bytes_per_step": int(Y.numel() * 2), "api": "rmm_matmul"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(), "clock_remeasured": remeasured,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = time_cpu_oracle()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus and not (args.impl == "reference"):
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("for --gpus > 1 launch with torch.distributed.run (one rank per GPU)")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_rmm(args)
+
+
+if __name__ == "__main__":
+    main()

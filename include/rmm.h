@@ -144,6 +144,14 @@ RMM_API rmm_status rmm_gemm(const void* A_I, int64_t ld_ai, const void* B, int64
                             int dtype, void* Y, int out_dtype, int64_t ldy,
                             void* ws, size_t ws_bytes, void* stream);
 
+/* Y = A_I · B_I on already-compacted bf16 operands: A_I [M x k] (ld_ai) and
+ * B_I [k x N] (ld_bi), i.e. the tensor-core stage of rmm_gemm without its row
+ * gather (Metodología › Mecanismo Central).  16-byte aligned A_I, B_I, Y;
+ * ld_ai, ld_bi multiples of 8.  No workspace. */
+RMM_API rmm_status rmm_gemm_compacted(const void* A_I, int64_t ld_ai, const void* B_I, int64_t ld_bi,
+                                      int64_t M, int64_t N, int64_t k, void* Y, int out_dtype,
+                                      int64_t ldy, void* stream);
+
 /* ------------------------------------------------------------------ whole path
  * The method end to end on one product: ss = score(A); I = topk(ss, k) with
  * k = rmm_k_from_rho(rho, d); A_I = compact(A, I); B_I = gather_rows(B, I);

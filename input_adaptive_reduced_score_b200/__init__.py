@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "lib", "LIB_PATH", "RMMError", "RMM_F32", "RMM_BF16", "rmm_abi_version", "rmm_k_from_rho",
     "rmm_device_error", "rmm_score", "rmm_score_workspace_size", "rmm_topk", "rmm_compact", "rmm_gather_rows",
-    "rmm_gemm", "rmm_gemm_workspace_size",
+    "rmm_gemm", "rmm_gemm_workspace_size", "rmm_gemm_compacted",
     "rmm_matmul", "rmm_matmul_workspace_size", "rmm_attention", "rmm_attention_workspace_size",
     "exported_symbols", "declared_symbols",
 ]
@@ -63,6 +63,7 @@ _sig("rmm_gather_rows", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_vp, c_i64, c_
 _sig("rmm_gemm_workspace_size", c_sz, c_int, c_i64, c_i64)
 _sig("rmm_gemm", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_int, c_vp, c_int, c_i64, c_vp,
      c_sz, c_vp)
+_sig("rmm_gemm_compacted", c_int, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_int, c_i64, c_vp)
 _sig("rmm_matmul_workspace_size", c_sz, c_int, c_i64, c_i64, c_i64, c_dbl)
 _sig("rmm_matmul", c_int, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_dbl, c_int, c_vp, c_int, c_i64, c_vp, c_vp,
      c_vp, c_sz, c_vp)
@@ -229,6 +230,23 @@ def rmm_gemm(A_I: torch.Tensor, B: torch.Tensor, idx: torch.Tensor, out: torch.T
     w, wn = _workspace(lib.rmm_gemm_workspace_size(dt, N, k), A_I.device, ws)
     _check(lib.rmm_gemm(_ptr(A_I), ld_ai, _ptr(B), ldb, _ptr(idx), d, M, N, k, dt, _ptr(out),
                         _dtype_code(out), ldy, _ptr(w), wn, _stream_ptr(stream)), "rmm_gemm")
+    return out
+
+
+def rmm_gemm_compacted(A_I: torch.Tensor, B_I: torch.Tensor, out: torch.Tensor = None, out_dtype=None,
+                       stream=None):
+    """Y = A_I · B_I on compacted bf16 operands A_I [M x k], B_I [k x N]."""
+    ld_ai = _row_major(A_I, "A_I")
+    ld_bi = _row_major(B_I, "B_I")
+    M, k = A_I.shape
+    N = B_I.shape[1]
+    if B_I.shape[0] != k:
+        raise ValueError("A_I and B_I disagree on k")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or A_I.dtype, device=A_I.device)
+    ldy = _row_major(out, "Y")
+    _check(lib.rmm_gemm_compacted(_ptr(A_I), ld_ai, _ptr(B_I), ld_bi, M, N, k, _ptr(out), _dtype_code(out), ldy,
+                                  _stream_ptr(stream)), "rmm_gemm_compacted")
     return out
 
 

@@ -280,6 +280,26 @@ rmm_status rmm_gemm(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, 
   return from_cuda(e, "rmm_gemm(bf16): launch");
 }
 
+rmm_status rmm_gemm_compacted(const void* A_I, int64_t ld_ai, const void* B_I, int64_t ld_bi, int64_t M, int64_t N,
+                              int64_t k, void* Y, int out_dtype, int64_t ldy, void* stream) {
+  clear_error();
+  if (!valid_dtype(out_dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm_compacted: out dtype %d", out_dtype);
+  if (M < 0 || N < 0 || k < 1 || ld_ai < k || ld_bi < N || ldy < N || M > kIntMax || N > kIntMax || k > kIntMax)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_gemm_compacted: bad sizes");
+  if (M == 0 || N == 0) return RMM_OK;
+  if (!A_I || !B_I || !Y) return fail(RMM_ERR_INVALID_ARG, "rmm_gemm_compacted: null pointer");
+  if (!aligned16(A_I) || !aligned16(B_I) || !aligned16(Y) || ld_ai % 8 || ld_bi % 8)
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm_compacted: needs 16-byte aligned operands, ld_ai/ld_bi multiples of 8");
+  if (((M + 127) / 128) * ((N + 255) / 256) > kIntMax)
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm_compacted: too many tiles");
+  unsigned* err = device_error_word();
+  if (!err) return RMM_ERR_CUDA;
+  const cudaError_t e =
+      launch_gemm_bf16_tc(A_I, ld_ai, B_I, ld_bi, M, N, k, Y, out_dtype, ldy, err, static_cast<cudaStream_t>(stream));
+  if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+  return from_cuda(e, "rmm_gemm_compacted: launch");
+}
+
 size_t rmm_matmul_workspace_size(int dtype, int64_t M, int64_t d, int64_t N, double rho) {
   if (!valid_dtype(dtype) || M < 0 || d < 1 || N < 0) return 0;
   const MatmulWs w = matmul_ws(dtype, M, d, N, rho);
