@@ -97,6 +97,27 @@ RMM_API rmm_status rmm_score(const void* A, int dtype, int64_t batch, int64_t M,
                      int64_t lda, int64_t batch_stride, float* ss, int64_t ld_ss,
                      int sqrt_out, void* ws, size_t ws_bytes, void* stream);
 
+/* rmm_score for callers that cannot allocate device memory: an inference-
+ * engine plugin handed only its input and output buffers, or a process whose
+ * device memory is all reserved up front by an external pool (where an extra
+ * cudaMalloc fails, and synchronises the device even when it succeeds).  The
+ * paper has no counterpart; this is a library-side convenience.
+ * Same arguments and result as rmm_score, minus the workspace: the row-split
+ * partial sums live in a fixed array of RMM_SCORE_NOALLOC_MAX_BYTES inside the
+ * library, which every GPU that loads the library holds until exit.  Shapes
+ * whose partial sums need more (rmm_score_workspace_size above the limit) are
+ * rejected with RMM_ERR_INVALID_ARG and a message.  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current); make that first call before any stream capture.  No
+ * call allocates or frees memory.  All calls share the array and each call
+ * overwrites it in full before reading it, so nothing has to be cleared
+ * between calls; calls that overlap on the GPU race on it and must be
+ * serialised by the caller. */
+#define RMM_SCORE_NOALLOC_MAX_BYTES ((size_t)8 << 20)
+RMM_API rmm_status rmm_score_noalloc(const void* A, int dtype, int64_t batch, int64_t M, int64_t d,
+                                     int64_t lda, int64_t batch_stride, float* ss, int64_t ld_ss,
+                                     int sqrt_out, void* stream);
+
 /* ------------------------------------------------------------------ top-k
  * For each of `batch` score rows (row b at scores + b*ld_s, length d), writes
  * the k indices with the largest scores to idx + b*ld_idx, in ascending index

@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "lib", "LIB_PATH", "RMMError", "RMM_F32", "RMM_BF16", "rmm_abi_version", "rmm_k_from_rho",
-    "rmm_device_error", "rmm_score", "rmm_score_workspace_size", "rmm_topk", "rmm_compact", "rmm_gather_rows",
+    "rmm_device_error", "rmm_score", "rmm_score_workspace_size", "rmm_score_noalloc", "rmm_topk", "rmm_compact", "rmm_gather_rows",
     "rmm_gemm", "rmm_gemm_workspace_size", "rmm_gemm_compacted",
     "rmm_matmul", "rmm_matmul_workspace_size", "rmm_attention", "rmm_attention_workspace_size",
     "exported_symbols", "declared_symbols",
@@ -57,6 +57,7 @@ _sig("rmm_k_from_rho", c_i64, c_dbl, c_i64)
 _sig("rmm_device_error", c_int, c_vp, c_int, ctypes.POINTER(ctypes.c_uint))
 _sig("rmm_score_workspace_size", c_sz, c_int, c_i64, c_i64, c_i64)
 _sig("rmm_score", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_int, c_vp, c_sz, c_vp)
+_sig("rmm_score_noalloc", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_int, c_vp)
 _sig("rmm_topk", c_int, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp)
 _sig("rmm_compact", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp)
 _sig("rmm_gather_rows", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp)
@@ -168,6 +169,23 @@ def rmm_score(A: torch.Tensor, out: torch.Tensor = None, sqrt_out: bool = False,
     w, wn = _workspace(wsb, A.device, ws)
     _check(lib.rmm_score(_ptr(A3), dt, b, M, d, A3.stride(1), A3.stride(0) if b > 1 else 0, _ptr(out2),
                          out2.stride(0), int(sqrt_out), _ptr(w), wn, _stream_ptr(stream)), "rmm_score")
+    return out if batched or out.dim() == 1 else out2[0]
+
+
+def rmm_score_noalloc(A: torch.Tensor, out: torch.Tensor = None, sqrt_out: bool = False, stream=None):
+    """rmm_score without a workspace argument: the partial sums use the
+    library's built-in scratch array (for callers that cannot allocate)."""
+    batched = A.dim() == 3
+    A3 = A if batched else A.unsqueeze(0)
+    if A3.stride(2) != 1:
+        raise ValueError("A must have unit column stride")
+    b, M, d = A3.shape
+    if out is None:
+        out = torch.empty((b, d), dtype=torch.float32, device=A.device)
+    out2 = out if out.dim() == 2 else out.view(1, -1)
+    _check(lib.rmm_score_noalloc(_ptr(A3), _dtype_code(A3), b, M, d, A3.stride(1), A3.stride(0) if b > 1 else 0,
+                                 _ptr(out2), out2.stride(0), int(sqrt_out), _stream_ptr(stream)),
+           "rmm_score_noalloc")
     return out if batched or out.dim() == 1 else out2[0]
 
 
