@@ -113,7 +113,7 @@ RMM_API rmm_status rmm_score(const void* A, int dtype, int64_t batch, int64_t M,
  * overwrites it in full before reading it, so nothing has to be cleared
  * between calls; calls that overlap on the GPU race on it and must be
  * serialised by the caller. */
-#define RMM_SCORE_NOALLOC_MAX_BYTES ((size_t)8 << 20)
+#define RMM_SCORE_NOALLOC_MAX_BYTES ((size_t)16 << 20)
 RMM_API rmm_status rmm_score_noalloc(const void* A, int dtype, int64_t batch, int64_t M, int64_t d,
                                      int64_t lda, int64_t batch_stride, float* ss, int64_t ld_ss,
                                      int sqrt_out, void* stream);

@@ -3,12 +3,11 @@
 //   compact_kernel      A_I[:, r] = A[:, I_r]   (column gather of the activation)
 //   gather_rows_kernel  B_I[r, :] = B[I_r, :]   (row gather of the weight)
 //
-// HBM-bound gather.  Each thread produces 8 consecutive output columns of one
-// row (one 16-byte store for bf16): it reads 8 indices, gathers the 8 source
-// elements through the read-only cache (the kept indices are increasing, so a
-// warp's 256 gathers cover a short run of the source row and reuse its
-// sectors), and writes them with one vector store.  A 256-thread CTA covers
-// 2048 output columns of one row.
+// HBM-bound gather.  Each thread produces 8 consecutive output columns (one
+// 16-byte store for bf16) of each of 8 rows: it reads its 8 indices once,
+// gathers the source elements through the read-only cache (the kept indices
+// are increasing, so a warp's 256 gathers cover a short run of the source row
+// and reuse its sectors), and writes them with vector stores.
 #include <cuda_bf16.h>
 
 #include "rmm_device.cuh"
@@ -19,45 +18,58 @@ namespace {
 
 constexpr int kCompactThreads = 256;
 constexpr int kPerThread = 8;
+constexpr int kRowsPerCta = 8;
 constexpr int64_t kColsPerCta = kCompactThreads * kPerThread;
 
+// A CTA covers 2048 output columns of 8 consecutive rows: each thread reads
+// its 8 indices once and gathers them from every row, so several rows'
+// gathers are in flight together.
 template <typename T>
 __global__ void __launch_bounds__(kCompactThreads) compact_kernel(const T* __restrict__ A, int64_t M, int64_t d,
                                                                   int64_t lda, const int32_t* __restrict__ idx,
                                                                   int64_t k, T* __restrict__ AI, int64_t ld_ai,
                                                                   int64_t chunks, bool vec_ok, unsigned* err) {
-  const int64_t row = static_cast<int64_t>(blockIdx.x) / chunks;
+  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) / chunks) * kRowsPerCta;
   const int64_t chunk = static_cast<int64_t>(blockIdx.x) % chunks;
   const int64_t c0 = chunk * kColsPerCta + static_cast<int64_t>(threadIdx.x) * kPerThread;
-  if (row >= M || c0 >= k) return;
-  const T* a = A + row * lda;
-  T* o = AI + row * ld_ai + c0;
-  alignas(16) T v[kPerThread];
+  if (row0 >= M || c0 >= k) return;
+  int32_t j[kPerThread];
   bool bad = false;
 #pragma unroll
   for (int e = 0; e < kPerThread; ++e) {
-    v[e] = T(0.f);
+    j[e] = -1;
     if (c0 + e < k) {
-      const int32_t j = __ldg(idx + c0 + e);
-      if (j >= 0 && j < d) {
-        v[e] = __ldg(a + j);
+      const int32_t v = __ldg(idx + c0 + e);
+      if (v >= 0 && v < d) {
+        j[e] = v;
       } else {
         bad = true;
       }
     }
   }
   if (bad) record_error(err, kDevErrBadIndex);
-  if (vec_ok && c0 + kPerThread <= k) {
-    if constexpr (sizeof(T) == 2) {
-      *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(v);
-    } else {
-      reinterpret_cast<float4*>(o)[0] = *reinterpret_cast<const float4*>(&v[0]);
-      reinterpret_cast<float4*>(o)[1] = *reinterpret_cast<const float4*>(&v[4]);
-    }
-  } else {
+  const bool full = vec_ok && c0 + kPerThread <= k;
+#pragma unroll 4
+  for (int rr = 0; rr < kRowsPerCta; ++rr) {
+    const int64_t row = row0 + rr;
+    if (row >= M) break;
+    const T* a = A + row * lda;
+    T* o = AI + row * ld_ai + c0;
+    alignas(16) T v[kPerThread];
 #pragma unroll
-    for (int e = 0; e < kPerThread; ++e)
-      if (c0 + e < k) o[e] = v[e];
+    for (int e = 0; e < kPerThread; ++e) v[e] = j[e] >= 0 ? __ldg(a + j[e]) : T(0.f);
+    if (full) {
+      if constexpr (sizeof(T) == 2) {
+        *reinterpret_cast<uint4*>(o) = *reinterpret_cast<const uint4*>(v);
+      } else {
+        reinterpret_cast<float4*>(o)[0] = *reinterpret_cast<const float4*>(&v[0]);
+        reinterpret_cast<float4*>(o)[1] = *reinterpret_cast<const float4*>(&v[4]);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < kPerThread; ++e)
+        if (c0 + e < k) o[e] = v[e];
+    }
   }
 }
 
@@ -115,7 +127,7 @@ cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64
                            int64_t k, void* A_I, int64_t ld_ai, unsigned* err, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
   const int64_t chunks = (k + kColsPerCta - 1) / kColsPerCta;
-  const int64_t blocks = M * chunks;
+  const int64_t blocks = ((M + kRowsPerCta - 1) / kRowsPerCta) * chunks;
   const size_t elt = dtype == 1 ? 2 : 4;
   const bool vec_ok = reinterpret_cast<uintptr_t>(A_I) % 16 == 0 && (ld_ai * elt) % 16 == 0;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;

@@ -3,12 +3,12 @@
 // s_j = ||A[:,j]||_2; the square keeps the ranking).
 //
 // HBM-bound design: each thread owns one 16-byte column vector (8 bf16 or 4
-// fp32 columns) and walks rows with 16-byte loads, so a warp reads 512
-// contiguous bytes of a row.  A 256-thread CTA is col_threads wide and
+// fp32 columns) and loads 16 rows of it at once, so a warp reads 512
+// contiguous bytes of a row per load.  A 256-thread CTA is col_threads wide and
 // row_groups tall; CTAs tile (column strip, row split, batch).  Squares of bf16
 // values are exact in fp32 and accumulate with one rounding per row (fma).
 // Row groups combine by a fixed pairwise tree in shared memory; row splits are
-// combined by a second kernel in a fixed blocked order.  No atomics, so the
+// combined by a second kernel in a fixed order.  No atomics, so the
 // result depends only on the shape.
 #include <cuda_bf16.h>
 
@@ -20,17 +20,20 @@ namespace rmm {
 namespace {
 
 constexpr int kScoreThreads = 256;
-constexpr int64_t kTargetCtas = 2368;  // 16 x 148: enough 256-thread CTAs to cover HBM latency
-constexpr int64_t kMinRowsPerSplit = 32;
-constexpr int64_t kMaxSplits = 64;
+// Every thread sums exactly kRowsPerThread rows of its column vector, with all
+// of those 16-byte loads issued before the first is consumed: one round of
+// memory latency per CTA.  A CTA therefore covers kRowsPerThread * row_groups
+// rows; the row splits this produces are summed by the finalize kernel.  The
+// plan depends only on the shape, so the summation order does too.
+constexpr int kRowsPerThread = 16;
+static_assert(kRowsPerThread % 8 == 0, "loads are issued eight at a time");
 
 template <typename T>
 struct Lanes;
 template <>
 struct Lanes<__nv_bfloat16> {
   static constexpr int kVec = 8;
-  __device__ static void load(const __nv_bfloat16* p, float (&x)[8]) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+  __device__ static void unpack(const uint4 v, float (&x)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -43,12 +46,11 @@ struct Lanes<__nv_bfloat16> {
 template <>
 struct Lanes<float> {
   static constexpr int kVec = 4;
-  __device__ static void load(const float* p, float (&x)[4]) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-    x[0] = v.x;
-    x[1] = v.y;
-    x[2] = v.z;
-    x[3] = v.w;
+  __device__ static void unpack(const uint4 v, float (&x)[4]) {
+    x[0] = __uint_as_float(v.x);
+    x[1] = __uint_as_float(v.y);
+    x[2] = __uint_as_float(v.z);
+    x[3] = __uint_as_float(v.w);
   }
   __device__ static float scalar(const float* p) { return __ldg(p); }
 };
@@ -75,27 +77,23 @@ __global__ void __launch_bounds__(kScoreThreads) score_partial_kernel(
 
   if (col0 < d) {
     if (vec_ok && col0 + V <= d) {
-      int64_t r = r0 + ty;
-      // four independent 16-byte loads in flight per thread
-      for (; r + 3 * row_groups < r1; r += 4 * row_groups) {
-        float x0[V], x1[V], x2[V], x3[V];
-        Lanes<T>::load(Ab + r * lda + col0, x0);
-        Lanes<T>::load(Ab + (r + row_groups) * lda + col0, x1);
-        Lanes<T>::load(Ab + (r + 2 * row_groups) * lda + col0, x2);
-        Lanes<T>::load(Ab + (r + 3 * row_groups) * lda + col0, x3);
+      // two rounds of eight independent 16-byte loads (more in flight costs
+      // registers, hence occupancy, for no gain)
 #pragma unroll
-        for (int e = 0; e < V; ++e) {
-          acc[e] = fmaf(x0[e], x0[e], acc[e]);
-          acc[e] = fmaf(x1[e], x1[e], acc[e]);
-          acc[e] = fmaf(x2[e], x2[e], acc[e]);
-          acc[e] = fmaf(x3[e], x3[e], acc[e]);
+      for (int u0 = 0; u0 < kRowsPerThread; u0 += 8) {
+        uint4 raw[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t r = r0 + ty + static_cast<int64_t>(u0 + u) * row_groups;
+          raw[u] = r < r1 ? __ldg(reinterpret_cast<const uint4*>(Ab + r * lda + col0)) : make_uint4(0, 0, 0, 0);
         }
-      }
-      for (; r < r1; r += row_groups) {
-        float x0[V];
-        Lanes<T>::load(Ab + r * lda + col0, x0);
 #pragma unroll
-        for (int e = 0; e < V; ++e) acc[e] = fmaf(x0[e], x0[e], acc[e]);
+        for (int u = 0; u < 8; ++u) {
+          float x[V];
+          Lanes<T>::unpack(raw[u], x);
+#pragma unroll
+          for (int e = 0; e < V; ++e) acc[e] = fmaf(x[e], x[e], acc[e]);
+        }
       }
     } else {
       for (int64_t r = r0 + ty; r < r1; r += row_groups) {
@@ -134,21 +132,37 @@ __global__ void __launch_bounds__(kScoreThreads) score_partial_kernel(
   }
 }
 
-// Sum the row-split partials of one column: blocks of 8 sequentially, then
-// the block sums sequentially (fixed order).  Grid: x = column blocks, y = batch.
-__global__ void score_finalize_kernel(const float* __restrict__ partial, int64_t d, int64_t splits,
-                                      float* __restrict__ ss, int64_t ld_ss, int sqrt_out) {
-  const int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (j >= d) return;
+// Sum the row-split partials: a 256-thread CTA covers 32 columns; thread
+// (c, g) adds splits g, g+8, g+16, ... of column c in increasing order, then
+// the 8 group sums combine by a fixed pairwise tree.  Grid: x = column
+// blocks of 32, y = batch.
+__global__ void __launch_bounds__(256) score_finalize_kernel(const float* __restrict__ partial, int64_t d,
+                                                             int64_t splits, float* __restrict__ ss, int64_t ld_ss,
+                                                             int sqrt_out) {
+  __shared__ float part[8][33];
+  const int c = threadIdx.x & 31, g = threadIdx.x >> 5;
+  const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + c;
   const float* p = partial + static_cast<int64_t>(blockIdx.y) * splits * d + j;
-  float total = 0.f;
-  for (int64_t s0 = 0; s0 < splits; s0 += 8) {
-    float blk = 0.f;
-    const int64_t s1 = min(splits, s0 + 8);
-    for (int64_t s = s0; s < s1; ++s) blk += p[s * d];
-    total += blk;
+  float acc = 0.f;
+  if (j < d) {
+    int64_t s = g;
+    for (; s + 24 < splits; s += 32) {  // four independent loads in flight, added in split order
+      const float a0 = __ldg(p + s * d), a1 = __ldg(p + (s + 8) * d);
+      const float a2 = __ldg(p + (s + 16) * d), a3 = __ldg(p + (s + 24) * d);
+      acc += a0;
+      acc += a1;
+      acc += a2;
+      acc += a3;
+    }
+    for (; s < splits; s += 8) acc += __ldg(p + s * d);
   }
-  ss[static_cast<int64_t>(blockIdx.y) * ld_ss + j] = sqrt_out ? sqrtf(total) : total;
+  part[g][c] = acc;
+  __syncthreads();
+  if (g == 0 && j < d) {
+    const float t = ((part[0][c] + part[1][c]) + (part[2][c] + part[3][c])) +
+                    ((part[4][c] + part[5][c]) + (part[6][c] + part[7][c]));
+    ss[static_cast<int64_t>(blockIdx.y) * ld_ss + j] = sqrt_out ? sqrtf(t) : t;
+  }
 }
 
 }  // namespace
@@ -162,11 +176,7 @@ ScorePlan score_plan(int dtype, int64_t batch, int64_t M, int64_t d) {
   p.col_threads = ct;
   p.row_groups = kScoreThreads / ct;
   p.strips = (vecs + ct - 1) / ct;
-  const int64_t base = std::max<int64_t>(1, p.strips * batch);
-  int64_t splits = (kTargetCtas + base - 1) / base;
-  splits = std::min(splits, std::max<int64_t>(1, (M + kMinRowsPerSplit - 1) / kMinRowsPerSplit));
-  splits = std::max<int64_t>(1, std::min(splits, kMaxSplits));
-  const int64_t rps = std::max<int64_t>(1, (M + splits - 1) / splits);
+  const int64_t rps = static_cast<int64_t>(kRowsPerThread) * p.row_groups;
   p.rows_per_split = rps;
   p.splits = M > 0 ? (M + rps - 1) / rps : 1;
   return p;
@@ -202,7 +212,7 @@ cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || direct) return e;
-  const dim3 g2(static_cast<unsigned>((d + 255) / 256), static_cast<unsigned>(batch));
+  const dim3 g2(static_cast<unsigned>((d + 31) / 32), static_cast<unsigned>(batch));
   score_finalize_kernel<<<g2, 256, 0, stream>>>(static_cast<const float*>(ws), d, p.splits, ss, ld_ss, sqrt_out);
   return cudaGetLastError();
 }

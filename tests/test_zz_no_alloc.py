@@ -15,15 +15,15 @@ import pytest
 import input_adaptive_reduced_score_b200 as R
 import workloads as W
 
-LIMIT = 8 << 20  # RMM_SCORE_NOALLOC_MAX_BYTES in include/rmm.h
+LIMIT = 16 << 20  # RMM_SCORE_NOALLOC_MAX_BYTES in include/rmm.h
 
 
 def test_oversized_shape_is_refused():
     """Refused on the host, before any device work (runs without a GPU)."""
-    # 2100 matrices of 128 x 512: two row splits each, 2100 x 2 x 512 x 4 B = 8.6 MB of partial sums
-    b, M, d = 2100, 128, 512
+    # 4160 x 65536: 65 row splits x 65536 columns x 4 B = 17 MB of partial sums
+    b, M, d = 1, 4160, 65536
     assert R.rmm_score_workspace_size(R.RMM_BF16, b, M, d) > LIMIT
-    st = R.lib.rmm_score_noalloc(ctypes.c_void_p(256), R.RMM_BF16, b, M, d, d, M * d, ctypes.c_void_p(256), d, 0,
+    st = R.lib.rmm_score_noalloc(ctypes.c_void_p(256), R.RMM_BF16, b, M, d, d, 0, ctypes.c_void_p(256), d, 0,
                                  ctypes.c_void_p(0))
     assert st == 1
     assert b"built-in" in R.lib.rmm_last_error()
