@@ -81,6 +81,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// mbar_wait taken by a whole warp with a warp-uniform result: true only if
+// every lane saw the phase complete.  Use it where a warp-synchronous
+// (.sync.aligned) instruction follows, so an abort can never split the warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               unsigned* err, unsigned site) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, err, site);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
 // ------------------------------------------------------------------ TMA / cp.async
 
 // 2-D tiled TMA load of one box into shared memory; completion is signalled on
@@ -91,6 +100,26 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, uint
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(tmap), "r"(bar), "r"(x), "r"(y)
       : "memory");
+}
+
+// 3-D tiled TMA load (x innermost); same alignment rule as tma_load_2d.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint32_t bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Barrier among `count` threads (a multiple of 32) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// 2^x, hardware approximation (maximum relative error about 2^-22); -inf gives +0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // TMA row gather: four rows (r0..r3) of a 2-D tensor, one box of columns

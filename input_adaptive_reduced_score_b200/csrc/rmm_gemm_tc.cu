@@ -163,11 +163,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
       const uint32_t b = it & 1, acc_phase = (it >> 1) & 1;
-      if (!mbar_wait(accempty(b), acc_phase ^ 1u, abort_flag, err, 2)) break;
+      if (!mbar_wait_warp(accempty(b), acc_phase ^ 1u, abort_flag, err, 2)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + b * BN;
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait(full(stage), phase, abort_flag, err, 3)) {
+        if (!mbar_wait_warp(full(stage), phase, abort_flag, err, 3)) {
           ok = false;
           break;
         }
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const uint32_t b = it & 1, acc_phase = (it >> 1) & 1;
-      if (!mbar_wait(accfull(b), acc_phase, abort_flag, err, 4)) break;
+      if (!mbar_wait_warp(accfull(b), acc_phase, abort_flag, err, 4)) break;
       tc_fence_after();
       const int m_blk = tile % num_m, n_blk = tile / num_m;
       const int row = m_blk * BM + qtr * 32 + lane;

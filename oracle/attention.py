@@ -31,7 +31,8 @@ import numpy as np
 
 from .rmm import k_from_rho, column_sq_norms, topk_indices
 
-__all__ = ["attention_head", "reduced_attention", "kv_head_of"]
+__all__ = ["attention_head", "reduced_attention", "kv_head_of", "head_dim_selection", "lse_rows",
+           "token_scores", "out_rows"]
 
 
 def kv_head_of(h: int, Hq: int, Hkv: int) -> int:
@@ -39,10 +40,14 @@ def kv_head_of(h: int, Hq: int, Hkv: int) -> int:
     return (h * Hkv) // Hq
 
 
-def attention_head(Q, K, V, rho_d: float, rho_t: float, causal: bool = True, scale=None):
+def attention_head(Q, K, V, rho_d: float, rho_t: float, causal: bool = True, scale=None,
+                   token_idx=None, return_p: bool = False):
     """One (batch, head): Q [S x D], K [S x D], V [S x D] in fp64.
 
-    Returns dict(O [S x D], idx_d [k_d], idx_t [k_t], lse [S], t [S], ssq [D]).
+    Returns dict(O [S x D], idx_d [k_d], idx_t [k_t], lse [S], t [S], ssq [D])
+    (plus P [S x S] when return_p).  `token_idx`, when given, replaces the
+    token selection (a test hook for cases where several sets are top-k
+    within floating-point error); everything else is unchanged.
     Steps follow the method's order: score Q's columns, keep the top head_dim
     indices, form the reduced logits, the causal softmax, score P's columns,
     keep the top tokens, form the reduced PV product.
@@ -69,10 +74,13 @@ def attention_head(Q, K, V, rho_d: float, rho_t: float, causal: bool = True, sca
     P = e / z
     # token selection on A = P (R4)
     t = np.einsum("ij,ij->j", P, P)
-    idx_t = topk_indices(t, k_from_rho(rho_t, S))
+    idx_t = topk_indices(t, k_from_rho(rho_t, S)) if token_idx is None else np.asarray(token_idx, np.int64)
     # reduced PV (R5)
     O = P[:, idx_t] @ V[idx_t, :]
-    return dict(O=O, idx_d=idx_d, idx_t=idx_t, lse=lse, t=t, ssq=ssq)
+    out = dict(O=O, idx_d=idx_d, idx_t=idx_t, lse=lse, t=t, ssq=ssq)
+    if return_p:
+        out["P"] = P
+    return out
 
 
 def reduced_attention(Q, K, V, rho_d: float, rho_t: float, causal: bool = True, scale=None,
@@ -102,4 +110,60 @@ def reduced_attention(Q, K, V, rho_d: float, rho_t: float, causal: bool = True, 
         r = attention_head(Q[b, h], K[b, g], V[b, g], rho_d, rho_t, causal, scale)
         for key in out:
             out[key][b, h] = r[key]
+    return out
+
+
+# ---------------------------------------------------------------- row / column restricted forms
+# The same definitions as attention_head, evaluated on chosen query rows or
+# key columns only, for sequences whose S x S matrix is too large to hold.
+# Each value is computed exactly as in attention_head; only the set of rows
+# or columns evaluated is restricted.
+
+def head_dim_selection(Q, rho_d: float):
+    """I_d of one (batch, head): top ceil(rho_d D) columns of Q by score (R1)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    return topk_indices(column_sq_norms(Q), k_from_rho(rho_d, Q.shape[1]))
+
+
+def lse_rows(Q, K, idx_d, rows, scale=None):
+    """lse_i = logsumexp_{j<=i} scale * Q[i, I_d] . K[j, I_d] for i in rows (R2, R3)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    scale = 1.0 / math.sqrt(Q.shape[1]) if scale is None else scale
+    out = np.empty(len(rows))
+    Kd = K[:, idx_d]
+    for n, i in enumerate(rows):
+        logits = scale * (Kd[: i + 1] @ Q[i, idx_d])
+        mx = logits.max()
+        out[n] = mx + np.log(np.sum(np.exp(logits - mx)))
+    return out
+
+
+def token_scores(Q, K, idx_d, lse, cols, scale=None):
+    """t_j = sum_{i>=j} P_ij^2 = sum_{i>=j} exp(2 (S_ij - lse_i)) for j in cols (R4),
+    given lse for every row."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    scale = 1.0 / math.sqrt(Q.shape[1]) if scale is None else scale
+    Qd = Q[:, idx_d]
+    out = np.empty(len(cols))
+    for n, j in enumerate(cols):
+        logits = scale * (Qd[j:] @ K[j, idx_d])
+        out[n] = np.sum(np.exp(2.0 * (logits - lse[j:])))
+    return out
+
+
+def out_rows(Q, K, V, idx_d, lse, idx_t, rows, scale=None):
+    """O_i = sum_{j in I_t, j<=i} exp(S_ij - lse_i) V_j for i in rows (R5)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    scale = 1.0 / math.sqrt(Q.shape[1]) if scale is None else scale
+    idx_t = np.asarray(idx_t, dtype=np.int64)
+    out = np.zeros((len(rows), V.shape[1]))
+    for n, i in enumerate(rows):
+        kept = idx_t[idx_t <= i]
+        if kept.size:
+            p = np.exp(scale * (K[kept][:, idx_d] @ Q[i, idx_d]) - lse[n])
+            out[n] = p @ V[kept]
     return out

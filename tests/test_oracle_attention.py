@@ -107,3 +107,34 @@ def test_planted_mistake_renormalised_pv_is_caught():
     kt = O.k_from_rho(0.3, S)
     renorm = np.array([V[:min(ii, kt - 1) + 1].mean(0) for ii in range(S)])
     assert not np.allclose(r["O"], renorm)
+
+
+def test_restricted_forms_agree_with_full_head():
+    S, D = 90, 16
+    Q, K, V = (_rand((S, D), s) for s in (13, 14, 15))
+    r = OA.attention_head(Q, K, V, 0.5, 0.4)
+    idx_d = OA.head_dim_selection(Q, 0.5)
+    np.testing.assert_array_equal(idx_d, r["idx_d"])
+    rows = np.arange(S)
+    lse = OA.lse_rows(Q, K, idx_d, rows)
+    np.testing.assert_allclose(lse, r["lse"], rtol=1e-13, atol=1e-13)
+    t = OA.token_scores(Q, K, idx_d, lse, np.arange(S))
+    np.testing.assert_allclose(t, r["t"], rtol=1e-12)
+    some = np.array([0, 7, 44, 89])
+    O = OA.out_rows(Q, K, V, idx_d, lse[some], r["idx_t"], some)
+    np.testing.assert_allclose(O, r["O"][some], rtol=1e-12, atol=1e-14)
+
+
+def test_restricted_forms_uniform_closed_form():
+    S, D = 40, 8
+    Q = _rand((S, D), 16)
+    K = np.zeros((S, D))
+    V = _rand((S, D), 17)
+    idx_d = OA.head_dim_selection(Q, 1.0)
+    lse = OA.lse_rows(Q, K, idx_d, np.arange(S))
+    np.testing.assert_allclose(lse, np.log(np.arange(1, S + 1)), atol=1e-14)
+    t = OA.token_scores(Q, K, idx_d, lse, [0, 5, S - 1])
+    ref = [sum(1.0 / (i + 1) ** 2 for i in range(j, S)) for j in (0, 5, S - 1)]
+    np.testing.assert_allclose(t, ref, rtol=1e-13)
+    O = OA.out_rows(Q, K, V, idx_d, lse[[3, 20]], [0, 2, 30], [3, 20])
+    np.testing.assert_allclose(O, [(V[0] + V[2]) / 4, (V[0] + V[2]) / 21], rtol=1e-13)
