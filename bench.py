@@ -259,6 +259,47 @@ def aggregate(local_ms, local_flops, world):
     return float(t.item()), float(f.item())
 
 
+ATTN = dict(B=1, Hq=32, Hkv=32, S=8192, D=128, rho_d=0.5, rho_t=0.5, seed=3)
+
+
+def measure_attention(R, workloads, bf16_tensor, dev, stream, flush, steps, timed):
+    """Reduced attention on the 32-head, 8192-token workload (same flush and
+    event protocol as the GEMM path), next to torch's causal SDPA."""
+    import torch
+    a = ATTN
+    inp = workloads.attention(a["seed"], a["B"], a["Hq"], a["Hkv"], a["S"], a["D"], a["rho_d"], a["rho_t"])
+    Q, K, V = (bf16_tensor(x, dev) for x in (inp.Q, inp.K, inp.V))
+    O = torch.empty_like(Q)
+    ws = torch.empty(R.rmm_attention_workspace_size(a["B"], a["Hq"], a["Hkv"], a["S"], a["D"], a["rho_d"],
+                                                    a["rho_t"]), dtype=torch.uint8, device=dev)
+
+    def rmm(ev):
+        ev[0].record(stream)
+        R.rmm_attention(Q, K, V, a["rho_d"], a["rho_t"], out=O, ws=ws)
+        ev[1].record(stream)
+
+    def sdpa(ev):
+        ev[0].record(stream)
+        torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=True)
+        ev[1].record(stream)
+
+    for fn in (rmm, sdpa):
+        for _ in range(3):
+            fn([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    rmm_ms = statistics.mean(p[0] for p in timed(rmm, steps, 2))
+    sdpa_ms = statistics.mean(p[0] for p in timed(sdpa, steps, 2))
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the attention runs")
+    S, D, H = a["S"], a["D"], a["B"] * a["Hq"]
+    dense_flops = 4.0 * (S * (S + 1) / 2) * D * H
+    return {"workload": f"causal attention B{a['B']} H{a['Hq']} S{S} D{D}, rho_d={a['rho_d']} rho_t={a['rho_t']}, "
+                        "Q/K/V N(0,1) x per-dim lognormal(0,0.5)",
+            "ms": rmm_ms, "sdpa_ms": sdpa_ms, "speedup_vs_sdpa": sdpa_ms / rmm_ms,
+            "dense_equivalent_tflops": dense_flops / (rmm_ms * 1e-3) / 1e12,
+            "sdpa_tflops": dense_flops / (sdpa_ms * 1e-3) / 1e12,
+            "gpu_launches_per_call": 12, "calls": steps}
+
+
 def run_rmm(args):
     import numpy as np
     import torch
@@ -379,6 +420,8 @@ def run_rmm(args):
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the dense / end-to-end runs")
 
+    attention = measure_attention(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 20), timed)
+
     peaks, peak_src = load_peaks()
     gemm_ms = stage_ms["gemm"]
     achieved = flops_step / (gemm_ms * 1e-3) / 1e12
@@ -418,6 +461,7 @@ def run_rmm(args):
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(X.numel() * 2),
                     "d2h_bytes_per_step": int(Y.numel() * 2), "api": "rmm_matmul"},
             "gpu_launches": launches_per_step * args.steps,
+            "attention": attention,
             "clocks": clk.summary(), "clock_remeasured": remeasured,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -307,3 +307,17 @@ def _full_cond(which):
         ks = [oracle.k_from_rho(r, inp.d) for r in inp.rhos]
         _CACHE[key], _ = widen_topk_gaps(inp.A, "bf16", ks)
     return _CACHE[key]
+
+
+# ------------------------------------------------------------------ 70B-shaped layer
+
+@pytest.mark.slow
+@pytest.mark.parametrize("which", ["q_proj", "k_proj", "up_proj", "down_proj"])
+def test_path_layer70b(which):
+    """The 70B-shaped layer's distinct projection shapes (q/o 2048x8192x8192,
+    k/v 2048x8192x1024 at rho 0.5; up/gate 2048x8192x28672 and down
+    2048x28672x8192 at rho 0.8), whole path, sampled rows."""
+    inp = W.layer70b_inputs(which)
+    ks = [oracle.k_from_rho(r, inp.d) for r in inp.rhos]
+    A2, _ = widen_topk_gaps(inp.A, "bf16", ks)
+    _check_path(inp, inp.rhos[0], rows=sample_rows(inp.M), cond=A2)
