@@ -454,7 +454,7 @@ def run_rmm(args):
             "dense_tflops": 2.0 * M * N * D / (dense_ms * 1e-3) / 1e12,
             "dense_equivalent_tflops": 2.0 * M * N * D / (path_ms * 1e-3) / 1e12,
             "path_roofline_frac": path_roof_ms / path_ms,
-            "roofline": {"kernel": "gemm_bf16_tc_kernel", "bound": "tensor", "achieved": achieved,
+            "roofline": {"kernel": "gemm_bf16_tc_pair_kernel", "bound": "tensor", "achieved": achieved,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
                          "traffic": traffic, "peak_source": f"{peak_src} (burst bf16)"},
             "kernels": kernels,

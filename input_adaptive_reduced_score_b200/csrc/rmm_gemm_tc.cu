@@ -20,6 +20,11 @@
 // All waits are bounded (rmm_device.cuh); on a timeout the kernel records an
 // error, drains its own copies and MMAs, frees TMEM and returns.
 //
+// Activations of 256 rows or more use the CTA-pair variant below (256 x 256
+// tiles, tcgen05.mma.cta_group::2), which halves each SM's share of B and
+// so cuts the operand bytes each SM pulls from L2 per MMA by a third; the
+// single-CTA kernel serves smaller M.
+//
 // Why B_I is gathered beforehand rather than inside this kernel: gathering
 // the k rows of B per k-block with tile::gather4 (64 four-row TMA gathers per
 // stage) or with 16-byte cp.async was measured on B200 at about 2.2 TB/s of
@@ -68,6 +73,42 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
     if (global_ns() - t0 > kDrainNs) return false;
   }
   return true;
+}
+
+// Store 32 fp32 accumulator values of one output row (columns col0 ..
+// col0+31, masked at N) as fp32 or bf16, with 16-byte stores when aligned.
+__device__ __forceinline__ void store_row32(void* Y, int out_f32, int64_t ldy, int y_vec_ok, int row, int col0, int N,
+                                            const uint32_t (&v)[32]) {
+  if (out_f32) {
+    float* y = static_cast<float*>(Y) + static_cast<int64_t>(row) * ldy + col0;
+    if (y_vec_ok && col0 + 32 <= N) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<float4*>(y)[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                      __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (col0 + e < N) y[e] = __uint_as_float(v[e]);
+    }
+  } else {
+    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y) + static_cast<int64_t>(row) * ldy + col0;
+    if (y_vec_ok && col0 + 32 <= N) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+        w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+        w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+        w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+        reinterpret_cast<uint4*>(y)[i] = w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (col0 + e < N) y[e] = __float2bfloat16_rn(__uint_as_float(v[e]));
+    }
+  }
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -214,39 +255,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(taddr + cc * 32, v);
         tmem_wait_ld();
         const int col0 = n_blk * BN + half * 128 + cc * 32;
-        if (row < M && col0 < N) {
-          if (out_f32) {
-            float* y = static_cast<float*>(Y) + static_cast<int64_t>(row) * ldy + col0;
-            if (y_vec_ok && col0 + 32 <= N) {
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                reinterpret_cast<float4*>(y)[i] =
-                    make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (col0 + e < N) y[e] = __uint_as_float(v[e]);
-            }
-          } else {
-            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y) + static_cast<int64_t>(row) * ldy + col0;
-            if (y_vec_ok && col0 + 32 <= N) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-                w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-                w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-                w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-                reinterpret_cast<uint4*>(y)[i] = w;
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (col0 + e < N) y[e] = __float2bfloat16_rn(__uint_as_float(v[e]));
-            }
-          }
-        }
+        if (row < M && col0 < N) store_row32(Y, out_f32, ldy, y_vec_ok, row, col0, N, v);
       }
       tc_fence_before();
       __syncwarp();
@@ -259,6 +268,209 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
+}
+
+// ---------------------------------------------------------------- CTA-pair kernel
+//
+// Same pipeline on a pair of SMs (a 2-CTA cluster) computing 256 x 256
+// tiles with tcgen05.mma.cta_group::2 (M = 256): each CTA loads 128 rows of
+// A_I and 128 of the tile's 256 columns of B_I per k-block (32 KB per SM per
+// stage instead of 48 KB for the same MMA work per SM), and each CTA's
+// tensor memory holds its 128 rows x 256 columns of the accumulator.
+//   - both CTAs' TMA loads signal the leader's (rank 0) full barrier, whose
+//     expected bytes the leader registers for both halves;
+//   - the leader's single MMA thread issues the pair MMAs; its commits arrive
+//     on the empty / accumulator-full barriers of both CTAs (multicast);
+//   - both CTAs' epilogue warps arrive on the leader's accumulator-empty
+//     barrier;
+//   - cluster barriers after set-up and before tensor memory is released.
+namespace pairk {
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 6;
+constexpr int A_STAGE = 128 * BK * 2;           // this CTA's 128 rows: 16 KB
+constexpr int B_CHUNK = BK * 128;               // 64 columns x 64 rows: 8 KB
+constexpr int B_STAGE = 2 * B_CHUNK;            // this CTA's 128 columns: 16 KB
+constexpr uint32_t STAGE_TX = 2 * (A_STAGE + B_STAGE);
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = (2 + EPI_WARPS) * 32;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + BAR_BYTES + 1024;
+
+struct PairBars {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t accfull[2];
+  uint64_t accempty[2];
+  uint64_t drain;
+  uint32_t tmem_slot;
+  int abort_flag;
+};
+static_assert(sizeof(PairBars) <= BAR_BYTES, "barrier block");
+}  // namespace pairk
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
+    gemm_bf16_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                             int M, int N, int K, void* __restrict__ Y, int out_f32, int64_t ldy, int y_vec_ok,
+                             unsigned* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+  const uint32_t base = smem_u32(smem);
+  pairk::PairBars* bars = reinterpret_cast<pairk::PairBars*>(smem + pairk::STAGES * (pairk::A_STAGE + pairk::B_STAGE));
+  volatile int* abort_flag = &bars->abort_flag;
+  auto sA = [&](uint32_t s) { return base + s * pairk::A_STAGE; };
+  auto sB = [&](uint32_t s) { return base + pairk::STAGES * pairk::A_STAGE + s * pairk::B_STAGE; };
+  auto full = [&](uint32_t s) { return smem_u32(&bars->full[s]); };
+  auto empty = [&](uint32_t s) { return smem_u32(&bars->empty[s]); };
+  auto accfull = [&](uint32_t b) { return smem_u32(&bars->accfull[b]); };
+  auto accempty = [&](uint32_t b) { return smem_u32(&bars->accempty[b]); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = static_cast<int>(cluster_id_x()), ncl = static_cast<int>(nclusters_x());
+  const int num_m = (M + pairk::BM - 1) / pairk::BM, num_n = (N + pairk::BN - 1) / pairk::BN;
+  const int num_tiles = num_m * num_n;
+  const int nk = (K + pairk::BK - 1) / pairk::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < pairk::STAGES; ++s) {
+      mbar_init(full(s), 1);   // leader's producer: arrive + both CTAs' bytes
+      mbar_init(empty(s), 1);  // pair commit (multicast)
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accfull(b), 1);               // pair commit (multicast)
+      mbar_init(accempty(b), 2 * pairk::EPI_WARPS);  // epilogue warps of both CTAs
+    }
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(&bars->tmem_slot), pairk::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < num_tiles; tile += ncl) {
+        const int m_blk = tile % num_m, n_blk = tile / num_m;
+        const int a_row = m_blk * pairk::BM + static_cast<int>(rank) * 128;
+        const int b_col = n_blk * pairk::BN + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, err, 41)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full_leader = mapa_shared(full(stage), 0);
+          if (leader) mbar_arrive_expect_tx(full(stage), pairk::STAGE_TX);
+          tma_load_2d_pair(sA(stage), &tmap_a, full_leader, kb * pairk::BK, a_row);
+          tma_load_2d_pair(sB(stage), &tmap_b, full_leader, b_col, kb * pairk::BK);
+          tma_load_2d_pair(sB(stage) + pairk::B_CHUNK, &tmap_b, full_leader, b_col + 64, kb * pairk::BK);
+          ++issued;
+          if (++stage == pairk::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (leader) {
+        // the pair's copies for the last stages must land before either CTA exits
+        uint32_t st = stage, ph = phase;
+        const uint32_t n = issued < pairk::STAGES ? issued : pairk::STAGES;
+        for (uint32_t j = 0; j < n; ++j) {
+          if (st == 0) {
+            st = pairk::STAGES - 1;
+            ph ^= 1u;
+          } else {
+            --st;
+          }
+          wait_drain(full(st), ph);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader CTA)
+    if (leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(pairk::BM, pairk::BN, /*a_mn=*/false, /*b_mn=*/true);
+      uint32_t stage = 0, phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < num_tiles; tile += ncl, ++it) {
+        const uint32_t b = it & 1, acc_phase = (it >> 1) & 1;
+        if (!mbar_wait_warp(accempty(b), acc_phase ^ 1u, abort_flag, err, 42)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * pairk::BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_warp(full(stage), phase, abort_flag, err, 43)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+#pragma unroll
+            for (int kk = 0; kk < pairk::BK / 16; ++kk) {
+              const uint64_t ad = sdesc_sw128(sA(stage) + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(sB(stage) + kk * 16 * 128, pairk::B_CHUNK, 1024);
+              mma_f16_ss_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            mma_commit_pair_multicast(empty(stage), 0x3);
+          }
+          __syncwarp();
+          if (++stage == pairk::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) mma_commit_pair_multicast(accfull(b), 0x3);
+        __syncwarp();
+      }
+      if (lane == 0) {
+        mma_commit_pair_multicast(smem_u32(&bars->drain), 0x1);
+        wait_drain(smem_u32(&bars->drain), 0);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int qtr = warp & 3;
+    const int half = (warp - 2) / 4;
+    int it = 0;
+    for (int tile = cid; tile < num_tiles; tile += ncl, ++it) {
+      const uint32_t b = it & 1, acc_phase = (it >> 1) & 1;
+      if (!mbar_wait_warp(accfull(b), acc_phase, abort_flag, err, 44)) break;
+      tc_fence_after();
+      const int m_blk = tile % num_m, n_blk = tile / num_m;
+      const int row = m_blk * pairk::BM + static_cast<int>(rank) * 128 + qtr * 32 + lane;
+      const uint32_t taddr = tmem_base + b * pairk::BN + half * 128 + (static_cast<uint32_t>(qtr * 32) << 16);
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(taddr + cc * 32, v);
+        tmem_wait_ld();
+        const int col0 = n_blk * pairk::BN + half * 128 + cc * 32;
+        if (row < M && col0 < N) store_row32(Y, out_f32, ldy, y_vec_ok, row, col0, N, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(accempty(b), 0));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();  // all MMAs, copies and remote arrivals of the pair are done
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, pairk::TMEM_COLS);
 }
 
 // ---------------------------------------------------------------- host side
@@ -288,7 +500,9 @@ bool configure_kernel_once() {
   std::lock_guard<std::mutex> lock(mu);
   if (!done[dev]) {
     if (cudaFuncSetAttribute(gemm_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-        cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(gemm_bf16_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pairk::SMEM_BYTES) != cudaSuccess)
       return false;
     done[dev] = true;
   }
@@ -330,11 +544,20 @@ cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I,
     return cudaErrorInvalidValue;
   }
   const int sms = device_sm_count();
-  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   const int out_f32 = out_dtype == 0 ? 1 : 0;
   const size_t oelt = out_f32 ? 4 : 2;
   const int y_vec_ok = (reinterpret_cast<uintptr_t>(Y) % 16 == 0) && ((ldy * oelt) % 16 == 0);
+  if (M >= pairk::BM) {
+    // 256 x 256 tiles on SM pairs: one 2-CTA cluster per pair of SMs
+    const int64_t tiles = ((M + pairk::BM - 1) / pairk::BM) * ((N + pairk::BN - 1) / pairk::BN);
+    const int clusters = static_cast<int>(tiles < sms / 2 ? tiles : sms / 2);
+    gemm_bf16_tc_pair_kernel<<<2 * clusters, pairk::THREADS, pairk::SMEM_BYTES, stream>>>(
+        tmap_a, tmap_b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(k), Y, out_f32, ldy, y_vec_ok,
+        err);
+    return cudaGetLastError();
+  }
+  const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmap_a, tmap_b, static_cast<int>(M),
                                                               static_cast<int>(N), static_cast<int>(k), Y, out_f32,
                                                               ldy, y_vec_ok, err);
