@@ -146,6 +146,18 @@ RMM_API rmm_status rmm_compact(const void* A, int dtype, int64_t M, int64_t d, i
 RMM_API rmm_status rmm_gather_rows(const void* B, int dtype, int64_t d, int64_t N, int64_t ldb,
                                    const int32_t* idx, int64_t k, void* B_I, int64_t ld_bi, void* stream);
 
+/* ------------------------------------------------------------------ both reduced operands
+ * A_I = A[:, idx] and B_I = B[idx, :] in one launch (bf16 only): the same
+ * results as rmm_compact followed by rmm_gather_rows, with the two copies
+ * overlapped (Metodología › Mecanismo Central: both operands of the reduced
+ * product are restricted to I).  A [M x d] (lda), B [d x N] (ldb), A_I
+ * [M x k] (ld_ai >= k), B_I [k x N] (ld_bi >= N).  B, B_I 16-byte aligned and
+ * ldb, ld_bi multiples of 8 (RMM_ERR_UNSUPPORTED otherwise).  Indices outside
+ * [0, d) give zeros and are flagged in the device error word. */
+RMM_API rmm_status rmm_compact_gather(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t M,
+                                      int64_t d, int64_t N, const int32_t* idx, int64_t k, void* A_I,
+                                      int64_t ld_ai, void* B_I, int64_t ld_bi, void* stream);
+
 /* ------------------------------------------------------------------ reduced GEMM
  * Y = A_I · B[idx, :]  (Metodología › Mecanismo Central), where A_I is the
  * compacted [M x k] activation (ld_ai), B the full [d x N] row-major operand

@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "lib", "LIB_PATH", "RMMError", "RMM_F32", "RMM_BF16", "rmm_abi_version", "rmm_k_from_rho",
-    "rmm_device_error", "rmm_score", "rmm_score_workspace_size", "rmm_score_noalloc", "rmm_topk", "rmm_compact", "rmm_gather_rows",
+    "rmm_device_error", "rmm_score", "rmm_score_workspace_size", "rmm_score_noalloc", "rmm_topk", "rmm_compact", "rmm_gather_rows", "rmm_compact_gather",
     "rmm_gemm", "rmm_gemm_workspace_size", "rmm_gemm_compacted",
     "rmm_matmul", "rmm_matmul_workspace_size", "rmm_attention", "rmm_attention_workspace_size",
     "exported_symbols", "declared_symbols",
@@ -61,6 +61,8 @@ _sig("rmm_score_noalloc", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_i64, c_i64,
 _sig("rmm_topk", c_int, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp)
 _sig("rmm_compact", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp)
 _sig("rmm_gather_rows", c_int, c_vp, c_int, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp)
+_sig("rmm_compact_gather", c_int, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64,
+     c_vp)
 _sig("rmm_gemm_workspace_size", c_sz, c_int, c_i64, c_i64)
 _sig("rmm_gemm", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_int, c_vp, c_int, c_i64, c_vp,
      c_sz, c_vp)
@@ -226,6 +228,27 @@ def rmm_gather_rows(B: torch.Tensor, idx: torch.Tensor, out: torch.Tensor = None
     _check(lib.rmm_gather_rows(_ptr(B), _dtype_code(B), d, N, ldb, _ptr(idx), k, _ptr(out), out.stride(0),
                                _stream_ptr(stream)), "rmm_gather_rows")
     return out
+
+
+def rmm_compact_gather(A: torch.Tensor, B: torch.Tensor, idx: torch.Tensor, out_a: torch.Tensor = None,
+                       out_b: torch.Tensor = None, stream=None):
+    """A_I = A[:, idx] and B_I = B[idx, :] in one launch (bf16); returns (A_I, B_I)."""
+    lda = _row_major(A, "A")
+    ldb = _row_major(B, "B")
+    M, d = A.shape
+    if B.shape[0] != d:
+        raise ValueError("A and B disagree on d")
+    N = B.shape[1]
+    k = idx.numel()
+    if out_a is None:
+        out_a = torch.empty((M, (k + 7) // 8 * 8), dtype=A.dtype, device=A.device)[:, :k]
+    if out_b is None:
+        out_b = torch.empty((k, (N + 7) // 8 * 8), dtype=B.dtype, device=B.device)[:, :N]
+    if A.dtype != torch.bfloat16 or B.dtype != torch.bfloat16:
+        raise TypeError("rmm_compact_gather takes bf16 operands")
+    _check(lib.rmm_compact_gather(_ptr(A), lda, _ptr(B), ldb, M, d, N, _ptr(idx), k, _ptr(out_a), out_a.stride(0),
+                                  _ptr(out_b), out_b.stride(0), _stream_ptr(stream)), "rmm_compact_gather")
+    return out_a, out_b
 
 
 def rmm_gemm_workspace_size(dtype: int, N: int, k: int) -> int:

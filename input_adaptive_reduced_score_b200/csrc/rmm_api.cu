@@ -244,6 +244,25 @@ rmm_status rmm_gather_rows(const void* B, int dtype, int64_t d, int64_t N, int64
                    "rmm_gather_rows: launch");
 }
 
+rmm_status rmm_compact_gather(const void* A, int64_t lda, const void* B, int64_t ldb, int64_t M, int64_t d,
+                              int64_t N, const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai, void* B_I,
+                              int64_t ld_bi, void* stream) {
+  clear_error();
+  if (M < 0 || N < 0 || d < 1 || lda < d || ldb < N || k < 1 || k > d || ld_ai < k || ld_bi < N || d > kIntMax)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_compact_gather: bad sizes");
+  if (M == 0 && N == 0) return RMM_OK;
+  if (!idx || (M > 0 && (!A || !A_I)) || (N > 0 && (!B || !B_I)))
+    return fail(RMM_ERR_INVALID_ARG, "rmm_compact_gather: null pointer");
+  if (N > 0 && (!aligned16(B) || !aligned16(B_I) || ldb % 8 || ld_bi % 8))
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_compact_gather: needs 16-byte aligned B/B_I, ldb and ld_bi multiples of 8");
+  if (k + ((M + 7) / 8) * ((k + 63) / 64) > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "rmm_compact_gather: grid");
+  unsigned* err = device_error_word();
+  if (!err) return RMM_ERR_CUDA;
+  return from_cuda(launch_compact_and_gather(A, M, d, lda, B, N, ldb, idx, k, A_I, ld_ai, B_I, ld_bi, err,
+                                             static_cast<cudaStream_t>(stream)),
+                   "rmm_compact_gather: launch");
+}
+
 rmm_status rmm_gemm(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, const int32_t* idx, int64_t d,
                     int64_t M, int64_t N, int64_t k, int dtype, void* Y, int out_dtype, int64_t ldy, void* ws,
                     size_t ws_bytes, void* stream) {
@@ -329,6 +348,14 @@ rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t ldb, in
   if (st != RMM_OK) return st;
   st = rmm_topk(ss, 1, d, d, k, idx, k, stream);
   if (st != RMM_OK) return st;
+  if (dtype == RMM_BF16 && M > 0 && N > 0 && aligned16(B) && ldb % 8 == 0) {
+    // both reduced operands in one launch, then the dense product on them
+    const int64_t ld_bi = round_up(N, 8);
+    void* bi = base + w.bi;
+    st = rmm_compact_gather(A, lda, B, ldb, M, d, N, idx, k, ai, w.ld_ai, bi, ld_bi, stream);
+    if (st != RMM_OK) return st;
+    return rmm_gemm_compacted(ai, w.ld_ai, bi, ld_bi, M, N, k, Y, out_dtype, ldy, stream);
+  }
   st = rmm_compact(A, dtype, M, d, lda, idx, k, ai, w.ld_ai, stream);
   if (st != RMM_OK) return st;
   return rmm_gemm(ai, w.ld_ai, B, ldb, idx, d, M, N, k, dtype, Y, out_dtype, ldy, base + w.bi, w.total - w.bi,

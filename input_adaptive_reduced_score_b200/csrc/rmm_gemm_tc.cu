@@ -37,6 +37,7 @@
 
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
+#include "rmm_launch.cuh"
 
 namespace rmm {
 namespace {
@@ -155,6 +156,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_slot;
+  // set-up above overlaps the previous kernel's tail; operands are read after
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -355,6 +359,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
   cluster_sync();  // barriers of both CTAs initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -551,17 +557,14 @@ cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I,
     // 256 x 256 tiles on SM pairs: one 2-CTA cluster per pair of SMs
     const int64_t tiles = ((M + pairk::BM - 1) / pairk::BM) * ((N + pairk::BN - 1) / pairk::BN);
     const int clusters = static_cast<int>(tiles < sms / 2 ? tiles : sms / 2);
-    gemm_bf16_tc_pair_kernel<<<2 * clusters, pairk::THREADS, pairk::SMEM_BYTES, stream>>>(
-        tmap_a, tmap_b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(k), Y, out_f32, ldy, y_vec_ok,
-        err);
-    return cudaGetLastError();
+    return launch_pdl(gemm_bf16_tc_pair_kernel, dim3(2 * clusters), dim3(pairk::THREADS), pairk::SMEM_BYTES,
+                      stream, tmap_a, tmap_b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(k), Y,
+                      out_f32, ldy, y_vec_ok, err);
   }
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  gemm_bf16_tc_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tmap_a, tmap_b, static_cast<int>(M),
-                                                              static_cast<int>(N), static_cast<int>(k), Y, out_f32,
-                                                              ldy, y_vec_ok, err);
-  return cudaGetLastError();
+  return launch_pdl(gemm_bf16_tc_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, tmap_a, tmap_b,
+                    static_cast<int>(M), static_cast<int>(N), static_cast<int>(k), Y, out_f32, ldy, y_vec_ok, err);
 }
 
 }  // namespace rmm

@@ -52,6 +52,12 @@ cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64
 cudaError_t launch_gather_rows(const void* B, int64_t d, int64_t row_bytes, int64_t ldb_bytes, const int32_t* idx,
                                int64_t k, void* B_I, int64_t ldbi_bytes, unsigned* err, cudaStream_t stream);
 
+// Both reduced operands in one launch (bf16): A_I = A[:, idx] and
+// B_I = B[idx, :]; B, B_I bases and pitches 16-byte aligned, N even.
+cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64_t lda, const void* B, int64_t N,
+                                      int64_t ldb, const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai,
+                                      void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream);
+
 // ---- reduced GEMM (rmm_gemm_tc.cu, rmm_gemm_simt.cu)
 // Returns cudaSuccess or an error; on a driver error in tensor-map encoding
 // the message is set and cudaErrorInvalidValue returned.

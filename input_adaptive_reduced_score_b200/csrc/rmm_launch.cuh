@@ -1,0 +1,36 @@
+// rmm_launch.cuh — kernel launches with programmatic dependent launch (PDL).
+//
+// Every librmm kernel starts with pdl_wait() before it touches global memory
+// written by earlier work on the stream, then calls pdl_trigger().  Launched
+// with programmatic stream serialisation, a kernel may therefore begin (and
+// run its set-up) while its predecessor drains, yet never reads before the
+// predecessor's writes are complete; launched without it, both calls are
+// no-ops.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <utility>
+
+namespace rmm {
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+}  // namespace rmm

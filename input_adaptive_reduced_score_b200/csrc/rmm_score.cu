@@ -15,6 +15,7 @@
 #include <algorithm>
 
 #include "rmm_internal.h"
+#include "rmm_launch.cuh"
 
 namespace rmm {
 namespace {
@@ -63,6 +64,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_partial_kernel(
     int64_t out_split_stride, int sqrt_out) {
   constexpr int V = Lanes<T>::kVec;
   __shared__ float red[kScoreThreads * V];
+  pdl_wait();
+  pdl_trigger();
   const int tx = threadIdx.x % col_threads;
   const int ty = threadIdx.x / col_threads;
   const int row_groups = kScoreThreads / col_threads;
@@ -140,6 +143,8 @@ __global__ void __launch_bounds__(256) score_finalize_kernel(const float* __rest
                                                              int64_t splits, float* __restrict__ ss, int64_t ld_ss,
                                                              int sqrt_out) {
   __shared__ float part[8][33];
+  pdl_wait();
+  pdl_trigger();
   const int c = threadIdx.x & 31, g = threadIdx.x >> 5;
   const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + c;
   const float* p = partial + static_cast<int64_t>(blockIdx.y) * splits * d + j;
@@ -201,20 +206,19 @@ cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int
   const int64_t out_bs = direct ? ld_ss : p.splits * d;
   const int64_t out_ss = direct ? 0 : d;
   const int sq = direct ? sqrt_out : 0;
+  cudaError_t e;
   if (dtype == 1) {
-    score_partial_kernel<__nv_bfloat16><<<grid, kScoreThreads, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(A), M, d, lda, batch_stride, p.col_threads, p.rows_per_split, vec_ok, out,
-        out_bs, out_ss, sq);
+    e = launch_pdl(score_partial_kernel<__nv_bfloat16>, grid, dim3(kScoreThreads), 0, stream,
+                   static_cast<const __nv_bfloat16*>(A), M, d, lda, batch_stride, p.col_threads, p.rows_per_split,
+                   vec_ok, out, out_bs, out_ss, sq);
   } else {
-    score_partial_kernel<float><<<grid, kScoreThreads, 0, stream>>>(static_cast<const float*>(A), M, d, lda,
-                                                                    batch_stride, p.col_threads, p.rows_per_split,
-                                                                    vec_ok, out, out_bs, out_ss, sq);
+    e = launch_pdl(score_partial_kernel<float>, grid, dim3(kScoreThreads), 0, stream, static_cast<const float*>(A),
+                   M, d, lda, batch_stride, p.col_threads, p.rows_per_split, vec_ok, out, out_bs, out_ss, sq);
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || direct) return e;
   const dim3 g2(static_cast<unsigned>((d + 31) / 32), static_cast<unsigned>(batch));
-  score_finalize_kernel<<<g2, 256, 0, stream>>>(static_cast<const float*>(ws), d, p.splits, ss, ld_ss, sqrt_out);
-  return cudaGetLastError();
+  return launch_pdl(score_finalize_kernel, g2, dim3(256), 0, stream, static_cast<const float*>(ws), d, p.splits, ss,
+                    ld_ss, sqrt_out);
 }
 
 }  // namespace rmm

@@ -13,6 +13,7 @@
 // a block-wide scan for output positions.
 // Integer work only: the result is the unique set defined by the rule.
 #include "rmm_internal.h"
+#include "rmm_launch.cuh"
 
 namespace rmm {
 namespace {
@@ -64,6 +65,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   const float* s = scores + static_cast<int64_t>(blockIdx.x) * ld_s;
   int32_t* out = idx + static_cast<int64_t>(blockIdx.x) * ld_idx;
   const int tid = threadIdx.x, lane = tid & 31;
+  pdl_wait();
+  pdl_trigger();
 
   if (kStaged) {
     for (int64_t j = tid; j < d; j += kTopkThreads) staged[j] = score_key(__ldg(s + j));
@@ -148,6 +151,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_search_kernel(const floa
   const float* s = scores + static_cast<int64_t>(blockIdx.x) * ld_s;
   int32_t* out = idx + static_cast<int64_t>(blockIdx.x) * ld_idx;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_trigger();
 
   uint32_t key[KPT];
   uint32_t valid = 0u;
@@ -235,24 +240,24 @@ cudaError_t launch_topk(const float* scores, int64_t batch, int64_t d, int64_t l
                         int64_t ld_idx, cudaStream_t stream) {
   const unsigned grid = static_cast<unsigned>(batch);
   if (d <= 1 * kTopkThreads) {
-    topk_search_kernel<1><<<grid, kTopkThreads, 0, stream>>>(scores, d, ld_s, k, idx, ld_idx);
-    return cudaGetLastError();
+    return launch_pdl(topk_search_kernel<1>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
+                      ld_idx);
   }
   if (d <= 2 * kTopkThreads) {
-    topk_search_kernel<2><<<grid, kTopkThreads, 0, stream>>>(scores, d, ld_s, k, idx, ld_idx);
-    return cudaGetLastError();
+    return launch_pdl(topk_search_kernel<2>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
+                      ld_idx);
   }
   if (d <= 4 * kTopkThreads) {
-    topk_search_kernel<4><<<grid, kTopkThreads, 0, stream>>>(scores, d, ld_s, k, idx, ld_idx);
-    return cudaGetLastError();
+    return launch_pdl(topk_search_kernel<4>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
+                      ld_idx);
   }
   if (d <= 8 * kTopkThreads) {
-    topk_search_kernel<8><<<grid, kTopkThreads, 0, stream>>>(scores, d, ld_s, k, idx, ld_idx);
-    return cudaGetLastError();
+    return launch_pdl(topk_search_kernel<8>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
+                      ld_idx);
   }
   if (d <= 16 * kTopkThreads) {
-    topk_search_kernel<16><<<grid, kTopkThreads, 0, stream>>>(scores, d, ld_s, k, idx, ld_idx);
-    return cudaGetLastError();
+    return launch_pdl(topk_search_kernel<16>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
+                      ld_idx);
   }
   const int64_t bytes = d * 4;
   if (bytes <= kMaxStagedBytes) {
@@ -261,12 +266,10 @@ cudaError_t launch_topk(const float* scores, int64_t batch, int64_t d, int64_t l
                                                  static_cast<int>(kMaxStagedBytes));
       if (e != cudaSuccess) return e;
     }
-    topk_kernel<true><<<static_cast<unsigned>(batch), kTopkThreads, static_cast<size_t>(bytes), stream>>>(
-        scores, d, ld_s, k, idx, ld_idx);
-  } else {
-    topk_kernel<false><<<static_cast<unsigned>(batch), kTopkThreads, 0, stream>>>(scores, d, ld_s, k, idx, ld_idx);
+    return launch_pdl(topk_kernel<true>, dim3(grid), dim3(kTopkThreads), static_cast<size_t>(bytes), stream, scores,
+                      d, ld_s, k, idx, ld_idx);
   }
-  return cudaGetLastError();
+  return launch_pdl(topk_kernel<false>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx, ld_idx);
 }
 
 }  // namespace rmm

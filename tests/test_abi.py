@@ -59,6 +59,9 @@ def test_validation_rejects_before_launch():
     assert _raw("rmm_gemm", vp(16), 8, vp(16), 8, vp(16), 8, 4, 8, 4, 1, vp(16), 1, 8, vp(0), 0, s) == 3  # no workspace
     assert _raw("rmm_gather_rows", vp(16), 1, 0, 8, 8, vp(16), 4, vp(16), 8, s) == 1    # d = 0
     assert _raw("rmm_gather_rows", vp(16), 1, 8, 8, 12, vp(16), 4, vp(16), 12, s) == 2  # pitch not 16-byte
+    assert _raw("rmm_compact_gather", vp(16), 8, vp(16), 8, 4, 8, 8, vp(0), 4, vp(16), 8, vp(16), 8, s) == 1  # null
+    assert _raw("rmm_compact_gather", vp(16), 8, vp(16), 12, 4, 8, 12, vp(16), 4, vp(16), 8, vp(16), 16, s) == 2
+    assert _raw("rmm_compact_gather", vp(16), 8, vp(16), 8, 4, 8, 8, vp(16), 9, vp(16), 9, vp(16), 8, s) == 1  # k > d
     assert _raw("rmm_matmul", vp(16), 8, vp(16), 8, 4, 8, 8, ctypes.c_double(1.5), 1, vp(16), 1, 8,
                 vp(0), vp(0), vp(16), 1 << 20, s) == 1
     assert _raw("rmm_matmul", vp(16), 8, vp(16), 8, 4, 8, 8, ctypes.c_double(0.5), 1, vp(16), 1, 8,

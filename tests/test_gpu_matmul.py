@@ -143,6 +143,39 @@ def test_compact_exact(dtype, M, d, k):
     no_device_error()
 
 
+@pytest.mark.parametrize("M,d,N,k", [(300, 1000, 700, 333), (4096, 4096, 1024, 2048), (3, 5, 2, 1),
+                                     (129, 2100, 701, 2100), (0, 64, 24, 10), (17, 96, 264, 65)])
+def test_compact_gather_exact(M, d, N, k):
+    """Both reduced operands in one launch equal A[:, I] and B[I, :] exactly."""
+    rng = np.random.default_rng(M + d + N)
+    A = W.llm_activation_bf16(5, max(M, 1), d)[:M]
+    Bb = W.weight_bf16(6, d, N)
+    idx = np.sort(rng.choice(d, k, replace=False)).astype(np.int32)
+    At = bf16_tensor(A) if M > 0 else torch.empty((0, d), dtype=torch.bfloat16, device="cuda")
+    Bt = _pitched(bf16_tensor(Bb))
+    it = torch.from_numpy(idx).cuda()
+    AI, BI = R.rmm_compact_gather(At, Bt, it)
+    np.testing.assert_array_equal(to_f64(AI), oracle.decode(A, "bf16")[:, idx])
+    np.testing.assert_array_equal(to_f64(BI), oracle.decode(Bb, "bf16")[idx, :])
+    no_device_error()
+
+
+def test_compact_gather_bad_index_gives_zeros_and_flag():
+    M, d, N, k = 40, 128, 72, 16
+    A = W.llm_activation_bf16(7, M, d)
+    Bb = W.weight_bf16(8, d, N)
+    idx = np.arange(k, dtype=np.int32)
+    idx[3] = -2
+    AI, BI = R.rmm_compact_gather(bf16_tensor(A), bf16_tensor(Bb), torch.from_numpy(idx).cuda())
+    assert R.rmm_device_error(clear=True) == 1
+    a, b = to_f64(AI), to_f64(BI)
+    assert np.all(a[:, 3] == 0) and np.all(b[3] == 0)
+    ok = np.delete(np.arange(k), 3)
+    np.testing.assert_array_equal(a[:, ok], oracle.decode(A, "bf16")[:, idx[ok]])
+    np.testing.assert_array_equal(b[ok], oracle.decode(Bb, "bf16")[idx[ok]])
+    no_device_error()
+
+
 # ------------------------------------------------------------------ reduced GEMM
 
 def _pitched(t):
