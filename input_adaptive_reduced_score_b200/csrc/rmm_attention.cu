@@ -44,7 +44,6 @@ constexpr int CHUNK_BYTES = TILE * 128;   // one [128 x 64] bf16 tile, 128-byte 
 constexpr int ATT_THREADS = 192;          // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr unsigned long long kDrainNs = 100000000ull;
 
 struct AttnParams {
   int S;            // tokens
@@ -56,14 +55,6 @@ struct AttnParams {
   int c_stages;     // pass C key/value ring depth (1 or 2, as shared memory allows)
   float scale_log2; // logit scale times log2(e)
 };
-
-__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
-  const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kDrainNs) return false;
-  }
-  return true;
-}
 
 // ------------------------------------------------------------------ prep kernels
 
@@ -213,7 +204,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           phase ^= 1u;
         }
       }
-      drain_wait(smem_u32(&bars->fixed_full), 0);
+      wait_drain(smem_u32(&bars->fixed_full), 0);
       uint32_t st = stage, ph = phase;
       for (uint32_t j = 0; j < (issued < QK_STAGES ? issued : QK_STAGES); ++j) {
         if (st == 0) {
@@ -222,7 +213,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         } else {
           --st;
         }
-        drain_wait(full(st), ph);
+        wait_drain(full(st), ph);
       }
     }
     __syncwarp();
@@ -255,7 +246,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     if (lane == 0) {
       mma_commit(smem_u32(&bars->drain));
-      drain_wait(smem_u32(&bars->drain), 0);
+      wait_drain(smem_u32(&bars->drain), 0);
     }
     __syncwarp();
   } else {
@@ -436,7 +427,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           phase ^= 1u;
         }
       }
-      drain_wait(smem_u32(&bars->qfull), 0);
+      wait_drain(smem_u32(&bars->qfull), 0);
       uint32_t st = stage, ph = phase;
       for (uint32_t j = 0; j < (issued < static_cast<uint32_t>(nst) ? issued : static_cast<uint32_t>(nst)); ++j) {
         if (st == 0) {
@@ -445,7 +436,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         } else {
           --st;
         }
-        drain_wait(kvfull(st), ph);
+        wait_drain(kvfull(st), ph);
       }
     }
     __syncwarp();
@@ -508,7 +499,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (lane == 0) {
       if (nrb > 0) mma_commit(smem_u32(&bars->ofull));
       mma_commit(smem_u32(&bars->drain));
-      drain_wait(smem_u32(&bars->drain), 0);
+      wait_drain(smem_u32(&bars->drain), 0);
     }
     __syncwarp();
   } else {

@@ -1,14 +1,22 @@
 // rmm_compact.cu — the reduced operands of A_{:,I} B_{I,:} (Reduced Matrix
 // Multiplication technical summary, Metodología › Mecanismo Central):
-//   compact_kernel      A_I[:, r] = A[:, I_r]   (column gather of the activation)
-//   gather_rows_kernel  B_I[r, :] = B[I_r, :]   (row gather of the weight)
+//   A_I[:, r] = A[:, I_r]   (column gather of the activation)
+//   B_I[r, :] = B[I_r, :]   (row gather of the weight)
 //
-// HBM-bound gather.  Each thread produces 8 consecutive output columns (one
-// 16-byte store for bf16) of each of 8 rows: it reads its 8 indices once,
-// gathers the source elements through the read-only cache (the kept indices
-// are increasing, so a warp's 256 gathers cover a short run of the source row
-// and reuse its sectors), and writes them with vector stores.
+// HBM-bound gathers.
+//  - bf16 A with 16-byte aligned rows: a block copies R whole rows of A into
+//    shared memory with one bulk copy per row (the copy engine reads them at
+//    full width); then the lanes of a warp take 32 consecutive output
+//    columns, read their sources from shared memory (increasing and close
+//    together, so without bank conflicts) and store 64 contiguous bytes.
+//    R is chosen so a block stages about 32 KB.
+//  - other layouts: each thread gathers its 8 output columns of 8 rows
+//    straight from global memory through the read-only cache.
+//  - B rows are whole contiguous rows: one block per kept row streams it with
+//    16-byte loads and stores.
 #include <cuda_bf16.h>
+
+#include <atomic>
 
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
@@ -73,6 +81,82 @@ __device__ __forceinline__ void compact_block(int64_t blk, const T* __restrict__
   }
 }
 
+// Staged compaction of R rows (bf16).  The caller guarantees: A and every row
+// start 16-byte aligned (lda a multiple of 8), d a multiple of 8, R * 2d bytes
+// of dynamic shared memory.
+constexpr int kStageTargetBytes = 32 * 1024;
+constexpr int64_t kMaxStagedRowBytes = 200 * 1024;
+
+__device__ __forceinline__ void compact_rows_block(int64_t blk, const uint16_t* __restrict__ A, int64_t M, int64_t d,
+                                                   int64_t lda, const int32_t* __restrict__ idx, int64_t k,
+                                                   uint16_t* __restrict__ AI, int64_t ld_ai, int R, unsigned* err,
+                                                   uint8_t* stage) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  const int64_t row0 = blk * R;
+  if (row0 >= M) return;  // block-uniform
+  const int rows = static_cast<int>(min(static_cast<int64_t>(R), M - row0));
+  const uint32_t row_bytes = static_cast<uint32_t>(2 * d);
+  const uint32_t sbase = smem_u32(stage);
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(b, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(b, static_cast<uint32_t>(rows) * row_bytes);
+    for (int r = 0; r < rows; ++r) bulk_load_1d(sbase + r * row_bytes, A + (row0 + r) * lda, row_bytes, b);
+  }
+  __syncthreads();
+  const uint16_t* srows = reinterpret_cast<const uint16_t*>(stage);
+  bool landed = false;
+  // Output columns in chunks of 2048: thread t writes columns
+  // cbase + i*256 + t (i < 8), so a warp's 32 lanes handle 32 consecutive
+  // output columns, whose sources are increasing and close together in the
+  // staged row (conflict-free shared-memory reads, 64-byte stores).  The
+  // indices of the next chunk are loaded before the current chunk's stores.
+  auto load_idx = [&](int64_t cbase, int32_t (&j)[kPerThread]) {
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      const int64_t c = cbase + i * kCompactThreads + threadIdx.x;
+      j[i] = -2;  // no such output column
+      if (c < k) {
+        const int32_t v = __ldg(idx + c);
+        if (v >= 0 && v < d) {
+          j[i] = v;
+        } else {
+          j[i] = -1;
+          bad = true;
+        }
+      }
+    }
+    if (bad) record_error(err, kDevErrBadIndex);
+  };
+  int32_t jn[kPerThread];
+  load_idx(0, jn);
+  for (int64_t cbase = 0; cbase < k; cbase += kColsPerCta) {
+    int32_t j[kPerThread];
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) j[i] = jn[i];
+    if (cbase + kColsPerCta < k) load_idx(cbase + kColsPerCta, jn);
+    if (!landed) {
+      // bounded wait; on expiry the site is recorded and no row is written
+      if (!mbar_wait(b, 0, &abort_flag, err, 61)) break;
+      landed = true;
+    }
+    for (int r = 0; r < rows; ++r) {
+      const uint16_t* sr = srows + static_cast<int64_t>(r) * d;
+      uint16_t* o = AI + (row0 + r) * ld_ai + cbase + threadIdx.x;
+#pragma unroll
+      for (int i = 0; i < kPerThread; ++i)
+        if (j[i] != -2) o[i * kCompactThreads] = j[i] >= 0 ? sr[j[i]] : static_cast<uint16_t>(0);
+    }
+  }
+  // thread 0 always has an output column, so it has waited for the copies;
+  // after an expired wait it waits once more, briefly, before the block retires
+  if (!landed && threadIdx.x == 0) wait_drain(b, 0);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kCompactThreads) compact_kernel(const T* __restrict__ A, int64_t M, int64_t d,
                                                                   int64_t lda, const int32_t* __restrict__ idx,
@@ -81,6 +165,17 @@ __global__ void __launch_bounds__(kCompactThreads) compact_kernel(const T* __res
   pdl_wait();
   pdl_trigger();
   compact_block<T>(blockIdx.x, A, M, d, lda, idx, k, AI, ld_ai, chunks, vec_ok, err);
+}
+
+__global__ void __launch_bounds__(kCompactThreads) compact_staged_kernel(const uint16_t* __restrict__ A, int64_t M,
+                                                                         int64_t d, int64_t lda,
+                                                                         const int32_t* __restrict__ idx, int64_t k,
+                                                                         uint16_t* __restrict__ AI, int64_t ld_ai,
+                                                                         int R, unsigned* err) {
+  extern __shared__ __align__(128) uint8_t stage[];
+  pdl_wait();
+  pdl_trigger();
+  compact_rows_block(blockIdx.x, A, M, d, lda, idx, k, AI, ld_ai, R, err, stage);
 }
 
 // One CTA per kept row: the row I_r of B is copied whole with 16-byte loads and
@@ -131,21 +226,53 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint4
 }
 
 // Both reduced operands in one grid: blocks [0, k) gather the kept rows of B,
-// the remaining blocks compact the kept columns of A (bf16), so the two HBM
+// the remaining blocks compact the kept columns of A (bf16; staged R rows per
+// block, or the direct gather of 8 rows x 2048 columns), so the two HBM
 // streams overlap.
+template <bool kStagedA>
 __global__ void __launch_bounds__(kGatherThreads) compact_gather_kernel(
     const uint4* __restrict__ B, int64_t d, int64_t vecs, int64_t tail_halves, int64_t ldb_vec,
-    uint4* __restrict__ BI, int64_t ldbi_vec, const __nv_bfloat16* __restrict__ A, int64_t M, int64_t lda,
-    __nv_bfloat16* __restrict__ AI, int64_t ld_ai, int64_t chunks, bool vec_ok, const int32_t* __restrict__ idx,
+    uint4* __restrict__ BI, int64_t ldbi_vec, const uint16_t* __restrict__ A, int64_t M, int64_t lda,
+    uint16_t* __restrict__ AI, int64_t ld_ai, int64_t chunks, int R, bool vec_ok, const int32_t* __restrict__ idx,
     int64_t k, unsigned* err) {
+  extern __shared__ __align__(128) uint8_t stage[];
   pdl_wait();
   pdl_trigger();
   const int64_t blk = blockIdx.x;
   if (blk < k) {
     gather_row_block(blk, B, d, vecs, tail_halves, ldb_vec, idx, k, BI, ldbi_vec, err);
+  } else if constexpr (kStagedA) {
+    compact_rows_block(blk - k, A, M, d, lda, idx, k, AI, ld_ai, R, err, stage);
   } else {
-    compact_block<__nv_bfloat16>(blk - k, A, M, d, lda, idx, k, AI, ld_ai, chunks, vec_ok, err);
+    compact_block<__nv_bfloat16>(blk - k, reinterpret_cast<const __nv_bfloat16*>(A), M, d, lda, idx, k,
+                                 reinterpret_cast<__nv_bfloat16*>(AI), ld_ai, chunks, vec_ok, err);
   }
+}
+
+// Rows per block of the staged compaction, or 0 when A's layout does not allow
+// whole-row bulk copies (16-byte aligned rows, d a multiple of 8, a row of at
+// most kMaxStagedRowBytes).
+int staged_rows(const void* A, int64_t d, int64_t lda) {
+  if (reinterpret_cast<uintptr_t>(A) % 16 || lda % 8 || d % 8) return 0;
+  const int64_t row_bytes = 2 * d;
+  if (row_bytes > kMaxStagedRowBytes) return 0;
+  const int64_t r = kStageTargetBytes / row_bytes;
+  return static_cast<int>(r < 1 ? 1 : (r > 8 ? 8 : r));
+}
+
+// Opt a kernel into kMaxStagedRowBytes of dynamic shared memory, once per device.
+template <auto Kernel>
+bool allow_staged_smem() {
+  static std::atomic<uint64_t> configured{0};  // bit per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const uint64_t bit = 1ull << dev;
+  if (configured.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kMaxStagedRowBytes)) !=
+      cudaSuccess)
+    return false;
+  configured.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
 }
 
 }  // namespace
@@ -162,10 +289,19 @@ cudaError_t launch_gather_rows(const void* B, int64_t d, int64_t row_bytes, int6
 cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64_t lda, const int32_t* idx,
                            int64_t k, void* A_I, int64_t ld_ai, unsigned* err, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
-  const int64_t chunks = (k + kColsPerCta - 1) / kColsPerCta;
-  const int64_t blocks = ((M + kRowsPerCta - 1) / kRowsPerCta) * chunks;
   const size_t elt = dtype == 1 ? 2 : 4;
   const bool vec_ok = reinterpret_cast<uintptr_t>(A_I) % 16 == 0 && (ld_ai * elt) % 16 == 0;
+  const int R = dtype == 1 ? staged_rows(A, d, lda) : 0;
+  if (R > 0) {
+    const int64_t blocks = (M + R - 1) / R;
+    const size_t smem = static_cast<size_t>(R) * 2 * d;
+    if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    if (smem > 48 * 1024 && !allow_staged_smem<compact_staged_kernel>()) return cudaErrorInvalidValue;
+    return launch_pdl(compact_staged_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kCompactThreads), smem, stream,
+                      static_cast<const uint16_t*>(A), M, d, lda, idx, k, static_cast<uint16_t*>(A_I), ld_ai, R, err);
+  }
+  const int64_t chunks = (k + kColsPerCta - 1) / kColsPerCta;
+  const int64_t blocks = ((M + kRowsPerCta - 1) / kRowsPerCta) * chunks;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   if (dtype == 1)
     return launch_pdl(compact_kernel<__nv_bfloat16>, dim3(static_cast<unsigned>(blocks)), dim3(kCompactThreads), 0,
@@ -179,16 +315,27 @@ cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64
 cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64_t lda, const void* B, int64_t N,
                                       int64_t ldb, const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai,
                                       void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream) {
+  const int R = staged_rows(A, d, lda);
   const int64_t chunks = (k + kColsPerCta - 1) / kColsPerCta;
-  const int64_t cblocks = M > 0 ? ((M + kRowsPerCta - 1) / kRowsPerCta) * chunks : 0;
+  const int64_t cblocks = M <= 0 ? 0 : (R > 0 ? (M + R - 1) / R : ((M + kRowsPerCta - 1) / kRowsPerCta) * chunks);
   const int64_t blocks = k + cblocks;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   const bool vec_ok = reinterpret_cast<uintptr_t>(A_I) % 16 == 0 && (ld_ai * 2) % 16 == 0;
   const int64_t row_bytes = N * 2;
-  return launch_pdl(compact_gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kGatherThreads), 0, stream,
-                    static_cast<const uint4*>(B), d, row_bytes / 16, (row_bytes % 16) / 2, ldb * 2 / 16,
-                    static_cast<uint4*>(B_I), ld_bi * 2 / 16, static_cast<const __nv_bfloat16*>(A), M, lda,
-                    static_cast<__nv_bfloat16*>(A_I), ld_ai, chunks, vec_ok, idx, k, err);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(kGatherThreads);
+  const uint4* b = static_cast<const uint4*>(B);
+  uint4* bi = static_cast<uint4*>(B_I);
+  const uint16_t* a = static_cast<const uint16_t*>(A);
+  uint16_t* ai = static_cast<uint16_t*>(A_I);
+  if (R > 0) {
+    const size_t smem = static_cast<size_t>(R) * 2 * d;
+    if (smem > 48 * 1024 && !allow_staged_smem<compact_gather_kernel<true>>()) return cudaErrorInvalidValue;
+    return launch_pdl(compact_gather_kernel<true>, grid, block, smem, stream, b, d, row_bytes / 16,
+                      (row_bytes % 16) / 2, ldb * 2 / 16, bi, ld_bi * 2 / 16, a, M, lda, ai, ld_ai, chunks, R, vec_ok,
+                      idx, k, err);
+  }
+  return launch_pdl(compact_gather_kernel<false>, grid, block, 0, stream, b, d, row_bytes / 16, (row_bytes % 16) / 2,
+                    ldb * 2 / 16, bi, ld_bi * 2 / 16, a, M, lda, ai, ld_ai, chunks, 0, vec_ok, idx, k, err);
 }
 
 }  // namespace rmm

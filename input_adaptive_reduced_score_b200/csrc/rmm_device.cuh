@@ -84,6 +84,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // mbar_wait taken by a whole warp with a warp-uniform result: true only if
 // every lane saw the phase complete.  Use it where a warp-synchronous
 // (.sync.aligned) instruction follows, so an abort can never split the warp.
+// Last, short wait before a CTA retires after an abort: lets copies or MMAs
+// already in flight land in (or finish reading) this CTA's shared memory.
+constexpr unsigned long long kDrainNs = 100000000ull;  // 100 ms
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_ns() - t0 > kDrainNs) return false;
+  }
+  return true;
+}
+
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                unsigned* err, unsigned site) {
   const bool ok = mbar_wait(bar, parity, abort_flag, err, site);
@@ -91,6 +102,15 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, vo
 }
 
 // ------------------------------------------------------------------ TMA / cp.async
+
+// Untiled bulk copy of `bytes` (a multiple of 16) from global memory to this
+// CTA's shared memory; both addresses 16-byte aligned.  Completion is
+// signalled on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
 
 // 2-D tiled TMA load of one box into shared memory; completion is signalled on
 // `bar` as transaction bytes.  The innermost coordinate x must be a multiple

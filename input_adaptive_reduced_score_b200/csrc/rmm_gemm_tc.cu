@@ -53,7 +53,6 @@ constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * (A_STAGE + B_STAGE) + BAR_BYTES + 1024;
-constexpr unsigned long long kDrainNs = 100000000ull;  // 100 ms
 
 static_assert(BK == 64 && BN == 256, "stage layout assumes 64 x 256 B stages");
 
@@ -68,13 +67,6 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= BAR_BYTES, "barrier block");
 
-__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
-  const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_ns() - t0 > kDrainNs) return false;
-  }
-  return true;
-}
 
 // Store 32 fp32 accumulator values of one output row (columns col0 ..
 // col0+31, masked at N) as fp32 or bf16, with 16-byte stores when aligned.
@@ -288,12 +280,18 @@ __global__ void __launch_bounds__(THREADS, 1)
 //   - both CTAs' epilogue warps arrive on the leader's accumulator-empty
 //     barrier;
 //   - cluster barriers after set-up and before tensor memory is released.
+// Work items: tiles below `split_from` are whole 256 x 256 tiles; each tile
+// from `split_from` on is done as two 256 x 128 halves (MMA N = 128, each
+// CTA holding one 64-column chunk of B).  The host splits the tiles of a last
+// partial wave when their halves still fit in one wave, so that wave ends in
+// about half the time.
 namespace pairk {
 constexpr int BM = 256, BN = 256, BK = 64, STAGES = 6;
 constexpr int A_STAGE = 128 * BK * 2;           // this CTA's 128 rows: 16 KB
 constexpr int B_CHUNK = BK * 128;               // 64 columns x 64 rows: 8 KB
 constexpr int B_STAGE = 2 * B_CHUNK;            // this CTA's 128 columns: 16 KB
 constexpr uint32_t STAGE_TX = 2 * (A_STAGE + B_STAGE);
+constexpr uint32_t STAGE_TX_HALF = 2 * (A_STAGE + B_CHUNK);
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = (2 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -309,12 +307,22 @@ struct PairBars {
   int abort_flag;
 };
 static_assert(sizeof(PairBars) <= BAR_BYTES, "barrier block");
+
+struct Item {
+  int m_blk, n0, width;  // tile rows m_blk*256.., columns n0 .. n0+width-1
+};
+__device__ __forceinline__ Item item_of(int i, int split_from, int num_m) {
+  if (i < split_from) return Item{i % num_m, (i / num_m) * BN, BN};
+  const int j = i - split_from;
+  const int tile = split_from + (j >> 1);
+  return Item{tile % num_m, (tile / num_m) * BN + (j & 1) * (BN / 2), BN / 2};
+}
 }  // namespace pairk
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
     gemm_bf16_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-                             int M, int N, int K, void* __restrict__ Y, int out_f32, int64_t ldy, int y_vec_ok,
-                             unsigned* err) {
+                             int M, int N, int K, int split_from, void* __restrict__ Y, int out_f32, int64_t ldy,
+                             int y_vec_ok, unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -333,7 +341,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
   const bool leader = rank == 0;
   const int cid = static_cast<int>(cluster_id_x()), ncl = static_cast<int>(nclusters_x());
   const int num_m = (M + pairk::BM - 1) / pairk::BM, num_n = (N + pairk::BN - 1) / pairk::BN;
-  const int num_tiles = num_m * num_n;
+  const int num_items = split_from + 2 * (num_m * num_n - split_from);
   const int nk = (K + pairk::BK - 1) / pairk::BK;
 
   if (threadIdx.x == 0) {
@@ -367,20 +375,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, issued = 0;
       bool ok = true;
-      for (int tile = cid; ok && tile < num_tiles; tile += ncl) {
-        const int m_blk = tile % num_m, n_blk = tile / num_m;
-        const int a_row = m_blk * pairk::BM + static_cast<int>(rank) * 128;
-        const int b_col = n_blk * pairk::BN + static_cast<int>(rank) * 128;
+      for (int i = cid; ok && i < num_items; i += ncl) {
+        const pairk::Item t = pairk::item_of(i, split_from, num_m);
+        const bool whole = t.width == pairk::BN;
+        const int a_row = t.m_blk * pairk::BM + static_cast<int>(rank) * 128;
+        const int b_col = t.n0 + static_cast<int>(rank) * (t.width / 2);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, err, 41)) {
             ok = false;
             break;
           }
           const uint32_t full_leader = mapa_shared(full(stage), 0);
-          if (leader) mbar_arrive_expect_tx(full(stage), pairk::STAGE_TX);
+          if (leader) mbar_arrive_expect_tx(full(stage), whole ? pairk::STAGE_TX : pairk::STAGE_TX_HALF);
           tma_load_2d_pair(sA(stage), &tmap_a, full_leader, kb * pairk::BK, a_row);
           tma_load_2d_pair(sB(stage), &tmap_b, full_leader, b_col, kb * pairk::BK);
-          tma_load_2d_pair(sB(stage) + pairk::B_CHUNK, &tmap_b, full_leader, b_col + 64, kb * pairk::BK);
+          if (whole)
+            tma_load_2d_pair(sB(stage) + pairk::B_CHUNK, &tmap_b, full_leader, b_col + 64, kb * pairk::BK);
           ++issued;
           if (++stage == pairk::STAGES) {
             stage = 0;
@@ -407,11 +417,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA)
     if (leader) {
-      constexpr uint32_t idesc = idesc_bf16_f32(pairk::BM, pairk::BN, /*a_mn=*/false, /*b_mn=*/true);
+      constexpr uint32_t idesc_whole = idesc_bf16_f32(pairk::BM, pairk::BN, /*a_mn=*/false, /*b_mn=*/true);
+      constexpr uint32_t idesc_half = idesc_bf16_f32(pairk::BM, pairk::BN / 2, /*a_mn=*/false, /*b_mn=*/true);
       uint32_t stage = 0, phase = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = cid; ok && tile < num_tiles; tile += ncl, ++it) {
+      for (int i = cid; ok && i < num_items; i += ncl, ++it) {
+        const uint32_t idesc = i < split_from ? idesc_whole : idesc_half;
         const uint32_t b = it & 1, acc_phase = (it >> 1) & 1;
         if (!mbar_wait_warp(accempty(b), acc_phase ^ 1u, abort_flag, err, 42)) break;
         tc_fence_after();
@@ -452,19 +464,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
     const int qtr = warp & 3;
     const int half = (warp - 2) / 4;
     int it = 0;
-    for (int tile = cid; tile < num_tiles; tile += ncl, ++it) {
+    for (int i = cid; i < num_items; i += ncl, ++it) {
       const uint32_t b = it & 1, acc_phase = (it >> 1) & 1;
       if (!mbar_wait_warp(accfull(b), acc_phase, abort_flag, err, 44)) break;
       tc_fence_after();
-      const int m_blk = tile % num_m, n_blk = tile / num_m;
-      const int row = m_blk * pairk::BM + static_cast<int>(rank) * 128 + qtr * 32 + lane;
-      const uint32_t taddr = tmem_base + b * pairk::BN + half * 128 + (static_cast<uint32_t>(qtr * 32) << 16);
+      const pairk::Item t = pairk::item_of(i, split_from, num_m);
+      const int hw = t.width / 2;  // accumulator columns per epilogue half
+      const int row = t.m_blk * pairk::BM + static_cast<int>(rank) * 128 + qtr * 32 + lane;
+      const uint32_t taddr = tmem_base + b * pairk::BN + half * hw + (static_cast<uint32_t>(qtr * 32) << 16);
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < hw / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(taddr + cc * 32, v);
         tmem_wait_ld();
-        const int col0 = n_blk * pairk::BN + half * 128 + cc * 32;
+        const int col0 = t.n0 + half * hw + cc * 32;
         if (row < M && col0 < N) store_row32(Y, out_f32, ldy, y_vec_ok, row, col0, N, v);
       }
       tc_fence_before();
@@ -556,10 +569,16 @@ cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I,
   if (M >= pairk::BM) {
     // 256 x 256 tiles on SM pairs: one 2-CTA cluster per pair of SMs
     const int64_t tiles = ((M + pairk::BM - 1) / pairk::BM) * ((N + pairk::BN - 1) / pairk::BN);
-    const int clusters = static_cast<int>(tiles < sms / 2 ? tiles : sms / 2);
+    const int64_t pairs = sms / 2;
+    // split the tiles of a last partial wave into halves when those fit in one wave
+    const int64_t rem = tiles % pairs;
+    const int64_t split_from = (rem > 0 && 2 * rem <= pairs) ? tiles - rem : tiles;
+    const int64_t items = split_from + 2 * (tiles - split_from);
+    if (items > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    const int clusters = static_cast<int>(items < pairs ? items : pairs);
     return launch_pdl(gemm_bf16_tc_pair_kernel, dim3(2 * clusters), dim3(pairk::THREADS), pairk::SMEM_BYTES,
-                      stream, tmap_a, tmap_b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(k), Y,
-                      out_f32, ldy, y_vec_ok, err);
+                      stream, tmap_a, tmap_b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(k),
+                      static_cast<int>(split_from), Y, out_f32, ldy, y_vec_ok, err);
   }
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);

@@ -3,15 +3,20 @@
 // keep the k indices with the highest scores).  The tie rule (lowest index
 // first) and the ascending output order are this library's reading.
 //
-// One 1024-thread CTA per score row; scores are mapped to order-preserving
-// uint32 keys.  The exact key T of the k-th largest score is found either by
-// a register-resident 4-ary search over the key range (rows of up to 16384)
-// or by a 4-pass MSB-first radix select (8-bit digits, shared-memory
-// histograms; keys staged once in shared memory when the row fits in 200 KB).
-// A final ordered sweep emits, in ascending index order, every index with
-// key > T and the first `need` indices with key == T, using warp ballots and
-// a block-wide scan for output positions.
-// Integer work only: the result is the unique set defined by the rule.
+// One CTA per score row; scores are mapped to order-preserving uint32 keys.
+// Rows of up to 51200 scores are staged once in shared memory and selected
+// by a histogram search: the key range [min, max] is cut into 2048 bins,
+// the bin holding the k-th largest key becomes the new range, and the search
+// stops when the range is a single key (at most three rounds for 32-bit
+// keys) or when the keys at or above the range's start are exactly k.  Each
+// round costs three block barriers.  The selected indices are then written in
+// ascending order in one sweep: each warp owns a contiguous block of indices,
+// one barrier exchanges the warps' counts, and ballots place each index.
+// Longer rows use a 4-pass MSB-first radix select that re-reads the scores
+// from global memory.  Integer work only: the result is the unique set
+// defined by the rule.
+#include <atomic>
+
 #include "rmm_internal.h"
 #include "rmm_launch.cuh"
 
@@ -52,13 +57,11 @@ __device__ __forceinline__ uint32_t block_flag_scan(bool flag, uint32_t* warp_cn
   return r;
 }
 
-// Keys of the row: staged in dynamic shared memory when it fits (one parallel
-// load, then every pass reads shared memory), else re-read from global memory.
-template <bool kStaged>
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restrict__ scores, int64_t d,
+// Rows too long to stage: 4-pass radix select over keys re-read from global
+// memory (8-bit digits, shared-memory histograms).
+__global__ void __launch_bounds__(kTopkThreads) topk_radix_kernel(const float* __restrict__ scores, int64_t d,
                                                              int64_t ld_s, int64_t k, int32_t* __restrict__ idx,
                                                              int64_t ld_idx) {
-  extern __shared__ uint32_t staged[];
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_cnt[33];
   __shared__ uint32_t sh_prefix, sh_need;
@@ -68,10 +71,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   pdl_wait();
   pdl_trigger();
 
-  if (kStaged) {
-    for (int64_t j = tid; j < d; j += kTopkThreads) staged[j] = score_key(__ldg(s + j));
-  }
-  auto key_at = [&](int64_t j) -> uint32_t { return kStaged ? staged[j] : score_key(__ldg(s + j)); };
+  auto key_at = [&](int64_t j) -> uint32_t { return score_key(__ldg(s + j)); };
 
   uint32_t prefix = 0u, mask = 0u, need = static_cast<uint32_t>(k);
   for (int pass = 0; pass < 4; ++pass) {
@@ -136,140 +136,233 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const float* __restr
   }
 }
 
-// Register-resident variant for d <= 1024 * KPT: thread t holds the keys of
-// indices t, t + 1024, ...  The threshold T (the k-th largest key) is found by
-// a 4-ary search over the 32-bit key range: each step counts, block-wide, the
-// keys at or above three probes (warp redux + one barrier, double-buffered
-// counts), keeping count(>= lo) >= k > count(>= hi).  Sixteen steps reach
-// hi = lo + 1, so T = lo exactly.  No atomics.
-template <int KPT>
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_search_kernel(const float* __restrict__ scores, int64_t d,
-                                                                       int64_t ld_s, int64_t k,
-                                                                       int32_t* __restrict__ idx, int64_t ld_idx) {
-  __shared__ uint32_t wcnt[2][32][4];
-  __shared__ uint32_t warp_cnt[33];
+constexpr int kBins = 2048;
+constexpr int64_t kMaxStagedKeys = 51200;  // 200 KB of keys + 8 KB of bins per CTA
+
+// Histogram search on keys staged in shared memory (rows of up to
+// kMaxStagedKeys scores).  Invariant of the search: count(key >= hi) =
+// `above` < k <= count(key >= lo).
+template <int NT>
+__global__ void __launch_bounds__(NT, 1) topk_hist_kernel(const float* __restrict__ scores, int64_t d64, int64_t ld_s,
+                                                           int64_t k64, int32_t* __restrict__ idx, int64_t ld_idx) {
+  constexpr int NW = NT / 32;
+  constexpr int BPT = kBins / NT;  // bins per thread, contiguous
+  static_assert(BPT == 2 || BPT == 8, "bin vectors are 2 or 8 words");
+  extern __shared__ __align__(16) uint32_t keys[];
+  __shared__ __align__(16) uint32_t hist[kBins];
+  __shared__ uint32_t wred[NW][2];  // per-warp min/max, then per-warp bin totals
+  __shared__ uint32_t wcnt[NW][2];  // per-warp (above, in-range) counts for the emission
+  __shared__ uint32_t sh_bin, sh_above, sh_done;
+  const int d = static_cast<int>(d64);
+  const uint32_t k = static_cast<uint32_t>(k64);
   const float* s = scores + static_cast<int64_t>(blockIdx.x) * ld_s;
   int32_t* out = idx + static_cast<int64_t>(blockIdx.x) * ld_idx;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const bool vec4 = (reinterpret_cast<uintptr_t>(s) & 15u) == 0 && (d & 3) == 0;
   pdl_wait();
   pdl_trigger();
 
-  uint32_t key[KPT];
-  uint32_t valid = 0u;
+  // stage the keys, zero the bins, find the key range; the loads of a batch
+  // are all issued before the first is used (one memory round trip per batch)
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  if (vec4) {
+    const int nv = d >> 2;
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+    for (int v0 = tid; v0 < nv; v0 += 4 * NT) {
+      float4 f[4];
 #pragma unroll
-  for (int i = 0; i < KPT; ++i) {
-    const int64_t j = tid + static_cast<int64_t>(i) * kTopkThreads;
-    key[i] = j < d ? score_key(__ldg(s + j)) : 0u;
-    if (j < d) valid |= 1u << i;
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * NT;
+        f[u] = v < nv ? __ldg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * NT;
+        if (v < nv) {
+          const uint4 q = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
+          reinterpret_cast<uint4*>(keys)[v] = q;
+          kmin = min(kmin, min(min(q.x, q.y), min(q.z, q.w)));
+          kmax = max(kmax, max(max(q.x, q.y), max(q.z, q.w)));
+        }
+      }
+    }
+  } else {
+    for (int j0 = tid; j0 < d; j0 += 8 * NT) {
+      float f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * NT;
+        f[u] = j < d ? __ldg(s + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * NT;
+        if (j < d) {
+          const uint32_t key = score_key(f[u]);
+          keys[j] = key;
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
+      }
+    }
   }
-  // every probe lies below 2^32 (probes < hi <= 2^32), so 32-bit compares suffice
-  auto count_ge = [&](uint64_t t) -> uint32_t {
-    const uint32_t t32 = static_cast<uint32_t>(t);
-    uint32_t c = 0u;
-#pragma unroll
-    for (int i = 0; i < KPT; ++i) c += ((valid >> i) & 1u) && key[i] >= t32 ? 1u : 0u;
-    return c;
-  };
+  for (int b = tid; b < kBins; b += NT) hist[b] = 0u;
+  kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+  kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+  if (lane == 0) {
+    wred[warp][0] = kmin;
+    wred[warp][1] = kmax;
+  }
+  __syncthreads();
+  uint64_t lo = __reduce_min_sync(0xFFFFFFFFu, lane < NW ? wred[lane][0] : 0xFFFFFFFFu);
+  uint64_t hi = static_cast<uint64_t>(__reduce_max_sync(0xFFFFFFFFu, lane < NW ? wred[lane][1] : 0u)) + 1u;
+  uint32_t above = 0u;
+  bool done = false;
 
-  uint64_t lo = 0ull, hi = 1ull << 32;  // count(>= lo) = d >= k; count(>= 2^32) = 0 < k
-  int buf = 0;
-  while (hi - lo > 1ull) {
-    const uint64_t w = hi - lo;
-    const uint64_t t1 = lo + w / 4, t2 = lo + w / 2, t3 = lo + (w * 3) / 4;
-    const uint32_t c1 = __reduce_add_sync(0xFFFFFFFFu, count_ge(t1));
-    const uint32_t c2 = __reduce_add_sync(0xFFFFFFFFu, count_ge(t2));
-    const uint32_t c3 = __reduce_add_sync(0xFFFFFFFFu, count_ge(t3));
-    if (lane == 0) {
-      wcnt[buf][warp][0] = c1;
-      wcnt[buf][warp][1] = c2;
-      wcnt[buf][warp][2] = c3;
+  // each round shrinks the range at least 2048-fold (or to one key), so four
+  // rounds always suffice for 32-bit keys; the bound is only a guard
+  for (int round = 0; round < 8 && hi - lo > 1u && !done; ++round) {
+    const uint64_t range = hi - lo;
+    const int nbits = 64 - __clzll(static_cast<long long>(range - 1u));  // ceil(log2(range))
+    const int shift = nbits > 11 ? nbits - 11 : 0;
+    for (int j = tid; j < d; j += NT) {
+      const uint32_t key = keys[j];
+      if (key >= lo && key < hi) atomicAdd(&hist[static_cast<uint32_t>((key - lo) >> shift)], 1u);
     }
     __syncthreads();
-    // every warp sums the 32 per-warp counts itself (no second barrier)
-    const uint32_t n1 = __reduce_add_sync(0xFFFFFFFFu, wcnt[buf][lane][0]);
-    const uint32_t n2 = __reduce_add_sync(0xFFFFFFFFu, wcnt[buf][lane][1]);
-    const uint32_t n3 = __reduce_add_sync(0xFFFFFFFFu, wcnt[buf][lane][2]);
-    const uint64_t kk = static_cast<uint64_t>(k);
-    if (n3 >= kk) {
-      lo = t3;
-    } else if (n2 >= kk) {
-      lo = t2;
-      hi = t3;
-    } else if (n1 >= kk) {
-      lo = t1;
-      hi = t2;
+    // this thread's bins [tid*BPT, tid*BPT + BPT), read and cleared for the next round
+    uint32_t c[BPT];
+    if constexpr (BPT == 2) {
+      const uint2 v = reinterpret_cast<const uint2*>(hist)[tid];
+      c[0] = v.x;
+      c[1] = v.y;
+      reinterpret_cast<uint2*>(hist)[tid] = make_uint2(0u, 0u);
     } else {
-      hi = t1;
+      const uint4 v0 = reinterpret_cast<const uint4*>(hist)[2 * tid];
+      const uint4 v1 = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
+      c[0] = v0.x; c[1] = v0.y; c[2] = v0.z; c[3] = v0.w;
+      c[4] = v1.x; c[5] = v1.y; c[6] = v1.z; c[7] = v1.w;
+      reinterpret_cast<uint4*>(hist)[2 * tid] = make_uint4(0u, 0u, 0u, 0u);
+      reinterpret_cast<uint4*>(hist)[2 * tid + 1] = make_uint4(0u, 0u, 0u, 0u);
     }
-    buf ^= 1;
+    uint32_t local = 0u;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) local += c[i];
+    uint32_t incl = local;  // keys in the bins of lanes >= this lane (this warp)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_down_sync(0xFFFFFFFFu, incl, o);
+      if (lane + o < 32) incl += n;
+    }
+    if (lane == 0) wred[warp][0] = incl;
+    __syncthreads();
+    const uint32_t wt = lane < NW ? wred[lane][0] : 0u;
+    uint32_t wincl = wt;  // keys in the bins of warps >= lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_down_sync(0xFFFFFFFFu, wincl, o);
+      if (lane + o < 32) wincl += n;
+    }
+    const uint32_t after_warp = __shfl_sync(0xFFFFFFFFu, wincl - wt, warp);
+    // walk this thread's bins from the top: exactly one bin in the block has
+    // above + (keys in higher bins) < k <= above + (keys in it and higher bins)
+    uint32_t higher = above + after_warp + (incl - local);
+#pragma unroll
+    for (int i = BPT - 1; i >= 0; --i) {
+      const uint32_t ge = higher + c[i];
+      if (higher < k && ge >= k) {
+        sh_bin = static_cast<uint32_t>(tid * BPT + i);
+        sh_above = higher;
+        sh_done = ge == k ? 1u : 0u;
+      }
+      higher = ge;
+    }
+    __syncthreads();
+    const uint64_t nlo = lo + (static_cast<uint64_t>(sh_bin) << shift);
+    const uint64_t nhi = nlo + (1ull << shift);
+    hi = nhi < hi ? nhi : hi;
+    lo = nlo;
+    above = sh_above;
+    done = sh_done != 0u;
   }
-  const uint32_t T = static_cast<uint32_t>(lo);
-  // keys strictly above T (all kept), then `need` keys equal to T, lowest index first
-  uint32_t gt = 0u;
-#pragma unroll
-  for (int i = 0; i < KPT; ++i) gt += ((valid >> i) & 1u) && key[i] > T ? 1u : 0u;
-  gt = __reduce_add_sync(0xFFFFFFFFu, gt);
-  if (lane == 0) wcnt[buf][warp][0] = gt;
-  __syncthreads();
-  const uint32_t n_gt = __reduce_add_sync(0xFFFFFFFFu, wcnt[buf][lane][0]);
-  const uint32_t need = static_cast<uint32_t>(k) - n_gt;
 
-  uint32_t eq_seen = 0u, written = 0u;
+  // Selected: every key >= hi (`above` of them) and, lowest index first,
+  // need = k - above of the keys in [lo, hi).  When the search stopped with
+  // exactly k keys at or above lo, that is all of them; otherwise [lo, hi)
+  // is the single key T of the k-th largest score.
+  const uint32_t need = k - above;
+  const int C = ((d + 32 * NW - 1) / (32 * NW)) * 32;  // indices per warp
+  const int j0 = warp * C, j1 = min(d, j0 + C);
+  uint32_t ngt = 0u, neq = 0u;
+  for (int base = j0; base < j1; base += 32) {
+    const int j = base + lane;
+    const uint32_t key = j < j1 ? keys[j] : 0u;
+    ngt += __popc(__ballot_sync(0xFFFFFFFFu, j < j1 && key >= hi));
+    neq += __popc(__ballot_sync(0xFFFFFFFFu, j < j1 && key >= lo && key < hi));
+  }
+  if (lane == 0) {
+    wcnt[warp][0] = ngt;
+    wcnt[warp][1] = neq;
+  }
+  __syncthreads();
+  const uint32_t g = lane < NW ? wcnt[lane][0] : 0u, e = lane < NW ? wcnt[lane][1] : 0u;
+  uint32_t gi = g, ei = e;
 #pragma unroll
-  for (int i = 0; i < KPT; ++i) {
-    const int64_t j = tid + static_cast<int64_t>(i) * kTopkThreads;
-    if (static_cast<int64_t>(i) * kTopkThreads >= d) break;  // block-uniform
-    const bool in = (valid >> i) & 1u;
-    const bool eq = in && key[i] == T;
-    uint32_t eq_total;
-    const uint32_t eq_rank = eq_seen + block_flag_scan(eq, warp_cnt, &eq_total);
-    const bool sel = in && (key[i] > T || (eq && eq_rank < need));
-    uint32_t sel_total;
-    const uint32_t pos = written + block_flag_scan(sel, warp_cnt, &sel_total);
-    if (sel) out[pos] = static_cast<int32_t>(j);
-    eq_seen += eq_total;
-    written += sel_total;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t gn = __shfl_up_sync(0xFFFFFFFFu, gi, o);
+    const uint32_t en = __shfl_up_sync(0xFFFFFFFFu, ei, o);
+    if (lane >= o) {
+      gi += gn;
+      ei += en;
+    }
+  }
+  const uint32_t gt_before = __shfl_sync(0xFFFFFFFFu, gi - g, warp);
+  uint32_t eq_run = __shfl_sync(0xFFFFFFFFu, ei - e, warp);
+  uint32_t pos = gt_before + min(eq_run, need);
+  for (int base = j0; base < j1; base += 32) {
+    const int j = base + lane;
+    const uint32_t key = j < j1 ? keys[j] : 0u;
+    const bool gt = j < j1 && key >= hi;
+    const bool eq = j < j1 && key >= lo && key < hi;
+    const uint32_t eb = __ballot_sync(0xFFFFFFFFu, eq);
+    const bool sel = gt || (eq && eq_run + __popc(eb & lt_mask) < need);
+    const uint32_t sb = __ballot_sync(0xFFFFFFFFu, sel);
+    if (sel) out[pos + __popc(sb & lt_mask)] = j;
+    pos += __popc(sb);
+    eq_run += __popc(eb);
   }
 }
 
-constexpr int64_t kMaxStagedBytes = 200 * 1024;
+// Opt the histogram kernel into kMaxStagedKeys * 4 bytes of dynamic shared
+// memory, once per device.
+template <int NT>
+bool allow_staged_rows() {
+  static std::atomic<uint64_t> configured{0};  // bit per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const uint64_t bit = 1ull << dev;
+  if (configured.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(topk_hist_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kMaxStagedKeys * 4)) != cudaSuccess)
+    return false;
+  configured.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
 
 }  // namespace
 
 cudaError_t launch_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k, int32_t* idx,
                         int64_t ld_idx, cudaStream_t stream) {
-  const unsigned grid = static_cast<unsigned>(batch);
-  if (d <= 1 * kTopkThreads) {
-    return launch_pdl(topk_search_kernel<1>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
-                      ld_idx);
+  const dim3 grid(static_cast<unsigned>(batch));
+  if (d <= kMaxStagedKeys) {
+    const size_t bytes = static_cast<size_t>(d) * 4;
+    if (d <= 2048)  // 8 KB of keys: no opt-in needed
+      return launch_pdl(topk_hist_kernel<256>, grid, dim3(256), bytes, stream, scores, d, ld_s, k, idx, ld_idx);
+    if (bytes > 48 * 1024 && !allow_staged_rows<1024>()) return cudaErrorInvalidValue;
+    return launch_pdl(topk_hist_kernel<1024>, grid, dim3(1024), bytes, stream, scores, d, ld_s, k, idx, ld_idx);
   }
-  if (d <= 2 * kTopkThreads) {
-    return launch_pdl(topk_search_kernel<2>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
-                      ld_idx);
-  }
-  if (d <= 4 * kTopkThreads) {
-    return launch_pdl(topk_search_kernel<4>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
-                      ld_idx);
-  }
-  if (d <= 8 * kTopkThreads) {
-    return launch_pdl(topk_search_kernel<8>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
-                      ld_idx);
-  }
-  if (d <= 16 * kTopkThreads) {
-    return launch_pdl(topk_search_kernel<16>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx,
-                      ld_idx);
-  }
-  const int64_t bytes = d * 4;
-  if (bytes <= kMaxStagedBytes) {
-    if (bytes > 48 * 1024) {
-      const cudaError_t e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(kMaxStagedBytes));
-      if (e != cudaSuccess) return e;
-    }
-    return launch_pdl(topk_kernel<true>, dim3(grid), dim3(kTopkThreads), static_cast<size_t>(bytes), stream, scores,
-                      d, ld_s, k, idx, ld_idx);
-  }
-  return launch_pdl(topk_kernel<false>, dim3(grid), dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx, ld_idx);
+  return launch_pdl(topk_radix_kernel, grid, dim3(kTopkThreads), 0, stream, scores, d, ld_s, k, idx, ld_idx);
 }
 
 }  // namespace rmm

@@ -99,6 +99,13 @@ def _topk_cases():
     cases += [("top ties", s, 2)]
     s = (rng.random(2048).astype(np.float32) * 2 ** -126)  # subnormals
     cases += [("subnormal", s, 1024)]
+    cases += [("negative", (rng.standard_normal(3001) * 5).astype(np.float32), 1500)]
+    s = np.concatenate([np.float32([3e38, 1e-38]), rng.random(5000).astype(np.float32)])
+    cases += [("wide range", s, 2000)]
+    s = rng.random(51200).astype(np.float32)             # longest row staged in shared memory
+    cases += [("staged max", s, 25600)]
+    s = rng.random(51201).astype(np.float32)             # first row length re-read from global memory
+    cases += [("global radix", s, 17)]
     return cases
 
 
@@ -140,6 +147,20 @@ def test_compact_exact(dtype, M, d, k):
     it = torch.from_numpy(idx).cuda()
     AI = R.rmm_compact(At, it)
     np.testing.assert_array_equal(to_f64(AI), oracle.decode(A, dtype)[:, idx])
+    no_device_error()
+
+
+@pytest.mark.parametrize("M,d,lda,k", [(37, 60000, 60000, 30001),   # 120 KB rows: one staged row per block
+                                       (19, 4096, 4104, 2048),      # padded pitch; last block of 3 rows
+                                       (70, 1024, 1030, 700)])      # pitch not a multiple of 8: direct gather
+def test_compact_staged_and_pitched(M, d, lda, k):
+    rng = np.random.default_rng(M * 7 + d)
+    A = W.llm_activation_bf16(11, M, d)
+    buf = torch.zeros((M, lda), dtype=torch.bfloat16, device="cuda")
+    buf[:, :d] = bf16_tensor(A)
+    idx = np.sort(rng.choice(d, k, replace=False)).astype(np.int32)
+    AI = R.rmm_compact(buf[:, :d], torch.from_numpy(idx).cuda())
+    np.testing.assert_array_equal(to_f64(AI), oracle.decode(A, "bf16")[:, idx])
     no_device_error()
 
 
@@ -196,6 +217,7 @@ GEMM_SHAPES = [
     (17, 96, 264, 65),        # N just past a tile, k just past a block
     (512, 4096, 1024, 2048),  # several tiles and k blocks
     (1000, 3000, 2000, 1500),
+    (1024, 1024, 7424, 512),  # 116 tiles of 256 x 256: a last wave too full to split into halves
 ]
 
 
