@@ -17,11 +17,13 @@
 //   5. token top-k of t, causal prefix counts              (rmm_topk kernels, attn_prefix_kernel)
 //   6. K_T = K_I[I_t], V_T = V_g[I_t] row gathers           (gather_heads_kernel)
 //   7. pass C: O_i = sum_{r: pos_r <= i} exp(S_ir - lse_i) V_T[r]  (attn_out_kernel)
-// with S_ij = scale * Q_I[i] . K_I[j].  Passes A-C are tcgen05 kernels: one
-// TMA lane, one MMA lane, four softmax/epilogue warps; the 128 x 128 logit
-// tile lives in tensor memory (double-buffered); pass C writes P as bf16 in
-// the 128-byte-swizzled K-major layout into shared memory and accumulates
-// O += P V_T in tensor memory.  Exponentials use the hardware ex2.
+// with S_ij = scale * Q_I[i] . K_I[j].  Passes A-C are tcgen05 kernels with
+// a TMA warp, an MMA warp and two softmax groups of four warps that take
+// alternate 128 x 128 logit tiles from tensor memory.  Pass C writes P as
+// bf16 back into tensor memory over the logits it has read and accumulates
+// O += P V_T in tensor memory.  Exponentials use the hardware ex2; the
+// scale is folded into packed (f32x2) FMAs; only tiles on the causal
+// diagonal or past the sequence end are masked.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -41,7 +43,8 @@ namespace {
 
 constexpr int TILE = 128;                 // rows of every tile (queries or keys)
 constexpr int CHUNK_BYTES = TILE * 128;   // one [128 x 64] bf16 tile, 128-byte rows: 16 KB
-constexpr int ATT_THREADS = 192;          // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int ATT_THREADS = 320;          // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (two groups of four)
+constexpr int SOFTMAX_THREADS = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -52,7 +55,8 @@ struct AttnParams {
   int kt;           // kept tokens
   int nqb;          // query (= key) blocks of 128
   int out_f32;      // O written as fp32 (else bf16)
-  int c_stages;     // pass C key/value ring depth (1 or 2, as shared memory allows)
+  int c_ks;         // pass C key ring depth (2..4, as shared memory allows)
+  int c_vs;         // pass C value ring depth (1..4, as shared memory allows)
   float scale_log2; // logit scale times log2(e)
 };
 
@@ -126,19 +130,23 @@ struct QkBars {
   uint64_t drain;
   uint32_t tmem_slot;
   int abort_flag;
-  float lsh[4][TILE];  // per softmax warp: log2-domain lse of the current query block
+  float lsh[8][TILE];  // pass B, per softmax warp: -2 lse log2(e) of the current query block
+  float cmb[2][TILE];  // the second softmax group's per-row state, handed to the first
 };
 
 // Pass A (kLse): CTA = one query block; the Q tile is loaded once and key
-//   blocks 0..qb stream through the ring; thread r of the softmax warps owns
-//   query row r and keeps a running max / sum in the log2 domain.
+//   blocks 0..qb stream through the ring; a softmax thread owns query row r
+//   and keeps a running max / sum in the log2 domain.
 // Pass B (kColScore): CTA = one key block; the K tile is loaded once and query
 //   blocks kb..nqb-1 stream through; the tile in tensor memory is S^T (lane =
-//   key), so thread r owns key r and sums exp(2 (S_ij - lse_i)) over its
-//   queries with no cross-thread reduction: a 128-term block sum added into a
-//   running total, queries in ascending order.
+//   key), so a softmax thread owns key r and sums exp(2 (S_ij - lse_i)) over
+//   its queries with no cross-thread reduction.
+// Two softmax groups of four warps take alternate stream blocks (group g
+// the blocks g, g+2, ..., in tensor-memory buffer g); at the end group 1
+// hands its per-row state to group 0 through shared memory.  Only blocks on
+// the causal diagonal or past the sequence end are masked.
 template <int MODE>
-__global__ void __launch_bounds__(ATT_THREADS, 1)
+__global__ void __launch_bounds__(ATT_THREADS, 2)
     attn_qk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    float* __restrict__ lse, float* __restrict__ tsc, AttnParams p, unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -250,24 +258,27 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     __syncwarp();
   } else {
-    const int qtr = warp & 3;
+    const int g = (warp - 2) >> 2;                  // softmax group
+    const int qtr = warp & 3;                       // tensor-memory lane quarter of this warp
     const int r = qtr * 32 + lane;                  // TMEM lane = tile row
     const int own = fixed_blk * TILE + r;           // this thread's query (A) or key (B)
     const uint32_t lane_off = static_cast<uint32_t>(qtr * 32) << 16;
+    const float sl = p.scale_log2;
     float m = -INFINITY, l = 0.f;                   // pass A state (log2 domain)
     float total = 0.f;                              // pass B state
-    for (int it = 0; it < n_stream; ++it) {
+    float* nl = bars->lsh[warp - 2];
+    for (int it = g; it < n_stream; it += 2) {
       const uint32_t b = it & 1, sph = (it >> 1) & 1;
-      const int sblk = first_stream + it;
-      float* lsh = bars->lsh[qtr];
+      const int sbase = (first_stream + it) * TILE;
+      const bool masked = first_stream + it == fixed_blk || sbase + TILE > p.S;
       if (MODE == kColScore) {
         // each warp keeps its own copy of the block's 128 lse values, so only
         // warp-level synchronisation is needed
         __syncwarp();
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int q = sblk * TILE + u * 32 + lane;
-          lsh[u * 32 + lane] = q < p.S ? lse[static_cast<int64_t>(bh) * p.S + q] * kLog2e : 0.f;
+          const int q = sbase + u * 32 + lane;
+          nl[u * 32 + lane] = q < p.S ? -2.f * kLog2e * lse[static_cast<int64_t>(bh) * p.S + q] : 0.f;
         }
         __syncwarp();
       }
@@ -277,32 +288,64 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t v[32];
+        __syncwarp();  // the tensor-memory load is warp-synchronous: reconverge first
         tmem_ld32(tmem_base + b * TILE + cc * 32 + lane_off, v);
         tmem_wait_ld();
-        if (MODE == kLse) {
-          float x[32];
-          float mx = -INFINITY;
+        if (masked) {
+          // pass A keeps keys j <= own, pass B queries i >= own; both j, i < S
+          const int c0 = sbase + cc * 32;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int j = sblk * TILE + cc * 32 + e;
-            x[e] = (j <= own && j < p.S) ? __uint_as_float(v[e]) * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[e]);
+            const int j = c0 + e;
+            const bool keep = (MODE == kLse ? j <= own : j >= own) && j < p.S;
+            if (!keep) v[e] = __float_as_uint(-INFINITY);
           }
-          if (mx > -INFINITY) {
-            const float mn = fmaxf(m, mx);
-            float add = 0.f;
+        }
+        uint64_t acc0 = f2_pack(0.f, 0.f), acc1 = acc0;
+        if (MODE == kLse) {
+          const float mx = max_of32(v) * sl;
+          if (mx > -INFINITY) {  // else nothing is kept in this chunk (lane-divergent; ALU work only)
+            if (mx > m) {
+              l *= fast_exp2(m - mx);
+              m = mx;
+            }
+            const uint64_t slp = f2_pack(sl, sl), nm = f2_pack(-m, -m);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) add += fast_exp2(x[e] - mn);
-            l = l * fast_exp2(m - mn) + add;
-            m = mn;
+            for (int e = 0; e < 16; ++e) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), slp, nm), x0, x1);
+              const uint64_t ex = f2_pack(fast_exp2(x0), fast_exp2(x1));
+              if (e & 1) {
+                acc1 = f2_add(acc1, ex);
+              } else {
+                acc0 = f2_add(acc0, ex);
+              }
+            }
           }
         } else {
+          const uint64_t sl2 = f2_pack(2.f * sl, 2.f * sl);
+          const float2* nlc = reinterpret_cast<const float2*>(nl + cc * 32);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int i = sblk * TILE + cc * 32 + e;
-            const float pe = fast_exp2(2.f * (__uint_as_float(v[e]) * p.scale_log2 - lsh[cc * 32 + e]));
-            blk += (i >= own && i < p.S) ? pe : 0.f;
+          for (int e = 0; e < 16; ++e) {
+            const float2 q = nlc[e];
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sl2,
+                             f2_pack(q.x, q.y)),
+                      x0, x1);
+            const uint64_t ex = f2_pack(fast_exp2(x0), fast_exp2(x1));
+            if (e & 1) {
+              acc1 = f2_add(acc1, ex);
+            } else {
+              acc0 = f2_add(acc0, ex);
+            }
           }
+        }
+        float s0, s1;
+        f2_unpack(f2_add(acc0, acc1), s0, s1);
+        if (MODE == kLse) {
+          l += s0 + s1;
+        } else {
+          blk += s0 + s1;
         }
       }
       total += blk;
@@ -310,11 +353,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(sempty(b));
     }
-    if (own < p.S) {
+    // group 1 hands its state to group 0; every softmax warp reaches this
+    // barrier exactly once (also after an aborted wait)
+    if (g == 1) {
+      bars->cmb[0][r] = MODE == kLse ? m : total;
+      bars->cmb[1][r] = l;
+    }
+    named_barrier(1, SOFTMAX_THREADS);
+    if (g == 0 && own < p.S) {
       if (MODE == kLse) {
-        lse[static_cast<int64_t>(bh) * p.S + own] = (m + log2f(l)) * kLn2;
+        const float m1 = bars->cmb[0][r], l1 = bars->cmb[1][r];
+        const float mm = fmaxf(m, m1);
+        const float ll = (m > -INFINITY ? l * fast_exp2(m - mm) : 0.f) + (m1 > -INFINITY ? l1 * fast_exp2(m1 - mm) : 0.f);
+        lse[static_cast<int64_t>(bh) * p.S + own] = (mm + log2f(ll)) * kLn2;
       } else {
-        tsc[static_cast<int64_t>(bh) * p.S + own] = total;
+        tsc[static_cast<int64_t>(bh) * p.S + own] = total + bars->cmb[0][r];
       }
     }
   }
@@ -328,27 +381,45 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 
 // ------------------------------------------------------------------ pass C
 
-constexpr int C_STAGES = 2;  // maximum key/value ring depth of pass C
+constexpr int C_MAX_KS = 4;  // key ring depth of pass C (at most)
+constexpr int C_MAX_VS = 4;  // value ring depth (at most)
+constexpr int C_SBUF = 3;    // logit / P buffers in tensor memory
 
 struct OutBars {
-  uint64_t kvfull[C_STAGES], kvempty[C_STAGES];
+  uint64_t kfull[C_MAX_KS], kempty[C_MAX_KS];
+  uint64_t vfull[C_MAX_VS], vempty[C_MAX_VS];
   uint64_t qfull;
-  uint64_t sfull[2], sempty[2];
-  uint64_t pfull[2], pempty[2];
+  uint64_t sfull[C_SBUF], pfull[C_SBUF];
   uint64_t ofull;
   uint64_t drain;
   uint32_t tmem_slot;
   int abort_flag;
-  int pos[4][TILE];  // per softmax warp: token positions of the current kept block
+  int pos[8][TILE];  // per softmax warp: token positions of the current kept block
 };
+
+// Waits, with a bounded wall time, for the last min(issued, n) loads of a
+// ring of n stages to land (load t used stage t % n, phase (t / n) & 1).
+__device__ __forceinline__ void drain_ring(const uint64_t* full, int issued, int n) {
+  for (int t = issued - 1; t >= 0 && t >= issued - n; --t) wait_drain(smem_u32(&full[t % n]), (t / n) & 1);
+}
 
 // CTA = one query block.  Kept tokens are processed 128 at a time (only the
 // blocks that hold a kept position <= the block's last query): S = Q_I K_T^T
 // into tensor memory; the softmax warps turn row i into P_ir = exp(S_ir -
-// lse_i) for kept positions <= i (else 0), store it as bf16 in the
-// K-major 128-byte-swizzled layout, and the MMA lane accumulates O += P V_T
-// (V_T read MN-major).  S and P are double-buffered so the softmax of block r
-// overlaps the PV product of block r-1.
+// lse_i) for kept positions <= i (else 0) and write it as bf16 back into the
+// same tensor-memory buffer (two per column, over the logits already read);
+// the MMA lane accumulates O += P V_T with P read from tensor memory and V_T
+// (MN-major) from shared memory.
+//   Tensor memory (512 columns): three logit / P buffers of 128 columns and O.
+//   - kept block j uses buffer j % 3; the MMA lane issues PV(j) as soon as
+//     softmax(j) is done and then S(j+3) into the same buffer: tcgen05 MMAs
+//     of one thread run in issue order, so PV(j) has read P(j) before S(j+3)
+//     writes there, and each softmax group finds its next logits ready;
+//   - two softmax groups of four warps take alternate kept blocks;
+//   - one producer lane streams keys, another values, each into its own ring;
+//   - the MMA role runs on one lane (it has no warp-synchronous instruction).
+// Only kept blocks that reach past the first query of this block are masked;
+// the two groups split the output columns in the epilogue.
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attn_out_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kt,
                     const __grid_constant__ CUtensorMap tm_vt, const float* __restrict__ lse,
@@ -359,39 +430,44 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
   const uint32_t base = smem_u32(smem);
   const int dc = p.D / 64;
+  const int ks = p.c_ks, vs = p.c_vs;
   const int q_bytes = p.kc * CHUNK_BYTES;
-  const int kv_bytes = (p.kc + dc) * CHUNK_BYTES;
+  const int k_bytes = p.kc * CHUNK_BYTES;
+  const int v_bytes = dc * CHUNK_BYTES;
   const uint32_t q_tile = base;
-  auto kv = [&](uint32_t s) { return base + q_bytes + s * kv_bytes; };
-  const int nst = p.c_stages;
-  const uint32_t p_base = base + q_bytes + nst * kv_bytes;  // two P buffers of 2 chunks
-  auto pbuf = [&](uint32_t b) { return p_base + b * 2 * CHUNK_BYTES; };
-  OutBars* bars = reinterpret_cast<OutBars*>(smem + q_bytes + nst * kv_bytes + 4 * CHUNK_BYTES);
+  auto kst = [&](int s) { return base + q_bytes + s * k_bytes; };
+  auto vst = [&](int s) { return base + q_bytes + ks * k_bytes + s * v_bytes; };
+  OutBars* bars = reinterpret_cast<OutBars*>(smem + q_bytes + ks * k_bytes + vs * v_bytes);
   volatile int* abort_flag = &bars->abort_flag;
-  auto kvfull = [&](uint32_t s) { return smem_u32(&bars->kvfull[s]); };
-  auto kvempty = [&](uint32_t s) { return smem_u32(&bars->kvempty[s]); };
-  auto sfull = [&](uint32_t b) { return smem_u32(&bars->sfull[b]); };
-  auto sempty = [&](uint32_t b) { return smem_u32(&bars->sempty[b]); };
-  auto pfull = [&](uint32_t b) { return smem_u32(&bars->pfull[b]); };
-  auto pempty = [&](uint32_t b) { return smem_u32(&bars->pempty[b]); };
+  auto kfull = [&](int s) { return smem_u32(&bars->kfull[s]); };
+  auto kempty = [&](int s) { return smem_u32(&bars->kempty[s]); };
+  auto vfull = [&](int s) { return smem_u32(&bars->vfull[s]); };
+  auto vempty = [&](int s) { return smem_u32(&bars->vempty[s]); };
+  auto sfull = [&](int b) { return smem_u32(&bars->sfull[b]); };
+  auto pfull = [&](int b) { return smem_u32(&bars->pfull[b]); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int qb = p.nqb - 1 - static_cast<int>(blockIdx.x);  // heaviest blocks first
   const int nv = __ldg(nvalid + static_cast<int64_t>(bh) * p.nqb + qb);
   const int nrb = (nv + TILE - 1) / TILE;
+  // kept positions before this block's first query: kept blocks made only of
+  // those need no causal mask
+  const int nbefore = qb > 0 ? __ldg(nvalid + static_cast<int64_t>(bh) * p.nqb + qb - 1) : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < nst; ++s) {
-      mbar_init(kvfull(s), 1);
-      mbar_init(kvempty(s), 1);
+    for (int s = 0; s < ks; ++s) {
+      mbar_init(kfull(s), 1);
+      mbar_init(kempty(s), 1);
+    }
+    for (int s = 0; s < vs; ++s) {
+      mbar_init(vfull(s), 1);
+      mbar_init(vempty(s), 1);
     }
     mbar_init(smem_u32(&bars->qfull), 1);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(sfull(b), 1);
-      mbar_init(sempty(b), 4);
-      mbar_init(pfull(b), 4);
-      mbar_init(pempty(b), 1);
+    for (int b = 0; b < C_SBUF; ++b) {
+      mbar_init(sfull(b), 1);  // commit of S
+      mbar_init(pfull(b), 4);  // one arrival per warp of the softmax group
     }
     mbar_init(smem_u32(&bars->ofull), 1);
     mbar_init(smem_u32(&bars->drain), 1);
@@ -406,164 +482,168 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_slot;
-  const uint32_t o_tmem = tmem_base + 2 * TILE;
+  const uint32_t o_tmem = tmem_base + C_SBUF * TILE;
+  auto buf_tmem = [&](int b) { return tmem_base + b * TILE; };
 
   if (warp == 0) {
+    // lane 0: Q, then the key ring; lane 1: the value ring
     if (lane == 0 && nrb > 0) {
       mbar_arrive_expect_tx(smem_u32(&bars->qfull), q_bytes);
       for (int c = 0; c < p.kc; ++c)
         tma_load_3d(q_tile + c * CHUNK_BYTES, &tm_q, smem_u32(&bars->qfull), c * 64, qb * TILE, bh);
-      uint32_t stage = 0, phase = 0, issued = 0;
-      for (int rb = 0; rb < nrb; ++rb) {
-        if (!mbar_wait(kvempty(stage), phase ^ 1u, abort_flag, err, 21)) break;
-        mbar_arrive_expect_tx(kvfull(stage), kv_bytes);
-        for (int c = 0; c < p.kc; ++c)
-          tma_load_3d(kv(stage) + c * CHUNK_BYTES, &tm_kt, kvfull(stage), c * 64, rb * TILE, bh);
-        for (int c = 0; c < dc; ++c)
-          tma_load_3d(kv(stage) + (p.kc + c) * CHUNK_BYTES, &tm_vt, kvfull(stage), c * 64, rb * TILE, bh);
-        ++issued;
-        if (++stage == static_cast<uint32_t>(nst)) {
-          stage = 0;
-          phase ^= 1u;
-        }
+      int n = 0;
+      for (int t = 0; t < nrb; ++t) {
+        const int st = t % ks;
+        if (!mbar_wait(kempty(st), ((t / ks) & 1) ^ 1u, abort_flag, err, 21)) break;
+        mbar_arrive_expect_tx(kfull(st), k_bytes);
+        for (int c = 0; c < p.kc; ++c) tma_load_3d(kst(st) + c * CHUNK_BYTES, &tm_kt, kfull(st), c * 64, t * TILE, bh);
+        ++n;
       }
       wait_drain(smem_u32(&bars->qfull), 0);
-      uint32_t st = stage, ph = phase;
-      for (uint32_t j = 0; j < (issued < static_cast<uint32_t>(nst) ? issued : static_cast<uint32_t>(nst)); ++j) {
-        if (st == 0) {
-          st = nst - 1;
-          ph ^= 1u;
-        } else {
-          --st;
-        }
-        wait_drain(kvfull(st), ph);
+      drain_ring(bars->kfull, n, ks);
+    } else if (lane == 1 && nrb > 0) {
+      int n = 0;
+      for (int t = 0; t < nrb; ++t) {
+        const int st = t % vs;
+        if (!mbar_wait(vempty(st), ((t / vs) & 1) ^ 1u, abort_flag, err, 29)) break;
+        mbar_arrive_expect_tx(vfull(st), v_bytes);
+        for (int c = 0; c < dc; ++c) tma_load_3d(vst(st) + c * CHUNK_BYTES, &tm_vt, vfull(st), c * 64, t * TILE, bh);
+        ++n;
       }
+      drain_ring(bars->vfull, n, vs);
     }
     __syncwarp();
   } else if (warp == 1) {
-    constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, false, false);
-    const uint32_t idesc_o = idesc_bf16_f32(TILE, p.D, false, true);
-    bool ok = nrb == 0 || mbar_wait_warp(smem_u32(&bars->qfull), 0, abort_flag, err, 22);
-    // O += P(r) V_T(r)
-    auto pv = [&](int r) -> bool {
-      const uint32_t b = r & 1, pph = (r >> 1) & 1;
-      const uint32_t st = r % nst;
-      if (!mbar_wait_warp(pfull(b), pph, abort_flag, err, 23)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-#pragma unroll
-        for (int kk = 0; kk < TILE / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(pbuf(b) + (kk / 4) * CHUNK_BYTES + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kv(st) + p.kc * CHUNK_BYTES + kk * 16 * 128, CHUNK_BYTES, 1024);
-          mma_f16_ss(o_tmem, ad, bd, idesc_o, (r | kk) != 0 ? 1u : 0u);
-        }
-        mma_commit(kvempty(st));
-        mma_commit(pempty(b));
-      }
-      __syncwarp();
-      return true;
-    };
-    for (int rb = 0; ok && rb < nrb; ++rb) {
-      const uint32_t b = rb & 1, sph = (rb >> 1) & 1;
-      const uint32_t st = rb % nst, kph = (rb / nst) & 1;
-      // with a single key/value stage, block rb can only be loaded once the
-      // PV product of rb-1 has released the stage: issue that product first
-      if (nst == 1 && rb >= 1 && !pv(rb - 1)) {
-        ok = false;
-        break;
-      }
-      if (!mbar_wait_warp(kvfull(st), kph, abort_flag, err, 24)) {
-        ok = false;
-        break;
-      }
-      if (!mbar_wait_warp(sempty(b), sph ^ 1u, abort_flag, err, 25)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (lane == 0) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, false, false);
+      const uint32_t idesc_o = idesc_bf16_f32(TILE, p.D, false, true);
+      bool ok = nrb == 0 || mbar_wait(smem_u32(&bars->qfull), 0, abort_flag, err, 22);
+      // S(t) = Q_I K_T(t)^T into buffer t % 3
+      auto issue_s = [&](int t) -> bool {
+        const int st = t % ks;
+        if (!mbar_wait(kfull(st), (t / ks) & 1, abort_flag, err, 24)) return false;
+        tc_fence_after();
         for (int c = 0; c < p.kc; ++c) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = sdesc_sw128(q_tile + c * CHUNK_BYTES + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(kv(st) + c * CHUNK_BYTES + kk * 32, 16, 1024);
-            mma_f16_ss(tmem_base + b * TILE, ad, bd, idesc_s, (c | kk) != 0 ? 1u : 0u);
+            const uint64_t bd = sdesc_sw128(kst(st) + c * CHUNK_BYTES + kk * 32, 16, 1024);
+            mma_f16_ss(buf_tmem(t % C_SBUF), ad, bd, idesc_s, (c | kk) != 0 ? 1u : 0u);
           }
         }
-        mma_commit(sfull(b));
+        mma_commit(kempty(st));
+        mma_commit(sfull(t % C_SBUF));
+        return true;
+      };
+      // O += P(t) V_T(t), P from the first 64 columns of buffer t % 3
+      auto issue_pv = [&](int t) -> bool {
+        const int st = t % vs;
+        if (!mbar_wait(vfull(st), (t / vs) & 1, abort_flag, err, 30)) return false;
+        tc_fence_after();
+        const uint32_t pt = buf_tmem(t % C_SBUF);
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) {
+          const uint64_t bd = sdesc_sw128(vst(st) + kk * 16 * 128, CHUNK_BYTES, 1024);
+          mma_f16_ts(o_tmem, pt + kk * 8, bd, idesc_o, (t | kk) != 0 ? 1u : 0u);
+        }
+        mma_commit(vempty(st));
+        return true;
+      };
+      for (int t = 0; ok && t < C_SBUF && t < nrb; ++t) ok = issue_s(t);
+      for (int j = 0; ok && j < nrb; ++j) {
+        ok = mbar_wait(pfull(j % C_SBUF), (j / C_SBUF) & 1, abort_flag, err, 23);
+        if (ok) tc_fence_after();
+        ok = ok && issue_pv(j);
+        if (ok && j + C_SBUF < nrb) ok = issue_s(j + C_SBUF);
       }
-      __syncwarp();
-      if (nst > 1 && rb >= 1 && !pv(rb - 1)) ok = false;
-    }
-    if (ok && nrb > 0) ok = pv(nrb - 1);
-    if (lane == 0) {
-      if (nrb > 0) mma_commit(smem_u32(&bars->ofull));
+      if (ok && nrb > 0) mma_commit(smem_u32(&bars->ofull));
       mma_commit(smem_u32(&bars->drain));
       wait_drain(smem_u32(&bars->drain), 0);
     }
     __syncwarp();
   } else {
-    const int qtr = warp & 3;
+    const int g = (warp - 2) >> 2;  // softmax group
+    const int qtr = warp & 3;       // tensor-memory lane quarter of this warp
     const int r = qtr * 32 + lane;
     const int i = qb * TILE + r;
     const uint32_t lane_off = static_cast<uint32_t>(qtr * 32) << 16;
     const float L2 = i < p.S ? lse[static_cast<int64_t>(bh) * p.S + i] * kLog2e : 0.f;
     const int32_t* pos_bh = pos + static_cast<int64_t>(bh) * p.kt;
+    const uint64_t slp = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(-L2, -L2);
+    int* psh = bars->pos[warp - 2];
     bool ok = true;
-    for (int rb = 0; rb < nrb; ++rb) {
-      const uint32_t b = rb & 1, sph = (rb >> 1) & 1;
-      int* psh = bars->pos[qtr];
-      __syncwarp();
+    for (int rb = g; ok && rb < nrb; rb += 2) {
+      const int b = rb % C_SBUF;
+      const uint32_t sph = (rb / C_SBUF) & 1;
+      const bool masked = rb * TILE + TILE > nbefore;
+      if (masked) {
+        __syncwarp();
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int kr = rb * TILE + u * 32 + lane;
-        psh[u * 32 + lane] = kr < p.kt ? __ldg(pos_bh + kr) : 0x7FFFFFFF;
+        for (int u = 0; u < 4; ++u) {
+          const int kr = rb * TILE + u * 32 + lane;
+          psh[u * 32 + lane] = kr < p.kt ? __ldg(pos_bh + kr) : 0x7FFFFFFF;
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      if (!mbar_wait_warp(sfull(b), sph, abort_flag, err, 26) ||
-          !mbar_wait_warp(pempty(b), sph ^ 1u, abort_flag, err, 27)) {
+      if (!mbar_wait_warp(sfull(b), sph, abort_flag, err, 26)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint8_t* prow = smem + (pbuf(b) - base) + r * 128;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tmem_base + b * TILE + cc * 32 + lane_off, v);
-        tmem_wait_ld();
-        uint32_t w[16];
+      // P goes over the logits of the same buffer: chunk cc's P (16 columns
+      // from 16 cc) only covers logits already read
+      const uint32_t s_addr = buf_tmem(b) + lane_off;
+      const uint32_t p_addr = s_addr;
+      // P for the 32 kept columns of chunk cc from the scores in v, packed two
+      // per tensor-memory column
+      auto exps = [&](int cc, const uint32_t (&v)[32], uint32_t (&w)[16]) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int q0 = cc * 32 + 2 * e;
-          const float p0 = psh[q0] <= i ? fast_exp2(__uint_as_float(v[2 * e]) * p.scale_log2 - L2) : 0.f;
-          const float p1 = psh[q0 + 1] <= i ? fast_exp2(__uint_as_float(v[2 * e + 1]) * p.scale_log2 - L2) : 0.f;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), slp, nl2), x0, x1);
+          float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          if (masked) {
+            if (psh[cc * 32 + 2 * e] > i) p0 = 0.f;
+            if (psh[cc * 32 + 2 * e + 1] > i) p1 = 0.f;
+          }
           w[e] = pack_bf16x2(p0, p1);
         }
-        // columns cc*32 .. cc*32+31: chunk cc/2, 16-byte pieces (cc%2)*4 .. +3, swizzled by row
-        uint8_t* crow = prow + (cc >> 1) * CHUNK_BYTES;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int piece = (cc & 1) * 4 + q;
-          *reinterpret_cast<uint4*>(crow + ((piece ^ (r & 7)) << 4)) =
-              make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        }
-      }
-      tc_fence_before();
-      fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+      };
+      uint32_t va[32], vb[32], w[16];
+      __syncwarp();  // tensor-memory accesses are warp-synchronous: reconverge first
+      tmem_ld32(s_addr, va);
+      tmem_wait_ld_into(va);
+      tmem_ld32(s_addr + 32, vb);
+      exps(0, va, w);
+      tmem_st16(p_addr, w);
+      tmem_wait_ld_into(vb);
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(sempty(b));
-        mbar_arrive(pfull(b));
-      }
+      tmem_ld32(s_addr + 64, va);
+      exps(1, vb, w);
+      tmem_st16(p_addr + 16, w);
+      tmem_wait_ld_into(va);
+      __syncwarp();
+      tmem_ld32(s_addr + 96, vb);
+      exps(2, va, w);
+      tmem_st16(p_addr + 32, w);
+      tmem_wait_ld_into(vb);
+      exps(3, vb, w);
+      tmem_st16(p_addr + 48, w);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull(b));
     }
-    // epilogue: O row i.  Every lane of the warp takes part in the tensor-memory
-    // loads (warp-synchronous); only rows i < S are stored.
+    // epilogue: O row i, columns [g D/2, (g+1) D/2).  Every lane of the warp
+    // takes part in the tensor-memory loads (warp-synchronous); only rows
+    // i < S are stored.
     const bool have = ok && nrb > 0 && mbar_wait_warp(smem_u32(&bars->ofull), 0, abort_flag, err, 28);
     if (have) tc_fence_after();
-    for (int cc = 0; cc < p.D / 32; ++cc) {
+    const int ncc = p.D / 64;  // 32-column chunks per group
+    for (int cc = g * ncc; cc < (g + 1) * ncc; ++cc) {
       uint32_t v[32];
       if (have) {
+        __syncwarp();
         tmem_ld32(o_tmem + cc * 32 + lane_off, v);
         tmem_wait_ld();
       } else {
@@ -806,16 +886,26 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
     if (e != cudaSuccess || (e = debug_step(stream, "row gathers")) != cudaSuccess) return e;
   }
   // 7. pass C
-  auto out_smem_for = [&](int stages) {
-    return kc * CHUNK_BYTES + stages * (kc + static_cast<int>(D / 64)) * CHUNK_BYTES + 4 * CHUNK_BYTES +
+  auto out_smem_for = [&](int ks, int vs) {
+    return kc * CHUNK_BYTES + ks * kc * CHUNK_BYTES + vs * static_cast<int>(D / 64) * CHUNK_BYTES +
            static_cast<int>(sizeof(OutBars)) + 1024;
   };
   int dev = 0, max_smem = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
-  prm.c_stages = out_smem_for(C_STAGES) <= max_smem ? C_STAGES : 1;
-  const int out_smem = out_smem_for(prm.c_stages);
+  // deepest key and value rings that fit (the value ring grows first)
+  prm.c_ks = 2;
+  prm.c_vs = 1;
+  for (int d = C_MAX_VS; d >= 1; --d) {
+    const int kd_ring = std::min(d, C_MAX_KS) < 2 ? 2 : std::min(d, C_MAX_KS);
+    if (out_smem_for(kd_ring, d) <= max_smem) {
+      prm.c_ks = kd_ring;
+      prm.c_vs = d;
+      break;
+    }
+  }
+  const int out_smem = out_smem_for(prm.c_ks, prm.c_vs);
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!set_smem(attn_out_kernel, out_smem)) {
@@ -829,3 +919,4 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
 }
 
 }  // namespace rmm
+
