@@ -301,6 +301,65 @@ def measure_attention(R, workloads, bf16_tensor, dev, stream, flush, steps, time
             "gpu_launches_per_call": 12, "calls": steps}
 
 
+def measure_decode(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, Wt, hbm_gbs):
+    """Decode-sized products (M = 1 and 16 activation rows) on the MLP up/gate
+    weight through rmm_matmul (one selection launch: scores, top-k and A_I;
+    then the row-streaming product that reads only the kept rows of W), next
+    to cuBLAS on the full W (same flush protocol).  The product is also timed
+    alone; its bandwidth counts its algorithmic bytes: the k kept rows of W,
+    A_I and Y."""
+    import torch
+    out = {}
+    for rows in (1, 16):
+        X = bf16_tensor(workloads.llm_activation_bf16(7 + rows, rows, D), dev)
+        k = R.rmm_k_from_rho(RHO, D)
+        ss = torch.empty(D, dtype=torch.float32, device=dev)
+        idx = torch.empty(k, dtype=torch.int32, device=dev)
+        AI = torch.empty((rows, (k + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)[:, :k]
+        Y = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+        Yd = torch.empty_like(Y)
+        sws = torch.empty(max(256, R.rmm_score_workspace_size(R.RMM_BF16, 1, rows, D)), dtype=torch.uint8, device=dev)
+        gws = torch.empty(R.rmm_gemm_workspace_size(R.RMM_BF16, N, k), dtype=torch.uint8, device=dev)
+
+        mws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, rows, D, N, RHO), dtype=torch.uint8, device=dev)
+
+        def rmm(ev):
+            # the whole path as a user calls it: one selection launch, then the product
+            ev[0].record(stream)
+            R.rmm_matmul(X, Wt, RHO, out=Y, idx_out=idx, ws=mws)
+            ev[1].record(stream)
+
+        def product(ev):
+            ev[0].record(stream)
+            R.rmm_gemm(AI, Wt, idx, out=Y, ws=gws)
+            ev[1].record(stream)
+
+        def dense(ev):
+            ev[0].record(stream)
+            torch.matmul(X, Wt, out=Yd)
+            ev[1].record(stream)
+
+        for _ in range(3):
+            rmm([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+            dense([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        R.rmm_compact(X, idx, out=AI)
+        for _ in range(3):
+            product([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        step_ms = statistics.mean(p[0] for p in timed(rmm, steps, 2))
+        prod_ms = statistics.mean(p[0] for p in timed(product, steps, 2))
+        dense_ms = statistics.mean(p[0] for p in timed(dense, steps, 2))
+        prod_bytes = 2.0 * k * N + 2.0 * rows * k + 2.0 * rows * N
+        gbs = prod_bytes / (prod_ms * 1e-3) / 1e9
+        out[f"M{rows}"] = {"step_us": step_ms * 1e3, "product_us": prod_ms * 1e3, "product_GB/s": gbs,
+                           "product_frac_hbm": gbs / hbm_gbs, "dense_us": dense_ms * 1e3,
+                           "speedup_vs_dense": dense_ms / step_ms}
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the decode runs")
+    out["workload"] = (f"decode rows x[1 or 16 x {D}] (lognormal channel scale, outliers) . W[{D}x{N}], rho={RHO}; "
+                       "W streamed from HBM (256 MiB flush between steps)")
+    return out
+
+
 def run_rmm(args):
     import numpy as np
     import torch
@@ -436,6 +495,8 @@ def run_rmm(args):
     attention = measure_attention(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 20), timed)
 
     peaks, peak_src = load_peaks()
+    decode = measure_decode(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed, Wt,
+                            peaks["hbm_gbs"])
     gemm_ms = stage_ms["gemm"]
     achieved = flops_step / (gemm_ms * 1e-3) / 1e12
     traffic = traffic_per_launch()
@@ -479,6 +540,7 @@ def run_rmm(args):
                     "d2h_bytes_per_step": int(Y.numel() * 2), "api": "rmm_matmul"},
             "gpu_launches": launches_per_step * args.steps,
             "attention": attention,
+            "decode": decode,
             "clocks": clk.summary(), "clock_remeasured": remeasured,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -124,7 +124,8 @@ RMM_API rmm_status rmm_score_noalloc(const void* A, int dtype, int64_t batch, in
  * order; equal scores are taken lowest index first (Metodología › Estrategia
  * de Selección keeps the top-k; the tie rule and the order are this library's
  * reading).  Scores must be finite; -0.0 ranks equal to +0.0.  The selection
- * is an exact radix select on the fp32 bit patterns, so the index set is the
+ * is exact on the fp32 bit patterns (a histogram search over the key range,
+ * or a radix select for rows longer than 51200), so the index set is the
  * unique one defined by that rule.  1 <= k <= d, ld_idx >= k, ld_s >= d.  */
 RMM_API rmm_status rmm_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k,
                     int32_t* idx, int64_t ld_idx, void* stream);
@@ -163,11 +164,15 @@ RMM_API rmm_status rmm_compact_gather(const void* A, int64_t lda, const void* B,
  * compacted [M x k] activation (ld_ai), B the full [d x N] row-major operand
  * (ldb >= N) whose rows idx[0..k) are the kept contraction indices, and Y is
  * [M x N] (ldy >= N) written as out_dtype (RMM_BF16 or RMM_F32).
- *  - dtype RMM_BF16: B's kept rows are first copied into workspace (a
- *    streaming row gather), then a persistent tcgen05 tensor-core kernel
- *    computes the product with fp32 accumulation in tensor memory.  Requires
- *    16-byte aligned A_I, B, Y, and ld_ai, ldb multiples of 8
- *    (RMM_ERR_UNSUPPORTED otherwise).  B must be finite.
+ *  - dtype RMM_BF16, M > 16: B's kept rows are first copied into workspace
+ *    (a streaming row gather), then a persistent tcgen05 tensor-core kernel
+ *    computes the product with fp32 accumulation in tensor memory.
+ *  - dtype RMM_BF16, M <= 16 (decode): the kept rows of B are read in place,
+ *    once each, by a row-streaming kernel with fp32 accumulation; the
+ *    workspace holds fp32 partial sums over ranges of kept rows, added in a
+ *    fixed order.
+ *    Both bf16 forms require 16-byte aligned A_I, B, Y, and ld_ai, ldb
+ *    multiples of 8 (RMM_ERR_UNSUPPORTED otherwise).  B must be finite.
  *  - dtype RMM_F32: fp32 FMA kernel (A_I, B fp32; Y fp32 only); no workspace.
  * Workspace: rmm_gemm_workspace_size(dtype, N, k) bytes, 256-byte aligned.
  * Out-of-range indices contribute zero and are flagged.  k >= 1. */

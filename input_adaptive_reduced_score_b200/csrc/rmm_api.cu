@@ -291,6 +291,15 @@ rmm_status rmm_gemm(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, 
     return fail(RMM_ERR_WORKSPACE, "rmm_gemm: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes, need);
   unsigned* err = device_error_word();
   if (!err) return RMM_ERR_CUDA;
+  if (M <= kGemvMaxM) {
+    // a few rows: the kept rows of B are read in place (no gathered copy)
+    const GemvPlan pl = gemv_plan(M, N, k, device_sm_count());
+    if (pl.partial_bytes > ws_bytes)
+      return fail(RMM_ERR_WORKSPACE, "rmm_gemm: workspace %zu < %zu bytes", ws_bytes, pl.partial_bytes);
+    const cudaError_t e = launch_gemv(A_I, ld_ai, B, ldb, idx, M, d, N, k, pl, static_cast<float*>(ws), Y, out_dtype,
+                                      ldy, err, s);
+    return from_cuda(e, "rmm_gemm(bf16, few rows): launch");
+  }
   const int64_t ld_bi = round_up(N, 8);
   cudaError_t e = launch_gather_rows(B, d, N * 2, ldb * 2, idx, k, ws, ld_bi * 2, err, s);
   if (e != cudaSuccess) return from_cuda(e, "rmm_gemm: row gather launch");
@@ -344,11 +353,19 @@ rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t ldb, in
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
   void* score_ws = base + w.score;
   void* ai = base + w.ai;
+  if (dtype == RMM_BF16 && M > 0 && N > 0 && select_rows_supported(M, d) && aligned16(B) && ldb % 8 == 0) {
+    // a few rows (decode): scores, selection and A_I in one launch, then the
+    // product that reads only the kept rows of B
+    const cudaError_t e = launch_select_rows(A, M, d, lda, k, idx, ss, ai, w.ld_ai, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return from_cuda(e, "rmm_matmul: row selection launch");
+    return rmm_gemm(ai, w.ld_ai, B, ldb, idx, d, M, N, k, dtype, Y, out_dtype, ldy, base + w.bi, w.total - w.bi,
+                    stream);
+  }
   rmm_status st = rmm_score(A, dtype, 1, M, d, lda, 0, ss, d, 0, score_ws, score_workspace_bytes(dtype, 1, M, d), stream);
   if (st != RMM_OK) return st;
   st = rmm_topk(ss, 1, d, d, k, idx, k, stream);
   if (st != RMM_OK) return st;
-  if (dtype == RMM_BF16 && M > 0 && N > 0 && aligned16(B) && ldb % 8 == 0) {
+  if (dtype == RMM_BF16 && M > kGemvMaxM && N > 0 && aligned16(B) && ldb % 8 == 0) {
     // both reduced operands in one launch, then the dense product on them
     const int64_t ld_bi = round_up(N, 8);
     void* bi = base + w.bi;

@@ -42,6 +42,12 @@ cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int
 cudaError_t launch_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k,
                         int32_t* idx, int64_t ld_idx, cudaStream_t stream);
 
+// A few bf16 activation rows: scores, top-k and A_I = A[:, idx] in one launch
+// (M <= 16, d <= 51200; A_I gets ld_ai >= k).  ss may be null.
+bool select_rows_supported(int64_t M, int64_t d);
+cudaError_t launch_select_rows(const void* A, int64_t M, int64_t d, int64_t lda, int64_t k, int32_t* idx, float* ss,
+                               void* A_I, int64_t ld_ai, cudaStream_t stream);
+
 // ---- compaction (rmm_compact.cu)
 cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64_t lda,
                            const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai, unsigned* err,
@@ -68,6 +74,21 @@ cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I,
 cudaError_t launch_gemm_f32_simt(const float* A_I, int64_t ld_ai, const float* B, int64_t ldb,
                                  const int32_t* idx, int64_t d, int64_t M, int64_t N, int64_t k,
                                  float* Y, int64_t ldy, unsigned* err, cudaStream_t stream);
+
+// ---- reduced product for M <= 16 rows (rmm_gemv.cu): kept rows of B read in place
+constexpr int64_t kGemvMaxM = 16;
+struct GemvPlan {
+  int64_t slices;        // column slices of 128
+  int splits;            // kept-row ranges
+  int rows_per_split;
+  bool clustered;        // the splits of a column slice form one cluster (no partials in memory)
+  size_t partial_bytes;  // fp32 partial sums in global memory (0 with one split or a cluster)
+};
+GemvPlan gemv_plan(int64_t M, int64_t N, int64_t k, int sms);
+// A_I bf16 [M x k] (ld_ai), B bf16 [d x N] (ldb, rows 8-byte aligned), idx [k].
+cudaError_t launch_gemv(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, const int32_t* idx, int64_t M,
+                        int64_t d, int64_t N, int64_t k, const GemvPlan& plan, float* partial, void* Y, int out_dtype,
+                        int64_t ldy, unsigned* err, cudaStream_t stream);
 
 // ---- reduced attention (rmm_attention.cu)
 size_t attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D, int64_t kd,

@@ -141,72 +141,21 @@ constexpr int64_t kMaxStagedKeys = 51200;  // 200 KB of keys + 8 KB of bins per 
 
 // Histogram search on keys staged in shared memory (rows of up to
 // kMaxStagedKeys scores).  Invariant of the search: count(key >= hi) =
-// `above` < k <= count(key >= lo).
+// `above` < k <= count(key >= lo).  The caller has written keys[0..d) and
+// passes each thread's minimum and maximum key; every thread of the block
+// calls this once.  Writes the k selected indices, ascending, to out.
 template <int NT>
-__global__ void __launch_bounds__(NT, 1) topk_hist_kernel(const float* __restrict__ scores, int64_t d64, int64_t ld_s,
-                                                           int64_t k64, int32_t* __restrict__ idx, int64_t ld_idx) {
+__device__ __forceinline__ void select_staged(const uint32_t* keys, int d, uint32_t k, uint32_t kmin, uint32_t kmax,
+                                              int32_t* __restrict__ out) {
   constexpr int NW = NT / 32;
   constexpr int BPT = kBins / NT;  // bins per thread, contiguous
   static_assert(BPT == 2 || BPT == 8, "bin vectors are 2 or 8 words");
-  extern __shared__ __align__(16) uint32_t keys[];
   __shared__ __align__(16) uint32_t hist[kBins];
   __shared__ uint32_t wred[NW][2];  // per-warp min/max, then per-warp bin totals
   __shared__ uint32_t wcnt[NW][2];  // per-warp (above, in-range) counts for the emission
   __shared__ uint32_t sh_bin, sh_above, sh_done;
-  const int d = static_cast<int>(d64);
-  const uint32_t k = static_cast<uint32_t>(k64);
-  const float* s = scores + static_cast<int64_t>(blockIdx.x) * ld_s;
-  int32_t* out = idx + static_cast<int64_t>(blockIdx.x) * ld_idx;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  const bool vec4 = (reinterpret_cast<uintptr_t>(s) & 15u) == 0 && (d & 3) == 0;
-  pdl_wait();
-  pdl_trigger();
-
-  // stage the keys, zero the bins, find the key range; the loads of a batch
-  // are all issued before the first is used (one memory round trip per batch)
-  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-  if (vec4) {
-    const int nv = d >> 2;
-    const float4* s4 = reinterpret_cast<const float4*>(s);
-    for (int v0 = tid; v0 < nv; v0 += 4 * NT) {
-      float4 f[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int v = v0 + u * NT;
-        f[u] = v < nv ? __ldg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int v = v0 + u * NT;
-        if (v < nv) {
-          const uint4 q = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
-          reinterpret_cast<uint4*>(keys)[v] = q;
-          kmin = min(kmin, min(min(q.x, q.y), min(q.z, q.w)));
-          kmax = max(kmax, max(max(q.x, q.y), max(q.z, q.w)));
-        }
-      }
-    }
-  } else {
-    for (int j0 = tid; j0 < d; j0 += 8 * NT) {
-      float f[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + u * NT;
-        f[u] = j < d ? __ldg(s + j) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + u * NT;
-        if (j < d) {
-          const uint32_t key = score_key(f[u]);
-          keys[j] = key;
-          kmin = min(kmin, key);
-          kmax = max(kmax, key);
-        }
-      }
-    }
-  }
   for (int b = tid; b < kBins; b += NT) hist[b] = 0u;
   kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
   kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
@@ -334,6 +283,140 @@ __global__ void __launch_bounds__(NT, 1) topk_hist_kernel(const float* __restric
   }
 }
 
+// One score row per CTA: stage its keys, then select_staged.
+template <int NT>
+__global__ void __launch_bounds__(NT, 1) topk_hist_kernel(const float* __restrict__ scores, int64_t d64, int64_t ld_s,
+                                                           int64_t k64, int32_t* __restrict__ idx, int64_t ld_idx) {
+  extern __shared__ __align__(16) uint32_t keys[];
+  const int d = static_cast<int>(d64);
+  const uint32_t k = static_cast<uint32_t>(k64);
+  const float* s = scores + static_cast<int64_t>(blockIdx.x) * ld_s;
+  int32_t* out = idx + static_cast<int64_t>(blockIdx.x) * ld_idx;
+  const int tid = threadIdx.x;
+  const bool vec4 = (reinterpret_cast<uintptr_t>(s) & 15u) == 0 && (d & 3) == 0;
+  pdl_wait();
+  pdl_trigger();
+
+  // stage the keys, zero the bins, find the key range; the loads of a batch
+  // are all issued before the first is used (one memory round trip per batch)
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  if (vec4) {
+    const int nv = d >> 2;
+    const float4* s4 = reinterpret_cast<const float4*>(s);
+    for (int v0 = tid; v0 < nv; v0 += 4 * NT) {
+      float4 f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * NT;
+        f[u] = v < nv ? __ldg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * NT;
+        if (v < nv) {
+          const uint4 q = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
+          reinterpret_cast<uint4*>(keys)[v] = q;
+          kmin = min(kmin, min(min(q.x, q.y), min(q.z, q.w)));
+          kmax = max(kmax, max(max(q.x, q.y), max(q.z, q.w)));
+        }
+      }
+    }
+  } else {
+    for (int j0 = tid; j0 < d; j0 += 8 * NT) {
+      float f[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * NT;
+        f[u] = j < d ? __ldg(s + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int j = j0 + u * NT;
+        if (j < d) {
+          const uint32_t key = score_key(f[u]);
+          keys[j] = key;
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
+      }
+    }
+  }
+  select_staged<NT>(keys, d, k, kmin, kmax, out);
+}
+
+// A few activation rows (decode): column scores of A [M x d], the top-k
+// selection and the compaction A_I = A[:, I] in one CTA of 1024 threads.
+// Scores are fp32 sums of the rows' exact squares in row order.  Optional
+// ss output.  keys in dynamic shared memory (d words, d <= kMaxStagedKeys).
+__global__ void __launch_bounds__(1024, 1)
+    select_rows_kernel(const uint16_t* __restrict__ A, int M, int64_t d64, int64_t lda, int64_t k64,
+                       int32_t* __restrict__ idx, float* __restrict__ ss, uint16_t* __restrict__ AI, int64_t ld_ai) {
+  extern __shared__ __align__(16) uint32_t keys[];
+  const int d = static_cast<int>(d64);
+  const int tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  const bool vec = (reinterpret_cast<uintptr_t>(A) & 15u) == 0 && (lda & 7) == 0 && (d & 7) == 0;
+  if (vec) {
+    for (int v = tid; v < d / 8; v += 1024) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int m = 0; m < M; ++m) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(A + static_cast<int64_t>(m) * lda) + v);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float lo = __uint_as_float(w[t] << 16), hi = __uint_as_float(w[t] & 0xFFFF0000u);
+          acc[2 * t] = fmaf(lo, lo, acc[2 * t]);
+          acc[2 * t + 1] = fmaf(hi, hi, acc[2 * t + 1]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t key = score_key(acc[e]);
+        keys[8 * v + e] = key;
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+        if (ss) ss[8 * v + e] = acc[e];
+      }
+    }
+  } else {
+    for (int j = tid; j < d; j += 1024) {
+      float acc = 0.f;
+      for (int m = 0; m < M; ++m) {
+        const float x = __uint_as_float(static_cast<uint32_t>(A[static_cast<int64_t>(m) * lda + j]) << 16);
+        acc = fmaf(x, x, acc);
+      }
+      const uint32_t key = score_key(acc);
+      keys[j] = key;
+      kmin = min(kmin, key);
+      kmax = max(kmax, key);
+      if (ss) ss[j] = acc;
+    }
+  }
+  const uint32_t k = static_cast<uint32_t>(k64);
+  select_staged<1024>(keys, d, k, kmin, kmax, idx);
+  __syncthreads();  // this block's index writes are visible to all its threads
+  for (int64_t e = tid; e < static_cast<int64_t>(M) * k; e += 1024) {
+    const int m = static_cast<int>(e / k);
+    const int64_t r = e % k;
+    AI[m * ld_ai + r] = A[static_cast<int64_t>(m) * lda + __ldg(idx + r)];
+  }
+}
+
+bool allow_select_rows() {
+  static std::atomic<uint64_t> configured{0};  // bit per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const uint64_t bit = 1ull << dev;
+  if (configured.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(select_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kMaxStagedKeys * 4)) != cudaSuccess)
+    return false;
+  configured.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+
 // Opt the histogram kernel into kMaxStagedKeys * 4 bytes of dynamic shared
 // memory, once per device.
 template <int NT>
@@ -351,6 +434,16 @@ bool allow_staged_rows() {
 }
 
 }  // namespace
+
+bool select_rows_supported(int64_t M, int64_t d) { return M >= 1 && M <= 16 && d >= 1 && d <= kMaxStagedKeys; }
+
+cudaError_t launch_select_rows(const void* A, int64_t M, int64_t d, int64_t lda, int64_t k, int32_t* idx, float* ss,
+                               void* A_I, int64_t ld_ai, cudaStream_t stream) {
+  const size_t bytes = static_cast<size_t>(d) * 4;
+  if (bytes > 48 * 1024 && !allow_select_rows()) return cudaErrorInvalidValue;
+  return launch_pdl(select_rows_kernel, dim3(1), dim3(1024), bytes, stream, static_cast<const uint16_t*>(A),
+                    static_cast<int>(M), d, lda, k, idx, ss, static_cast<uint16_t*>(A_I), ld_ai);
+}
 
 cudaError_t launch_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k, int32_t* idx,
                         int64_t ld_idx, cudaStream_t stream) {

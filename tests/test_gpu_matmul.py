@@ -243,6 +243,95 @@ def test_gemm_bf16_parity(M, d, N, k, out_dtype):
     no_device_error()
 
 
+DECODE_SHAPES = [  # M, d, N, k: a few activation rows (decode); kept rows of B read in place
+    (1, 4096, 4096, 2048),
+    (2, 1000, 700, 333),       # ragged N and k
+    (3, 512, 8, 1),            # one kept row
+    (5, 4096, 1032, 4096),     # every row kept
+    (8, 2048, 14336, 1024),
+    (13, 4096, 264, 2867),
+    (16, 4096, 4096, 2048),
+]
+
+
+@pytest.mark.parametrize("M,d,N,k", DECODE_SHAPES)
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_gemm_few_rows_parity(M, d, N, k, out_dtype):
+    inp = W.scaled_matmul_bf16(31 + M, M, d, N)
+    rng = np.random.default_rng(M * 11 + k)
+    idx = np.sort(rng.choice(d, k, replace=False)).astype(np.int32)
+    A = oracle.decode(inp.A, "bf16")
+    Bm = oracle.decode(inp.B, "bf16")
+    At, Bt = bf16_tensor(inp.A), _pitched(bf16_tensor(inp.B))
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(At, it)
+    Y = R.rmm_gemm(AI, Bt, it, out_dtype=out_dtype)
+    ref = A[:, idx] @ Bm[idx, :]
+    if out_dtype == torch.float32:
+        # fp32 sums of exact bf16 products, k terms in some order
+        bound = k * 2.0 ** -24 * (np.abs(A[:, idx]) @ np.abs(Bm[idx, :])) + 1e-30
+        assert np.all(np.abs(to_f64(Y) - ref) <= bound)
+    else:
+        check_bf16_output(to_f64(Y), ref, np.abs(A[:, idx]) @ np.abs(Bm[idx, :]), k)
+    no_device_error()
+
+
+def test_gemm_few_rows_bad_index_flagged():
+    M, d, N, k = 4, 256, 128, 64
+    inp = W.scaled_matmul_bf16(77, M, d, N)
+    idx = np.arange(k, dtype=np.int32)
+    idx[9] = d + 5
+    At, Bt = bf16_tensor(inp.A), bf16_tensor(inp.B)
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(At, it)
+    assert R.rmm_device_error(clear=True) == 1
+    R.rmm_gemm(AI, Bt, it, out_dtype=torch.float32)
+    assert R.rmm_device_error(clear=True) == 1
+    no_device_error()
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_path_decode_rows(M):
+    """Whole path at decode sizes on the MLP up/gate and down shapes."""
+    for inp in (W.llm_activation_bf16(41 + M, M, 4096), W.llm_activation_bf16(43 + M, M, 14336)):
+        d = inp.shape[1]
+        Wb = W.weight_bf16(5, d, 4096 if d == 14336 else 14336)
+        A = oracle.decode(inp, "bf16")
+        Bm = oracle.decode(Wb, "bf16")
+        cond, _ = widen_topk_gaps(inp, "bf16", [oracle.k_from_rho(0.5, d)])
+        Ac = oracle.decode(cond, "bf16")
+        k = oracle.k_from_rho(0.5, d)
+        idx = oracle.topk_indices(oracle.column_sq_norms(Ac), k)
+        idx_out = torch.empty(k, dtype=torch.int32, device="cuda")
+        ss_out = torch.empty(d, dtype=torch.float32, device="cuda")
+        Y = R.rmm_matmul(bf16_tensor(cond), bf16_tensor(Wb), 0.5, idx_out=idx_out, ss_out=ss_out)
+        np.testing.assert_array_equal(idx_out.cpu().numpy(), idx)
+        np.testing.assert_allclose(to_f64(ss_out), oracle.column_sq_norms(Ac), rtol=1e-5)
+        ref = Ac[:, idx] @ Bm[idx, :]
+        check_bf16_output(to_f64(Y), ref, np.abs(Ac[:, idx]) @ np.abs(Bm[idx, :]), k)
+    no_device_error()
+
+
+def test_path_decode_unaligned_rows():
+    """Few rows with a row pitch that is not a multiple of 8 (the fused
+    selection's scalar path) and d not a multiple of 8."""
+    M, d, N, rho = 3, 1001, 264, 0.4
+    A_bits = W.llm_activation_bf16(91, M, d)
+    k = oracle.k_from_rho(rho, d)
+    cond, _ = widen_topk_gaps(A_bits, "bf16", [k])
+    Ac = oracle.decode(cond, "bf16")
+    Wb = W.weight_bf16(92, d, N)
+    Bm = oracle.decode(Wb, "bf16")
+    buf = torch.zeros((M, d + 2), dtype=torch.bfloat16, device="cuda")
+    buf[:, :d] = bf16_tensor(cond)
+    idx_out = torch.empty(k, dtype=torch.int32, device="cuda")
+    Y = R.rmm_matmul(buf[:, :d], _pitched(bf16_tensor(Wb)), rho, idx_out=idx_out)
+    idx = oracle.topk_indices(oracle.column_sq_norms(Ac), k)
+    np.testing.assert_array_equal(idx_out.cpu().numpy(), idx)
+    check_bf16_output(to_f64(Y), Ac[:, idx] @ Bm[idx, :], np.abs(Ac[:, idx]) @ np.abs(Bm[idx, :]), k)
+    no_device_error()
+
+
 def test_gemm_writes_only_its_window():
     """Guard bands: Y is a window of a larger buffer; nothing outside changes."""
     M, d, N, k = 200, 640, 300, 200
