@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["bench", "attention", "decode"], default="bench",
+                    help="attention / decode: run only that workload a few times and exit (a short "
+                         "program for profiler captures; prints no JSON line)")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -551,8 +554,47 @@ def run_rmm(args):
         torch.distributed.destroy_process_group()
 
 
+def run_case(case):
+    """Short runs for profiler captures: the reduced-attention workload called
+    three times, or the decode products (1 and 16 rows on the MLP up/gate
+    weight) called twelve times each with a 256 MiB write in between."""
+    import numpy as np
+    import torch
+    import input_adaptive_reduced_score_b200 as R
+    import workloads
+    from tests.helpers import bf16_tensor
+    dev = torch.device("cuda", 0)
+    if case == "attention":
+        a = ATTN
+        inp = workloads.attention(a["seed"], a["B"], a["Hq"], a["Hkv"], a["S"], a["D"], a["rho_d"], a["rho_t"])
+        Q, K, V = (bf16_tensor(x, dev) for x in (inp.Q, inp.K, inp.V))
+        O = torch.empty_like(Q)
+        ws = torch.empty(R.rmm_attention_workspace_size(a["B"], a["Hq"], a["Hkv"], a["S"], a["D"], a["rho_d"],
+                                                        a["rho_t"]), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            R.rmm_attention(Q, K, V, a["rho_d"], a["rho_t"], out=O, ws=ws)
+    else:
+        k = R.rmm_k_from_rho(RHO, D)
+        Wt = bf16_tensor(workloads.weight_bf16(1, D, N), dev)
+        idx = torch.from_numpy(np.sort(np.random.default_rng(0).choice(D, k, replace=False)).astype(np.int32)).to(dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        gws = torch.empty(R.rmm_gemm_workspace_size(R.RMM_BF16, N, k), dtype=torch.uint8, device=dev)
+        for rows in (1, 16):
+            AI = R.rmm_compact(bf16_tensor(workloads.llm_activation_bf16(7, rows, D), dev), idx)
+            Y = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+            for _ in range(12):
+                flush.zero_()
+                R.rmm_gemm(AI, Wt, idx, out=Y, ws=gws)
+    torch.cuda.synchronize()
+    if R.rmm_device_error() != 0:
+        raise SystemExit("device error")
+
+
 def main():
     args = parse_args()
+    if args.case != "bench":
+        run_case(args.case)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if world != args.gpus and not (args.impl == "reference"):
         if world == 1 and args.gpus > 1:
