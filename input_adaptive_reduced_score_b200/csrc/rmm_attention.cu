@@ -55,8 +55,9 @@ struct AttnParams {
   int kt;           // kept tokens
   int nqb;          // query (= key) blocks of 128
   int out_f32;      // O written as fp32 (else bf16)
-  int c_ks;         // pass C key ring depth (2..4, as shared memory allows)
-  int c_vs;         // pass C value ring depth (1..4, as shared memory allows)
+  int c_ks;         // pass C key ring depth (as shared memory allows)
+  int c_vs;         // pass C value ring depth (as shared memory allows)
+  int c_ps;         // pass C on SM pairs: P buffers in shared memory (2 or 3)
   float scale_log2; // logit scale times log2(e)
 };
 
@@ -678,6 +679,307 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ pass C on SM pairs
+//
+// The same product for two adjacent query blocks on a pair of SMs (a 2-CTA
+// cluster) with tcgen05.mma.cta_group::2 (M = 256): measured on B200, an
+// M256 N128 K16 pair step takes ~68 cycles against ~114 for M128 N128 on
+// one SM, and each SM loads only half of every key block and half of every
+// value block (no multicast: each CTA loads its own halves).
+//   - the leader (rank 0) takes the heavier query block; both CTAs walk the
+//     leader's kept blocks (the lighter block's extra ones are fully masked);
+//   - S = Q_I K_T^T: each CTA's A is its own 128 query rows, its B the 64
+//     keys [j*128 + rank*64, +64) of kept block j; each CTA's tensor memory
+//     gets its 128 rows x 128 keys;
+//   - P (bf16) goes to each CTA's shared memory; O += P V_T: each CTA's B is
+//     its 64 of V's 128 columns, each CTA's tensor memory gets its rows of O;
+//   - every load signals the leader's barriers; the leader's MMA lane waits
+//     on them, and its commits reach both CTAs (multicast); the softmax
+//     groups of both CTAs arrive on the leader's P barrier;
+//   - three logit buffers: after softmax(j) (both CTAs) the leader issues
+//     S(j+3) into buffer j % 3 (softmax(j) has read it) and then PV(j);
+//   - key stage j % 3 is free when S(j) is done and value stage j % c_ps
+//     when PV(j) is done, so the producers wait on the logit and P barriers
+//     (one commit each per kept block instead of two).
+// Every wait is bounded; every path reaches the final cluster barrier.
+constexpr int CP_KS = C_SBUF;  // key ring depth = logit buffers (a key stage is freed with its logits)
+constexpr int CP_MAX_PS = 3;   // P buffers = value ring depth (a value stage is freed with its P)
+constexpr int CP_HALF_ROWS = TILE / 2;                 // keys of a kept block per CTA
+constexpr int CP_KCHUNK_BYTES = CP_HALF_ROWS * 128;    // [64 x 64] bf16, 128-byte rows: 8 KB
+
+struct PairOutBars {
+  uint64_t kfull[CP_KS];
+  uint64_t vfull[CP_MAX_PS];
+  uint64_t qfull;
+  uint64_t sfull[C_SBUF];
+  uint64_t pfull[CP_MAX_PS], pempty[CP_MAX_PS];
+  uint64_t ofull;
+  uint64_t drain;
+  uint32_t tmem_slot;
+  int abort_flag;
+  int pos[8][TILE];
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
+    attn_out_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
+                         const __grid_constant__ CUtensorMap tm_vt, const float* __restrict__ lse,
+                         const int32_t* __restrict__ pos, const int* __restrict__ nvalid, void* __restrict__ O,
+                         AttnParams p, unsigned* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
+  const uint32_t base = smem_u32(smem);
+  constexpr int ks = CP_KS;
+  const int ps = p.c_ps, vs = ps;
+  const int q_bytes = p.kc * CHUNK_BYTES;
+  const int k_bytes = p.kc * CP_KCHUNK_BYTES;  // this CTA's half of a key block
+  const int v_bytes = CHUNK_BYTES;             // this CTA's 64 columns of a value block
+  const uint32_t q_tile = base;
+  auto kst = [&](int s) { return base + q_bytes + s * k_bytes; };
+  auto vst = [&](int s) { return base + q_bytes + ks * k_bytes + s * v_bytes; };
+  const uint32_t p_base = base + q_bytes + ks * k_bytes + vs * v_bytes;  // P buffers of 2 chunks
+  auto pbuf = [&](int b) { return p_base + b * 2 * CHUNK_BYTES; };
+  PairOutBars* bars =
+      reinterpret_cast<PairOutBars*>(smem + q_bytes + ks * k_bytes + vs * v_bytes + ps * 2 * CHUNK_BYTES);
+  volatile int* abort_flag = &bars->abort_flag;
+  auto kfull = [&](int s) { return smem_u32(&bars->kfull[s]); };
+  auto vfull = [&](int s) { return smem_u32(&bars->vfull[s]); };
+  auto sfull = [&](int b) { return smem_u32(&bars->sfull[b]); };
+  auto pfull = [&](int b) { return smem_u32(&bars->pfull[b]); };
+  auto pempty = [&](int b) { return smem_u32(&bars->pempty[b]); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int bh = blockIdx.y;
+  const int pair = static_cast<int>(blockIdx.x) >> 1;
+  const int qb0 = p.nqb - 1 - 2 * pair;                   // the leader's (heavier) block
+  const int qb = qb0 - static_cast<int>(rank);            // this CTA's block (-1: none)
+  const int* nv_bh = nvalid + static_cast<int64_t>(bh) * p.nqb;
+  const int nrb = (__ldg(nv_bh + qb0) + TILE - 1) / TILE;  // kept blocks both CTAs walk
+  const int nbefore = qb > 0 ? __ldg(nv_bh + qb - 1) : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ks; ++s) mbar_init(kfull(s), 1);  // leader: its producer's arrive + both CTAs' bytes
+    for (int s = 0; s < vs; ++s) mbar_init(vfull(s), 1);
+    mbar_init(smem_u32(&bars->qfull), 1);
+    for (int b = 0; b < C_SBUF; ++b) mbar_init(sfull(b), 1);  // multicast commit
+    for (int b = 0; b < ps; ++b) {
+      mbar_init(pfull(b), 8);   // leader: four warps of a softmax group in each CTA
+      mbar_init(pempty(b), 1);  // multicast commit
+    }
+    mbar_init(smem_u32(&bars->ofull), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(&bars->tmem_slot), 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_slot;
+  const uint32_t o_tmem = tmem_base + C_SBUF * TILE;
+  auto buf_tmem = [&](int b) { return tmem_base + b * TILE; };
+
+  if (warp == 0) {
+    // lane 0: Q, then this CTA's key halves; lane 1: its value halves.  The
+    // leader's lanes register both CTAs' bytes on its barriers.
+    if (lane == 0 && nrb > 0) {
+      const uint32_t qf = mapa_shared(smem_u32(&bars->qfull), 0);
+      if (leader) mbar_arrive_expect_tx(smem_u32(&bars->qfull), 2 * q_bytes);
+      for (int c = 0; c < p.kc; ++c) tma_load_3d_pair(q_tile + c * CHUNK_BYTES, &tm_q, qf, c * 64, qb * TILE, bh);
+      int n = 0;
+      for (int t = 0; t < nrb; ++t) {
+        const int st = t % ks;  // freed by S(t - 3): the logits of buffer st
+        if (!mbar_wait(sfull(st), ((t / ks) & 1) ^ 1u, abort_flag, err, 31)) break;
+        const uint32_t kf = mapa_shared(kfull(st), 0);
+        if (leader) mbar_arrive_expect_tx(kfull(st), 2 * k_bytes);
+        for (int c = 0; c < p.kc; ++c)
+          tma_load_3d_pair(kst(st) + c * CP_KCHUNK_BYTES, &tm_kh, kf, c * 64,
+                           t * TILE + static_cast<int>(rank) * CP_HALF_ROWS, bh);
+        ++n;
+      }
+      if (leader) {
+        wait_drain(smem_u32(&bars->qfull), 0);
+        drain_ring(bars->kfull, n, ks);
+      }
+    } else if (lane == 1 && nrb > 0) {
+      int n = 0;
+      for (int t = 0; t < nrb; ++t) {
+        const int st = t % vs;  // freed by PV(t - c_ps): P buffer st
+        if (!mbar_wait(pempty(st), ((t / vs) & 1) ^ 1u, abort_flag, err, 32)) break;
+        const uint32_t vf = mapa_shared(vfull(st), 0);
+        if (leader) mbar_arrive_expect_tx(vfull(st), 2 * v_bytes);
+        tma_load_3d_pair(vst(st), &tm_vt, vf, static_cast<int>(rank) * 64, t * TILE, bh);
+        ++n;
+      }
+      if (leader) drain_ring(bars->vfull, n, vs);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(2 * TILE, TILE, false, false);
+      const uint32_t idesc_o = idesc_bf16_f32(2 * TILE, p.D, false, true);
+      bool ok = nrb == 0 || mbar_wait(smem_u32(&bars->qfull), 0, abort_flag, err, 33);
+      auto issue_s = [&](int t) -> bool {
+        const int st = t % ks;
+        if (!mbar_wait(kfull(st), (t / ks) & 1, abort_flag, err, 34)) return false;
+        tc_fence_after();
+        for (int c = 0; c < p.kc; ++c) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sdesc_sw128(q_tile + c * CHUNK_BYTES + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(kst(st) + c * CP_KCHUNK_BYTES + kk * 32, 16, 1024);
+            mma_f16_ss_pair(buf_tmem(t % C_SBUF), ad, bd, idesc_s, (c | kk) != 0 ? 1u : 0u);
+          }
+        }
+        mma_commit_pair_multicast(sfull(t % C_SBUF), 0x3);
+        return true;
+      };
+      auto issue_pv = [&](int t) -> bool {
+        const int st = t % vs, pb = t % ps;
+        if (!mbar_wait(vfull(st), (t / vs) & 1, abort_flag, err, 35)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < TILE / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(pbuf(pb) + (kk / 4) * CHUNK_BYTES + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(vst(st) + kk * 16 * 128, CHUNK_BYTES, 1024);
+          mma_f16_ss_pair(o_tmem, ad, bd, idesc_o, (t | kk) != 0 ? 1u : 0u);
+        }
+        mma_commit_pair_multicast(pempty(pb), 0x3);
+        return true;
+      };
+      for (int t = 0; ok && t < C_SBUF && t < nrb; ++t) ok = issue_s(t);
+      for (int j = 0; ok && j < nrb; ++j) {
+        ok = mbar_wait(pfull(j % ps), (j / ps) & 1, abort_flag, err, 36);
+        if (ok) tc_fence_after();
+        if (ok && j + C_SBUF < nrb) ok = issue_s(j + C_SBUF);
+        ok = ok && issue_pv(j);
+      }
+      if (ok && nrb > 0) mma_commit_pair_multicast(smem_u32(&bars->ofull), 0x3);
+      mma_commit_pair_multicast(smem_u32(&bars->drain), 0x1);
+      wait_drain(smem_u32(&bars->drain), 0);
+    }
+    __syncwarp();
+  } else {
+    const int g = (warp - 2) >> 2;  // softmax group
+    const int qtr = warp & 3;       // tensor-memory lane quarter of this warp
+    const int r = qtr * 32 + lane;
+    const int i = qb * TILE + r;    // this thread's query (negative for the spare CTA of an odd count)
+    const bool row_ok = i >= 0 && i < p.S;
+    const uint32_t lane_off = static_cast<uint32_t>(qtr * 32) << 16;
+    const float L2 = row_ok ? lse[static_cast<int64_t>(bh) * p.S + i] * kLog2e : 0.f;
+    const int32_t* pos_bh = pos + static_cast<int64_t>(bh) * p.kt;
+    const uint64_t slp = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(-L2, -L2);
+    int* psh = bars->pos[warp - 2];
+    bool ok = true;
+    for (int rb = g; ok && rb < nrb; rb += 2) {
+      const int b = rb % C_SBUF, pb = rb % ps;
+      const uint32_t sph = (rb / C_SBUF) & 1, pph = (rb / ps) & 1;
+      const bool masked = rb * TILE + TILE > nbefore;
+      if (masked) {
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int kr = rb * TILE + u * 32 + lane;
+          psh[u * 32 + lane] = kr < p.kt ? __ldg(pos_bh + kr) : 0x7FFFFFFF;
+        }
+        __syncwarp();
+      }
+      if (!mbar_wait_warp(sfull(b), sph, abort_flag, err, 37) ||
+          !mbar_wait_warp(pempty(pb), pph ^ 1u, abort_flag, err, 38)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t s_addr = buf_tmem(b) + lane_off;
+      uint8_t* prow = smem + (pbuf(pb) - base) + r * 128;
+      auto emit = [&](int cc, const uint32_t (&v)[32]) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), slp, nl2), x0, x1);
+          float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          if (masked) {
+            if (psh[cc * 32 + 2 * e] > i) p0 = 0.f;
+            if (psh[cc * 32 + 2 * e + 1] > i) p1 = 0.f;
+          }
+          w[e] = pack_bf16x2(p0, p1);
+        }
+        uint8_t* crow = prow + (cc >> 1) * CHUNK_BYTES;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int piece = (cc & 1) * 4 + q;
+          *reinterpret_cast<uint4*>(crow + ((piece ^ (r & 7)) << 4)) =
+              make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+      };
+      uint32_t va[32], vb[32];
+      __syncwarp();  // tensor-memory loads are warp-synchronous: reconverge first
+      tmem_ld32(s_addr, va);
+      tmem_wait_ld_into(va);
+      tmem_ld32(s_addr + 32, vb);
+      emit(0, va);
+      tmem_wait_ld_into(vb);
+      __syncwarp();
+      tmem_ld32(s_addr + 64, va);
+      emit(1, vb);
+      tmem_wait_ld_into(va);
+      __syncwarp();
+      tmem_ld32(s_addr + 96, vb);
+      emit(2, va);
+      tmem_wait_ld_into(vb);
+      emit(3, vb);
+      tc_fence_before();
+      fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(pfull(pb), 0));
+    }
+    // epilogue: O row i, columns [g D/2, (g+1) D/2)
+    const bool have = ok && nrb > 0 && mbar_wait_warp(smem_u32(&bars->ofull), 0, abort_flag, err, 39);
+    if (have) tc_fence_after();
+    const int ncc = p.D / 64;
+    for (int cc = g * ncc; cc < (g + 1) * ncc; ++cc) {
+      uint32_t v[32];
+      if (have) {
+        __syncwarp();
+        tmem_ld32(o_tmem + cc * 32 + lane_off, v);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
+      }
+      if (!row_ok) continue;
+      const int64_t off = (static_cast<int64_t>(bh) * p.S + i) * p.D + cc * 32;
+      if (p.out_f32) {
+        float4* y = reinterpret_cast<float4*>(static_cast<float*>(O) + off);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          y[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
+                             __uint_as_float(v[4 * q + 3]));
+      } else {
+        uint4* y = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(O) + off);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          y[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+      }
+    }
+    tc_fence_before();
+  }
+
+  tc_fence_before();
+  cluster_sync();  // all MMAs, copies and remote arrivals of the pair are done
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -698,8 +1000,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D bf16 map over [heads][rows][pitch] with logical row length `cols`;
-// boxes of 64 columns x 128 rows x 1 head, 128-byte swizzle.
-bool encode_heads(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int64_t heads, int64_t pitch) {
+// boxes of 64 columns x box_rows rows x 1 head, 128-byte swizzle.
+bool encode_heads(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int64_t heads, int64_t pitch,
+                  int box_rows = TILE) {
   EncodeTiledFn encode = encode_fn();
   if (!encode) {
     set_error("rmm_attention: cuTensorMapEncodeTiled entry point unavailable");
@@ -708,7 +1011,7 @@ bool encode_heads(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows,
   const cuuint64_t gdim[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(heads)};
   const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(pitch) * 2, static_cast<cuuint64_t>(pitch * rows) * 2};
-  const cuuint32_t box[3] = {64, TILE, 1};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), gdim, gstride, box,
                             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -885,15 +1188,38 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
     e = cudaGetLastError();
     if (e != cudaSuccess || (e = debug_step(stream, "row gathers")) != cudaSuccess) return e;
   }
-  // 7. pass C
-  auto out_smem_for = [&](int ks, int vs) {
-    return kc * CHUNK_BYTES + ks * kc * CHUNK_BYTES + vs * static_cast<int>(D / 64) * CHUNK_BYTES +
-           static_cast<int>(sizeof(OutBars)) + 1024;
-  };
+  // 7. pass C: on SM pairs when D = 128 (a pair's CTA takes 64 of V's columns)
   int dev = 0, max_smem = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess ||
       (e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
+  if (D == 128) {
+    // key ring of 3 (one per logit buffer); value ring = P buffers, 3 when they fit
+    auto pair_smem_for = [&](int ps) {
+      return kc * CHUNK_BYTES + CP_KS * kc * CP_KCHUNK_BYTES + ps * CHUNK_BYTES + ps * 2 * CHUNK_BYTES +
+             static_cast<int>(sizeof(PairOutBars)) + 1024;
+    };
+    prm.c_ps = pair_smem_for(3) <= max_smem ? 3 : 2;
+    const int pair_smem = pair_smem_for(prm.c_ps);
+    CUtensorMap tm_kh;
+    if (!encode_heads(&tm_kh, kt_rows, kd, kt, BH, w.ldk, CP_HALF_ROWS)) return cudaErrorInvalidValue;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      if (!set_smem(attn_out_pair_kernel, pair_smem)) {
+        set_error("rmm_attention: cannot set %d bytes of shared memory for pass C", pair_smem);
+        return cudaErrorInvalidValue;
+      }
+    }
+    const dim3 grid_pair(static_cast<unsigned>(2 * ((nqb + 1) / 2)), static_cast<unsigned>(BH));
+    attn_out_pair_kernel<<<grid_pair, ATT_THREADS, pair_smem, stream>>>(tm_q, tm_kh, tm_vt, lse, idx_t, nvalid, O,
+                                                                         prm, err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return debug_step(stream, "pass C (output, SM pairs)");
+  }
+  auto out_smem_for = [&](int ks, int vs) {
+    return kc * CHUNK_BYTES + ks * kc * CHUNK_BYTES + vs * static_cast<int>(D / 64) * CHUNK_BYTES +
+           static_cast<int>(sizeof(OutBars)) + 1024;
+  };
   // deepest key and value rings that fit (the value ring grows first)
   prm.c_ks = 2;
   prm.c_vs = 1;
