@@ -204,6 +204,37 @@ RMM_API rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t
                       void* Y, int out_dtype, int64_t ldy, int32_t* idx_out, float* ss_out,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ int8 weights
+ * The reduced product with an int8 weight (Resultados Experimentales ›
+ * Compatibilidad: the method works with INT8 weight quantisation).  The
+ * page fixes no scheme; the one taken here is symmetric weight-only
+ * quantisation with one fp32 scale per output column:
+ *     B[j, n] = Bq[j, n] * b_scale[n],   Bq int8 [d x N] (ldb bytes),
+ * so  Y = A_I · B[idx, :] = (A_I · Bq[idx, :]) * b_scale  (column-wise).
+ * The selection is unchanged: it reads the activation only.
+ *  - M <= 16: the kept int8 rows are read in place (half the bytes of bf16),
+ *    widened exactly to fp32, and each column's sum is scaled at the end.
+ *  - M > 16: the kept rows are gathered into workspace as exact bf16
+ *    integers, the tcgen05 product runs on them, and the epilogue scales
+ *    each column before rounding to out_dtype.
+ * A_I bf16 [M x k] (ld_ai, a multiple of 8), Bq (ldb a multiple of 16), Y
+ * (ldy) 16-byte aligned, else RMM_ERR_UNSUPPORTED.  b_scale [N] fp32,
+ * finite.  Workspace: rmm_gemm_w8_workspace_size(N, k) bytes, 256-byte
+ * aligned.  Out-of-range indices contribute zero and are flagged. */
+RMM_API size_t rmm_gemm_w8_workspace_size(int64_t N, int64_t k);
+RMM_API rmm_status rmm_gemm_w8(const void* A_I, int64_t ld_ai, const int8_t* Bq, int64_t ldb, const float* b_scale,
+                               const int32_t* idx, int64_t d, int64_t M, int64_t N, int64_t k, void* Y,
+                               int out_dtype, int64_t ldy, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole path with an int8 weight: ss = score(A) (bf16 A [M x d], lda);
+ * I = topk(ss, k), k = rmm_k_from_rho(rho, d); Y = A_I · (Bq[I, :] *
+ * b_scale).  idx_out and ss_out as in rmm_matmul.  Workspace:
+ * rmm_matmul_w8_workspace_size bytes, 256-byte aligned. */
+RMM_API size_t rmm_matmul_w8_workspace_size(int64_t M, int64_t d, int64_t N, double rho);
+RMM_API rmm_status rmm_matmul_w8(const void* A, int64_t lda, const int8_t* Bq, int64_t ldb, const float* b_scale,
+                                 int64_t M, int64_t d, int64_t N, double rho, void* Y, int out_dtype, int64_t ldy,
+                                 int32_t* idx_out, float* ss_out, void* ws, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------ reduced attention
  * Causal attention with both reductions of Metodología › Alcance de
  * Aplicación, for Q [B, Hq, S, D] and K, V [B, Hkv, S, D] bf16, contiguous

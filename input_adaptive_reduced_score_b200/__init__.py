@@ -22,7 +22,8 @@ __all__ = [
     "lib", "LIB_PATH", "RMMError", "RMM_F32", "RMM_BF16", "rmm_abi_version", "rmm_k_from_rho",
     "rmm_device_error", "rmm_score", "rmm_score_workspace_size", "rmm_score_noalloc", "rmm_topk", "rmm_compact", "rmm_gather_rows", "rmm_compact_gather",
     "rmm_gemm", "rmm_gemm_workspace_size", "rmm_gemm_compacted",
-    "rmm_matmul", "rmm_matmul_workspace_size", "rmm_attention", "rmm_attention_workspace_size",
+    "rmm_matmul", "rmm_matmul_workspace_size", "rmm_gemm_w8", "rmm_gemm_w8_workspace_size", "rmm_matmul_w8",
+    "rmm_matmul_w8_workspace_size", "rmm_attention", "rmm_attention_workspace_size",
     "exported_symbols", "declared_symbols",
 ]
 
@@ -69,6 +70,12 @@ _sig("rmm_gemm", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i
 _sig("rmm_gemm_compacted", c_int, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_int, c_i64, c_vp)
 _sig("rmm_matmul_workspace_size", c_sz, c_int, c_i64, c_i64, c_i64, c_dbl)
 _sig("rmm_matmul", c_int, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_i64, c_dbl, c_int, c_vp, c_int, c_i64, c_vp, c_vp,
+     c_vp, c_sz, c_vp)
+_sig("rmm_gemm_w8_workspace_size", c_sz, c_i64, c_i64)
+_sig("rmm_gemm_w8", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_int, c_i64, c_vp,
+     c_sz, c_vp)
+_sig("rmm_matmul_w8_workspace_size", c_sz, c_i64, c_i64, c_i64, c_dbl)
+_sig("rmm_matmul_w8", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_dbl, c_vp, c_int, c_i64, c_vp, c_vp,
      c_vp, c_sz, c_vp)
 _sig("rmm_attention_workspace_size", c_sz, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl)
 _sig("rmm_attention", c_int, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl, c_flt, c_vp, c_int,
@@ -310,6 +317,57 @@ def rmm_matmul(A: torch.Tensor, B: torch.Tensor, rho: float, out: torch.Tensor =
     w, wn = _workspace(wsb, A.device, ws)
     _check(lib.rmm_matmul(_ptr(A), lda, _ptr(B), ldb, M, d, N, float(rho), dt, _ptr(out), _dtype_code(out), ldy,
                           _ptr(idx_out), _ptr(ss_out), _ptr(w), wn, _stream_ptr(stream)), "rmm_matmul")
+    return out
+
+
+def _int8_weight(Bq: torch.Tensor, b_scale: torch.Tensor):
+    if Bq.dtype != torch.int8:
+        raise TypeError("Bq must be int8")
+    if b_scale.dtype != torch.float32 or b_scale.numel() != Bq.shape[1] or not b_scale.is_contiguous():
+        raise ValueError("b_scale must be a contiguous fp32 vector of N column scales")
+    return _row_major(Bq, "Bq")
+
+
+def rmm_gemm_w8_workspace_size(N: int, k: int) -> int:
+    return lib.rmm_gemm_w8_workspace_size(N, k)
+
+
+def rmm_gemm_w8(A_I: torch.Tensor, Bq: torch.Tensor, b_scale: torch.Tensor, idx: torch.Tensor,
+                out: torch.Tensor = None, out_dtype=None, ws=None, stream=None):
+    """Y = A_I · (Bq[idx, :] * b_scale), A_I bf16 [M x k], Bq int8 [d x N], b_scale fp32 [N]."""
+    ld_ai = _row_major(A_I, "A_I")
+    ldb = _int8_weight(Bq, b_scale)
+    M, k = A_I.shape
+    d, N = Bq.shape
+    if idx.numel() != k:
+        raise ValueError("idx must hold k indices")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or A_I.dtype, device=A_I.device)
+    ldy = _row_major(out, "Y")
+    w, wn = _workspace(lib.rmm_gemm_w8_workspace_size(N, k), A_I.device, ws)
+    _check(lib.rmm_gemm_w8(_ptr(A_I), ld_ai, _ptr(Bq), ldb, _ptr(b_scale), _ptr(idx), d, M, N, k, _ptr(out),
+                           _dtype_code(out), ldy, _ptr(w), wn, _stream_ptr(stream)), "rmm_gemm_w8")
+    return out
+
+
+def rmm_matmul_w8_workspace_size(M: int, d: int, N: int, rho: float) -> int:
+    return lib.rmm_matmul_w8_workspace_size(M, d, N, float(rho))
+
+
+def rmm_matmul_w8(A: torch.Tensor, Bq: torch.Tensor, b_scale: torch.Tensor, rho: float, out: torch.Tensor = None,
+                  out_dtype=None, idx_out: torch.Tensor = None, ss_out: torch.Tensor = None, ws=None, stream=None):
+    """The whole path with an int8 weight: score -> top-k -> compaction -> reduced product."""
+    lda = _row_major(A, "A")
+    ldb = _int8_weight(Bq, b_scale)
+    M, d = A.shape
+    N = Bq.shape[1]
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype or A.dtype, device=A.device)
+    ldy = _row_major(out, "Y")
+    w, wn = _workspace(lib.rmm_matmul_w8_workspace_size(M, d, N, float(rho)), A.device, ws)
+    _check(lib.rmm_matmul_w8(_ptr(A), lda, _ptr(Bq), ldb, _ptr(b_scale), M, d, N, float(rho), _ptr(out),
+                             _dtype_code(out), ldy, _ptr(idx_out), _ptr(ss_out), _ptr(w), wn, _stream_ptr(stream)),
+           "rmm_matmul_w8")
     return out
 
 

@@ -379,6 +379,102 @@ rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t ldb, in
                   stream);
 }
 
+size_t rmm_gemm_w8_workspace_size(int64_t N, int64_t k) { return rmm_gemm_workspace_size(RMM_BF16, N, k); }
+
+rmm_status rmm_gemm_w8(const void* A_I, int64_t ld_ai, const int8_t* Bq, int64_t ldb, const float* b_scale,
+                       const int32_t* idx, int64_t d, int64_t M, int64_t N, int64_t k, void* Y, int out_dtype,
+                       int64_t ldy, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (!valid_dtype(out_dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm_w8: out dtype %d", out_dtype);
+  if (M < 0 || N < 0 || d < 1 || k < 1 || k > d || ld_ai < k || ldb < N || ldy < N || M > kIntMax ||
+      N > kIntMax || d > kIntMax)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_gemm_w8: bad sizes");
+  if (M == 0 || N == 0) return RMM_OK;
+  if (!A_I || !Bq || !b_scale || !idx || !Y) return fail(RMM_ERR_INVALID_ARG, "rmm_gemm_w8: null pointer");
+  if (!aligned16(A_I) || !aligned16(Bq) || !aligned16(Y) || ld_ai % 8 || ldb % 16)
+    return fail(RMM_ERR_UNSUPPORTED,
+                "rmm_gemm_w8: needs 16-byte aligned A_I/Bq/Y, ld_ai a multiple of 8 and ldb of 16");
+  if (((M + 127) / 128) * ((N + 255) / 256) > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "rmm_gemm_w8: too many tiles");
+  const size_t need = rmm_gemm_w8_workspace_size(N, k);
+  if (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
+    return fail(RMM_ERR_WORKSPACE, "rmm_gemm_w8: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes, need);
+  unsigned* err = device_error_word();
+  if (!err) return RMM_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M <= kGemvMaxM) {
+    const GemvPlan pl = gemv_plan(M, N, k, device_sm_count());
+    if (pl.partial_bytes > ws_bytes)
+      return fail(RMM_ERR_WORKSPACE, "rmm_gemm_w8: workspace %zu < %zu bytes", ws_bytes, pl.partial_bytes);
+    return from_cuda(launch_gemv(A_I, ld_ai, Bq, ldb, idx, M, d, N, k, pl, static_cast<float*>(ws), Y, out_dtype, ldy,
+                                 err, s, b_scale),
+                     "rmm_gemm_w8(few rows): launch");
+  }
+  const int64_t ld_bi = round_up(N, 8);
+  cudaError_t e = launch_gather_rows_i8(Bq, d, N, ldb, idx, k, ws, ld_bi, err, s);
+  if (e != cudaSuccess) return from_cuda(e, "rmm_gemm_w8: row gather launch");
+  e = launch_gemm_bf16_tc(A_I, ld_ai, ws, ld_bi, M, N, k, Y, out_dtype, ldy, err, s, b_scale);
+  if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+  return from_cuda(e, "rmm_gemm_w8: launch");
+}
+
+size_t rmm_matmul_w8_workspace_size(int64_t M, int64_t d, int64_t N, double rho) {
+  return rmm_matmul_workspace_size(RMM_BF16, M, d, N, rho);
+}
+
+rmm_status rmm_matmul_w8(const void* A, int64_t lda, const int8_t* Bq, int64_t ldb, const float* b_scale, int64_t M,
+                         int64_t d, int64_t N, double rho, void* Y, int out_dtype, int64_t ldy, int32_t* idx_out,
+                         float* ss_out, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (!valid_dtype(out_dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_w8: out dtype %d", out_dtype);
+  const int64_t k = k_from_rho_impl(rho, d);
+  if (k < 1) return fail(RMM_ERR_INVALID_ARG, "rmm_matmul_w8: rho %g outside (0,1] or d < 1", rho);
+  if (M < 0 || N < 0 || lda < d || ldb < N || ldy < N) return fail(RMM_ERR_INVALID_ARG, "rmm_matmul_w8: bad sizes");
+  if (!A || !Bq || !b_scale || !Y) return fail(RMM_ERR_INVALID_ARG, "rmm_matmul_w8: null pointer");
+  if (!aligned16(Bq) || ldb % 16)
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_w8: needs a 16-byte aligned Bq and ldb a multiple of 16");
+  const MatmulWs w = matmul_ws(RMM_BF16, M, d, N, rho);
+  if (!ws || ws_bytes < w.total || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
+    return fail(RMM_ERR_WORKSPACE, "rmm_matmul_w8: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes,
+                w.total);
+  char* base = static_cast<char*>(ws);
+  float* ss = ss_out ? ss_out : reinterpret_cast<float*>(base + w.ss);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+  void* ai = base + w.ai;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M > 0 && N > 0 && select_rows_supported(M, d)) {
+    const cudaError_t e = launch_select_rows(A, M, d, lda, k, idx, ss, ai, w.ld_ai, s);
+    if (e != cudaSuccess) return from_cuda(e, "rmm_matmul_w8: row selection launch");
+    return rmm_gemm_w8(ai, w.ld_ai, Bq, ldb, b_scale, idx, d, M, N, k, Y, out_dtype, ldy, base + w.bi,
+                       w.total - w.bi, stream);
+  }
+  rmm_status st = rmm_score(A, RMM_BF16, 1, M, d, lda, 0, ss, d, 0, base + w.score,
+                            score_workspace_bytes(RMM_BF16, 1, M, d), stream);
+  if (st != RMM_OK) return st;
+  st = rmm_topk(ss, 1, d, d, k, idx, k, stream);
+  if (st != RMM_OK) return st;
+  if (M > kGemvMaxM && N > 0) {
+    // both reduced operands in one launch (the int8 rows widened to bf16),
+    // then the tensor-core product with the column scales in its epilogue
+    const int64_t ld_bi = round_up(N, 8);
+    void* bi = base + w.bi;
+    if (k + ((M + 7) / 8) * ((k + 63) / 64) > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_w8: grid");
+    if (((M + 127) / 128) * ((N + 255) / 256) > kIntMax)
+      return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_w8: too many tiles");
+    if (!aligned16(Y)) return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_w8: needs a 16-byte aligned Y");
+    unsigned* err = device_error_word();
+    if (!err) return RMM_ERR_CUDA;
+    cudaError_t e = launch_compact_and_gather(A, M, d, lda, Bq, N, ldb, idx, k, ai, w.ld_ai, bi, ld_bi, err, s, true);
+    if (e != cudaSuccess) return from_cuda(e, "rmm_matmul_w8: compaction launch");
+    e = launch_gemm_bf16_tc(ai, w.ld_ai, bi, ld_bi, M, N, k, Y, out_dtype, ldy, err, s, b_scale);
+    if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+    return from_cuda(e, "rmm_matmul_w8: launch");
+  }
+  st = rmm_compact(A, RMM_BF16, M, d, lda, idx, k, ai, w.ld_ai, stream);
+  if (st != RMM_OK) return st;
+  return rmm_gemm_w8(ai, w.ld_ai, Bq, ldb, b_scale, idx, d, M, N, k, Y, out_dtype, ldy, base + w.bi, w.total - w.bi,
+                     stream);
+}
+
 size_t rmm_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D, double rho_d,
                                     double rho_t) {
   const int64_t kd = k_from_rho_impl(rho_d, D), kt = k_from_rho_impl(rho_t, S);

@@ -13,7 +13,9 @@
 //  - other layouts: each thread gathers its 8 output columns of 8 rows
 //    straight from global memory through the read-only cache.
 //  - B rows are whole contiguous rows: one block per kept row streams it with
-//    16-byte loads and stores.
+//    16-byte loads and stores.  An int8 B (weight-only quantisation) is
+//    widened to exact bf16 values on the way; its scales are applied by the
+//    product.
 #include <cuda_bf16.h>
 
 #include <atomic>
@@ -215,6 +217,66 @@ __device__ __forceinline__ void gather_row_block(int64_t r, const uint4* __restr
   for (; v < vecs; v += kGatherThreads) dst[v] = __ldcs(src + v);
 }
 
+// The int8 form (weight-only quantised B): row I_r of the int8 matrix is read
+// with 16-byte loads (16 values) and written as 16 exact bf16 values (two
+// 16-byte stores); the per-column scale is applied later, in the product's
+// epilogue.  A row length that is not a multiple of 16 ends with byte loads.
+__device__ __forceinline__ void gather_row_block_i8(int64_t r, const uint4* __restrict__ Bq, int64_t d, int64_t vecs,
+                                                    int64_t tail_bytes, int64_t ldb_vec,
+                                                    const int32_t* __restrict__ idx, int64_t k,
+                                                    uint4* __restrict__ BI, int64_t ldbi_vec, unsigned* err) {
+  if (r >= k) return;
+  const int32_t j = __ldg(idx + r);
+  uint4* dst = BI + r * ldbi_vec;
+  __nv_bfloat16* dst_tail = reinterpret_cast<__nv_bfloat16*>(dst + 2 * vecs);
+  if (j < 0 || j >= d) {
+    if (threadIdx.x == 0) record_error(err, kDevErrBadIndex);
+    for (int64_t v = threadIdx.x; v < 2 * vecs; v += kGatherThreads) dst[v] = make_uint4(0, 0, 0, 0);
+    if (threadIdx.x < tail_bytes) dst_tail[threadIdx.x] = __float2bfloat16_rn(0.f);
+    return;
+  }
+  const uint4* src = Bq + static_cast<int64_t>(j) * ldb_vec;
+  if (threadIdx.x < tail_bytes)
+    dst_tail[threadIdx.x] =
+        __float2bfloat16_rn(static_cast<float>(reinterpret_cast<const int8_t*>(src + vecs)[threadIdx.x]));
+  auto put = [&](int64_t v, const uint4& q) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float f[4];
+      i8x4_to_f32(w[e], f);
+      o[2 * e] = pack_bf16x2(f[0], f[1]);
+      o[2 * e + 1] = pack_bf16x2(f[2], f[3]);
+    }
+    dst[2 * v] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[2 * v + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+  };
+  int64_t v = threadIdx.x;
+  for (; v + 3 * kGatherThreads < vecs; v += 4 * kGatherThreads) {
+    const uint4 a0 = __ldcs(src + v);
+    const uint4 a1 = __ldcs(src + v + kGatherThreads);
+    const uint4 a2 = __ldcs(src + v + 2 * kGatherThreads);
+    const uint4 a3 = __ldcs(src + v + 3 * kGatherThreads);
+    put(v, a0);
+    put(v + kGatherThreads, a1);
+    put(v + 2 * kGatherThreads, a2);
+    put(v + 3 * kGatherThreads, a3);
+  }
+  for (; v < vecs; v += kGatherThreads) put(v, __ldcs(src + v));
+}
+
+__global__ void __launch_bounds__(kGatherThreads) gather_rows_i8_kernel(const uint4* __restrict__ Bq, int64_t d,
+                                                                          int64_t vecs, int64_t tail_bytes,
+                                                                          int64_t ldb_vec,
+                                                                          const int32_t* __restrict__ idx, int64_t k,
+                                                                          uint4* __restrict__ BI, int64_t ldbi_vec,
+                                                                          unsigned* err) {
+  pdl_wait();
+  pdl_trigger();
+  gather_row_block_i8(blockIdx.x, Bq, d, vecs, tail_bytes, ldb_vec, idx, k, BI, ldbi_vec, err);
+}
+
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint4* __restrict__ B, int64_t d,
                                                                        int64_t vecs, int64_t tail_halves,
                                                                        int64_t ldb_vec, const int32_t* __restrict__ idx,
@@ -229,9 +291,11 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint4
 // the remaining blocks compact the kept columns of A (bf16; staged R rows per
 // block, or the direct gather of 8 rows x 2048 columns), so the two HBM
 // streams overlap.
-template <bool kStagedA>
+// kW8: B is int8 (vecs counts 16-value vectors, tail_elems trailing bytes)
+// and B_I is written as bf16; otherwise B is bf16 (tail_elems trailing halves).
+template <bool kStagedA, bool kW8>
 __global__ void __launch_bounds__(kGatherThreads) compact_gather_kernel(
-    const uint4* __restrict__ B, int64_t d, int64_t vecs, int64_t tail_halves, int64_t ldb_vec,
+    const uint4* __restrict__ B, int64_t d, int64_t vecs, int64_t tail_elems, int64_t ldb_vec,
     uint4* __restrict__ BI, int64_t ldbi_vec, const uint16_t* __restrict__ A, int64_t M, int64_t lda,
     uint16_t* __restrict__ AI, int64_t ld_ai, int64_t chunks, int R, bool vec_ok, const int32_t* __restrict__ idx,
     int64_t k, unsigned* err) {
@@ -240,7 +304,10 @@ __global__ void __launch_bounds__(kGatherThreads) compact_gather_kernel(
   pdl_trigger();
   const int64_t blk = blockIdx.x;
   if (blk < k) {
-    gather_row_block(blk, B, d, vecs, tail_halves, ldb_vec, idx, k, BI, ldbi_vec, err);
+    if constexpr (kW8)
+      gather_row_block_i8(blk, B, d, vecs, tail_elems, ldb_vec, idx, k, BI, ldbi_vec, err);
+    else
+      gather_row_block(blk, B, d, vecs, tail_elems, ldb_vec, idx, k, BI, ldbi_vec, err);
   } else if constexpr (kStagedA) {
     compact_rows_block(blk - k, A, M, d, lda, idx, k, AI, ld_ai, R, err, stage);
   } else {
@@ -314,28 +381,46 @@ cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64
 
 cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64_t lda, const void* B, int64_t N,
                                       int64_t ldb, const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai,
-                                      void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream) {
+                                      void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream, bool b_int8) {
   const int R = staged_rows(A, d, lda);
   const int64_t chunks = (k + kColsPerCta - 1) / kColsPerCta;
   const int64_t cblocks = M <= 0 ? 0 : (R > 0 ? (M + R - 1) / R : ((M + kRowsPerCta - 1) / kRowsPerCta) * chunks);
   const int64_t blocks = k + cblocks;
   if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   const bool vec_ok = reinterpret_cast<uintptr_t>(A_I) % 16 == 0 && (ld_ai * 2) % 16 == 0;
-  const int64_t row_bytes = N * 2;
+  const int64_t belt = b_int8 ? 1 : 2;
+  const int64_t row_bytes = N * belt;
+  const int64_t vecs = row_bytes / 16, tail = (row_bytes % 16) / belt;
+  const int64_t ldb_vec = ldb * belt / 16, ldbi_vec = ld_bi * 2 / 16;
   const dim3 grid(static_cast<unsigned>(blocks)), block(kGatherThreads);
   const uint4* b = static_cast<const uint4*>(B);
   uint4* bi = static_cast<uint4*>(B_I);
   const uint16_t* a = static_cast<const uint16_t*>(A);
   uint16_t* ai = static_cast<uint16_t*>(A_I);
+  auto go = [&](auto kernel, size_t smem, int r) {
+    return launch_pdl(kernel, grid, block, smem, stream, b, d, vecs, tail, ldb_vec, bi, ldbi_vec, a, M, lda, ai, ld_ai,
+                      chunks, r, vec_ok, idx, k, err);
+  };
   if (R > 0) {
     const size_t smem = static_cast<size_t>(R) * 2 * d;
-    if (smem > 48 * 1024 && !allow_staged_smem<compact_gather_kernel<true>>()) return cudaErrorInvalidValue;
-    return launch_pdl(compact_gather_kernel<true>, grid, block, smem, stream, b, d, row_bytes / 16,
-                      (row_bytes % 16) / 2, ldb * 2 / 16, bi, ld_bi * 2 / 16, a, M, lda, ai, ld_ai, chunks, R, vec_ok,
-                      idx, k, err);
+    if (b_int8) {
+      if (smem > 48 * 1024 && !allow_staged_smem<compact_gather_kernel<true, true>>()) return cudaErrorInvalidValue;
+      return go(compact_gather_kernel<true, true>, smem, R);
+    }
+    if (smem > 48 * 1024 && !allow_staged_smem<compact_gather_kernel<true, false>>()) return cudaErrorInvalidValue;
+    return go(compact_gather_kernel<true, false>, smem, R);
   }
-  return launch_pdl(compact_gather_kernel<false>, grid, block, 0, stream, b, d, row_bytes / 16, (row_bytes % 16) / 2,
-                    ldb * 2 / 16, bi, ld_bi * 2 / 16, a, M, lda, ai, ld_ai, chunks, 0, vec_ok, idx, k, err);
+  if (b_int8) return go(compact_gather_kernel<false, true>, 0, 0);
+  return go(compact_gather_kernel<false, false>, 0, 0);
+}
+
+cudaError_t launch_gather_rows_i8(const void* Bq, int64_t d, int64_t N, int64_t ldb, const int32_t* idx, int64_t k,
+                                  void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream) {
+  if (k == 0 || N == 0) return cudaSuccess;
+  if (k > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  return launch_pdl(gather_rows_i8_kernel, dim3(static_cast<unsigned>(k)), dim3(kGatherThreads), 0, stream,
+                    static_cast<const uint4*>(Bq), d, N / 16, N % 16, ldb / 16, idx, k, static_cast<uint4*>(B_I),
+                    ld_bi * 2 / 16, err);
 }
 
 }  // namespace rmm

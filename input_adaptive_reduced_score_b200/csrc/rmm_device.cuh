@@ -437,4 +437,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Four signed 8-bit integers packed in w (byte 0 first) to exact fp32 values.
+// Each byte, offset by 128 (an xor of its sign bit), becomes the low mantissa
+// byte of 2^23: the float 2^23 + (q + 128), from which 2^23 + 128 is
+// subtracted exactly.  One byte permute per value and a packed subtract per
+// pair, with no integer-to-float conversion unit involved.
+__device__ __forceinline__ void i8x4_to_f32(uint32_t w, float (&f)[4]) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint64_t bias = f2_pack(-8388736.f, -8388736.f);
+  const uint64_t lo = f2_add(f2_pack(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540)),
+                                     __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541))),
+                             bias);
+  const uint64_t hi = f2_add(f2_pack(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7542)),
+                                     __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7543))),
+                             bias);
+  f2_unpack(lo, f[0], f[1]);
+  f2_unpack(hi, f[2], f[3]);
+}
+
 }  // namespace rmm

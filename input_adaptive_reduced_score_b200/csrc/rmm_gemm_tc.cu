@@ -16,7 +16,9 @@
 //              release stages and publish finished accumulators.
 //   warps 2-9  epilogue: two warps per TMEM lane quarter, each draining 128
 //              of the 256 columns with tcgen05.ld, converting, and storing rows
-//              of Y with 16-byte stores.
+//              of Y with 16-byte stores.  With an int8 weight (B_I widened to
+//              exact bf16 integers by the gather) the epilogue multiplies each
+//              column by its scale first.
 // All waits are bounded (rmm_device.cuh); on a timeout the kernel records an
 // error, drains its own copies and MMAs, frees TMEM and returns.
 //
@@ -68,6 +70,26 @@ struct Bars {
 static_assert(sizeof(Bars) <= BAR_BYTES, "barrier block");
 
 
+// Multiply 32 accumulator values (columns col0 .. col0+31, masked at N) by
+// their column scales (the per-column scales of an int8 weight).  Every lane
+// of the warp reads the same 32 scales.
+__device__ __forceinline__ void scale_row32(const float* __restrict__ col_scale, int col0, int N, uint32_t (&v)[32]) {
+  if (col0 + 32 <= N && (reinterpret_cast<uintptr_t>(col_scale) & 15) == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 c = __ldg(reinterpret_cast<const float4*>(col_scale + col0) + i);
+      v[4 * i] = __float_as_uint(__uint_as_float(v[4 * i]) * c.x);
+      v[4 * i + 1] = __float_as_uint(__uint_as_float(v[4 * i + 1]) * c.y);
+      v[4 * i + 2] = __float_as_uint(__uint_as_float(v[4 * i + 2]) * c.z);
+      v[4 * i + 3] = __float_as_uint(__uint_as_float(v[4 * i + 3]) * c.w);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      if (col0 + e < N) v[e] = __float_as_uint(__uint_as_float(v[e]) * __ldg(col_scale + col0 + e));
+  }
+}
+
 // Store 32 fp32 accumulator values of one output row (columns col0 ..
 // col0+31, masked at N) as fp32 or bf16, with 16-byte stores when aligned.
 __device__ __forceinline__ void store_row32(void* Y, int out_f32, int64_t ldy, int y_vec_ok, int row, int col0, int N,
@@ -106,7 +128,8 @@ __device__ __forceinline__ void store_row32(void* Y, int out_f32, int64_t ldy, i
 
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b, int M,
-                        int N, int K, void* __restrict__ Y, int out_f32, int64_t ldy, int y_vec_ok, unsigned* err) {
+                        int N, int K, void* __restrict__ Y, int out_f32, int64_t ldy, int y_vec_ok,
+                        const float* __restrict__ col_scale, unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -251,7 +274,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(taddr + cc * 32, v);
         tmem_wait_ld();
         const int col0 = n_blk * BN + half * 128 + cc * 32;
-        if (row < M && col0 < N) store_row32(Y, out_f32, ldy, y_vec_ok, row, col0, N, v);
+        if (row < M && col0 < N) {
+          if (col_scale) scale_row32(col_scale, col0, N, v);
+          store_row32(Y, out_f32, ldy, y_vec_ok, row, col0, N, v);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -322,7 +348,7 @@ __device__ __forceinline__ Item item_of(int i, int split_from, int num_m) {
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
     gemm_bf16_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                              int M, int N, int K, int split_from, void* __restrict__ Y, int out_f32, int64_t ldy,
-                             int y_vec_ok, unsigned* err) {
+                             int y_vec_ok, const float* __restrict__ col_scale, unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -478,7 +504,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
         tmem_ld32(taddr + cc * 32, v);
         tmem_wait_ld();
         const int col0 = t.n0 + half * hw + cc * 32;
-        if (row < M && col0 < N) store_row32(Y, out_f32, ldy, y_vec_ok, row, col0, N, v);
+        if (row < M && col0 < N) {
+          if (col_scale) scale_row32(col_scale, col0, N, v);
+          store_row32(Y, out_f32, ldy, y_vec_ok, row, col0, N, v);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -553,7 +582,8 @@ bool encode_2d(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, in
 }  // namespace
 
 cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I, int64_t ld_bi, int64_t M, int64_t N,
-                                int64_t k, void* Y, int out_dtype, int64_t ldy, unsigned* err, cudaStream_t stream) {
+                                int64_t k, void* Y, int out_dtype, int64_t ldy, unsigned* err, cudaStream_t stream,
+                                const float* col_scale) {
   if (M == 0 || N == 0) return cudaSuccess;
   CUtensorMap tmap_a, tmap_b;
   if (!encode_2d(&tmap_a, A_I, k, M, ld_ai, BK, BM, "A_I")) return cudaErrorInvalidValue;
@@ -578,12 +608,13 @@ cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I,
     const int clusters = static_cast<int>(items < pairs ? items : pairs);
     return launch_pdl(gemm_bf16_tc_pair_kernel, dim3(2 * clusters), dim3(pairk::THREADS), pairk::SMEM_BYTES,
                       stream, tmap_a, tmap_b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(k),
-                      static_cast<int>(split_from), Y, out_f32, ldy, y_vec_ok, err);
+                      static_cast<int>(split_from), Y, out_f32, ldy, y_vec_ok, col_scale, err);
   }
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   return launch_pdl(gemm_bf16_tc_kernel, dim3(grid), dim3(THREADS), SMEM_BYTES, stream, tmap_a, tmap_b,
-                    static_cast<int>(M), static_cast<int>(N), static_cast<int>(k), Y, out_f32, ldy, y_vec_ok, err);
+                    static_cast<int>(M), static_cast<int>(N), static_cast<int>(k), Y, out_f32, ldy, y_vec_ok, col_scale,
+                    err);
 }
 
 }  // namespace rmm

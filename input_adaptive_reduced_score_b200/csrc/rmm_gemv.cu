@@ -16,6 +16,11 @@
 // of the outputs, in split order, through distributed shared memory; beyond 8
 // splits the sums go through global memory and a second kernel adds them in
 // split order.  Either way the result depends only on the shape.
+//
+// An int8 weight (weight-only quantisation with one fp32 scale per output
+// column; Resultados Experimentales › Compatibilidad) takes the same path
+// with half the bytes per row: each lane loads 8 (or 4) int8 values, widens
+// them exactly to fp32, and the column scale multiplies the finished sum.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -36,25 +41,29 @@ constexpr int kGemvMaxCluster = 8;  // splits reduced through distributed shared
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Columns per lane: 8 (16-byte loads) up to 8 activation rows, else 4
-// (8-byte loads), so the accumulators stay at MT x CPL <= 64 registers.
-template <int MT>
+// Columns per lane: 8 up to 8 activation rows, else 4, so the accumulators
+// stay at MT x CPL <= 64 registers; a lane's load is CPL weights (16 or 8
+// bytes of bf16, 8 or 4 bytes of int8).
+template <int MT, bool kW8 = false>
 struct GemvShape {
   static constexpr int CPL = MT <= 8 ? 8 : 4;
   static constexpr int COLS = 32 * CPL;            // columns of Y per block
   static constexpr int U = MT == 8 ? 4 : 8;        // rows per batch (two batches in flight per warp)
-  using Vec = typename std::conditional<CPL == 8, uint4, uint2>::type;
+  using Vec16 = typename std::conditional<CPL == 8, uint4, uint2>::type;
+  using Vec8 = typename std::conditional<CPL == 8, uint2, unsigned int>::type;
+  using Vec = typename std::conditional<kW8, Vec8, Vec16>::type;
 };
 
 // grid: x = column slice, y = row split.  Dynamic shared memory:
 // max(rows x (MT + 1), warps x MT x COLS) words.
-template <int MT>
+// kW8: B is int8 (ldb in bytes) and b_scale[c] multiplies column c.
+template <int MT, bool kW8>
 __global__ void __launch_bounds__(kGemvThreads, 2)
-    gemv_rows_kernel(const uint16_t* __restrict__ AI, int64_t ld_ai, const uint16_t* __restrict__ B, int64_t ldb,
-                     const int32_t* __restrict__ idx, int M, int64_t d, int64_t N, int64_t k, int rows_per_split,
-                     float* __restrict__ partial, void* __restrict__ Y, int out_f32, int64_t ldy, int clustered,
-                     unsigned* err) {
-  using Sh = GemvShape<MT>;
+    gemv_rows_kernel(const uint16_t* __restrict__ AI, int64_t ld_ai, const void* __restrict__ Bv, int64_t ldb,
+                     const float* __restrict__ b_scale, const int32_t* __restrict__ idx, int M, int64_t d, int64_t N,
+                     int64_t k, int rows_per_split, float* __restrict__ partial, void* __restrict__ Y, int out_f32,
+                     int64_t ldy, int clustered, unsigned* err) {
+  using Sh = GemvShape<MT, kW8>;
   using Vec = typename Sh::Vec;
   constexpr int CPL = Sh::CPL, COLS = Sh::COLS, U = Sh::U;
   extern __shared__ __align__(16) float sm[];
@@ -99,7 +108,12 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
       w[u] = Vec{};
       if (rr < nrows) {
         const int32_t j = sidx[rr];
-        if (j >= 0 && col_ok) w[u] = __ldcs(reinterpret_cast<const Vec*>(B + static_cast<int64_t>(j) * ldb + c0));
+        if (j >= 0 && col_ok) {
+          if constexpr (kW8)
+            w[u] = __ldcs(reinterpret_cast<const Vec*>(static_cast<const int8_t*>(Bv) + static_cast<int64_t>(j) * ldb + c0));
+          else
+            w[u] = __ldcs(reinterpret_cast<const Vec*>(static_cast<const uint16_t*>(Bv) + static_cast<int64_t>(j) * ldb + c0));
+        }
       }
     }
   };
@@ -110,10 +124,20 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
       if (rr < nrows) {
         float b[CPL];
         const uint32_t* wv = reinterpret_cast<const uint32_t*>(&w[u]);
+        if constexpr (kW8) {
 #pragma unroll
-        for (int q = 0; q < CPL / 2; ++q) {
-          b[2 * q] = bf16_lo(wv[q]);
-          b[2 * q + 1] = bf16_hi(wv[q]);
+          for (int q = 0; q < CPL / 4; ++q) {
+            float f[4];
+            i8x4_to_f32(wv[q], f);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) b[4 * q + e] = f[e];
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < CPL / 2; ++q) {
+            b[2 * q] = bf16_lo(wv[q]);
+            b[2 * q + 1] = bf16_hi(wv[q]);
+          }
         }
         const float* a = sm + rr * MT;
 #pragma unroll
@@ -169,6 +193,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
     const int m = e / COLS, cl = e % COLS;
     const int64_t c = static_cast<int64_t>(blockIdx.x) * COLS + cl;
     if (m >= M || c >= N) return;
+    if constexpr (kW8) v *= __ldg(b_scale + c);
     if (out_f32) {
       static_cast<float*>(Y)[static_cast<int64_t>(m) * ldy + c] = v;
     } else {
@@ -200,9 +225,11 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
   }
 }
 
-// Y[m, c] = sum over splits (in order) of partial[split][m][c].
+// Y[m, c] = sum over splits (in order) of partial[split][m][c], times
+// b_scale[c] when given.
 __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float* __restrict__ partial, int splits, int M,
-                                                          int64_t N, void* __restrict__ Y, int out_f32, int64_t ldy) {
+                                                          int64_t N, const float* __restrict__ b_scale,
+                                                          void* __restrict__ Y, int out_f32, int64_t ldy) {
   pdl_wait();
   pdl_trigger();
   const int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
@@ -211,6 +238,7 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float* __restric
   const int64_t c = e % N;
   float s = 0.f;
   for (int t = 0; t < splits; ++t) s += __ldg(partial + static_cast<int64_t>(t) * M * N + e);
+  if (b_scale) s *= __ldg(b_scale + c);
   if (out_f32) {
     static_cast<float*>(Y)[static_cast<int64_t>(m) * ldy + c] = s;
   } else {
@@ -236,15 +264,16 @@ GemvPlan plan_mt(int64_t M, int64_t N, int64_t k, int sms) {
   return p;
 }
 
-template <int MT>
-cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const uint16_t* B, int64_t ldb, const int32_t* idx,
-                           int M, int64_t d, int64_t N, int64_t k, const GemvPlan& pl, float* partial, void* Y,
-                           int out_f32, int64_t ldy, unsigned* err, cudaStream_t stream) {
+template <int MT, bool kW8>
+cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const void* B, int64_t ldb, const float* b_scale,
+                           const int32_t* idx, int M, int64_t d, int64_t N, int64_t k, const GemvPlan& pl,
+                           float* partial, void* Y, int out_f32, int64_t ldy, unsigned* err, cudaStream_t stream) {
   const size_t smem =
       static_cast<size_t>(std::max(pl.rows_per_split * (MT + 1), kGemvWarps * MT * GemvShape<MT>::COLS)) * 4;
   if (smem > 48 * 1024) {
     const cudaError_t e =
-        cudaFuncSetAttribute(gemv_rows_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaFuncSetAttribute(gemv_rows_kernel<MT, kW8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
   const dim3 grid(static_cast<unsigned>(pl.slices), static_cast<unsigned>(pl.splits));
@@ -264,16 +293,16 @@ cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const uint16_t* B,
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, gemv_rows_kernel<MT>, AI, ld_ai, B, ldb, idx, M, d, N, k, pl.rows_per_split, partial, Y,
-                           out_f32, ldy, 1, err);
+    e = cudaLaunchKernelEx(&cfg, gemv_rows_kernel<MT, kW8>, AI, ld_ai, B, ldb, b_scale, idx, M, d, N, k,
+                           pl.rows_per_split, partial, Y, out_f32, ldy, 1, err);
     return e;
   }
-  e = launch_pdl(gemv_rows_kernel<MT>, grid, dim3(kGemvThreads), smem, stream, AI, ld_ai, B, ldb, idx, M, d, N, k,
-                 pl.rows_per_split, partial, Y, out_f32, ldy, 0, err);
+  e = launch_pdl(gemv_rows_kernel<MT, kW8>, grid, dim3(kGemvThreads), smem, stream, AI, ld_ai, B, ldb, b_scale, idx,
+                 M, d, N, k, pl.rows_per_split, partial, Y, out_f32, ldy, 0, err);
   if (e != cudaSuccess || pl.splits == 1) return e;
   const int64_t outs = static_cast<int64_t>(M) * N;
   return launch_pdl(gemv_reduce_kernel, dim3(static_cast<unsigned>((outs + 255) / 256)), dim3(256), 0, stream,
-                    static_cast<const float*>(partial), pl.splits, M, N, Y, out_f32, ldy);
+                    static_cast<const float*>(partial), pl.splits, M, N, kW8 ? b_scale : nullptr, Y, out_f32, ldy);
 }
 
 }  // namespace
@@ -288,17 +317,24 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t k, int sms) {
 
 cudaError_t launch_gemv(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, const int32_t* idx, int64_t M,
                         int64_t d, int64_t N, int64_t k, const GemvPlan& pl, float* partial, void* Y, int out_dtype,
-                        int64_t ldy, unsigned* err, cudaStream_t stream) {
+                        int64_t ldy, unsigned* err, cudaStream_t stream, const float* b_scale) {
   if (M == 0 || N == 0) return cudaSuccess;
   const uint16_t* ai = static_cast<const uint16_t*>(A_I);
-  const uint16_t* b = static_cast<const uint16_t*>(B);
   const int out_f32 = out_dtype == 0 ? 1 : 0;
   const int m = static_cast<int>(M);
-  if (M <= 1) return launch_gemv_mt<1>(ai, ld_ai, b, ldb, idx, m, d, N, k, pl, partial, Y, out_f32, ldy, err, stream);
-  if (M <= 2) return launch_gemv_mt<2>(ai, ld_ai, b, ldb, idx, m, d, N, k, pl, partial, Y, out_f32, ldy, err, stream);
-  if (M <= 4) return launch_gemv_mt<4>(ai, ld_ai, b, ldb, idx, m, d, N, k, pl, partial, Y, out_f32, ldy, err, stream);
-  if (M <= 8) return launch_gemv_mt<8>(ai, ld_ai, b, ldb, idx, m, d, N, k, pl, partial, Y, out_f32, ldy, err, stream);
-  return launch_gemv_mt<16>(ai, ld_ai, b, ldb, idx, m, d, N, k, pl, partial, Y, out_f32, ldy, err, stream);
+  auto go = [&](auto mt) {
+    constexpr int MT = decltype(mt)::value;
+    if (b_scale)
+      return launch_gemv_mt<MT, true>(ai, ld_ai, B, ldb, b_scale, idx, m, d, N, k, pl, partial, Y, out_f32, ldy, err,
+                                      stream);
+    return launch_gemv_mt<MT, false>(ai, ld_ai, B, ldb, nullptr, idx, m, d, N, k, pl, partial, Y, out_f32, ldy, err,
+                                     stream);
+  };
+  if (M <= 1) return go(std::integral_constant<int, 1>{});
+  if (M <= 2) return go(std::integral_constant<int, 2>{});
+  if (M <= 4) return go(std::integral_constant<int, 4>{});
+  if (M <= 8) return go(std::integral_constant<int, 8>{});
+  return go(std::integral_constant<int, 16>{});
 }
 
 }  // namespace rmm

@@ -58,19 +58,28 @@ cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64
 cudaError_t launch_gather_rows(const void* B, int64_t d, int64_t row_bytes, int64_t ldb_bytes, const int32_t* idx,
                                int64_t k, void* B_I, int64_t ldbi_bytes, unsigned* err, cudaStream_t stream);
 
-// Both reduced operands in one launch (bf16): A_I = A[:, idx] and
-// B_I = B[idx, :]; B, B_I bases and pitches 16-byte aligned, N even.
+// Both reduced operands in one launch (bf16 A): A_I = A[:, idx] and
+// B_I = B[idx, :]; B, B_I bases and pitches 16-byte aligned.  b_int8: B is
+// int8 [d x N] (ldb in bytes, a multiple of 16) and B_I is written as bf16.
 cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64_t lda, const void* B, int64_t N,
                                       int64_t ldb, const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai,
-                                      void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream);
+                                      void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream,
+                                      bool b_int8 = false);
+
+// Row gather of an int8 B [d x N] (ldb bytes, multiple of 16; 16-byte aligned)
+// into bf16 B_I [k x N] (ld_bi elements, multiple of 8; 16-byte aligned).
+cudaError_t launch_gather_rows_i8(const void* Bq, int64_t d, int64_t N, int64_t ldb, const int32_t* idx, int64_t k,
+                                  void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream);
 
 // ---- reduced GEMM (rmm_gemm_tc.cu, rmm_gemm_simt.cu)
 // Returns cudaSuccess or an error; on a driver error in tensor-map encoding
 // the message is set and cudaErrorInvalidValue returned.
 // Dense tcgen05 GEMM on the compacted operands: Y = A_I [M x k] · B_I [k x N].
+// col_scale (may be null): fp32 [N], multiplies column n of the product
+// before it is stored (the per-column scales of an int8 weight).
 cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I, int64_t ld_bi, int64_t M,
                                 int64_t N, int64_t k, void* Y, int out_dtype, int64_t ldy, unsigned* err,
-                                cudaStream_t stream);
+                                cudaStream_t stream, const float* col_scale = nullptr);
 cudaError_t launch_gemm_f32_simt(const float* A_I, int64_t ld_ai, const float* B, int64_t ldb,
                                  const int32_t* idx, int64_t d, int64_t M, int64_t N, int64_t k,
                                  float* Y, int64_t ldy, unsigned* err, cudaStream_t stream);
@@ -85,10 +94,12 @@ struct GemvPlan {
   size_t partial_bytes;  // fp32 partial sums in global memory (0 with one split or a cluster)
 };
 GemvPlan gemv_plan(int64_t M, int64_t N, int64_t k, int sms);
-// A_I bf16 [M x k] (ld_ai), B bf16 [d x N] (ldb, rows 8-byte aligned), idx [k].
+// A_I bf16 [M x k] (ld_ai), B bf16 [d x N] (ldb, rows 16-byte aligned), idx [k].
+// b_scale non-null: B is int8 (ldb bytes, rows 16-byte aligned) and column n
+// of the product is multiplied by b_scale[n].
 cudaError_t launch_gemv(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, const int32_t* idx, int64_t M,
                         int64_t d, int64_t N, int64_t k, const GemvPlan& plan, float* partial, void* Y, int out_dtype,
-                        int64_t ldy, unsigned* err, cudaStream_t stream);
+                        int64_t ldy, unsigned* err, cudaStream_t stream, const float* b_scale = nullptr);
 
 // ---- reduced attention (rmm_attention.cu)
 size_t attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D, int64_t kd,

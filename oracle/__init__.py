@@ -22,5 +22,6 @@ functions are pinned to those readings, and the readings themselves are
 """
 from . import rmm, attention, conditioning  # noqa: F401
 from .rmm import (k_from_rho, column_sq_norms, column_norms, topk_indices,  # noqa: F401
-                  reduced_matmul, dense_matmul, rmm as rmm_path, decode)
+                  reduced_matmul, dense_matmul, rmm as rmm_path, decode,
+                  dequantize_w8, reduced_matmul_w8, rmm_w8)
 from .attention import reduced_attention, attention_head, kv_head_of  # noqa: F401

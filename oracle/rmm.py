@@ -20,7 +20,8 @@ import math
 import numpy as np
 
 __all__ = ["k_from_rho", "column_sq_norms", "column_norms", "topk_indices",
-           "reduced_matmul", "dense_matmul", "rmm", "decode"]
+           "reduced_matmul", "dense_matmul", "rmm", "decode", "dequantize_w8",
+           "reduced_matmul_w8", "rmm_w8"]
 
 
 def decode(x, dtype: str) -> np.ndarray:
@@ -117,3 +118,51 @@ def rmm(A, B, rho: float):
     k = k_from_rho(rho, A.shape[1])
     idx = topk_indices(ss, k)
     return reduced_matmul(A, B, idx), idx, ss
+
+
+def dequantize_w8(Bq, scale) -> np.ndarray:
+    """The weight an int8 matrix stands for: B[j, n] = Bq[j, n] * scale[n], fp64.
+
+    Resultados Experimentales › Compatibilidad: the method is reported to work
+    with INT8 weight quantisation.  READING (the page names no scheme):
+    symmetric weight-only quantisation with one scale per output column n of
+    the [d x N] weight, no zero point.
+    """
+    q = np.asarray(Bq)
+    if q.dtype != np.int8:
+        raise ValueError("Bq must be int8")
+    s = np.asarray(scale, dtype=np.float64)
+    if s.ndim != 1 or s.shape[0] != q.shape[1]:
+        raise ValueError("one scale per column of Bq")
+    if not np.all(np.isfinite(s)):
+        raise ValueError("non-finite scale")
+    return q.astype(np.float64) * s[None, :]
+
+
+def reduced_matmul_w8(A, Bq, scale, idx) -> np.ndarray:
+    """Y = A[:, I] B[I, :] with B the int8 weight's dequantised values, fp64.
+
+    Metodología › Mecanismo Central (the reduced product) applied to the
+    weight of Resultados Experimentales › Compatibilidad (see dequantize_w8).
+    The rows are restricted to I first, then dequantised.
+    """
+    idx = np.asarray(idx, dtype=np.int64)
+    q = np.asarray(Bq)
+    A = np.asarray(A, dtype=np.float64)
+    if A.shape[1] != q.shape[0]:
+        raise ValueError("contraction dimensions differ")
+    return A[:, idx] @ dequantize_w8(q[idx, :], scale)
+
+
+def rmm_w8(A, Bq, scale, rho: float):
+    """Whole path with an int8 weight: scores of A -> top-k -> reduced product.
+
+    The selection reads only the activation (Metodología › Estrategia de
+    Selección), so it is the same index set as for any other weight.
+    Returns (Y, I, ss).
+    """
+    A = np.asarray(A, dtype=np.float64)
+    ss = column_sq_norms(A)
+    k = k_from_rho(rho, A.shape[1])
+    idx = topk_indices(ss, k)
+    return reduced_matmul_w8(A, Bq, scale, idx), idx, ss

@@ -250,3 +250,109 @@ def test_pins_catch_planted_mistakes():
     assert not _pins_hold(reduced=lambda A, B, i: A[:, i[:-1]] @ B[i[:-1], :])
     # off-by-one in the gather
     assert not _pins_hold(reduced=lambda A, B, i: A[:, i] @ B[np.minimum(i + 1, B.shape[0] - 1), :])
+
+
+# ------------------------------------------------------------------ int8 weight
+
+
+def _w8_bruteforce(A, Bq, scale, rho):
+    """Whole int8-weight path by enumeration and explicit loops: the k-subset
+    with the largest sum of squared column norms (lowest indices first among
+    equals), then Y[m][n] = sum over kept j of A[m][j] * Bq[j][n] * scale[n]."""
+    M, d = A.shape
+    N = Bq.shape[1]
+    k = math.ceil(rho * d - 1e-9 * d)
+    ss = [sum(A[m][j] ** 2 for m in range(M)) for j in range(d)]
+    best = None
+    for sub in itertools.combinations(range(d), k):
+        key = (-sum(ss[j] for j in sub), sub)
+        if best is None or key < best:
+            best = key
+    I = best[1]
+    Y = [[0.0] * N for _ in range(M)]
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for j in I:
+                acc += A[m][j] * float(Bq[j][n]) * float(scale[n])
+            Y[m][n] = acc
+    return np.array(Y), np.array(I)
+
+
+@pytest.mark.parametrize("trial", range(4))
+def test_w8_bruteforce_small(trial):
+    rng = np.random.default_rng(100 + trial)
+    M, d, N = 3, 8, 5
+    A = rng.standard_normal((M, d)) * rng.uniform(0.2, 3.0, size=d)[None, :]
+    Bq = rng.integers(-127, 128, size=(d, N)).astype(np.int8)
+    scale = rng.uniform(1e-3, 5e-2, size=N).astype(np.float32)
+    for rho in (0.25, 0.5, 0.75):
+        Y, idx, _ = O.rmm_w8(A, Bq, scale, rho)
+        Yb, Ib = _w8_bruteforce(A, Bq, scale, rho)
+        np.testing.assert_array_equal(idx, Ib)
+        np.testing.assert_allclose(Y, Yb, rtol=1e-12, atol=1e-15)
+
+
+def test_w8_rho_one_factors_column_scale():
+    """rho = 1: the product is the dense int8 product with column n scaled by
+    scale[n] afterwards (distributivity; pins per-column, not per-row, scales)."""
+    rng = np.random.default_rng(11)
+    A = rng.standard_normal((6, 9))
+    Bq = rng.integers(-127, 128, size=(9, 7)).astype(np.int8)
+    scale = rng.uniform(0.5, 2.0, size=7).astype(np.float32)
+    Y, idx, _ = O.rmm_w8(A, Bq, scale, 1.0)
+    np.testing.assert_array_equal(idx, np.arange(9))
+    dense_int = np.einsum("mj,jn->mn", A, Bq.astype(np.float64))
+    np.testing.assert_allclose(Y, dense_int * scale.astype(np.float64)[None, :], rtol=1e-13, atol=1e-13)
+
+
+def test_w8_unit_scale_is_plain_reduced_product():
+    rng = np.random.default_rng(12)
+    A = rng.standard_normal((4, 10)) * np.arange(1, 11)[None, :]
+    Bq = rng.integers(-127, 128, size=(10, 3)).astype(np.int8)
+    Y, idx, _ = O.rmm_w8(A, Bq, np.ones(3, np.float32), 0.4)
+    Y2, idx2, _ = O.rmm(A, Bq.astype(np.float64), 0.4)
+    np.testing.assert_array_equal(idx, idx2)
+    np.testing.assert_array_equal(Y, Y2)
+
+
+@pytest.mark.parametrize("rho", [0.3, 0.6])
+def test_w8_error_bound(rho):
+    """The error bound of the reduced product holds for the dequantised weight."""
+    rng = np.random.default_rng(13)
+    A = rng.standard_normal((16, 24)) * np.exp(rng.standard_normal(24))[None, :]
+    Bq, scale = W.weight_int8(5, 24, 11)
+    B = O.dequantize_w8(Bq, scale)
+    Y, idx, _ = O.rmm_w8(A, Bq, scale, rho)
+    rest = np.setdiff1d(np.arange(24), idx)
+    err = np.linalg.norm(A @ B - Y)
+    assert err <= np.linalg.norm(A[:, rest]) * np.linalg.norm(B[rest, :], 2) * (1 + 1e-9)
+
+
+def test_weight_int8_is_absmax_storage():
+    """Generated int8 weights use the full symmetric range per column."""
+    q, s = W.weight_int8(3, 200, 33)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert np.all(np.abs(q.astype(np.int32)) <= 127)
+    assert np.all(np.max(np.abs(q.astype(np.int32)), axis=0) == 127)
+    assert np.all(s > 0)
+
+
+def test_w8_pins_catch_planted_mistakes():
+    """Each plausible mistake in the int8 product fails the brute-force pin."""
+    rng = np.random.default_rng(200)
+    M, d, N = 3, 8, 5
+    A = rng.standard_normal((M, d)) * rng.uniform(0.2, 3.0, size=d)[None, :]
+    Bq = rng.integers(-127, 128, size=(d, N)).astype(np.int8)
+    scale = rng.uniform(1e-3, 5e-2, size=N).astype(np.float32)
+    Yb, Ib = _w8_bruteforce(A, Bq, scale, 0.5)
+
+    def holds(prod):
+        Y = prod(A[:, Ib], Bq[Ib, :].astype(np.float64), scale.astype(np.float64))
+        return np.allclose(Y, Yb, rtol=1e-12, atol=1e-15)
+
+    assert holds(lambda a, q, s: a @ (q * s[None, :]))
+    assert not holds(lambda a, q, s: a @ q)                                       # scale dropped
+    assert not holds(lambda a, q, s: a @ (q * s[0]))                              # first column's scale for all
+    assert not holds(lambda a, q, s: (a @ q) / s[None, :])                        # scale inverted
+    assert not holds(lambda a, q, s: a @ (q * np.resize(s, q.shape[0])[:, None]))  # per-row scale

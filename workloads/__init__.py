@@ -50,7 +50,7 @@ def bf16_bits_to_f32(bits) -> np.ndarray:
 
 TENSOR_IDS = {
     "A": 1, "B": 2, "X": 3, "W": 4, "G": 5, "U": 6, "Q": 7, "K": 8, "V": 9,
-    "colscale": 10, "outliers": 11, "qscale": 12, "kscale": 13, "vscale": 14,
+    "colscale": 10, "outliers": 11, "qscale": 12, "kscale": 13, "vscale": 14, "W8": 15,
 }
 
 
@@ -188,6 +188,28 @@ def scaled_matmul_bf16(seed: int, M: int, d: int, N: int, rhos=(0.5,), outlier_f
     X = llm_activation_bf16(seed, M, d, outlier_frac=outlier_frac)
     W = weight_bf16(seed, d, N, std=0.02)
     return MatmulInputs(f"bf16 {M}x{d}x{N}", "bf16", X, W, tuple(rhos), seed)
+
+
+def weight_int8(seed: int, rows: int, cols: int, std: float = 0.02, group: int = 0):
+    """Int8 weight [rows x cols] with one fp32 scale per column, stored the way
+    a symmetric absmax quantiser stores an N(0, std^2) weight:
+    scale[n] = max_j |W[j, n]| / 127 (rounded to fp32), q = W / scale[n]
+    rounded half-to-even and clipped to [-127, 127].  Returns (q int8, scale
+    fp32).  Weight storage format only; nothing of the reduced product."""
+    W = _normal(substream(seed, "W8", group), (rows, cols)) * std
+    scale = (np.max(np.abs(W), axis=0) / 127.0).astype(np.float32)
+    q = np.clip(np.rint(W / scale.astype(np.float64)[None, :]), -127, 127).astype(np.int8)
+    return q, scale
+
+
+def mlp_up_w8(seed: int = 1, tokens: int = 4096, hidden: int = 4096, ffn: int = 14336) -> MatmulInputs:
+    """MLP up/gate projection with an int8 weight: X as in ``mlp_up`` (bf16) and
+    W [hidden x ffn] int8 with per-column scales (``weight_int8``), which are
+    kept in ``meta["b_scale"]``."""
+    X = llm_activation_bf16(seed, tokens, hidden)
+    q, scale = weight_int8(seed, hidden, ffn)
+    return MatmulInputs(f"MLP up/gate projection {tokens}x{hidden}x{ffn} bf16 x int8", "bf16", X, q,
+                        (0.5,), seed, meta={"b_scale": scale})
 
 
 @dataclass
