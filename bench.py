@@ -53,8 +53,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["bench", "attention", "decode"], default="bench",
-                    help="attention / decode: run only that workload a few times and exit (a short "
+    ap.add_argument("--case", choices=["bench", "attention", "decode", "w8"], default="bench",
+                    help="attention / decode / w8: run only that workload a few times and exit (a short "
                          "program for profiler captures; prints no JSON line)")
     a = ap.parse_args()
     if a.warmup < 3:
@@ -363,6 +363,64 @@ def measure_decode(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, 
     return out
 
 
+def measure_w8(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, X, hbm_gbs):
+    """The same products with an int8 weight (per-column fp32 scales):
+    rmm_matmul_w8 on the MLP up/gate activation (selection, one launch that
+    compacts A and widens the kept int8 rows to bf16, the tensor-core product
+    with the scales in its epilogue), and the decode product on 1 and 16 rows
+    (kept int8 rows read in place).  Product bandwidth counts its algorithmic
+    bytes: k kept int8 rows, the scales, A_I and Y."""
+    import torch
+    q, sc = workloads.weight_int8(1, D, N)
+    Wq = torch.from_numpy(q).to(dev)
+    S = torch.from_numpy(sc).to(dev)
+    k = R.rmm_k_from_rho(RHO, D)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    mws = torch.empty(R.rmm_matmul_w8_workspace_size(M, D, N, RHO), dtype=torch.uint8, device=dev)
+
+    def path(ev):
+        ev[0].record(stream)
+        R.rmm_matmul_w8(X, Wq, S, RHO, out=Y, ws=mws)
+        ev[1].record(stream)
+    for _ in range(3):
+        path([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    ms = statistics.mean(p[0] for p in timed(path, steps, 2))
+    out = {"prefill": {"ms": ms, "effective_tflops": 2.0 * M * N * k / (ms * 1e-3) / 1e12,
+                       "gpu_launches_per_call": 4}}
+    gws = torch.empty(R.rmm_gemm_w8_workspace_size(N, k), dtype=torch.uint8, device=dev)
+    for rows in (1, 16):
+        Xr = bf16_tensor(workloads.llm_activation_bf16(7 + rows, rows, D), dev)
+        idx = torch.empty(k, dtype=torch.int32, device=dev)
+        Yr = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+        rws = torch.empty(R.rmm_matmul_w8_workspace_size(rows, D, N, RHO), dtype=torch.uint8, device=dev)
+
+        def step(ev):
+            ev[0].record(stream)
+            R.rmm_matmul_w8(Xr, Wq, S, RHO, out=Yr, idx_out=idx, ws=rws)
+            ev[1].record(stream)
+        for _ in range(3):
+            step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        AI = R.rmm_compact(Xr, idx)
+
+        def product(ev):
+            ev[0].record(stream)
+            R.rmm_gemm_w8(AI, Wq, S, idx, out=Yr, ws=gws)
+            ev[1].record(stream)
+        for _ in range(3):
+            product([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        step_ms = statistics.mean(p[0] for p in timed(step, steps, 2))
+        prod_ms = statistics.mean(p[0] for p in timed(product, steps, 2))
+        prod_bytes = 1.0 * k * N + 4.0 * N + 2.0 * rows * k + 2.0 * rows * N
+        gbs = prod_bytes / (prod_ms * 1e-3) / 1e9
+        out[f"M{rows}"] = {"step_us": step_ms * 1e3, "product_us": prod_ms * 1e3, "product_GB/s": gbs,
+                           "product_frac_hbm": gbs / hbm_gbs}
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the int8-weight runs")
+    out["workload"] = (f"X[{M} or 1 or 16 x {D}] bf16 . W[{D}x{N}] int8 with per-column fp32 scales "
+                       f"(symmetric absmax storage of N(0, 0.02^2)), rho={RHO}; 256 MiB flush between steps")
+    return out
+
+
 def run_rmm(args):
     import numpy as np
     import torch
@@ -500,6 +558,7 @@ def run_rmm(args):
     peaks, peak_src = load_peaks()
     decode = measure_decode(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed, Wt,
                             peaks["hbm_gbs"])
+    w8 = measure_w8(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed, X, peaks["hbm_gbs"])
     gemm_ms = stage_ms["gemm"]
     achieved = flops_step / (gemm_ms * 1e-3) / 1e12
     traffic = traffic_per_launch()
@@ -544,6 +603,7 @@ def run_rmm(args):
             "gpu_launches": launches_per_step * args.steps,
             "attention": attention,
             "decode": decode,
+            "int8_weight": w8,
             "clocks": clk.summary(), "clock_remeasured": remeasured,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -573,6 +633,23 @@ def run_case(case):
                                                         a["rho_t"]), dtype=torch.uint8, device=dev)
         for _ in range(3):
             R.rmm_attention(Q, K, V, a["rho_d"], a["rho_t"], out=O, ws=ws)
+    elif case == "w8":
+        q, sc = workloads.weight_int8(1, D, N)
+        Wq, S = torch.from_numpy(q).to(dev), torch.from_numpy(sc).to(dev)
+        X = bf16_tensor(workloads.llm_activation_bf16(1, M, D), dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            flush.zero_()
+            R.rmm_matmul_w8(X, Wq, S, RHO, out=Y)
+        k = R.rmm_k_from_rho(RHO, D)
+        idx = torch.from_numpy(np.sort(np.random.default_rng(0).choice(D, k, replace=False)).astype(np.int32)).to(dev)
+        for rows in (1, 16):
+            AI = R.rmm_compact(bf16_tensor(workloads.llm_activation_bf16(7, rows, D), dev), idx)
+            Yr = torch.empty((rows, N), dtype=torch.bfloat16, device=dev)
+            for _ in range(12):
+                flush.zero_()
+                R.rmm_gemm_w8(AI, Wq, S, idx, out=Yr)
     else:
         k = R.rmm_k_from_rho(RHO, D)
         Wt = bf16_tensor(workloads.weight_bf16(1, D, N), dev)

@@ -21,6 +21,13 @@
 // column; Resultados Experimentales › Compatibilidad) takes the same path
 // with half the bytes per row: each lane loads 8 (or 4) int8 values, widens
 // them exactly to fp32, and the column scale multiplies the finished sum.
+//
+// Up to 8 activation rows the rows are streamed rather than loaded into
+// registers (gemv_stream_kernel): each warp keeps six stages of four kept
+// rows in flight as 16-byte asynchronous copies into its own ring in shared
+// memory, so a block has 192 rows in flight without holding them in
+// registers.  The register-loading kernel serves 9 to 16 rows, where the
+// FMAs rather than the loads set the time.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -48,7 +55,10 @@ template <int MT, bool kW8 = false>
 struct GemvShape {
   static constexpr int CPL = MT <= 8 ? 8 : 4;
   static constexpr int COLS = 32 * CPL;            // columns of Y per block
-  static constexpr int U = MT == 8 ? 4 : 8;        // rows per batch (two batches in flight per warp)
+  // rows per batch (two batches in flight per warp); int8 rows are half the
+  // bytes, so up to 4 activation rows they take twice the batch in the same
+  // registers
+  static constexpr int U = (MT == 8 ? 4 : 8) * (kW8 && MT <= 4 ? 2 : 1);
   using Vec16 = typename std::conditional<CPL == 8, uint4, uint2>::type;
   using Vec8 = typename std::conditional<CPL == 8, uint2, unsigned int>::type;
   using Vec = typename std::conditional<kW8, Vec8, Vec16>::type;
@@ -225,6 +235,231 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
   }
 }
 
+// ---------------------------------------------------------------- streamed rows (M <= 8)
+
+constexpr int kStreamWarps = 8;
+constexpr int kStreamThreads = 32 * kStreamWarps;
+constexpr int kStreamRowsPerStage = 4;              // kept rows per stage of a warp
+constexpr int kStreamStages = 6;                    // stages in flight per warp
+constexpr int kStreamCols = 256;                    // columns of Y per block
+constexpr int kStreamAiBytes = 16 * 1024;           // A_I staging (fp32 [row][m]) per block: two blocks fit an SM
+
+template <bool kW8>
+constexpr int stream_row_bytes() { return kStreamCols * (kW8 ? 1 : 2); }
+
+template <bool kW8>
+constexpr size_t stream_ring_bytes() {
+  return static_cast<size_t>(kStreamWarps) * kStreamStages * kStreamRowsPerStage * stream_row_bytes<kW8>();
+}
+
+// Dynamic shared memory: each warp's ring of stages, then A_I as fp32
+// [row][MT], then the rows' indices; the warp sums of the epilogue reuse the
+// start of it once every copy has landed.
+template <int MT, bool kW8>
+size_t stream_smem_bytes(int rows_per_split) {
+  const size_t stage_ai = static_cast<size_t>(rows_per_split) * (MT + 1) * 4;
+  const size_t red = static_cast<size_t>(kStreamWarps) * MT * kStreamCols * 4;
+  return std::max(stream_ring_bytes<kW8>() + stage_ai, red);
+}
+
+// 16-byte asynchronous copy global -> shared; src_bytes < 16 fills the rest
+// with zeros (0: no read at all).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// grid: x = column slice of 256, y = row split.  Warp w takes the split's
+// kept rows w, w + 8, w + 16, ..., four per stage, and keeps six stages of
+// 16-byte asynchronous copies in flight (no registers held, no copy engine
+// requests); a row whose index is out of range is copied as zeros.
+template <int MT, bool kW8>
+__global__ void __launch_bounds__(kStreamThreads, 2)
+    gemv_stream_kernel(const uint16_t* __restrict__ AI, int64_t ld_ai, const void* __restrict__ Bv, int64_t ldb,
+                       const float* __restrict__ b_scale, const int32_t* __restrict__ idx, int M, int64_t d,
+                       int64_t N, int64_t k, int rows_per_split, float* __restrict__ partial, void* __restrict__ Y,
+                       int out_f32, int64_t ldy, int clustered, unsigned* err) {
+  constexpr int ELT = kW8 ? 1 : 2;
+  constexpr int ROWB = stream_row_bytes<kW8>();
+  constexpr int CPL = kStreamCols / 32;  // 8 columns per lane
+  constexpr int COLS = kStreamCols;
+  constexpr int RPS = kStreamRowsPerStage;
+  constexpr int S = kStreamStages;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int nrows = static_cast<int>(k - r0 < rows_per_split ? k - r0 : rows_per_split);
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * COLS;
+  const int ncols = static_cast<int>(N - c0 < COLS ? N - c0 : COLS);
+  float* sa = reinterpret_cast<float*>(smem + stream_ring_bytes<kW8>());  // A_I [row][MT]
+  int32_t* sidx = reinterpret_cast<int32_t*>(sa + static_cast<size_t>(rows_per_split) * MT);
+  pdl_wait();
+  pdl_trigger();
+  for (int m = 0; m < MT; ++m)
+    for (int rr = threadIdx.x; rr < nrows; rr += kStreamThreads)
+      sa[rr * MT + m] =
+          m < M ? __uint_as_float(static_cast<uint32_t>(AI[static_cast<int64_t>(m) * ld_ai + r0 + rr]) << 16) : 0.f;
+  bool bad = false;
+  for (int rr = threadIdx.x; rr < nrows; rr += kStreamThreads) {
+    const int32_t j = __ldg(idx + r0 + rr);
+    const bool ok = j >= 0 && j < d;
+    bad |= !ok;
+    sidx[rr] = ok ? j : -1;
+  }
+  if (bad) record_error(err, kDevErrBadIndex);
+  __syncthreads();
+
+  // this lane's 16-byte piece of a row slice: bf16, piece = lane (its own 8
+  // columns); int8, 16 lanes per row, two rows per instruction
+  const char* B8 = static_cast<const char*>(Bv);
+  const uint32_t ring = smem_u32(smem) + static_cast<uint32_t>(warp * S * RPS * ROWB);
+  const int rows_w = nrows > warp ? (nrows - warp + kStreamWarps - 1) / kStreamWarps : 0;
+  const int nst = (rows_w + RPS - 1) / RPS;
+  auto issue = [&](int st) {
+    if (st < nst) {
+      const uint32_t base = ring + static_cast<uint32_t>((st % S) * RPS * ROWB);
+      if constexpr (kW8) {
+#pragma unroll
+        for (int h = 0; h < RPS / 2; ++h) {
+          const int u = 2 * h + (lane >> 4), piece = lane & 15;
+          const int i = st * RPS + u;
+          const int rr = warp + i * kStreamWarps;
+          const int32_t j = i < rows_w ? sidx[rr] : -1;
+          const int rem = ncols - piece * 16;
+          const uint32_t nb = j < 0 || rem <= 0 ? 0u : static_cast<uint32_t>(rem < 16 ? rem : 16);
+          const void* src = nb ? static_cast<const void*>(B8 + static_cast<int64_t>(j) * ldb + c0 + piece * 16) : Bv;
+          cp_async16(base + u * ROWB + piece * 16, src, nb);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < RPS; ++u) {
+          const int i = st * RPS + u;
+          const int rr = warp + i * kStreamWarps;
+          const int32_t j = i < rows_w ? sidx[rr] : -1;
+          const int rem = ncols - lane * CPL;
+          const uint32_t nb = j < 0 || rem <= 0 ? 0u : static_cast<uint32_t>((rem < CPL ? rem : CPL) * 2);
+          const void* src = nb ? static_cast<const void*>(B8 + (static_cast<int64_t>(j) * ldb + c0 + lane * CPL) * 2)
+                               : Bv;
+          cp_async16(base + u * ROWB + lane * 16, src, nb);
+        }
+      }
+    }
+    cp_async_commit();  // one group per stage, empty past the end, so the wait count stays fixed
+  };
+
+  float acc[MT][CPL];
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) acc[m][c] = 0.f;
+
+#pragma unroll
+  for (int st = 0; st < S - 1; ++st) issue(st);
+  for (int st = 0; st < nst; ++st) {
+    issue(st + S - 1);
+    cp_async_wait<S - 1>();  // stage st has landed (this lane's copies)
+    __syncwarp();            // ... and every lane's
+    const uint8_t* base = smem + warp * S * RPS * ROWB + (st % S) * RPS * ROWB + lane * CPL * ELT;
+#pragma unroll
+    for (int u = 0; u < RPS; ++u) {
+      const int i = st * RPS + u;
+      if (i < rows_w) {
+        const int rr = warp + i * kStreamWarps;
+        float b[CPL];
+        if constexpr (kW8) {
+          const uint2 w = *reinterpret_cast<const uint2*>(base + u * ROWB);
+          float f[4];
+          i8x4_to_f32(w.x, f);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) b[e] = f[e];
+          i8x4_to_f32(w.y, f);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) b[4 + e] = f[e];
+        } else {
+          const uint4 w = *reinterpret_cast<const uint4*>(base + u * ROWB);
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            b[2 * e] = bf16_lo(wv[e]);
+            b[2 * e + 1] = bf16_hi(wv[e]);
+          }
+        }
+        const float* a = sa + rr * MT;
+#pragma unroll
+        for (int m4 = 0; m4 < MT; m4 += 4) {
+          float av[4];
+          if (MT >= 4) {
+            const float4 v = *reinterpret_cast<const float4*>(a + m4);
+            av[0] = v.x; av[1] = v.y; av[2] = v.z; av[3] = v.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) av[e] = e < MT ? a[e] : 0.f;
+          }
+#pragma unroll
+          for (int e = 0; e < 4 && m4 + e < MT; ++e)
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) acc[m4 + e][c] = fmaf(av[e], b[c], acc[m4 + e][c]);
+        }
+      }
+    }
+    __syncwarp();  // every lane has read the stage before a later issue overwrites it
+  }
+  cp_async_wait<0>();
+  __syncthreads();  // the rings and the staging are free
+
+  // warp sums in a fixed order: red[m][c] = sum over warps
+  float* red = reinterpret_cast<float*>(smem);
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int c = 0; c < CPL; c += 4)
+      *reinterpret_cast<float4*>(red + (warp * MT + m) * COLS + lane * CPL + c) =
+          make_float4(acc[m][c], acc[m][c + 1], acc[m][c + 2], acc[m][c + 3]);
+  __syncthreads();
+  const int nout = MT * COLS;
+  for (int e = threadIdx.x; e < nout; e += kStreamThreads) {
+    float sum = 0.f;
+#pragma unroll
+    for (int wq = 0; wq < kStreamWarps; ++wq) sum += red[wq * nout + e];
+    red[e] = sum;
+  }
+  auto store = [&](int e, float v) {
+    const int m = e / COLS, cl = e % COLS;
+    const int64_t c = c0 + cl;
+    if (m >= M || c >= N) return;
+    if constexpr (kW8) v *= __ldg(b_scale + c);
+    if (out_f32) {
+      static_cast<float*>(Y)[static_cast<int64_t>(m) * ldy + c] = v;
+    } else {
+      static_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(m) * ldy + c] = __float2bfloat16_rn(v);
+    }
+  };
+  if (gridDim.y == 1) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < nout; e += kStreamThreads) store(e, red[e]);
+  } else if (clustered) {
+    cluster_sync();
+    const uint32_t nsplit = gridDim.y, rank = cluster_ctarank();
+    const uint32_t red_s = smem_u32(red);
+    for (int e = static_cast<int>(rank) * kStreamThreads + threadIdx.x; e < nout;
+         e += static_cast<int>(nsplit) * kStreamThreads) {
+      float v = 0.f;
+      for (uint32_t q = 0; q < nsplit; ++q) v += ld_dsmem_f32(mapa_shared(red_s + e * 4, q));
+      store(e, v);
+    }
+    cluster_sync();  // no block leaves while another may still read its shared memory
+  } else {
+    __syncthreads();
+    for (int e = threadIdx.x; e < nout; e += kStreamThreads) {
+      const int m = e / COLS, cl = e % COLS;
+      const int64_t c = c0 + cl;
+      if (m < M && c < N) partial[(static_cast<int64_t>(blockIdx.y) * M + m) * N + c] = red[e];
+    }
+  }
+}
+
 // Y[m, c] = sum over splits (in order) of partial[split][m][c], times
 // b_scale[c] when given.
 __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float* __restrict__ partial, int splits, int M,
@@ -251,8 +486,10 @@ GemvPlan plan_mt(int64_t M, int64_t N, int64_t k, int sms) {
   GemvPlan p{};
   p.slices = (N + GemvShape<MT>::COLS - 1) / GemvShape<MT>::COLS;
   // one wave of two blocks per SM (a partial second wave would double the
-  // time); each split at least 32 rows and at most what ~96 KB of staging holds
-  const int64_t max_rows = std::min<int64_t>(kGemvMaxRows, (96 * 1024) / ((MT + 1) * 4) / 8 * 8);
+  // time); each split at least 32 rows and at most what the A_I staging holds
+  // (~96 KB for the register-loading kernel, 16 KB beside the streaming ring)
+  const int64_t stage_bytes = MT <= 8 ? kStreamAiBytes : 96 * 1024;
+  const int64_t max_rows = std::min<int64_t>(kGemvMaxRows, stage_bytes / ((MT + 1) * 4) / 8 * 8);
   int64_t splits = std::max<int64_t>(1, 2 * static_cast<int64_t>(std::max(sms, 1)) / p.slices);
   splits = std::min<int64_t>(splits, kGemvMaxCluster);  // splits of a slice form one cluster
   splits = std::min<int64_t>(splits, std::max<int64_t>(1, k / 32));
@@ -268,12 +505,21 @@ template <int MT, bool kW8>
 cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const void* B, int64_t ldb, const float* b_scale,
                            const int32_t* idx, int M, int64_t d, int64_t N, int64_t k, const GemvPlan& pl,
                            float* partial, void* Y, int out_f32, int64_t ldy, unsigned* err, cudaStream_t stream) {
+  constexpr bool kStream = MT <= 8;
+  static_assert(!kStream || GemvShape<MT, kW8>::COLS == kStreamCols, "one column slicing for both kernels");
+  auto kernel = [] {
+    if constexpr (kStream)
+      return gemv_stream_kernel<MT, kW8>;
+    else
+      return gemv_rows_kernel<MT, kW8>;
+  }();
+  const int threads = kStream ? kStreamThreads : kGemvThreads;
   const size_t smem =
-      static_cast<size_t>(std::max(pl.rows_per_split * (MT + 1), kGemvWarps * MT * GemvShape<MT>::COLS)) * 4;
+      kStream ? stream_smem_bytes<MT, kW8>(pl.rows_per_split)
+              : static_cast<size_t>(std::max(pl.rows_per_split * (MT + 1), kGemvWarps * MT * GemvShape<MT>::COLS)) * 4;
   if (smem > 48 * 1024) {
     const cudaError_t e =
-        cudaFuncSetAttribute(gemv_rows_kernel<MT, kW8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
   const dim3 grid(static_cast<unsigned>(pl.slices), static_cast<unsigned>(pl.splits));
@@ -281,7 +527,7 @@ cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const void* B, int
   if (pl.clustered) {
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = grid;
-    cfg.blockDim = dim3(kGemvThreads);
+    cfg.blockDim = dim3(threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -293,12 +539,12 @@ cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const void* B, int
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, gemv_rows_kernel<MT, kW8>, AI, ld_ai, B, ldb, b_scale, idx, M, d, N, k,
-                           pl.rows_per_split, partial, Y, out_f32, ldy, 1, err);
+    e = cudaLaunchKernelEx(&cfg, kernel, AI, ld_ai, B, ldb, b_scale, idx, M, d, N, k, pl.rows_per_split, partial, Y,
+                           out_f32, ldy, 1, err);
     return e;
   }
-  e = launch_pdl(gemv_rows_kernel<MT, kW8>, grid, dim3(kGemvThreads), smem, stream, AI, ld_ai, B, ldb, b_scale, idx,
-                 M, d, N, k, pl.rows_per_split, partial, Y, out_f32, ldy, 0, err);
+  e = launch_pdl(kernel, grid, dim3(threads), smem, stream, AI, ld_ai, B, ldb, b_scale, idx, M, d, N, k,
+                 pl.rows_per_split, partial, Y, out_f32, ldy, 0, err);
   if (e != cudaSuccess || pl.splits == 1) return e;
   const int64_t outs = static_cast<int64_t>(M) * N;
   return launch_pdl(gemv_reduce_kernel, dim3(static_cast<unsigned>((outs + 255) / 256)), dim3(256), 0, stream,

@@ -465,3 +465,131 @@ def test_path_layer70b(which):
     ks = [oracle.k_from_rho(r, inp.d) for r in inp.rhos]
     A2, _ = widen_topk_gaps(inp.A, "bf16", ks)
     _check_path(inp, inp.rhos[0], rows=sample_rows(inp.M), cond=A2)
+
+
+# ------------------------------------------------------------------ int8 weight (weight-only quantisation)
+
+def _pitched16(t):
+    """int8 matrix in a buffer whose row pitch is a multiple of 16 bytes."""
+    n = t.shape[1]
+    if n % 16 == 0:
+        return t
+    buf = torch.zeros((t.shape[0], (n + 15) // 16 * 16), dtype=t.dtype, device=t.device)
+    buf[:, :n] = t
+    return buf[:, :n]
+
+
+def _check_w8(got, A_I, q_I, s, k, out_dtype):
+    """Oracle comparison for A_I · (q_I * s): the products a*q are exact in fp32
+    (8 + 7 significant bits), the k-term fp32 sum and the scale multiply add
+    at most (k + 1) * 2^-24 * sum |a q s| per element."""
+    ref = A_I @ (q_I.astype(np.float64) * s.astype(np.float64)[None, :])
+    absprod = np.abs(A_I) @ (np.abs(q_I.astype(np.float64)) * s.astype(np.float64)[None, :])
+    if out_dtype == torch.float32:
+        bound = (k + 1) * 2.0 ** -24 * absprod + 1e-30
+        assert np.all(np.abs(got - ref) <= bound)
+        if got.size >= 4096:
+            assert rel_fro(got, ref) <= 1e-5
+        return
+    check_bf16_output(got, ref, absprod, k + 1)
+
+
+W8_SHAPES = [  # M, d, N, k
+    (1, 4096, 4096, 2048),     # decode: kept int8 rows read in place
+    (3, 1000, 700, 333),       # ragged N (pitched rows) and k
+    (8, 2048, 14336, 1024),
+    (16, 4096, 4096, 2048),
+    (17, 96, 272, 65),         # tensor-core path: N just past a tile, k just past a block
+    (300, 1000, 700, 333),     # ragged M, N, k
+    (512, 4096, 1024, 2048),   # CTA-pair tensor-core path
+]
+
+
+@pytest.mark.parametrize("M,d,N,k", W8_SHAPES)
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_gemm_w8_parity(M, d, N, k, out_dtype):
+    A_bits = W.llm_activation_bf16(61 + M, M, d)
+    q, s = W.weight_int8(62 + M, d, N)
+    rng = np.random.default_rng(M * 7 + k)
+    idx = np.sort(rng.choice(d, k, replace=False)).astype(np.int32)
+    A = oracle.decode(A_bits, "bf16")
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(bf16_tensor(A_bits), it)
+    qt = _pitched16(torch.from_numpy(q).cuda())
+    st = torch.from_numpy(s).cuda()
+    Y = R.rmm_gemm_w8(AI, qt, st, it, out_dtype=out_dtype)
+    _check_w8(to_f64(Y), A[:, idx], q[idx], s, k, out_dtype)
+    # the oracle's own int8 product agrees with the check's reference
+    np.testing.assert_allclose(oracle.reduced_matmul_w8(A, q, s, idx),
+                               A[:, idx] @ (q[idx].astype(np.float64) * s.astype(np.float64)), rtol=1e-12)
+    no_device_error()
+
+
+@pytest.mark.parametrize("M", [1, 16, 300])
+def test_path_w8(M):
+    """Whole path with an int8 weight: selection bit-exact, product within bounds."""
+    d, N, rho = 4096, 1040, 0.5
+    A_bits = W.llm_activation_bf16(71 + M, M, d)
+    k = oracle.k_from_rho(rho, d)
+    cond, _ = widen_topk_gaps(A_bits, "bf16", [k])
+    Ac = oracle.decode(cond, "bf16")
+    q, s = W.weight_int8(72, d, N)
+    idx_out = torch.empty(k, dtype=torch.int32, device="cuda")
+    Y = R.rmm_matmul_w8(bf16_tensor(cond), torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(), rho,
+                        idx_out=idx_out)
+    Yo, idx, _ = oracle.rmm_w8(Ac, q, s, rho)
+    np.testing.assert_array_equal(idx_out.cpu().numpy(), idx)
+    _check_w8(to_f64(Y), Ac[:, idx], q[idx], s, k, torch.bfloat16)
+    assert rel_fro(to_f64(Y), Yo) <= 2e-3
+    no_device_error()
+
+
+def test_path_w8_mlp_up_full():
+    """MLP up/gate projection 4096 x 4096 x 14336 with an int8 weight at rho = 0.5,
+    the launch configuration the benchmark times; sampled rows vs the oracle."""
+    inp = W.mlp_up_w8()
+    k = oracle.k_from_rho(0.5, inp.d)
+    cond, _ = widen_topk_gaps(inp.A, "bf16", [k])
+    Ac = oracle.decode(cond, "bf16")
+    q, s = inp.B, inp.meta["b_scale"]
+    idx_out = torch.empty(k, dtype=torch.int32, device="cuda")
+    Y = R.rmm_matmul_w8(bf16_tensor(cond), torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(), 0.5,
+                        idx_out=idx_out)
+    idx = oracle.topk_indices(oracle.column_sq_norms(Ac), k)
+    np.testing.assert_array_equal(idx_out.cpu().numpy(), idx)
+    rows = sample_rows(inp.M)
+    _check_w8(to_f64(Y)[rows], Ac[rows][:, idx], q[idx], s, k, torch.bfloat16)
+    no_device_error()
+
+
+@pytest.mark.parametrize("M", [2, 200])
+def test_gemm_w8_bad_index_flagged(M):
+    d, N, k = 256, 128, 64
+    A_bits = W.llm_activation_bf16(81, M, d)
+    q, s = W.weight_int8(82, d, N)
+    idx = np.arange(k, dtype=np.int32)
+    idx[5] = d + 3
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(bf16_tensor(A_bits), it)
+    assert R.rmm_device_error(clear=True) == 1
+    Y = R.rmm_gemm_w8(AI, torch.from_numpy(q).cuda(), torch.from_numpy(s).cuda(), it, out_dtype=torch.float32)
+    assert R.rmm_device_error(clear=True) == 1
+    # the bad index contributes nothing; the rest is the product over the good ones
+    good = np.delete(np.arange(k), 5)
+    A = oracle.decode(A_bits, "bf16")
+    _check_w8(to_f64(Y), to_f64(AI)[:, good], q[idx[good]], s, k, torch.float32)
+    no_device_error()
+
+
+def test_gemm_w8_rejects_bad_layouts():
+    A_I = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
+    it = torch.arange(64, dtype=torch.int32, device="cuda")
+    s = torch.ones(24, dtype=torch.float32, device="cuda")
+    q = torch.zeros((128, 24), dtype=torch.int8, device="cuda")   # row pitch 24 bytes
+    with pytest.raises(R.RMMError):
+        R.rmm_gemm_w8(A_I, q, s, it)
+    with pytest.raises(ValueError):
+        R.rmm_gemm_w8(A_I, _pitched16(q), s[:10], it)
+    with pytest.raises(TypeError):
+        R.rmm_gemm_w8(A_I, _pitched16(q).to(torch.int16), s, it)
+    no_device_error()
