@@ -10,6 +10,7 @@ Modules:
   rmm           scores, top-k selection and the reduced product
   attention     reduced attention (head_dim reduction in QK^T, token
                 reduction in PV)
+  decode_attention  the same for one new query token over a KV cache
   conditioning  deterministic score-gap widening of generated inputs, so the
                 fp32 GPU ranking and the fp64 oracle ranking must agree
 
@@ -20,8 +21,9 @@ reduce to library routines, error bounds).  The attention READINGS R1-R6
 functions are pinned to those readings, and the readings themselves are
 "parity unpinned" against the page.
 """
-from . import rmm, attention, conditioning  # noqa: F401
+from . import rmm, attention, decode_attention, conditioning  # noqa: F401
 from .rmm import (k_from_rho, column_sq_norms, column_norms, topk_indices,  # noqa: F401
                   reduced_matmul, dense_matmul, rmm as rmm_path, decode,
                   dequantize_w8, reduced_matmul_w8, rmm_w8)
 from .attention import reduced_attention, attention_head, kv_head_of  # noqa: F401
+from .decode_attention import decode_attention_head  # noqa: F401

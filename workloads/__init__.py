@@ -262,3 +262,52 @@ def attention(seed: int = 3, B: int = 1, Hq: int = 32, Hkv: int = 32, S: int = 8
         V[:, g] = f32_to_bf16_bits(Vg)
     name = f"reduced attention B{B} Hq{Hq} Hkv{Hkv} S{S} D{D}"
     return AttentionInputs(name, Q, K, V, rho_d, rho_t, seed, attempts)
+
+
+@dataclass
+class DecodeAttentionInputs:
+    """One new query token per sequence over a KV cache: q [B,Hq,D] and caches
+    K/V [B,Hkv,Lmax,D] (bf16 bits, contiguous) holding L valid tokens."""
+    name: str
+    q: np.ndarray
+    K: np.ndarray
+    V: np.ndarray
+    L: int
+    rho_d: float
+    rho_t: float
+    seed: int
+    attempts: list = field(default_factory=list)
+
+    @property
+    def shape(self):
+        B, Hq, D = self.q.shape
+        return B, Hq, self.K.shape[1], self.L, self.K.shape[2], D
+
+
+def decode_attention(seed: int = 5, B: int = 1, Hq: int = 32, Hkv: int = 8, L: int = 32768, D: int = 128,
+                     rho_d: float = 0.5, rho_t: float = 0.5, Lmax: int = None, attempts=None) -> DecodeAttentionInputs:
+    """Decode-step workload: per kv-group g, q (its Hq/Hkv heads), K and V drawn
+    as N(0,1) times a per-(head, dim) lognormal(0, 0.5) scale, as in the
+    prefill workload.  Cache rows L..Lmax-1 (unused capacity) hold 1e4, so a
+    read past the valid length would show.  ``attempts[g]`` selects the
+    redraw attempt of kv-group g."""
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    Lmax = L if Lmax is None else Lmax
+    if not (1 <= L <= Lmax):
+        raise ValueError("need 1 <= L <= Lmax")
+    G = Hq // Hkv
+    attempts = list(attempts) if attempts is not None else [0] * Hkv
+    q = np.empty((B, Hq, D), np.uint16)
+    K = np.full((B, Hkv, Lmax, D), f32_to_bf16_bits(np.float32(1e4)), np.uint16)
+    V = np.full((B, Hkv, Lmax, D), f32_to_bf16_bits(np.float32(1e4)), np.uint16)
+    for g in range(Hkv):
+        a = attempts[g]
+        qs = np.exp(0.5 * _normal(substream(seed, "qscale", g, a), (G, D)))
+        ks = np.exp(0.5 * _normal(substream(seed, "kscale", g, a), D))
+        vs = np.exp(0.5 * _normal(substream(seed, "vscale", g, a), D))
+        q[:, g * G:(g + 1) * G] = f32_to_bf16_bits(_normal(substream(seed, "Q", g, a), (B, G, D)) * qs[None])
+        K[:, g, :L] = f32_to_bf16_bits(_normal(substream(seed, "K", g, a), (B, L, D)) * ks[None, None, :])
+        V[:, g, :L] = f32_to_bf16_bits(_normal(substream(seed, "V", g, a), (B, L, D)) * vs[None, None, :])
+    return DecodeAttentionInputs(f"decode attention B{B} Hq{Hq} Hkv{Hkv} L{L} D{D}", q, K, V, L, rho_d, rho_t,
+                                 seed, attempts)
