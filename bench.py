@@ -53,9 +53,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["bench", "attention", "decode", "w8"], default="bench",
-                    help="attention / decode / w8: run only that workload a few times and exit (a short "
-                         "program for profiler captures; prints no JSON line)")
+    ap.add_argument("--case", choices=["bench", "attention", "decode", "w8", "decode_attention"], default="bench",
+                    help="attention / decode / w8 / decode_attention: run only that workload a few times and exit "
+                         "(a short program for profiler captures; prints no JSON line)")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -421,6 +421,59 @@ def measure_w8(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, X, h
     return out
 
 
+DEC_ATTN = {"seed": 5, "Hq": 32, "Hkv": 8, "L": 32768, "D": 128, "rho_d": 0.5, "rho_t": 0.5}
+
+
+def measure_decode_attention(R, workloads, bf16_tensor, dev, stream, steps, timed, hbm_gbs):
+    """One decode step of reduced attention (GQA 32/8 heads, D = 128, a 32768-token
+    cache) for 1 and 8 sequences, next to torch's SDPA on the full cache.
+    Bandwidth counts the algorithmic bytes: every key row (the head_dim
+    selection differs per q-head, so every key sector is needed), the union
+    over a kv-group's q-heads of their kept value rows, q and O."""
+    import numpy as np
+    import torch
+    a = DEC_ATTN
+    out = {}
+    for B in (1, 8):
+        inp = workloads.decode_attention(a["seed"], B, a["Hq"], a["Hkv"], a["L"], a["D"], a["rho_d"], a["rho_t"])
+        q, K, V = (bf16_tensor(x, dev) for x in (inp.q, inp.K, inp.V))
+        kt = R.rmm_k_from_rho(a["rho_t"], a["L"])
+        O = torch.empty((B, a["Hq"], a["D"]), dtype=torch.bfloat16, device=dev)
+        idx_t = torch.empty((B * a["Hq"], kt), dtype=torch.int32, device=dev)
+        ws = torch.empty(R.rmm_decode_attention_workspace_size(B, a["Hq"], a["L"], a["D"], a["rho_t"], False, True),
+                         dtype=torch.uint8, device=dev)
+
+        def rmm(ev):
+            ev[0].record(stream)
+            R.rmm_decode_attention(q, K, V, a["L"], a["rho_d"], a["rho_t"], out=O, idx_t=idx_t, ws=ws)
+            ev[1].record(stream)
+        q4 = q.view(B, a["Hq"], 1, a["D"])
+
+        def sdpa(ev):
+            ev[0].record(stream)
+            torch.nn.functional.scaled_dot_product_attention(q4, K, V, enable_gqa=True)
+            ev[1].record(stream)
+        for _ in range(3):
+            rmm([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+            sdpa([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        rmm_us = statistics.mean(p[0] for p in timed(rmm, steps, 2)) * 1e3
+        sdpa_us = statistics.mean(p[0] for p in timed(sdpa, steps, 2)) * 1e3
+        it = idx_t.cpu().numpy().reshape(B, a["Hkv"], a["Hq"] // a["Hkv"], kt)
+        union = sum(len(np.unique(it[b, g])) for b in range(B) for g in range(a["Hkv"]))
+        row = a["D"] * 2
+        alg = B * a["Hkv"] * a["L"] * row + union * row + 2 * B * a["Hq"] * row
+        gbs = alg / (rmm_us * 1e-6) / 1e9
+        out[f"B{B}"] = {"rmm_us": rmm_us, "sdpa_us": sdpa_us, "speedup_vs_sdpa": sdpa_us / rmm_us,
+                        "algorithmic_MB": alg / 1e6, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs,
+                        "kept_value_rows_union_frac": union / (B * a["Hkv"] * a["L"]), "gpu_launches_per_call": 3}
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the decode-attention runs")
+    out["workload"] = (f"decode step: q[B x {a['Hq']} x {a['D']}] over K/V caches [B x {a['Hkv']} x {a['L']} x "
+                       f"{a['D']}] bf16, rho_d={a['rho_d']} rho_t={a['rho_t']}; caches larger than L2 (B=8), "
+                       "256 MiB write flush between steps")
+    return out
+
+
 def run_rmm(args):
     import numpy as np
     import torch
@@ -559,6 +612,8 @@ def run_rmm(args):
     decode = measure_decode(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed, Wt,
                             peaks["hbm_gbs"])
     w8 = measure_w8(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed, X, peaks["hbm_gbs"])
+    dec_attn = measure_decode_attention(R, workloads, bf16_tensor, dev, stream, min(args.steps, 30), timed,
+                                        peaks["hbm_gbs"])
     gemm_ms = stage_ms["gemm"]
     achieved = flops_step / (gemm_ms * 1e-3) / 1e12
     traffic = traffic_per_launch()
@@ -604,6 +659,7 @@ def run_rmm(args):
             "attention": attention,
             "decode": decode,
             "int8_weight": w8,
+            "decode_attention": dec_attn,
             "clocks": clk.summary(), "clock_remeasured": remeasured,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -633,6 +689,16 @@ def run_case(case):
                                                         a["rho_t"]), dtype=torch.uint8, device=dev)
         for _ in range(3):
             R.rmm_attention(Q, K, V, a["rho_d"], a["rho_t"], out=O, ws=ws)
+    elif case == "decode_attention":
+        a = DEC_ATTN
+        for B in (1, 8):
+            inp = workloads.decode_attention(a["seed"], B, a["Hq"], a["Hkv"], a["L"], a["D"], a["rho_d"], a["rho_t"])
+            q, K, V = (bf16_tensor(x, dev) for x in (inp.q, inp.K, inp.V))
+            O = torch.empty((B, a["Hq"], a["D"]), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty(R.rmm_decode_attention_workspace_size(B, a["Hq"], a["L"], a["D"], a["rho_t"]),
+                             dtype=torch.uint8, device=dev)
+            for _ in range(3):
+                R.rmm_decode_attention(q, K, V, a["L"], a["rho_d"], a["rho_t"], out=O, ws=ws)
     elif case == "w8":
         q, sc = workloads.weight_int8(1, D, N)
         Wq, S = torch.from_numpy(q).to(dev), torch.from_numpy(sc).to(dev)

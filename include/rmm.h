@@ -259,6 +259,34 @@ RMM_API rmm_status rmm_attention(const void* Q, const void* K, const void* V,
                          void* O, int out_dtype, int32_t* idx_d, int32_t* idx_t,
                          float* lse, float* tscore, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ reduced decode attention
+ * One new query token per sequence attending to a KV cache, with both
+ * reductions of Metodología › Alcance de Aplicación applied to its single
+ * query row (the autoregressive setting of Resultados Experimentales):
+ *   1. per (b, h): I_d = top k_d = ceil(rho_d*D) of q[b,h,c]^2 (lowest index
+ *      on ties);
+ *   2. s_j = scale * sum_{c in I_d} q[b,h,c] K[b,g,j,c] for the L cached
+ *      tokens j < L (g = h*Hkv/Hq; scale <= 0 selects 1/sqrt(D));
+ *      lse = logsumexp_j s_j;  P_j = exp(s_j - lse);
+ *   3. t_j = P_j^2 (squared column norms of the one-row P); I_t = top
+ *      k_t = ceil(rho_t*L) tokens (lowest index on ties);
+ *   4. O[b,h,:] = sum_{j in I_t} P_j V[b,g,j,:]  (P not renormalised).
+ * q [B, Hq, D] and O [B, Hq, D] (out_dtype) contiguous; K, V [B, Hkv, Lmax,
+ * D] bf16 contiguous caches of capacity Lmax holding L valid tokens (rows
+ * L..Lmax-1 are never read).  All four 16-byte aligned.  D in {64, 128},
+ * Hq = G * Hkv with G (q-heads per kv-head) in {1, 2, 4, 8, 16}, else
+ * RMM_ERR_UNSUPPORTED.  Optional outputs (may be NULL): idx_d [B*Hq, k_d],
+ * idx_t [B*Hq, k_t] ascending, lse [B*Hq], logits [B*Hq, L] (the s_j; when
+ * given it also serves as the kernels' logit buffer).  Workspace:
+ * rmm_decode_attention_workspace_size(B, Hq, L, D, rho_t, logits != NULL,
+ * idx_t != NULL) bytes, 256-byte aligned. */
+RMM_API size_t rmm_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t L, int64_t D, double rho_t,
+                                                   int with_logits, int with_idx_t);
+RMM_API rmm_status rmm_decode_attention(const void* q, const void* K, const void* V, int64_t B, int64_t Hq,
+                                        int64_t Hkv, int64_t L, int64_t Lmax, int64_t D, double rho_d, double rho_t,
+                                        float scale, void* O, int out_dtype, int32_t* idx_d, int32_t* idx_t,
+                                        float* lse, float* logits, void* ws, size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

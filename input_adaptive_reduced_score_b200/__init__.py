@@ -23,7 +23,8 @@ __all__ = [
     "rmm_device_error", "rmm_score", "rmm_score_workspace_size", "rmm_score_noalloc", "rmm_topk", "rmm_compact", "rmm_gather_rows", "rmm_compact_gather",
     "rmm_gemm", "rmm_gemm_workspace_size", "rmm_gemm_compacted",
     "rmm_matmul", "rmm_matmul_workspace_size", "rmm_gemm_w8", "rmm_gemm_w8_workspace_size", "rmm_matmul_w8",
-    "rmm_matmul_w8_workspace_size", "rmm_attention", "rmm_attention_workspace_size",
+    "rmm_matmul_w8_workspace_size", "rmm_attention", "rmm_attention_workspace_size", "rmm_decode_attention",
+    "rmm_decode_attention_workspace_size",
     "exported_symbols", "declared_symbols",
 ]
 
@@ -77,6 +78,9 @@ _sig("rmm_gemm_w8", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_i64, c
 _sig("rmm_matmul_w8_workspace_size", c_sz, c_i64, c_i64, c_i64, c_dbl)
 _sig("rmm_matmul_w8", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_dbl, c_vp, c_int, c_i64, c_vp, c_vp,
      c_vp, c_sz, c_vp)
+_sig("rmm_decode_attention_workspace_size", c_sz, c_i64, c_i64, c_i64, c_i64, c_dbl, c_int, c_int)
+_sig("rmm_decode_attention", c_int, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl, c_flt,
+     c_vp, c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp)
 _sig("rmm_attention_workspace_size", c_sz, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl)
 _sig("rmm_attention", c_int, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl, c_flt, c_vp, c_int,
      c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp)
@@ -390,4 +394,31 @@ def rmm_attention(Q, K, V, rho_d: float, rho_t: float, scale: float = 0.0, out=N
     _check(lib.rmm_attention(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, S, D, float(rho_d), float(rho_t), float(scale),
                              _ptr(out), _dtype_code(out), _ptr(idx_d), _ptr(idx_t), _ptr(lse), _ptr(tscore),
                              _ptr(w), wn, _stream_ptr(stream)), "rmm_attention")
+    return out
+
+
+def rmm_decode_attention_workspace_size(B, Hq, L, D, rho_t, with_logits=False, with_idx_t=False) -> int:
+    return lib.rmm_decode_attention_workspace_size(B, Hq, L, D, float(rho_t), int(bool(with_logits)),
+                                                   int(bool(with_idx_t)))
+
+
+def rmm_decode_attention(q, K, V, L: int, rho_d: float, rho_t: float, scale: float = 0.0, out=None, out_dtype=None,
+                         idx_d=None, idx_t=None, lse=None, logits=None, ws=None, stream=None):
+    """Reduced attention of one new query token per sequence over a KV cache:
+    q [B,Hq,D], caches K/V [B,Hkv,Lmax,D] (bf16, contiguous) holding L tokens."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous() or q.dim() != 3:
+        raise ValueError("q must be a contiguous [B, Hq, D] bf16 tensor")
+    for t, n in ((K, "K"), (V, "V")):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{n} must be a contiguous [B, Hkv, Lmax, D] bf16 tensor")
+    B, Hq, D = q.shape
+    Hkv, Lmax = K.shape[1], K.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=out_dtype or torch.bfloat16, device=q.device)
+    wsb = lib.rmm_decode_attention_workspace_size(B, Hq, L, D, float(rho_t), int(logits is not None),
+                                                  int(idx_t is not None))
+    w, wn = _workspace(wsb, q.device, ws)
+    _check(lib.rmm_decode_attention(_ptr(q), _ptr(K), _ptr(V), B, Hq, Hkv, L, Lmax, D, float(rho_d), float(rho_t),
+                                    float(scale), _ptr(out), _dtype_code(out), _ptr(idx_d), _ptr(idx_t), _ptr(lse),
+                                    _ptr(logits), _ptr(w), wn, _stream_ptr(stream)), "rmm_decode_attention")
     return out

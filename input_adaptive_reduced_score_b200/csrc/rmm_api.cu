@@ -475,6 +475,44 @@ rmm_status rmm_matmul_w8(const void* A, int64_t lda, const int8_t* Bq, int64_t l
                      stream);
 }
 
+size_t rmm_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t L, int64_t D, double rho_t,
+                                           int with_logits, int with_idx_t) {
+  const int64_t kt = k_from_rho_impl(rho_t, L);
+  if (B < 1 || Hq < 1 || kt < 1 || (D != 64 && D != 128)) return 0;
+  return decode_attention_workspace_bytes(B, Hq, L, D, kt, !with_logits, !with_idx_t);
+}
+
+rmm_status rmm_decode_attention(const void* q, const void* K, const void* V, int64_t B, int64_t Hq, int64_t Hkv,
+                                int64_t L, int64_t Lmax, int64_t D, double rho_d, double rho_t, float scale, void* O,
+                                int out_dtype, int32_t* idx_d, int32_t* idx_t, float* lse, float* logits, void* ws,
+                                size_t ws_bytes, void* stream) {
+  clear_error();
+  if (!valid_dtype(out_dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_decode_attention: out dtype %d", out_dtype);
+  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || Lmax < L || Hq % Hkv)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_decode_attention: bad sizes");
+  if (D != 64 && D != 128) return fail(RMM_ERR_UNSUPPORTED, "rmm_decode_attention: D must be 64 or 128");
+  if (!decode_attention_group_supported(Hq / Hkv))
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_decode_attention: q-heads per kv-head must be 1, 2, 4, 8 or 16");
+  if (B * Hq > 65535 || B * Hkv > 65535 || B * Hq * L > kIntMax || B * Hkv * Lmax * D > (int64_t{1} << 40) ||
+      Lmax > kIntMax)
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_decode_attention: sizes beyond the kernels' grid");
+  const int64_t kd = k_from_rho_impl(rho_d, D), kt = k_from_rho_impl(rho_t, L);
+  if (kd < 1 || kt < 1) return fail(RMM_ERR_INVALID_ARG, "rmm_decode_attention: rho outside (0,1]");
+  if (!q || !K || !V || !O) return fail(RMM_ERR_INVALID_ARG, "rmm_decode_attention: null pointer");
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(O))
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_decode_attention: q, K, V and O must be 16-byte aligned");
+  const size_t need = decode_attention_workspace_bytes(B, Hq, L, D, kt, logits == nullptr, idx_t == nullptr);
+  if (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
+    return fail(RMM_ERR_WORKSPACE, "rmm_decode_attention: workspace %zu < %zu bytes or not 256-byte aligned",
+                ws_bytes, need);
+  unsigned* err = device_error_word();
+  if (!err) return RMM_ERR_CUDA;
+  const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  const cudaError_t e = launch_decode_attention(q, K, V, B, Hq, Hkv, L, Lmax, D, kd, kt, sc, O, out_dtype, idx_d,
+                                                idx_t, lse, logits, ws, err, static_cast<cudaStream_t>(stream));
+  return from_cuda(e, "rmm_decode_attention: launch");
+}
+
 size_t rmm_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D, double rho_d,
                                     double rho_t) {
   const int64_t kd = k_from_rho_impl(rho_d, D), kt = k_from_rho_impl(rho_t, S);

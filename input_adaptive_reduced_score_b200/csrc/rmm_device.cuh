@@ -112,6 +112,16 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
                : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared (no copy engine involved);
+// src_bytes < 16 fills the rest with zeros (0: nothing is read).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed copy groups are pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // 2-D tiled TMA load of one box into shared memory; completion is signalled on
 // `bar` as transaction bytes.  The innermost coordinate x must be a multiple
 // of 16 bytes' worth of elements (the callers pass multiples of 64 bf16).

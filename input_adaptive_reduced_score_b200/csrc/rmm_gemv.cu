@@ -262,15 +262,6 @@ size_t stream_smem_bytes(int rows_per_split) {
   return std::max(stream_ring_bytes<kW8>() + stage_ai, red);
 }
 
-// 16-byte asynchronous copy global -> shared; src_bytes < 16 fills the rest
-// with zeros (0: no read at all).
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
 // grid: x = column slice of 256, y = row split.  Warp w takes the split's
 // kept rows w, w + 8, w + 16, ..., four per stage, and keeps six stages of
 // 16-byte asynchronous copies in flight (no registers held, no copy engine

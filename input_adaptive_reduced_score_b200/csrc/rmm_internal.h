@@ -109,4 +109,15 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
                              void* O, int out_dtype, int32_t* idx_d, int32_t* idx_t, float* lse,
                              float* tscore, void* ws, unsigned* err, cudaStream_t stream);
 
+// ---- reduced decode attention (rmm_decode_attention.cu)
+// own_logits / own_idx: the logits buffer [B*Hq, L] / token index buffer
+// [B*Hq, kt] live in the workspace (the caller did not pass them).
+bool decode_attention_group_supported(int64_t G);  // q-heads per kv-head: 1, 2, 4, 8 or 16
+size_t decode_attention_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int64_t D, int64_t kt, bool own_logits,
+                                        bool own_idx);
+cudaError_t launch_decode_attention(const void* q, const void* K, const void* V, int64_t B, int64_t Hq, int64_t Hkv,
+                                    int64_t L, int64_t Lmax, int64_t D, int64_t kd, int64_t kt, float scale, void* O,
+                                    int out_dtype, int32_t* idx_d, int32_t* idx_t, float* lse, float* logits,
+                                    void* ws, unsigned* err, cudaStream_t stream);
+
 }  // namespace rmm
