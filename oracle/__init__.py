@@ -11,6 +11,8 @@ Modules:
   attention     reduced attention (head_dim reduction in QK^T, token
                 reduction in PV)
   decode_attention  the same for one new query token over a KV cache
+  block         products sharing one selection; a gated MLP block with every
+                product reduced
   conditioning  deterministic score-gap widening of generated inputs, so the
                 fp32 GPU ranking and the fp64 oracle ranking must agree
 
@@ -21,7 +23,7 @@ reduce to library routines, error bounds).  The attention READINGS R1-R6
 functions are pinned to those readings, and the readings themselves are
 "parity unpinned" against the page.
 """
-from . import rmm, attention, decode_attention, conditioning  # noqa: F401
+from . import rmm, attention, decode_attention, block, conditioning  # noqa: F401
 from .rmm import (k_from_rho, column_sq_norms, column_norms, topk_indices,  # noqa: F401
                   reduced_matmul, dense_matmul, rmm as rmm_path, decode,
                   dequantize_w8, reduced_matmul_w8, rmm_w8)
