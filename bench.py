@@ -421,6 +421,83 @@ def measure_w8(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, X, h
     return out
 
 
+def measure_block(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, X):
+    """The block driver on the MLP up/gate activation X [4096 x 4096]:
+    (1) q/k/v-shaped products (W 4096 x 4096, 4096 x 1024, 4096 x 1024) at
+    rho = 0.5 with one shared selection (rmm_matmul_multi) against three
+    rmm_matmul calls; (2) the gated MLP block (d_ff = 14336, rho_up = 0.8,
+    rho_down = 0.5; up/gate share one selection, the down projection's scores
+    come from the fused SiLU * U producer) against the same chain built from
+    rmm_matmul calls and a torch SiLU * U, and against dense cuBLAS."""
+    import torch
+    out = {}
+    Ws = [bf16_tensor(workloads.weight_bf16(9, D, n, group=i), dev) for i, n in enumerate((D, 1024, 1024))]
+    Ys = [torch.empty((M, w.shape[1]), dtype=torch.bfloat16, device=dev) for w in Ws]
+    mws = torch.empty(R.rmm_matmul_multi_workspace_size(M, D, D, 0.5), dtype=torch.uint8, device=dev)
+    sws = [torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, M, D, w.shape[1], 0.5), dtype=torch.uint8, device=dev)
+           for w in Ws]
+
+    def shared(ev):
+        ev[0].record(stream)
+        R.rmm_matmul_multi(X, Ws, 0.5, outs=Ys, ws=mws)
+        ev[1].record(stream)
+
+    def separate(ev):
+        ev[0].record(stream)
+        for w, y, ws_ in zip(Ws, Ys, sws):
+            R.rmm_matmul(X, w, 0.5, out=y, ws=ws_)
+        ev[1].record(stream)
+    for _ in range(3):
+        shared([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        separate([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    out["qkv_shared_selection"] = {"shared_us": statistics.mean(p[0] for p in timed(shared, steps, 2)) * 1e3,
+                                   "separate_us": statistics.mean(p[0] for p in timed(separate, steps, 2)) * 1e3}
+    del Ws, Ys, mws, sws
+    F = 14336
+    Wu = bf16_tensor(workloads.weight_bf16(10, D, F, group=0), dev)
+    Wg = bf16_tensor(workloads.weight_bf16(10, D, F, group=1), dev)
+    Wd = bf16_tensor(workloads.weight_bf16(10, F, D, group=2), dev)
+    Y = torch.empty((M, D), dtype=torch.bfloat16, device=dev)
+    bws = torch.empty(R.rmm_mlp_block_workspace_size(M, D, F, 0.8, 0.5), dtype=torch.uint8, device=dev)
+    U = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+    G = torch.empty_like(U)
+    uws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, M, D, F, 0.8), dtype=torch.uint8, device=dev)
+    dws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, M, F, D, 0.5), dtype=torch.uint8, device=dev)
+
+    def block(ev):
+        ev[0].record(stream)
+        R.rmm_mlp_block(X, Wu, Wg, Wd, 0.8, 0.5, out=Y, ws=bws)
+        ev[1].record(stream)
+
+    def chain(ev):
+        ev[0].record(stream)
+        R.rmm_matmul(X, Wu, 0.8, out=U, ws=uws)
+        R.rmm_matmul(X, Wg, 0.8, out=G, ws=uws)
+        H = torch.nn.functional.silu(G) * U
+        R.rmm_matmul(H, Wd, 0.5, out=Y, ws=dws)
+        ev[1].record(stream)
+
+    def dense(ev):
+        ev[0].record(stream)
+        torch.matmul(torch.nn.functional.silu(X @ Wg) * (X @ Wu), Wd, out=Y)
+        ev[1].record(stream)
+    for _ in range(3):
+        for f in (block, chain, dense):
+            f([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    bl = statistics.mean(p[0] for p in timed(block, steps, 2))
+    ch = statistics.mean(p[0] for p in timed(chain, steps, 2))
+    de = statistics.mean(p[0] for p in timed(dense, steps, 2))
+    red_flops = 2.0 * M * F * R.rmm_k_from_rho(0.8, D) * 2 + 2.0 * M * D * R.rmm_k_from_rho(0.5, F)
+    out["mlp_block"] = {"block_us": bl * 1e3, "chain_of_rmm_matmul_us": ch * 1e3, "dense_cublas_us": de * 1e3,
+                        "speedup_vs_dense": de / bl, "effective_tflops": red_flops / (bl * 1e-3) / 1e12,
+                        "gpu_launches_per_call": 11}
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the block runs")
+    out["workload"] = (f"X[{M}x{D}] bf16 (MLP up/gate activation); q/k/v-shaped W at rho 0.5; gated MLP "
+                       f"d_ff={F}, rho_up=0.8, rho_down=0.5; 256 MiB flush between steps")
+    return out
+
+
 DEC_ATTN = {"seed": 5, "Hq": 32, "Hkv": 8, "L": 32768, "D": 128, "rho_d": 0.5, "rho_t": 0.5}
 
 
@@ -465,7 +542,7 @@ def measure_decode_attention(R, workloads, bf16_tensor, dev, stream, steps, time
         gbs = alg / (rmm_us * 1e-6) / 1e9
         out[f"B{B}"] = {"rmm_us": rmm_us, "sdpa_us": sdpa_us, "speedup_vs_sdpa": sdpa_us / rmm_us,
                         "algorithmic_MB": alg / 1e6, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs,
-                        "kept_value_rows_union_frac": union / (B * a["Hkv"] * a["L"]), "gpu_launches_per_call": 3}
+                        "kept_value_rows_union_frac": union / (B * a["Hkv"] * a["L"]), "gpu_launches_per_call": 6}
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the decode-attention runs")
     out["workload"] = (f"decode step: q[B x {a['Hq']} x {a['D']}] over K/V caches [B x {a['Hkv']} x {a['L']} x "
@@ -614,6 +691,7 @@ def run_rmm(args):
     w8 = measure_w8(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed, X, peaks["hbm_gbs"])
     dec_attn = measure_decode_attention(R, workloads, bf16_tensor, dev, stream, min(args.steps, 30), timed,
                                         peaks["hbm_gbs"])
+    block = measure_block(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 30), timed, X)
     gemm_ms = stage_ms["gemm"]
     achieved = flops_step / (gemm_ms * 1e-3) / 1e12
     traffic = traffic_per_launch()
@@ -660,6 +738,7 @@ def run_rmm(args):
             "decode": decode,
             "int8_weight": w8,
             "decode_attention": dec_attn,
+            "block_driver": block,
             "clocks": clk.summary(), "clock_remeasured": remeasured,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -235,6 +235,57 @@ RMM_API rmm_status rmm_matmul_w8(const void* A, int64_t lda, const int8_t* Bq, i
                                  int64_t M, int64_t d, int64_t N, double rho, void* Y, int out_dtype, int64_t ldy,
                                  int32_t* idx_out, float* ss_out, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ block driver
+ * Several products that read the same activation share one selection
+ * (Metodología › Mecanismo Central: I depends on A alone), e.g. the q, k and
+ * v projections of an attention input or the up and gate projections of an
+ * MLP input; each component keeps its own rho, since the pages find the
+ * attention-side products more reducible than the MLP ones and, within the
+ * MLP, the up projection the most sensitive and the down projection the
+ * most robust (Contribuciones Clave › Perspectivas Mecanísticas).
+ *
+ * rmm_matmul_multi: Y[i] = A[:, I] · B[i][I, :] for i < nprod with one
+ * I = topk(ss(A), k), k = rmm_k_from_rho(rho, d): one score pass (or none:
+ * ss_in, the d column scores of A, may be given, e.g. by
+ * rmm_silu_mul_score), one top-k, one compaction of A, then per product the
+ * row gather of B[i] and the product (M > 16: tcgen05 GEMM; M <= 16: kept rows
+ * read in place).  A bf16 [M x d] (lda); B[i] bf16 [d x N[i]] (ldb[i] a
+ * multiple of 8, 16-byte aligned); Y[i] [M x N[i]] (ldy[i], 16-byte aligned)
+ * in out_dtype.  idx_out (k, may be NULL) gets I; ss_out (d, may be NULL)
+ * the computed scores (not written when ss_in is given).  Workspace:
+ * rmm_matmul_multi_workspace_size(M, d, max N[i], rho) bytes. */
+RMM_API size_t rmm_matmul_multi_workspace_size(int64_t M, int64_t d, int64_t N_max, double rho);
+RMM_API rmm_status rmm_matmul_multi(const void* A, int64_t lda, int64_t M, int64_t d, double rho, int nprod,
+                                    const void* const* B, const int64_t* ldb, const int64_t* N, void* const* Y,
+                                    const int64_t* ldy, int out_dtype, const float* ss_in, int32_t* idx_out,
+                                    float* ss_out, void* ws, size_t ws_bytes, void* stream);
+
+/* The activation of an MLP's down projection with its column scores in the
+ * same pass: H = bf16(SiLU(G) ⊙ U), SiLU(g) = g / (1 + e^-g) in fp32, and
+ * ss_out[j] = sum_i H[i,j]^2 over the stored (rounded) H, summed in fp32 in
+ * an order fixed by the shape.  G (gate output), U (up output), H bf16
+ * [M x N] with pitches multiples of 8, 16-byte aligned.  Workspace:
+ * rmm_silu_mul_score_workspace_size(M, N) bytes (may be 0). */
+RMM_API size_t rmm_silu_mul_score_workspace_size(int64_t M, int64_t N);
+RMM_API rmm_status rmm_silu_mul_score(const void* G, int64_t ldg, const void* U, int64_t ldu, int64_t M, int64_t N,
+                                      void* H, int64_t ldh, float* ss_out, void* ws, size_t ws_bytes, void* stream);
+
+/* A gated MLP block with every product reduced:
+ *   U = X_I W_up[I,:], G = X_I W_gate[I,:] with one I from X (rho_up);
+ *   H = SiLU(G) ⊙ U with its column scores fused into the producer;
+ *   Y = H_J W_down[J,:] with J = topk(ss(H)) (rho_down).
+ * X bf16 [M x d_model] (ldx); W_up, W_gate bf16 [d_model x d_ff] (ld_up,
+ * ld_gate multiples of 8); W_down bf16 [d_ff x d_model] (ld_down a multiple
+ * of 8); Y [M x d_model] (ldy) in out_dtype; all 16-byte aligned.  U, G, H
+ * are bf16 in the workspace.  idx_up (k_up) and idx_down (k_down) may be
+ * NULL.  Workspace: rmm_mlp_block_workspace_size bytes. */
+RMM_API size_t rmm_mlp_block_workspace_size(int64_t M, int64_t d_model, int64_t d_ff, double rho_up, double rho_down);
+RMM_API rmm_status rmm_mlp_block(const void* X, int64_t ldx, int64_t M, int64_t d_model, int64_t d_ff,
+                                 const void* W_up, int64_t ld_up, const void* W_gate, int64_t ld_gate,
+                                 const void* W_down, int64_t ld_down, double rho_up, double rho_down, void* Y,
+                                 int out_dtype, int64_t ldy, int32_t* idx_up, int32_t* idx_down, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------ reduced attention
  * Causal attention with both reductions of Metodología › Alcance de
  * Aplicación, for Q [B, Hq, S, D] and K, V [B, Hkv, S, D] bf16, contiguous

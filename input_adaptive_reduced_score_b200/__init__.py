@@ -24,7 +24,8 @@ __all__ = [
     "rmm_gemm", "rmm_gemm_workspace_size", "rmm_gemm_compacted",
     "rmm_matmul", "rmm_matmul_workspace_size", "rmm_gemm_w8", "rmm_gemm_w8_workspace_size", "rmm_matmul_w8",
     "rmm_matmul_w8_workspace_size", "rmm_attention", "rmm_attention_workspace_size", "rmm_decode_attention",
-    "rmm_decode_attention_workspace_size",
+    "rmm_decode_attention_workspace_size", "rmm_matmul_multi", "rmm_matmul_multi_workspace_size",
+    "rmm_silu_mul_score", "rmm_silu_mul_score_workspace_size", "rmm_mlp_block", "rmm_mlp_block_workspace_size",
     "exported_symbols", "declared_symbols",
 ]
 
@@ -81,6 +82,14 @@ _sig("rmm_matmul_w8", c_int, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64
 _sig("rmm_decode_attention_workspace_size", c_sz, c_i64, c_i64, c_i64, c_i64, c_dbl, c_int, c_int)
 _sig("rmm_decode_attention", c_int, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl, c_flt,
      c_vp, c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp)
+_sig("rmm_matmul_multi_workspace_size", c_sz, c_i64, c_i64, c_i64, c_dbl)
+_sig("rmm_matmul_multi", c_int, c_vp, c_i64, c_i64, c_i64, c_dbl, c_int, c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp,
+     c_vp, c_vp, c_vp, c_sz, c_vp)
+_sig("rmm_silu_mul_score_workspace_size", c_sz, c_i64, c_i64)
+_sig("rmm_silu_mul_score", c_int, c_vp, c_i64, c_vp, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_vp, c_sz, c_vp)
+_sig("rmm_mlp_block_workspace_size", c_sz, c_i64, c_i64, c_i64, c_dbl, c_dbl)
+_sig("rmm_mlp_block", c_int, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_dbl, c_dbl,
+     c_vp, c_int, c_i64, c_vp, c_vp, c_vp, c_sz, c_vp)
 _sig("rmm_attention_workspace_size", c_sz, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl)
 _sig("rmm_attention", c_int, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl, c_flt, c_vp, c_int,
      c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp)
@@ -421,4 +430,73 @@ def rmm_decode_attention(q, K, V, L: int, rho_d: float, rho_t: float, scale: flo
     _check(lib.rmm_decode_attention(_ptr(q), _ptr(K), _ptr(V), B, Hq, Hkv, L, Lmax, D, float(rho_d), float(rho_t),
                                     float(scale), _ptr(out), _dtype_code(out), _ptr(idx_d), _ptr(idx_t), _ptr(lse),
                                     _ptr(logits), _ptr(w), wn, _stream_ptr(stream)), "rmm_decode_attention")
+    return out
+
+
+def rmm_matmul_multi_workspace_size(M: int, d: int, N_max: int, rho: float) -> int:
+    return lib.rmm_matmul_multi_workspace_size(M, d, N_max, float(rho))
+
+
+def rmm_matmul_multi(A: torch.Tensor, Bs, rho: float, outs=None, out_dtype=None, ss_in: torch.Tensor = None,
+                     idx_out: torch.Tensor = None, ss_out: torch.Tensor = None, ws=None, stream=None):
+    """Y[i] = A[:, I] @ Bs[i][I, :] with one selection I shared by every weight."""
+    lda = _row_major(A, "A")
+    M, d = A.shape
+    n = len(Bs)
+    if outs is None:
+        outs = [torch.empty((M, B.shape[1]), dtype=out_dtype or A.dtype, device=A.device) for B in Bs]
+    ldb = [_row_major(B, "B") for B in Bs]
+    ldy = [_row_major(Y, "Y") for Y in outs]
+    Ns = [B.shape[1] for B in Bs]
+    arr_p = (ctypes.c_void_p * n)(*[_ptr(B) for B in Bs])
+    arr_y = (ctypes.c_void_p * n)(*[_ptr(Y) for Y in outs])
+    arr_ldb = (ctypes.c_int64 * n)(*ldb)
+    arr_n = (ctypes.c_int64 * n)(*Ns)
+    arr_ldy = (ctypes.c_int64 * n)(*ldy)
+    w, wn = _workspace(lib.rmm_matmul_multi_workspace_size(M, d, max(Ns), float(rho)), A.device, ws)
+    _check(lib.rmm_matmul_multi(_ptr(A), lda, M, d, float(rho), n, ctypes.cast(arr_p, c_vp), ctypes.cast(arr_ldb, c_vp),
+                                ctypes.cast(arr_n, c_vp), ctypes.cast(arr_y, c_vp), ctypes.cast(arr_ldy, c_vp),
+                                _dtype_code(outs[0]), _ptr(ss_in), _ptr(idx_out), _ptr(ss_out), _ptr(w), wn,
+                                _stream_ptr(stream)), "rmm_matmul_multi")
+    return outs
+
+
+def rmm_silu_mul_score_workspace_size(M: int, N: int) -> int:
+    return lib.rmm_silu_mul_score_workspace_size(M, N)
+
+
+def rmm_silu_mul_score(G: torch.Tensor, U: torch.Tensor, out: torch.Tensor = None, ss_out: torch.Tensor = None,
+                       ws=None, stream=None):
+    """H = bf16(SiLU(G) * U) and the column scores of H in one pass; returns (H, ss)."""
+    ldg, ldu = _row_major(G, "G"), _row_major(U, "U")
+    M, N = G.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=G.device)
+    if ss_out is None:
+        ss_out = torch.empty(N, dtype=torch.float32, device=G.device)
+    w, wn = _workspace(lib.rmm_silu_mul_score_workspace_size(M, N), G.device, ws)
+    _check(lib.rmm_silu_mul_score(_ptr(G), ldg, _ptr(U), ldu, M, N, _ptr(out), _row_major(out, "H"), _ptr(ss_out),
+                                  _ptr(w), wn, _stream_ptr(stream)), "rmm_silu_mul_score")
+    return out, ss_out
+
+
+def rmm_mlp_block_workspace_size(M: int, d_model: int, d_ff: int, rho_up: float, rho_down: float) -> int:
+    return lib.rmm_mlp_block_workspace_size(M, d_model, d_ff, float(rho_up), float(rho_down))
+
+
+def rmm_mlp_block(X: torch.Tensor, W_up: torch.Tensor, W_gate: torch.Tensor, W_down: torch.Tensor, rho_up: float,
+                  rho_down: float, out: torch.Tensor = None, out_dtype=None, idx_up: torch.Tensor = None,
+                  idx_down: torch.Tensor = None, ws=None, stream=None):
+    """Gated MLP block, every product reduced: Y = RMM(SiLU(RMM(X, W_gate)) * RMM(X, W_up), W_down)."""
+    ldx = _row_major(X, "X")
+    M, d_model = X.shape
+    d_ff = W_up.shape[1]
+    if out is None:
+        out = torch.empty((M, d_model), dtype=out_dtype or X.dtype, device=X.device)
+    w, wn = _workspace(lib.rmm_mlp_block_workspace_size(M, d_model, d_ff, float(rho_up), float(rho_down)),
+                       X.device, ws)
+    _check(lib.rmm_mlp_block(_ptr(X), ldx, M, d_model, d_ff, _ptr(W_up), _row_major(W_up, "W_up"), _ptr(W_gate),
+                             _row_major(W_gate, "W_gate"), _ptr(W_down), _row_major(W_down, "W_down"),
+                             float(rho_up), float(rho_down), _ptr(out), _dtype_code(out), _row_major(out, "Y"),
+                             _ptr(idx_up), _ptr(idx_down), _ptr(w), wn, _stream_ptr(stream)), "rmm_mlp_block")
     return out

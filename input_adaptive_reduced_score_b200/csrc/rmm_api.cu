@@ -2,6 +2,7 @@
 // argument validation, workspace carving, launches, error reporting.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -135,6 +136,35 @@ MatmulWs matmul_ws(int dtype, int64_t M, int64_t d, int64_t N, double rho) {
   return w;
 }
 
+}  // namespace
+
+extern "C" size_t rmm_matmul_multi_workspace_size(int64_t M, int64_t d, int64_t N_max, double rho);
+extern "C" size_t rmm_silu_mul_score_workspace_size(int64_t M, int64_t N);
+namespace {
+struct MlpWs {
+  size_t u, g, h, ss, inner, total;
+  int64_t ld_ff;
+};
+MlpWs mlp_ws(int64_t M, int64_t d_model, int64_t d_ff, double rho_up, double rho_down) {
+  MlpWs w{};
+  w.ld_ff = round_up(d_ff, 8);
+  const size_t act = align_up(static_cast<size_t>(M) * w.ld_ff * 2, kWsAlign);
+  size_t off = 0;
+  w.u = off;
+  off += act;
+  w.g = off;
+  off += act;
+  w.h = off;
+  off += act;
+  w.ss = off;
+  off += align_up(static_cast<size_t>(d_ff) * 4, kWsAlign);
+  w.inner = off;
+  const size_t inner = std::max({rmm_matmul_multi_workspace_size(M, d_model, d_ff, rho_up),
+                                 rmm_matmul_multi_workspace_size(M, d_ff, d_model, rho_down),
+                                 rmm_silu_mul_score_workspace_size(M, d_ff)});
+  w.total = off + inner;
+  return w;
+}
 }  // namespace
 
 extern "C" {
@@ -473,6 +503,151 @@ rmm_status rmm_matmul_w8(const void* A, int64_t lda, const int8_t* Bq, int64_t l
   if (st != RMM_OK) return st;
   return rmm_gemm_w8(ai, w.ld_ai, Bq, ldb, b_scale, idx, d, M, N, k, Y, out_dtype, ldy, base + w.bi, w.total - w.bi,
                      stream);
+}
+
+// ------------------------------------------------------------------ block driver
+
+size_t rmm_silu_mul_score_workspace_size(int64_t M, int64_t N) {
+  if (M < 0 || N < 1) return 0;
+  return score_workspace_bytes(RMM_BF16, 1, M, N);
+}
+
+rmm_status rmm_silu_mul_score(const void* G, int64_t ldg, const void* U, int64_t ldu, int64_t M, int64_t N, void* H,
+                              int64_t ldh, float* ss_out, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (M < 0 || N < 1 || ldg < N || ldu < N || ldh < N || M > kIntMax * 16)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_silu_mul_score: bad sizes");
+  if (!G || !U || !H || !ss_out) return fail(RMM_ERR_INVALID_ARG, "rmm_silu_mul_score: null pointer");
+  if (!aligned16(G) || !aligned16(U) || !aligned16(H) || ldg % 8 || ldu % 8 || ldh % 8)
+    return fail(RMM_ERR_UNSUPPORTED, "rmm_silu_mul_score: needs 16-byte aligned G/U/H and pitches multiples of 8");
+  const size_t need = rmm_silu_mul_score_workspace_size(M, N);
+  if (need && (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % kWsAlign))
+    return fail(RMM_ERR_WORKSPACE, "rmm_silu_mul_score: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes,
+                need);
+  return from_cuda(launch_silu_mul_score(G, ldg, U, ldu, H, ldh, M, N, ss_out, ws, static_cast<cudaStream_t>(stream)),
+                   "rmm_silu_mul_score: launch");
+}
+
+size_t rmm_matmul_multi_workspace_size(int64_t M, int64_t d, int64_t N_max, double rho) {
+  return rmm_matmul_workspace_size(RMM_BF16, M, d, N_max, rho);
+}
+
+rmm_status rmm_matmul_multi(const void* A, int64_t lda, int64_t M, int64_t d, double rho, int nprod,
+                            const void* const* B, const int64_t* ldb, const int64_t* N, void* const* Y,
+                            const int64_t* ldy, int out_dtype, const float* ss_in, int32_t* idx_out, float* ss_out,
+                            void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (!valid_dtype(out_dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_multi: out dtype %d", out_dtype);
+  const int64_t k = k_from_rho_impl(rho, d);
+  if (k < 1) return fail(RMM_ERR_INVALID_ARG, "rmm_matmul_multi: rho %g outside (0,1] or d < 1", rho);
+  if (nprod < 1 || !B || !ldb || !N || !Y || !ldy || M < 0 || lda < d || !A)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_matmul_multi: bad arguments");
+  int64_t nmax = 0;
+  for (int i = 0; i < nprod; ++i) {
+    if (!B[i] || !Y[i] || N[i] < 1 || ldb[i] < N[i] || ldy[i] < N[i])
+      return fail(RMM_ERR_INVALID_ARG, "rmm_matmul_multi: bad product %d", i);
+    if (!aligned16(B[i]) || ldb[i] % 8 || !aligned16(Y[i]))
+      return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_multi: product %d needs 16-byte aligned B and Y, ldb % 8 == 0", i);
+    nmax = std::max(nmax, N[i]);
+  }
+  const MatmulWs w = matmul_ws(RMM_BF16, M, d, nmax, rho);
+  if (!ws || ws_bytes < w.total || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
+    return fail(RMM_ERR_WORKSPACE, "rmm_matmul_multi: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes,
+                w.total);
+  char* base = static_cast<char*>(ws);
+  float* ss = ss_out ? ss_out : reinterpret_cast<float*>(base + w.ss);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+  void* ai = base + w.ai;
+  void* bi = base + w.bi;
+  const size_t bi_bytes = w.total - w.bi;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rmm_status st = RMM_OK;
+  bool compacted = false;
+  if (M == 0) return RMM_OK;
+  // one selection for every product
+  if (ss_in) {
+    st = rmm_topk(ss_in, 1, d, d, k, idx, k, stream);
+  } else if (select_rows_supported(M, d)) {
+    const cudaError_t e = launch_select_rows(A, M, d, lda, k, idx, ss, ai, w.ld_ai, s);
+    if (e != cudaSuccess) return from_cuda(e, "rmm_matmul_multi: row selection launch");
+    compacted = true;
+  } else {
+    st = rmm_score(A, RMM_BF16, 1, M, d, lda, 0, ss, d, 0, base + w.score, score_workspace_bytes(RMM_BF16, 1, M, d),
+                   stream);
+    if (st == RMM_OK) st = rmm_topk(ss, 1, d, d, k, idx, k, stream);
+  }
+  if (st != RMM_OK) return st;
+  for (int i = 0; i < nprod; ++i) {
+    if (M <= kGemvMaxM) {
+      if (!compacted) {
+        st = rmm_compact(A, RMM_BF16, M, d, lda, idx, k, ai, w.ld_ai, stream);
+        if (st != RMM_OK) return st;
+        compacted = true;
+      }
+      st = rmm_gemm(ai, w.ld_ai, B[i], ldb[i], idx, d, M, N[i], k, RMM_BF16, Y[i], out_dtype, ldy[i], bi, bi_bytes,
+                    stream);
+    } else {
+      const int64_t ld_bi = round_up(N[i], 8);
+      if (!compacted) {
+        st = rmm_compact_gather(A, lda, B[i], ldb[i], M, d, N[i], idx, k, ai, w.ld_ai, bi, ld_bi, stream);
+        compacted = true;
+      } else {
+        st = rmm_gather_rows(B[i], RMM_BF16, d, N[i], ldb[i], idx, k, bi, ld_bi, stream);
+      }
+      if (st == RMM_OK) st = rmm_gemm_compacted(ai, w.ld_ai, bi, ld_bi, M, N[i], k, Y[i], out_dtype, ldy[i], stream);
+    }
+    if (st != RMM_OK) return st;
+  }
+  return RMM_OK;
+}
+
+
+size_t rmm_mlp_block_workspace_size(int64_t M, int64_t d_model, int64_t d_ff, double rho_up, double rho_down) {
+  if (M < 1 || d_model < 1 || d_ff < 1 || k_from_rho_impl(rho_up, d_model) < 1 || k_from_rho_impl(rho_down, d_ff) < 1)
+    return 0;
+  return mlp_ws(M, d_model, d_ff, rho_up, rho_down).total;
+}
+
+rmm_status rmm_mlp_block(const void* X, int64_t ldx, int64_t M, int64_t d_model, int64_t d_ff, const void* W_up,
+                         int64_t ld_up, const void* W_gate, int64_t ld_gate, const void* W_down, int64_t ld_down,
+                         double rho_up, double rho_down, void* Y, int out_dtype, int64_t ldy, int32_t* idx_up,
+                         int32_t* idx_down, void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (M < 1 || d_model < 1 || d_ff < 1 || !X || !W_up || !W_gate || !W_down || !Y)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_mlp_block: bad arguments");
+  if (k_from_rho_impl(rho_up, d_model) < 1 || k_from_rho_impl(rho_down, d_ff) < 1)
+    return fail(RMM_ERR_INVALID_ARG, "rmm_mlp_block: rho outside (0,1]");
+  const MlpWs w = mlp_ws(M, d_model, d_ff, rho_up, rho_down);
+  if (!ws || ws_bytes < w.total || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
+    return fail(RMM_ERR_WORKSPACE, "rmm_mlp_block: workspace %zu < %zu bytes or not 256-byte aligned", ws_bytes,
+                w.total);
+  char* base = static_cast<char*>(ws);
+  void* U = base + w.u;
+  void* G = base + w.g;
+  void* H = base + w.h;
+  float* ssH = reinterpret_cast<float*>(base + w.ss);
+  void* inner = base + w.inner;
+  const size_t inner_bytes = w.total - w.inner;
+  // up and gate: one selection on X for both
+  const void* Bs[2] = {W_up, W_gate};
+  const int64_t ldbs[2] = {ld_up, ld_gate};
+  const int64_t Ns[2] = {d_ff, d_ff};
+  void* Ys[2] = {U, G};
+  const int64_t ldys[2] = {w.ld_ff, w.ld_ff};
+  rmm_status st = rmm_matmul_multi(X, ldx, M, d_model, rho_up, 2, Bs, ldbs, Ns, Ys, ldys, RMM_BF16, nullptr, idx_up,
+                                   nullptr, inner, inner_bytes, stream);
+  if (st != RMM_OK) return st;
+  // H = SiLU(G) * U with the down projection's column scores in the same pass
+  st = rmm_silu_mul_score(G, w.ld_ff, U, w.ld_ff, M, d_ff, H, w.ld_ff, ssH, inner, inner_bytes, stream);
+  if (st != RMM_OK) return st;
+  // down: selection from the fused scores
+  const void* Bd[1] = {W_down};
+  const int64_t ldbd[1] = {ld_down};
+  const int64_t Nd[1] = {d_model};
+  void* Yd[1] = {Y};
+  const int64_t ldyd[1] = {ldy};
+  return rmm_matmul_multi(H, w.ld_ff, M, d_ff, rho_down, 1, Bd, ldbd, Nd, Yd, ldyd, out_dtype, ssH, idx_down, nullptr,
+                          inner, inner_bytes, stream);
 }
 
 size_t rmm_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t L, int64_t D, double rho_t,

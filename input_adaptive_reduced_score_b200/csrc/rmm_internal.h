@@ -38,6 +38,12 @@ cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int
                          int64_t batch_stride, float* ss, int64_t ld_ss, int sqrt_out, void* ws,
                          cudaStream_t stream);
 
+// H = bf16(SiLU(G) * U) and ss_j = sum_i H[i,j]^2 in one pass over [M x d]
+// bf16 G, U, H (16-byte aligned, pitches multiples of 8); the workspace holds
+// score_workspace_bytes(1, 1, M, d) bytes of row-split partials.
+cudaError_t launch_silu_mul_score(const void* G, int64_t ldg, const void* U, int64_t ldu, void* H, int64_t ldh,
+                                  int64_t M, int64_t d, float* ss, void* ws, cudaStream_t stream);
+
 // ---- top-k (rmm_topk.cu)
 cudaError_t launch_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k,
                         int32_t* idx, int64_t ld_idx, cudaStream_t stream);

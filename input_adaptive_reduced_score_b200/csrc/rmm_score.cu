@@ -10,6 +10,11 @@
 // Row groups combine by a fixed pairwise tree in shared memory; row splits are
 // combined by a second kernel in a fixed order.  No atomics, so the
 // result depends only on the shape.
+//
+// silu_mul_score_kernel fuses the score of the MLP down projection into the
+// producer of its activation: H = SiLU(G) * U (G, U the gate and up outputs,
+// bf16), rounded to bf16 and stored, and ss_j = sum_i H[i,j]^2 of the stored
+// values, on the same plan, so H is read back by nobody before the top-k.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -135,6 +140,91 @@ __global__ void __launch_bounds__(kScoreThreads) score_partial_kernel(
   }
 }
 
+// H = bf16(SiLU(G) * U) with SiLU(g) = g / (1 + e^-g) in fp32, and the
+// column sums of the stored H's squares, on the bf16 score plan (16-byte
+// vectors; G, U, H 16-byte aligned with row pitches multiples of 8).
+// Grid: x = column strip, y = row split.
+__global__ void __launch_bounds__(kScoreThreads) silu_mul_score_kernel(
+    const __nv_bfloat16* __restrict__ G, int64_t ldg, const __nv_bfloat16* __restrict__ U, int64_t ldu,
+    __nv_bfloat16* __restrict__ H, int64_t ldh, int64_t M, int64_t d, int col_threads, int64_t rows_per_split,
+    float* __restrict__ out, int64_t out_split_stride) {
+  constexpr int V = 8;
+  __shared__ float red[kScoreThreads * V];
+  pdl_wait();
+  pdl_trigger();
+  const int tx = threadIdx.x % col_threads;
+  const int ty = threadIdx.x / col_threads;
+  const int row_groups = kScoreThreads / col_threads;
+  const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * col_threads + tx) * V;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(M, r0 + rows_per_split);
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  auto produce = [&](float gv, float uv) {
+    const float h = gv / (1.f + expf(-gv)) * uv;
+    return __float2bfloat16_rn(h);
+  };
+  if (col0 < d) {
+    if (col0 + V <= d) {
+#pragma unroll
+      for (int u0 = 0; u0 < kRowsPerThread; u0 += 4) {
+        uint4 rg[4], ru[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t r = r0 + ty + static_cast<int64_t>(u0 + u) * row_groups;
+          rg[u] = r < r1 ? __ldg(reinterpret_cast<const uint4*>(G + r * ldg + col0)) : make_uint4(0, 0, 0, 0);
+          ru[u] = r < r1 ? __ldg(reinterpret_cast<const uint4*>(U + r * ldu + col0)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t r = r0 + ty + static_cast<int64_t>(u0 + u) * row_groups;
+          float gx[V], ux[V];
+          Lanes<__nv_bfloat16>::unpack(rg[u], gx);
+          Lanes<__nv_bfloat16>::unpack(ru[u], ux);
+          uint32_t packed[4];
+#pragma unroll
+          for (int e = 0; e < V; e += 2) {
+            const __nv_bfloat16 h0 = produce(gx[e], ux[e]), h1 = produce(gx[e + 1], ux[e + 1]);
+            const float f0 = __bfloat162float(h0), f1 = __bfloat162float(h1);
+            acc[e] = fmaf(f0, f0, acc[e]);
+            acc[e + 1] = fmaf(f1, f1, acc[e + 1]);
+            packed[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                            (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+          }
+          if (r < r1)
+            *reinterpret_cast<uint4*>(H + r * ldh + col0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+      }
+    } else {
+      for (int64_t r = r0 + ty; r < r1; r += row_groups) {
+        for (int e = 0; e < V && col0 + e < d; ++e) {
+          const __nv_bfloat16 h = produce(__bfloat162float(G[r * ldg + col0 + e]), __bfloat162float(U[r * ldu + col0 + e]));
+          H[r * ldh + col0 + e] = h;
+          const float f = __bfloat162float(h);
+          acc[e] = fmaf(f, f, acc[e]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < V; ++e) red[(ty * col_threads + tx) * V + e] = acc[e];
+  __syncthreads();
+  for (int s = row_groups / 2; s >= 1; s >>= 1) {
+    if (ty < s) {
+#pragma unroll
+      for (int e = 0; e < V; ++e) red[(ty * col_threads + tx) * V + e] += red[((ty + s) * col_threads + tx) * V + e];
+    }
+    __syncthreads();
+  }
+  if (ty == 0) {
+    float* o = out + static_cast<int64_t>(blockIdx.y) * out_split_stride;
+#pragma unroll
+    for (int e = 0; e < V; ++e)
+      if (col0 + e < d) o[col0 + e] = red[tx * V + e];
+  }
+}
+
 // Sum the row-split partials: a 256-thread CTA covers 32 columns; thread
 // (c, g) adds splits g, g+8, g+16, ... of column c in increasing order, then
 // the 8 group sums combine by a fixed pairwise tree.  Grid: x = column
@@ -219,6 +309,22 @@ cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int
   const dim3 g2(static_cast<unsigned>((d + 31) / 32), static_cast<unsigned>(batch));
   return launch_pdl(score_finalize_kernel, g2, dim3(256), 0, stream, static_cast<const float*>(ws), d, p.splits, ss,
                     ld_ss, sqrt_out);
+}
+
+cudaError_t launch_silu_mul_score(const void* G, int64_t ldg, const void* U, int64_t ldu, void* H, int64_t ldh,
+                                  int64_t M, int64_t d, float* ss, void* ws, cudaStream_t stream) {
+  const ScorePlan p = score_plan(1, 1, M, d);
+  const dim3 grid(static_cast<unsigned>(p.strips), static_cast<unsigned>(p.splits));
+  const bool direct = p.splits <= 1;
+  float* out = direct ? ss : static_cast<float*>(ws);
+  cudaError_t e = launch_pdl(silu_mul_score_kernel, grid, dim3(kScoreThreads), 0, stream,
+                             static_cast<const __nv_bfloat16*>(G), ldg, static_cast<const __nv_bfloat16*>(U), ldu,
+                             static_cast<__nv_bfloat16*>(H), ldh, M, d, p.col_threads, p.rows_per_split, out,
+                             direct ? int64_t{0} : d);
+  if (e != cudaSuccess || direct) return e;
+  const dim3 g2(static_cast<unsigned>((d + 31) / 32), 1u);
+  return launch_pdl(score_finalize_kernel, g2, dim3(256), 0, stream, static_cast<const float*>(ws), d, p.splits, ss,
+                    d, 0);
 }
 
 }  // namespace rmm

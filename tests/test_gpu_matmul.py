@@ -15,7 +15,7 @@ import torch
 import oracle
 import workloads as W
 from oracle.conditioning import widen_topk_gaps
-from tests.helpers import bf16_tensor, check_bf16_output, rel_fro, sample_rows, to_device, to_f64
+from tests.helpers import bf16_tensor, bf16_ulp, check_bf16_output, rel_fro, sample_rows, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -592,4 +592,103 @@ def test_gemm_w8_rejects_bad_layouts():
         R.rmm_gemm_w8(A_I, _pitched16(q), s[:10], it)
     with pytest.raises(TypeError):
         R.rmm_gemm_w8(A_I, _pitched16(q).to(torch.int16), s, it)
+    no_device_error()
+
+
+# ------------------------------------------------------------------ block driver
+
+@pytest.mark.parametrize("M", [5, 300, 1024])
+def test_matmul_multi_shared_selection(M):
+    """q/k/v-style products on one activation: one index set, every product
+    against the oracle."""
+    d, Ns, rho = 1024, (512, 128, 264), 0.5
+    A_bits = W.llm_activation_bf16(101 + M, M, d)
+    k = oracle.k_from_rho(rho, d)
+    cond, _ = widen_topk_gaps(A_bits, "bf16", [k])
+    Ac = oracle.decode(cond, "bf16")
+    Wb = [W.weight_bf16(102, d, n, group=i) for i, n in enumerate(Ns)]
+    Bm = [oracle.decode(w, "bf16") for w in Wb]
+    idx_out = torch.empty(k, dtype=torch.int32, device="cuda")
+    Ys = R.rmm_matmul_multi(bf16_tensor(cond), [_pitched(bf16_tensor(w)) for w in Wb], rho, idx_out=idx_out)
+    refs, idx, _ = oracle.block.matmul_shared(Ac, Bm, rho)
+    np.testing.assert_array_equal(idx_out.cpu().numpy(), idx)
+    for Y, ref, B in zip(Ys, refs, Bm):
+        check_bf16_output(to_f64(Y), ref, np.abs(Ac[:, idx]) @ np.abs(B[idx, :]), k)
+    no_device_error()
+
+
+def test_matmul_multi_given_scores():
+    """Selection from caller-given scores (no score pass)."""
+    M, d, N, rho = 64, 512, 256, 0.3
+    A_bits = W.llm_activation_bf16(111, M, d)
+    k = oracle.k_from_rho(rho, d)
+    cond, _ = widen_topk_gaps(A_bits, "bf16", [k])
+    Ac = oracle.decode(cond, "bf16")
+    ss = oracle.column_sq_norms(Ac)
+    Wb = W.weight_bf16(112, d, N)
+    idx_out = torch.empty(k, dtype=torch.int32, device="cuda")
+    (Y,) = R.rmm_matmul_multi(bf16_tensor(cond), [bf16_tensor(Wb)], rho, idx_out=idx_out,
+                              ss_in=torch.from_numpy(ss.astype(np.float32)).cuda())
+    idx = oracle.topk_indices(ss, k)
+    np.testing.assert_array_equal(idx_out.cpu().numpy(), idx)
+    Bm = oracle.decode(Wb, "bf16")
+    check_bf16_output(to_f64(Y), Ac[:, idx] @ Bm[idx, :], np.abs(Ac[:, idx]) @ np.abs(Bm[idx, :]), k)
+    no_device_error()
+
+
+def _gate_up(seed, M, N):
+    rng = np.random.default_rng(seed)
+    G = W.f32_to_bf16_bits(rng.standard_normal((M, N)) * 2.0)
+    U = W.f32_to_bf16_bits(rng.standard_normal((M, N)))
+    return G, U
+
+
+@pytest.mark.parametrize("M,N", [(300, 1000), (4096, 2048), (7, 13)])
+def test_silu_mul_score(M, N):
+    """H within one bf16 ulp of the oracle (fp32 SiLU rounds differently near
+    a bf16 rounding boundary, so a few elements may differ by one ulp), the
+    fused scores within 1e-3 of the oracle's scores of its own H."""
+    G, U = _gate_up(120 + M, M, N)
+    Gt, Ut = bf16_tensor(G), bf16_tensor(U)
+    if N % 8:
+        Gt, Ut = _pitched(Gt), _pitched(Ut)
+    H = torch.zeros((M, (N + 7) // 8 * 8), dtype=torch.bfloat16, device="cuda")[:, :N]
+    H, ss = R.rmm_silu_mul_score(Gt, Ut, out=H)
+    ref = oracle.block.silu_mul_bf16(oracle.decode(G, "bf16"), oracle.decode(U, "bf16"))
+    got = to_f64(H)
+    diff = np.abs(got - ref)
+    assert np.all(diff <= bf16_ulp(ref) + 1e-30)
+    assert np.mean(diff > 0) < 1e-3
+    np.testing.assert_allclose(to_f64(ss), oracle.column_sq_norms(ref), rtol=1e-3, atol=1e-30)
+    no_device_error()
+
+
+@pytest.mark.parametrize("M", [4, 512])
+def test_mlp_block(M):
+    """The gated MLP block end to end.  The up/gate selection reads X (gaps
+    widened): bit-exact.  The down selection reads the computed H, whose fp32
+    rounding may differ from the oracle's by one ulp in a few elements: every
+    index where the sets differ must lie within 1e-3 relative of the oracle's
+    boundary score, and Y within 5e-3 relative Frobenius of the oracle."""
+    dm, dff, rho_up, rho_down = 1024, 2816, 0.8, 0.5
+    X_bits = W.llm_activation_bf16(130 + M, M, dm)
+    ku = oracle.k_from_rho(rho_up, dm)
+    cond, _ = widen_topk_gaps(X_bits, "bf16", [ku])
+    Xc = oracle.decode(cond, "bf16")
+    Wu = W.weight_bf16(131, dm, dff, group=0)
+    Wg = W.weight_bf16(131, dm, dff, group=1)
+    Wd = W.weight_bf16(131, dff, dm, group=2)
+    kd = oracle.k_from_rho(rho_down, dff)
+    idx_up = torch.empty(ku, dtype=torch.int32, device="cuda")
+    idx_down = torch.empty(kd, dtype=torch.int32, device="cuda")
+    Y = R.rmm_mlp_block(bf16_tensor(cond), bf16_tensor(Wu), bf16_tensor(Wg), bf16_tensor(Wd), rho_up, rho_down,
+                        idx_up=idx_up, idx_down=idx_down)
+    r = oracle.block.mlp_block(Xc, *(oracle.decode(w, "bf16") for w in (Wu, Wg, Wd)), rho_up, rho_down)
+    np.testing.assert_array_equal(idx_up.cpu().numpy(), r["I"])
+    got_j = idx_down.cpu().numpy()
+    assert np.all(np.diff(got_j) > 0)
+    diff = np.setxor1d(got_j, r["J"])
+    thr = np.sort(r["ssH"])[::-1][kd - 1]
+    assert np.all(np.abs(r["ssH"][diff] - thr) <= 1e-3 * thr), (diff, r["ssH"][diff], thr)
+    assert rel_fro(to_f64(Y), r["Y"]) <= 5e-3
     no_device_error()
