@@ -4,30 +4,30 @@
 // autoregressive generation, Resultados Experimentales).
 //
 // HBM-bound: only the k kept rows of B are read, each once, in place (no
-// gathered copy).  A block owns 256 columns of Y (128 above 8 activation
-// rows) and a range of kept rows; its 8 warps take alternate rows of the
-// range, every lane loading 8 columns (16 bytes; 4 columns, 8 bytes, above 8
-// rows) of a row and accumulating them into fp32 sums.  The block's
-// kept-row indices and A_I values are staged in shared memory first (A_I as
-// fp32, [row][m], so one vector load serves four activation rows), so each
-// batch of row loads goes out without waiting for its indices.  Warps are summed in a fixed order in shared
-// memory.  Row ranges (splits) of one column slice run as one thread-block
-// cluster (up to 8 blocks): each block adds every split's sums for its share
-// of the outputs, in split order, through distributed shared memory; beyond 8
+// gathered copy).  A block owns 256 columns of Y and a range of kept rows;
+// the block's kept-row indices and A_I values are staged in shared memory
+// first.  Two kernels:
+//  - up to 4 activation rows, gemv_stream_kernel: each warp keeps six stages
+//    of four kept rows in flight as 16-byte asynchronous copies into its own
+//    ring in shared memory (192 rows in flight per block without holding
+//    them in registers); every lane then reads its 8 columns and accumulates
+//    fp32 FMAs; warps are summed in a fixed order.
+//  - 5 to 16 rows, gemv_mma_kernel: the FMAs (8 per row and column) would
+//    set the time, so the block runs mma.sync m16n8k16 (16 activation rows
+//    are one tile's M): stages of 32 kept rows x 256 columns arrive by
+//    cp.async, A_I comes from shared memory with ldmatrix and each stage's
+//    row-major weight tile with ldmatrix.trans; each warp owns 32 columns.
+// Row ranges (splits) of one column slice run as one thread-block cluster
+// (up to 8 blocks): each block adds every split's sums for its share of the
+// outputs, in split order, through distributed shared memory; beyond 8
 // splits the sums go through global memory and a second kernel adds them in
 // split order.  Either way the result depends only on the shape.
 //
 // An int8 weight (weight-only quantisation with one fp32 scale per output
-// column; Resultados Experimentales › Compatibilidad) takes the same path
-// with half the bytes per row: each lane loads 8 (or 4) int8 values, widens
-// them exactly to fp32, and the column scale multiplies the finished sum.
-//
-// Up to 8 activation rows the rows are streamed rather than loaded into
-// registers (gemv_stream_kernel): each warp keeps six stages of four kept
-// rows in flight as 16-byte asynchronous copies into its own ring in shared
-// memory, so a block has 192 rows in flight without holding them in
-// registers.  The register-loading kernel serves 9 to 16 rows, where the
-// FMAs rather than the loads set the time.
+// column; Resultados Experimentales › Compatibilidad) takes the same paths
+// with half the bytes per row: the stream kernel widens 8 int8 values per
+// lane exactly to fp32, the tensor-core kernel widens each stage to bf16
+// (exact) in shared memory; the column scale multiplies the finished sum.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -40,202 +40,13 @@
 namespace rmm {
 namespace {
 
-constexpr int kGemvThreads = 256;
-constexpr int kGemvWarps = kGemvThreads / 32;
 constexpr int kGemvMaxRows = 4096;  // kept rows per block (the staging buffer bounds it further)
 constexpr int kGemvMaxCluster = 8;  // splits reduced through distributed shared memory (portable cluster size)
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Columns per lane: 8 up to 8 activation rows, else 4, so the accumulators
-// stay at MT x CPL <= 64 registers; a lane's load is CPL weights (16 or 8
-// bytes of bf16, 8 or 4 bytes of int8).
-template <int MT, bool kW8 = false>
-struct GemvShape {
-  static constexpr int CPL = MT <= 8 ? 8 : 4;
-  static constexpr int COLS = 32 * CPL;            // columns of Y per block
-  // rows per batch (two batches in flight per warp); int8 rows are half the
-  // bytes, so up to 4 activation rows they take twice the batch in the same
-  // registers
-  static constexpr int U = (MT == 8 ? 4 : 8) * (kW8 && MT <= 4 ? 2 : 1);
-  using Vec16 = typename std::conditional<CPL == 8, uint4, uint2>::type;
-  using Vec8 = typename std::conditional<CPL == 8, uint2, unsigned int>::type;
-  using Vec = typename std::conditional<kW8, Vec8, Vec16>::type;
-};
-
-// grid: x = column slice, y = row split.  Dynamic shared memory:
-// max(rows x (MT + 1), warps x MT x COLS) words.
-// kW8: B is int8 (ldb in bytes) and b_scale[c] multiplies column c.
-template <int MT, bool kW8>
-__global__ void __launch_bounds__(kGemvThreads, 2)
-    gemv_rows_kernel(const uint16_t* __restrict__ AI, int64_t ld_ai, const void* __restrict__ Bv, int64_t ldb,
-                     const float* __restrict__ b_scale, const int32_t* __restrict__ idx, int M, int64_t d, int64_t N,
-                     int64_t k, int rows_per_split, float* __restrict__ partial, void* __restrict__ Y, int out_f32,
-                     int64_t ldy, int clustered, unsigned* err) {
-  using Sh = GemvShape<MT, kW8>;
-  using Vec = typename Sh::Vec;
-  constexpr int CPL = Sh::CPL, COLS = Sh::COLS, U = Sh::U;
-  extern __shared__ __align__(16) float sm[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
-  const int nrows = static_cast<int>(k - r0 < rows_per_split ? k - r0 : rows_per_split);
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * COLS + lane * CPL;
-  pdl_wait();
-  pdl_trigger();
-
-  // stage A_I[:, r0 .. r0 + nrows) as fp32 [row][m] (rows of MT, zero past
-  // M; read along rows, so coalesced) and the rows' indices after it (-1 for
-  // an index outside [0, d))
-  int32_t* sidx = reinterpret_cast<int32_t*>(sm + nrows * MT);
-  for (int m = 0; m < MT; ++m)
-    for (int rr = threadIdx.x; rr < nrows; rr += kGemvThreads)
-      sm[rr * MT + m] =
-          m < M ? __uint_as_float(static_cast<uint32_t>(AI[static_cast<int64_t>(m) * ld_ai + r0 + rr]) << 16) : 0.f;
-  bool bad = false;
-  for (int rr = threadIdx.x; rr < nrows; rr += kGemvThreads) {
-    const int32_t j = __ldg(idx + r0 + rr);
-    const bool ok = j >= 0 && j < d;
-    bad |= !ok;
-    sidx[rr] = ok ? j : -1;
-  }
-  if (bad) record_error(err, kDevErrBadIndex);
-  __syncthreads();
-
-  float acc[MT][CPL];
-#pragma unroll
-  for (int m = 0; m < MT; ++m)
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) acc[m][c] = 0.f;
-
-  const bool col_ok = c0 < N;
-  // batch t holds rows warp + (t*U + u)*8, u < U; the loads of batch t+1 are
-  // issued before batch t is consumed (two register buffers)
-  auto load = [&](int t, Vec (&w)[U]) {
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int rr = warp + (t * U + u) * kGemvWarps;
-      w[u] = Vec{};
-      if (rr < nrows) {
-        const int32_t j = sidx[rr];
-        if (j >= 0 && col_ok) {
-          if constexpr (kW8)
-            w[u] = __ldcs(reinterpret_cast<const Vec*>(static_cast<const int8_t*>(Bv) + static_cast<int64_t>(j) * ldb + c0));
-          else
-            w[u] = __ldcs(reinterpret_cast<const Vec*>(static_cast<const uint16_t*>(Bv) + static_cast<int64_t>(j) * ldb + c0));
-        }
-      }
-    }
-  };
-  auto consume = [&](int t, const Vec (&w)[U]) {
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int rr = warp + (t * U + u) * kGemvWarps;
-      if (rr < nrows) {
-        float b[CPL];
-        const uint32_t* wv = reinterpret_cast<const uint32_t*>(&w[u]);
-        if constexpr (kW8) {
-#pragma unroll
-          for (int q = 0; q < CPL / 4; ++q) {
-            float f[4];
-            i8x4_to_f32(wv[q], f);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) b[4 * q + e] = f[e];
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < CPL / 2; ++q) {
-            b[2 * q] = bf16_lo(wv[q]);
-            b[2 * q + 1] = bf16_hi(wv[q]);
-          }
-        }
-        const float* a = sm + rr * MT;
-#pragma unroll
-        for (int m4 = 0; m4 < MT; m4 += 4) {
-          float av[4];
-          if (MT >= 4) {
-            const float4 q = *reinterpret_cast<const float4*>(a + m4);
-            av[0] = q.x; av[1] = q.y; av[2] = q.z; av[3] = q.w;
-          } else {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) av[q] = q < MT ? a[q] : 0.f;
-          }
-#pragma unroll
-          for (int q = 0; q < 4 && m4 + q < MT; ++q)
-#pragma unroll
-            for (int c = 0; c < CPL; ++c) acc[m4 + q][c] = fmaf(av[q], b[c], acc[m4 + q][c]);
-        }
-      }
-    }
-  };
-  const int rows_w = (nrows - warp + kGemvWarps - 1) / kGemvWarps;  // rows of this warp
-  const int nbatch = (rows_w + U - 1) / U;
-  Vec wa[U], wb[U];
-  if (nbatch > 0) load(0, wa);
-  for (int t = 0; t < nbatch; t += 2) {
-    if (t + 1 < nbatch) load(t + 1, wb);
-    consume(t, wa);
-    if (t + 1 < nbatch) {
-      if (t + 2 < nbatch) load(t + 2, wa);
-      consume(t + 1, wb);
-    }
-  }
-
-  // sum the warps in a fixed order (the staging buffer is reused): red[m][c]
-  // (in warp 0's slot) = sum over warps
-  __syncthreads();
-  float* red = sm;  // [warp][m][COLS]
-#pragma unroll
-  for (int m = 0; m < MT; ++m)
-#pragma unroll
-    for (int c = 0; c < CPL; c += 4)
-      *reinterpret_cast<float4*>(red + (warp * MT + m) * COLS + lane * CPL + c) =
-          make_float4(acc[m][c], acc[m][c + 1], acc[m][c + 2], acc[m][c + 3]);
-  __syncthreads();
-  const int nout = MT * COLS;
-  for (int e = threadIdx.x; e < nout; e += kGemvThreads) {
-    float sum = 0.f;
-#pragma unroll
-    for (int wq = 0; wq < kGemvWarps; ++wq) sum += red[wq * nout + e];
-    red[e] = sum;
-  }
-  auto store = [&](int e, float v) {
-    const int m = e / COLS, cl = e % COLS;
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * COLS + cl;
-    if (m >= M || c >= N) return;
-    if constexpr (kW8) v *= __ldg(b_scale + c);
-    if (out_f32) {
-      static_cast<float*>(Y)[static_cast<int64_t>(m) * ldy + c] = v;
-    } else {
-      static_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(m) * ldy + c] = __float2bfloat16_rn(v);
-    }
-  };
-  if (gridDim.y == 1) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < nout; e += kGemvThreads) store(e, red[e]);
-  } else if (clustered) {
-    // the splits of this column slice form the cluster (rank = split)
-    cluster_sync();
-    const uint32_t nsplit = gridDim.y, rank = cluster_ctarank();
-    const uint32_t red_s = smem_u32(red);
-    for (int e = static_cast<int>(rank) * kGemvThreads + threadIdx.x; e < nout;
-         e += static_cast<int>(nsplit) * kGemvThreads) {
-      float v = 0.f;
-      for (uint32_t q = 0; q < nsplit; ++q) v += ld_dsmem_f32(mapa_shared(red_s + e * 4, q));
-      store(e, v);
-    }
-    cluster_sync();  // no block leaves while another may still read its shared memory
-  } else {
-    __syncthreads();
-    for (int e = threadIdx.x; e < nout; e += kGemvThreads) {
-      const int m = e / COLS, cl = e % COLS;
-      const int64_t c = static_cast<int64_t>(blockIdx.x) * COLS + cl;
-      if (m < M && c < N) partial[(static_cast<int64_t>(blockIdx.y) * M + m) * N + c] = red[e];
-    }
-  }
-}
-
-// ---------------------------------------------------------------- streamed rows (M <= 8)
+// ---------------------------------------------------------------- streamed rows (M <= 4)
 
 constexpr int kStreamWarps = 8;
 constexpr int kStreamThreads = 32 * kStreamWarps;
@@ -451,6 +262,216 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
   }
 }
 
+// ---------------------------------------------------------------- 9 to 16 rows on the tensor cores
+
+constexpr int kMmaThreads = 256;
+constexpr int kMmaCols = 256;          // columns of Y per block, 32 per warp
+constexpr int kMmaRowsPerStage = 32;   // kept rows per stage: two k16 steps
+template <bool kW8>
+constexpr int mma_stages() { return kW8 ? 8 : 5; }  // two blocks fit an SM
+constexpr int kMmaAiBytes = 32 * 1024; // A_I staging (bf16 [16][rows]) per block
+
+template <bool kW8>
+constexpr int mma_stage_pitch() { return kMmaCols * (kW8 ? 1 : 2) + 16; }  // bytes per staged row
+constexpr int kMmaWidePitch = kMmaCols * 2 + 16;                           // widened int8 row
+
+template <bool kW8>
+size_t mma_smem_bytes(int rows_per_split) {
+  const size_t ring = static_cast<size_t>(mma_stages<kW8>()) * kMmaRowsPerStage * mma_stage_pitch<kW8>();
+  const size_t wide = kW8 ? static_cast<size_t>(kMmaRowsPerStage) * kMmaWidePitch : 0;
+  const size_t ai = static_cast<size_t>(16) * ((rows_per_split + 31) / 32 * 32 * 2 + 16);
+  const size_t idx = static_cast<size_t>(rows_per_split + 32) * 4;
+  const size_t red = static_cast<size_t>(16) * kMmaCols * 4;
+  return std::max(ring + wide + ai + idx, red + ai + idx);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// grid: x = column slice of 256, y = row split; M <= 16 (rows past M are zero).
+template <bool kW8>
+__global__ void __launch_bounds__(kMmaThreads, 2)
+    gemv_mma_kernel(const uint16_t* __restrict__ AI, int64_t ld_ai, const void* __restrict__ Bv, int64_t ldb,
+                    const float* __restrict__ b_scale, const int32_t* __restrict__ idx, int M, int64_t d, int64_t N,
+                    int64_t k, int rows_per_split, float* __restrict__ partial, void* __restrict__ Y, int out_f32,
+                    int64_t ldy, int clustered, unsigned* err) {
+  constexpr int ELT = kW8 ? 1 : 2;
+  constexpr int PITCH = mma_stage_pitch<kW8>();
+  constexpr int RPS = kMmaRowsPerStage;
+  constexpr int S = mma_stages<kW8>();
+  constexpr int COLS = kMmaCols;
+  constexpr int CHUNKS = RPS * COLS * ELT / 16;  // 16-byte copies per stage
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int nrows = static_cast<int>(k - r0 < rows_per_split ? k - r0 : rows_per_split);
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * COLS;
+  const int ncols = static_cast<int>(N - c0 < COLS ? N - c0 : COLS);
+  const int rows16 = (rows_per_split + RPS - 1) / RPS * RPS;  // staged rows, whole stages
+  const int ai_pitch = rows16 * 2 + 16;  // bytes per A_I row (bf16), padded
+  const size_t ring_bytes = static_cast<size_t>(S) * RPS * PITCH;
+  const size_t wide_bytes = kW8 ? static_cast<size_t>(RPS) * kMmaWidePitch : 0;
+  uint8_t* wide = smem + ring_bytes;
+  uint8_t* sai = smem + std::max(ring_bytes + wide_bytes, static_cast<size_t>(16) * COLS * 4);
+  int32_t* sidx = reinterpret_cast<int32_t*>(sai + static_cast<size_t>(16) * ai_pitch);
+  pdl_wait();
+  pdl_trigger();
+
+  // A_I rows (zero past M and past the split's rows) and the kept indices
+  // (-1 for an index outside [0, d) and past the split's rows)
+  for (int e = threadIdx.x; e < 16 * rows16; e += kMmaThreads) {
+    const int m = e / rows16, r = e % rows16;
+    const uint16_t v = (m < M && r < nrows) ? AI[static_cast<int64_t>(m) * ld_ai + r0 + r] : uint16_t{0};
+    *reinterpret_cast<uint16_t*>(sai + m * ai_pitch + r * 2) = v;
+  }
+  bool bad = false;
+  for (int r = threadIdx.x; r < rows16; r += kMmaThreads) {
+    int32_t j = -1;
+    if (r < nrows) {
+      j = __ldg(idx + r0 + r);
+      if (j < 0 || j >= d) {
+        bad = true;
+        j = -1;
+      }
+    }
+    sidx[r] = j;
+  }
+  if (bad) record_error(err, kDevErrBadIndex);
+  __syncthreads();
+
+  const char* B8 = static_cast<const char*>(Bv);
+  const int nst = (nrows + RPS - 1) / RPS;
+  const uint32_t ring = smem_u32(smem);
+  auto issue = [&](int st) {
+    if (st < nst) {
+      const uint32_t base = ring + static_cast<uint32_t>((st % S) * RPS * PITCH);
+      for (int e = threadIdx.x; e < CHUNKS; e += kMmaThreads) {
+        const int r = e / (COLS * ELT / 16), piece = e % (COLS * ELT / 16);
+        const int32_t j = sidx[st * RPS + r];
+        const int rem = (ncols - piece * (16 / ELT)) * ELT;  // bytes of this piece inside the matrix
+        const uint32_t nb = j < 0 || rem <= 0 ? 0u : static_cast<uint32_t>(rem < 16 ? rem : 16);
+        const void* src = nb ? static_cast<const void*>(B8 + (static_cast<int64_t>(j) * ldb + c0) * ELT + piece * 16)
+                             : Bv;
+        cp_async16(base + r * PITCH + piece * 16, src, nb);
+      }
+    }
+    cp_async_commit();
+  };
+
+  float acc[4][4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+  const uint32_t ai_base = smem_u32(sai);
+  const uint32_t wide_base = smem_u32(wide);
+#pragma unroll
+  for (int st = 0; st < S - 1; ++st) issue(st);
+  for (int st = 0; st < nst; ++st) {
+    issue(st + S - 1);
+    cp_async_wait<S - 1>();
+    __syncthreads();  // every thread's copies of stage st have landed
+    uint32_t tile = ring + static_cast<uint32_t>((st % S) * RPS * PITCH);
+    uint32_t tpitch = PITCH;
+    if constexpr (kW8) {
+      // widen the int8 stage to bf16 (exact) in a separate buffer
+      const uint8_t* src = smem + (st % S) * RPS * PITCH;
+      for (int e = threadIdx.x; e < RPS * COLS / 4; e += kMmaThreads) {
+        const int r = e / (COLS / 4), c4 = e % (COLS / 4);
+        float f[4];
+        i8x4_to_f32(*reinterpret_cast<const uint32_t*>(src + r * PITCH + c4 * 4), f);
+        *reinterpret_cast<uint2*>(wide + r * kMmaWidePitch + c4 * 8) =
+            make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+      }
+      __syncthreads();
+      tile = wide_base;
+      tpitch = kMmaWidePitch;
+    }
+#pragma unroll
+    for (int ks = 0; ks < RPS / 16; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(ai_base + ((lane & 7) + ((lane >> 3) & 1) * 8) * ai_pitch + (st * RPS + ks * 16 + (lane >> 4) * 8) * 2,
+              a);
+#pragma unroll
+      for (int t2 = 0; t2 < 2; ++t2) {
+        // two 8-column tiles: lanes 0-15 address rows k 0-15 of the first,
+        // lanes 16-31 the same rows of the second
+        uint32_t b[4];
+        const int n0 = warp * 32 + t2 * 16 + (lane >> 4) * 8;
+        ldsm_x4_trans(tile + (ks * 16 + (lane & 15)) * tpitch + n0 * 2, b);
+        mma_16816(acc[2 * t2], a, b[0], b[1]);
+        mma_16816(acc[2 * t2 + 1], a, b[2], b[3]);
+      }
+    }
+    __syncthreads();  // the stage (and the widened copy) may be refilled now
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // this block's [16 x 256] sums: warp w owns columns 32 w .. 32 w + 31
+  float* red = reinterpret_cast<float*>(smem);
+  {
+    const int g = lane >> 2, c2 = (lane & 3) * 2;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int col = warp * 32 + t * 8 + c2;
+      red[g * COLS + col] = acc[t][0];
+      red[g * COLS + col + 1] = acc[t][1];
+      red[(g + 8) * COLS + col] = acc[t][2];
+      red[(g + 8) * COLS + col + 1] = acc[t][3];
+    }
+  }
+  const int nout = 16 * COLS;
+  auto store = [&](int e, float v) {
+    const int m = e / COLS, cl = e % COLS;
+    const int64_t c = c0 + cl;
+    if (m >= M || c >= N) return;
+    if constexpr (kW8) v *= __ldg(b_scale + c);
+    if (out_f32) {
+      static_cast<float*>(Y)[static_cast<int64_t>(m) * ldy + c] = v;
+    } else {
+      static_cast<__nv_bfloat16*>(Y)[static_cast<int64_t>(m) * ldy + c] = __float2bfloat16_rn(v);
+    }
+  };
+  if (gridDim.y == 1) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < nout; e += kMmaThreads) store(e, red[e]);
+  } else if (clustered) {
+    cluster_sync();
+    const uint32_t nsplit = gridDim.y, rank = cluster_ctarank();
+    const uint32_t red_s = smem_u32(red);
+    for (int e = static_cast<int>(rank) * kMmaThreads + threadIdx.x; e < nout;
+         e += static_cast<int>(nsplit) * kMmaThreads) {
+      float v = 0.f;
+      for (uint32_t q = 0; q < nsplit; ++q) v += ld_dsmem_f32(mapa_shared(red_s + e * 4, q));
+      store(e, v);
+    }
+    cluster_sync();  // no block leaves while another may still read its shared memory
+  } else {
+    __syncthreads();
+    for (int e = threadIdx.x; e < nout; e += kMmaThreads) {
+      const int m = e / COLS, cl = e % COLS;
+      const int64_t c = c0 + cl;
+      if (m < M && c < N) partial[(static_cast<int64_t>(blockIdx.y) * M + m) * N + c] = red[e];
+    }
+  }
+}
+
 // Y[m, c] = sum over splits (in order) of partial[split][m][c], times
 // b_scale[c] when given.
 __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float* __restrict__ partial, int splits, int M,
@@ -475,12 +496,13 @@ __global__ void __launch_bounds__(256) gemv_reduce_kernel(const float* __restric
 template <int MT>
 GemvPlan plan_mt(int64_t M, int64_t N, int64_t k, int sms) {
   GemvPlan p{};
-  p.slices = (N + GemvShape<MT>::COLS - 1) / GemvShape<MT>::COLS;
+  constexpr int64_t cols = MT <= 4 ? kStreamCols : kMmaCols;
+  p.slices = (N + cols - 1) / cols;
   // one wave of two blocks per SM (a partial second wave would double the
   // time); each split at least 32 rows and at most what the A_I staging holds
   // (~96 KB for the register-loading kernel, 16 KB beside the streaming ring)
-  const int64_t stage_bytes = MT <= 8 ? kStreamAiBytes : 96 * 1024;
-  const int64_t max_rows = std::min<int64_t>(kGemvMaxRows, stage_bytes / ((MT + 1) * 4) / 8 * 8);
+  const int64_t max_rows = MT <= 4 ? std::min<int64_t>(kGemvMaxRows, kStreamAiBytes / ((MT + 1) * 4) / 8 * 8)
+                                    : kMmaAiBytes / (16 * 2) / 32 * 32;
   int64_t splits = std::max<int64_t>(1, 2 * static_cast<int64_t>(std::max(sms, 1)) / p.slices);
   splits = std::min<int64_t>(splits, kGemvMaxCluster);  // splits of a slice form one cluster
   splits = std::min<int64_t>(splits, std::max<int64_t>(1, k / 32));
@@ -496,19 +518,16 @@ template <int MT, bool kW8>
 cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const void* B, int64_t ldb, const float* b_scale,
                            const int32_t* idx, int M, int64_t d, int64_t N, int64_t k, const GemvPlan& pl,
                            float* partial, void* Y, int out_f32, int64_t ldy, unsigned* err, cudaStream_t stream) {
-  constexpr bool kStream = MT <= 8;
-  static_assert(!kStream || GemvShape<MT, kW8>::COLS == kStreamCols, "one column slicing for both kernels");
+  constexpr bool kStream = MT <= 4;
   auto kernel = [] {
     if constexpr (kStream)
       return gemv_stream_kernel<MT, kW8>;
     else
-      return gemv_rows_kernel<MT, kW8>;
+      return gemv_mma_kernel<kW8>;
   }();
-  const int threads = kStream ? kStreamThreads : kGemvThreads;
-  const size_t smem =
-      kStream ? stream_smem_bytes<MT, kW8>(pl.rows_per_split)
-              : static_cast<size_t>(std::max(pl.rows_per_split * (MT + 1), kGemvWarps * MT * GemvShape<MT>::COLS)) * 4;
-  if (smem > 48 * 1024) {
+  const int threads = kStream ? kStreamThreads : kMmaThreads;
+  const size_t smem = kStream ? stream_smem_bytes<MT, kW8>(pl.rows_per_split) : mma_smem_bytes<kW8>(pl.rows_per_split);
+  {
     const cudaError_t e =
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
