@@ -53,8 +53,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["bench", "attention", "decode", "w8", "decode_attention"], default="bench",
-                    help="attention / decode / w8 / decode_attention: run only that workload a few times and exit "
+    ap.add_argument("--case", choices=["bench", "attention", "decode", "w8", "decode_attention", "block"],
+                    default="bench",
+                    help="attention / decode / w8 / decode_attention / block: run only that workload a few times and exit "
                          "(a short program for profiler captures; prints no JSON line)")
     a = ap.parse_args()
     if a.warmup < 3:
@@ -775,6 +776,19 @@ def run_case(case):
                                                         a["rho_t"]), dtype=torch.uint8, device=dev)
         for _ in range(3):
             R.rmm_attention(Q, K, V, a["rho_d"], a["rho_t"], out=O, ws=ws)
+    elif case == "block":
+        X = bf16_tensor(workloads.llm_activation_bf16(1, M, D), dev)
+        Ws = [bf16_tensor(workloads.weight_bf16(9, D, n, group=i), dev) for i, n in enumerate((D, 1024, 1024))]
+        F = 14336
+        Wu = bf16_tensor(workloads.weight_bf16(10, D, F, group=0), dev)
+        Wg = bf16_tensor(workloads.weight_bf16(10, D, F, group=1), dev)
+        Wd = bf16_tensor(workloads.weight_bf16(10, F, D, group=2), dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            flush.zero_()
+            R.rmm_matmul_multi(X, Ws, 0.5)
+            flush.zero_()
+            R.rmm_mlp_block(X, Wu, Wg, Wd, 0.8, 0.5)
     elif case == "decode_attention":
         a = DEC_ATTN
         for B in (1, 8):
