@@ -583,7 +583,7 @@ def run_rmm(args):
     sws = torch.empty(max(sws_n, 256), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = (2 if sws_n else 1) + 3
+    launches_per_step = 4  # score (one cluster launch for aligned bf16), top-k, compaction + gather, GEMM
     kernel_calls = {
         "score": lambda: R.rmm_score(X, out=ss, ws=sws),
         "topk": lambda: R.rmm_topk(ss, k, out=idx),

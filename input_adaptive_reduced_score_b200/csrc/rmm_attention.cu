@@ -165,9 +165,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 2)
   auto sempty = [&](uint32_t b) { return smem_u32(&bars->sempty[b]); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
+  // grid (heads, blocks): the hardware hands out x fastest, so every head's
+  // heaviest block goes out before any lighter one (no heavy tail)
+  const int bh = blockIdx.x;
   // pass A: heaviest query blocks first; pass B: key block kb (kb = 0 is the heaviest)
-  const int fixed_blk = MODE == kLse ? p.nqb - 1 - static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x);
+  const int fixed_blk = MODE == kLse ? p.nqb - 1 - static_cast<int>(blockIdx.y) : static_cast<int>(blockIdx.y);
   const int n_stream = MODE == kLse ? fixed_blk + 1 : p.nqb - fixed_blk;
   const int first_stream = MODE == kLse ? 0 : fixed_blk;
 
@@ -448,8 +450,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   auto pfull = [&](int b) { return smem_u32(&bars->pfull[b]); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int qb = p.nqb - 1 - static_cast<int>(blockIdx.x);  // heaviest blocks first
+  const int bh = blockIdx.x;                                 // grid (heads, blocks)
+  const int qb = p.nqb - 1 - static_cast<int>(blockIdx.y);  // heaviest blocks first
   const int nv = __ldg(nvalid + static_cast<int64_t>(bh) * p.nqb + qb);
   const int nrb = (nv + TILE - 1) / TILE;
   // kept positions before this block's first query: kept blocks made only of
@@ -751,8 +753,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
-  const int bh = blockIdx.y;
-  const int pair = static_cast<int>(blockIdx.x) >> 1;
+  const int bh = static_cast<int>(blockIdx.x) >> 1;  // grid (2 x heads, pairs): heaviest pairs of all heads first
+  const int pair = static_cast<int>(blockIdx.y);
   const int qb0 = p.nqb - 1 - 2 * pair;                   // the leader's (heavier) block
   const int qb = qb0 - static_cast<int>(rank);            // this CTA's block (-1: none)
   const int* nv_bh = nvalid + static_cast<int64_t>(bh) * p.nqb;
@@ -1159,7 +1161,8 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
       return cudaErrorInvalidValue;
     }
   }
-  const dim3 grid_qk(static_cast<unsigned>(nqb), static_cast<unsigned>(BH));
+  if (nqb > 65535) return cudaErrorInvalidConfiguration;
+  const dim3 grid_qk(static_cast<unsigned>(BH), static_cast<unsigned>(nqb));
   attn_qk_kernel<kLse><<<grid_qk, ATT_THREADS, qk_smem, stream>>>(tm_q, tm_k, lse, tsc, prm, err);
   if ((e = cudaGetLastError()) != cudaSuccess || (e = debug_step(stream, "pass A (lse)")) != cudaSuccess) return e;
   attn_qk_kernel<kColScore><<<grid_qk, ATT_THREADS, qk_smem, stream>>>(tm_q, tm_k, lse, tsc, prm, err);
@@ -1210,7 +1213,7 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
         return cudaErrorInvalidValue;
       }
     }
-    const dim3 grid_pair(static_cast<unsigned>(2 * ((nqb + 1) / 2)), static_cast<unsigned>(BH));
+    const dim3 grid_pair(static_cast<unsigned>(2 * BH), static_cast<unsigned>((nqb + 1) / 2));
     attn_out_pair_kernel<<<grid_pair, ATT_THREADS, pair_smem, stream>>>(tm_q, tm_kh, tm_vt, lse, idx_t, nvalid, O,
                                                                          prm, err);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -11,6 +11,14 @@
 // combined by a second kernel in a fixed order.  No atomics, so the
 // result depends only on the shape.
 //
+// For bf16 with 16-byte aligned rows, score_cluster_kernel does it in one
+// launch: at most 8 row splits of a column strip run as one thread-block
+// cluster and are added in split order through distributed shared memory;
+// column strips are narrowed until there are about two CTAs per SM, and
+// every thread keeps 16 loads in flight.  (The two-kernel form spent a third
+// of its partial pass ramping and draining one wave, and its finalize pass
+// was a launch of pure latency.)
+//
 // silu_mul_score_kernel fuses the score of the MLP down projection into the
 // producer of its activation: H = SiLU(G) * U (G, U the gate and up outputs,
 // bf16), rounded to bf16 and stored, and ss_j = sum_i H[i,j]^2 of the stored
@@ -19,6 +27,7 @@
 
 #include <algorithm>
 
+#include "rmm_device.cuh"
 #include "rmm_internal.h"
 #include "rmm_launch.cuh"
 
@@ -138,6 +147,88 @@ __global__ void __launch_bounds__(kScoreThreads) score_partial_kernel(
       }
     }
   }
+}
+
+// Grid: x = column strip, y = row split (the cluster), z = batch.
+__global__ void __launch_bounds__(kScoreThreads) score_cluster_kernel(
+    const __nv_bfloat16* __restrict__ A, int64_t M, int64_t d, int64_t lda, int64_t batch_stride, int col_threads,
+    int64_t rows_per_split, float* __restrict__ ss, int64_t ld_ss, int sqrt_out) {
+  constexpr int V = 8;
+  constexpr int U = 16;  // loads in flight per thread
+  __shared__ float red[kScoreThreads * V];
+  pdl_wait();
+  pdl_trigger();
+  const int tx = threadIdx.x % col_threads;
+  const int ty = threadIdx.x / col_threads;
+  const int row_groups = kScoreThreads / col_threads;
+  const int64_t col0 = (static_cast<int64_t>(blockIdx.x) * col_threads + tx) * V;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
+  const int64_t r1 = min(M, r0 + rows_per_split);
+  const __nv_bfloat16* Ab = A + static_cast<int64_t>(blockIdx.z) * batch_stride;
+  float acc[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  if (col0 < d) {
+    if (col0 + V <= d) {
+      for (int64_t rb = r0 + ty; rb < r1; rb += static_cast<int64_t>(U) * row_groups) {
+        uint4 raw[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int64_t r = rb + static_cast<int64_t>(u) * row_groups;
+          raw[u] = r < r1 ? __ldg(reinterpret_cast<const uint4*>(Ab + r * lda + col0)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          float x[V];
+          Lanes<__nv_bfloat16>::unpack(raw[u], x);
+#pragma unroll
+          for (int e = 0; e < V; ++e) acc[e] = fmaf(x[e], x[e], acc[e]);
+        }
+      }
+    } else {
+      for (int64_t r = r0 + ty; r < r1; r += row_groups) {
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          if (col0 + e < d) {
+            const float x = __bfloat162float(Ab[r * lda + col0 + e]);
+            acc[e] = fmaf(x, x, acc[e]);
+          }
+        }
+      }
+    }
+  }
+  // pairwise tree over the row groups (fixed order): the CTA's sums end in
+  // red[0 .. col_threads * V)
+#pragma unroll
+  for (int e = 0; e < V; ++e) red[(ty * col_threads + tx) * V + e] = acc[e];
+  __syncthreads();
+  for (int st = row_groups / 2; st >= 1; st >>= 1) {
+    if (ty < st) {
+#pragma unroll
+      for (int e = 0; e < V; ++e) red[(ty * col_threads + tx) * V + e] += red[((ty + st) * col_threads + tx) * V + e];
+    }
+    __syncthreads();
+  }
+  const int ncols = col_threads * V;
+  const int64_t cbase = static_cast<int64_t>(blockIdx.x) * ncols;
+  float* out = ss + static_cast<int64_t>(blockIdx.z) * ld_ss;
+  if (gridDim.y == 1) {
+    for (int e = threadIdx.x; e < ncols; e += kScoreThreads)
+      if (cbase + e < d) out[cbase + e] = sqrt_out ? sqrtf(red[e]) : red[e];
+    return;
+  }
+  // the splits of this strip are the cluster (rank = split): each CTA adds
+  // every split's sums for its share of the columns, in split order
+  cluster_sync();
+  const uint32_t nsplit = gridDim.y, rank = cluster_ctarank();
+  const uint32_t red_s = smem_u32(red);
+  for (int e = static_cast<int>(rank) * kScoreThreads + threadIdx.x; e < ncols;
+       e += static_cast<int>(nsplit) * kScoreThreads) {
+    float v = 0.f;
+    for (uint32_t q = 0; q < nsplit; ++q) v += ld_dsmem_f32(mapa_shared(red_s + e * 4, q));
+    if (cbase + e < d) out[cbase + e] = sqrt_out ? sqrtf(v) : v;
+  }
+  cluster_sync();  // no CTA leaves while another may still read its shared memory
 }
 
 // H = bf16(SiLU(G) * U) with SiLU(g) = g / (1 + e^-g) in fp32, and the
@@ -283,6 +374,34 @@ size_t score_workspace_bytes(int dtype, int64_t batch, int64_t M, int64_t d) {
   return align_up(static_cast<size_t>(batch) * p.splits * d * sizeof(float), kWsAlign);
 }
 
+namespace {
+
+// One-launch plan for bf16: the widest column strip (col_threads) that still
+// gives about two CTAs per SM, and up to 8 row splits (one cluster).
+struct ClusterScorePlan {
+  int col_threads;
+  int64_t strips, splits, rows_per_split;
+};
+
+ClusterScorePlan cluster_score_plan(int64_t batch, int64_t M, int64_t d) {
+  const int sms = std::max(device_sm_count(), 1);
+  const int64_t vecs = (d + 7) / 8;
+  int ct0 = 4;
+  while (ct0 < 64 && ct0 < vecs) ct0 <<= 1;  // no wider than the row
+  ClusterScorePlan best{};
+  for (int ct = ct0; ct >= 4; ct >>= 1) {
+    const int rg = kScoreThreads / ct;
+    int64_t splits = (M + 16 * rg - 1) / (16 * rg);
+    splits = std::min<int64_t>(std::max<int64_t>(splits, 1), 8);
+    const int64_t strips = (vecs + ct - 1) / ct;
+    best = {ct, strips, splits, (M + splits - 1) / splits};
+    if (strips * splits * batch >= 2 * sms) break;
+  }
+  return best;
+}
+
+}  // namespace
+
 cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
                          int64_t batch_stride, float* ss, int64_t ld_ss, int sqrt_out, void* ws,
                          cudaStream_t stream) {
@@ -290,6 +409,28 @@ cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int
   const size_t elt = dtype == 1 ? 2 : 4;
   const bool vec_ok = (reinterpret_cast<uintptr_t>(A) % 16 == 0) && ((lda * elt) % 16 == 0) &&
                       (batch == 1 || (batch_stride * elt) % 16 == 0);
+  if (dtype == 1 && vec_ok && M > 0 && batch <= 65535) {
+    const ClusterScorePlan c = cluster_score_plan(batch, M, d);
+    if (c.strips <= 0x7FFFFFFFLL) {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(static_cast<unsigned>(c.strips), static_cast<unsigned>(c.splits),
+                         static_cast<unsigned>(batch));
+      cfg.blockDim = dim3(kScoreThreads);
+      cfg.dynamicSmemBytes = 0;
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = 1;
+      attr[1].val.clusterDim.y = static_cast<unsigned>(c.splits);
+      attr[1].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      return cudaLaunchKernelEx(&cfg, score_cluster_kernel, static_cast<const __nv_bfloat16*>(A), M, d, lda,
+                                batch_stride, c.col_threads, c.rows_per_split, ss, ld_ss, sqrt_out);
+    }
+  }
   const dim3 grid(static_cast<unsigned>(p.strips), static_cast<unsigned>(p.splits), static_cast<unsigned>(batch));
   const bool direct = p.splits <= 1;
   float* out = direct ? ss : static_cast<float*>(ws);
