@@ -664,22 +664,50 @@ def run_rmm(args):
         torch.matmul(X, Wt, out=Y)
     dense_ms = statistics.mean(p[0] for p in timed(dense, min(args.steps, 100), 2))
 
-    # end to end through the public API: pinned host X in, pinned host Y out
-    Xh = X.cpu().pin_memory()
-    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    Xd = torch.empty_like(X)
+    # end to end through the public API, every step moving its X in from
+    # pinned host memory and its Y out to pinned host memory.  Steps are
+    # pipelined over three streams with two device buffers each: step i's X
+    # is copied in while step i-1 computes and step i-2's Y is copied out
+    # (the copies use the two PCIe directions and the copy engines; each step
+    # still writes the 256 MiB flush before its product).  Time = events
+    # around the whole sequence / steps.
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    Xh = [X.cpu().pin_memory() for _ in range(2)]
+    Yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    Xd = [torch.empty_like(X) for _ in range(2)]
+    Yd = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)]
     mws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, M, D, N, RHO), dtype=torch.uint8, device=dev)
 
-    def e2e(ev):
-        ev[0].record(stream)
-        Xd.copy_(Xh, non_blocking=True)
-        R.rmm_matmul(Xd, Wt, RHO, out=Y, ws=mws)
-        Yh.copy_(Y, non_blocking=True)
-        ev[1].record(stream)
-    for _ in range(3):
-        e2e([torch.cuda.Event(enable_timing=True) for _ in range(2)])
-    e2e_ms = [p[0] for p in timed(e2e, args.e2e_steps, 2)]
-    e2e_tot, e2e_flops = aggregate(sum(e2e_ms), flops_step * len(e2e_ms), world)
+    def e2e_pipeline(K):
+        ev = [[torch.cuda.Event() for _ in range(3)] for _ in range(K)]  # in, compute, out
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(K):
+            b = i % 2
+            s_in.wait_event(t0 if i < 2 else ev[i - 2][1])  # compute i-2 has read Xd[b]
+            with torch.cuda.stream(s_in):
+                Xd[b].copy_(Xh[b], non_blocking=True)
+            ev[i][0].record(s_in)
+            stream.wait_event(ev[i][0])
+            if i >= 2:
+                stream.wait_event(ev[i - 2][2])  # copy-out i-2 has read Yd[b]
+            flush.zero_()
+            R.rmm_matmul(Xd[b], Wt, RHO, out=Yd[b], ws=mws, stream=stream)
+            ev[i][1].record(stream)
+            s_out.wait_event(ev[i][1])
+            with torch.cuda.stream(s_out):
+                Yh[b].copy_(Yd[b], non_blocking=True)
+            ev[i][2].record(s_out)
+        stream.wait_event(ev[K - 1][2])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return t0.elapsed_time(t1)
+    e2e_pipeline(3)
+    e2e_total_ms = e2e_pipeline(args.e2e_steps)
+    e2e_tot, e2e_flops = aggregate(e2e_total_ms, flops_step * args.e2e_steps, world)
     e2e_value = e2e_flops / (e2e_tot * 1e-3) / 1e12
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the dense / end-to-end runs")
@@ -740,7 +768,9 @@ def run_rmm(args):
                          "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
             "kernels": kernels,
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(X.numel() * 2),
-                    "d2h_bytes_per_step": int(Y.numel() * 2), "api": "rmm_matmul"},
+                    "d2h_bytes_per_step": int(Y.numel() * 2), "api": "rmm_matmul",
+                    "ms_per_step": e2e_tot / args.e2e_steps,
+                    "schedule": "steps pipelined over copy-in, compute and copy-out streams (double buffers)"},
             "gpu_launches": launches_per_step * args.steps,
             "attention": attention,
             "decode": decode,
