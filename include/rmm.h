@@ -301,7 +301,9 @@ RMM_API rmm_status rmm_mlp_block(const void* X, int64_t ldx, int64_t M, int64_t 
  *      with no kept token in its window gets a zero row).
  * O is [B, Hq, S, D] written as out_dtype.  Optional outputs (may be NULL):
  * idx_d [B*Hq, k_d], idx_t [B*Hq, k_t], lse [B*Hq, S], tscore [B*Hq, S].
- * Requires D in {64, 128} and S >= 1. Workspace: rmm_attention_workspace_size. */
+ * Requires D in {64, 128}, 1 <= S <= 65535 * 128 and B * Hq <= 65535 (the
+ * grids' limits; RMM_ERR_INVALID_ARG otherwise).  Workspace:
+ * rmm_attention_workspace_size. */
 RMM_API size_t rmm_attention_workspace_size(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D,
                                     double rho_d, double rho_t);
 RMM_API rmm_status rmm_attention(const void* Q, const void* K, const void* V,

@@ -701,7 +701,7 @@ rmm_status rmm_attention(const void* Q, const void* K, const void* V, int64_t B,
   clear_error();
   if (!valid_dtype(out_dtype)) return fail(RMM_ERR_UNSUPPORTED, "rmm_attention: out dtype %d", out_dtype);
   if (!Q || !K || !V || !O) return fail(RMM_ERR_INVALID_ARG, "rmm_attention: null pointer");
-  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || S < 1 || S > (1LL << 24) || B * Hq > 65535)
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv || S < 1 || S > 65535LL * 128 || B * Hq > 65535)
     return fail(RMM_ERR_INVALID_ARG, "rmm_attention: bad sizes");
   if (D != 64 && D != 128) return fail(RMM_ERR_UNSUPPORTED, "rmm_attention: head_dim %lld (64 or 128 only)", (long long)D);
   const int64_t kd = k_from_rho_impl(rho_d, D), kt = k_from_rho_impl(rho_t, S);
