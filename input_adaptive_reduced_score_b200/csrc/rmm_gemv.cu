@@ -31,6 +31,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <atomic>
 #include <type_traits>
 
 #include "rmm_device.cuh"
@@ -41,6 +42,7 @@ namespace rmm {
 namespace {
 
 constexpr int kGemvMaxRows = 4096;  // kept rows per block (the staging buffer bounds it further)
+constexpr int kGemvMaxSmem = 200 * 1024;  // dynamic shared memory the decode kernels are opted into
 constexpr int kGemvMaxCluster = 8;  // splits reduced through distributed shared memory (portable cluster size)
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -51,7 +53,10 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 constexpr int kStreamWarps = 8;
 constexpr int kStreamThreads = 32 * kStreamWarps;
 constexpr int kStreamRowsPerStage = 4;              // kept rows per stage of a warp
-constexpr int kStreamStages = 6;                    // stages in flight per warp
+// stages in flight per warp (twelve for int8 rows, filling the same ring,
+// measured no faster: the one-row product is bound by fixed latency)
+template <bool kW8>
+constexpr int stream_stages() { return 6; }
 constexpr int kStreamCols = 256;                    // columns of Y per block
 constexpr int kStreamAiBytes = 16 * 1024;           // A_I staging (fp32 [row][m]) per block: two blocks fit an SM
 
@@ -60,7 +65,7 @@ constexpr int stream_row_bytes() { return kStreamCols * (kW8 ? 1 : 2); }
 
 template <bool kW8>
 constexpr size_t stream_ring_bytes() {
-  return static_cast<size_t>(kStreamWarps) * kStreamStages * kStreamRowsPerStage * stream_row_bytes<kW8>();
+  return static_cast<size_t>(kStreamWarps) * stream_stages<kW8>() * kStreamRowsPerStage * stream_row_bytes<kW8>();
 }
 
 // Dynamic shared memory: each warp's ring of stages, then A_I as fp32
@@ -88,7 +93,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
   constexpr int CPL = kStreamCols / 32;  // 8 columns per lane
   constexpr int COLS = kStreamCols;
   constexpr int RPS = kStreamRowsPerStage;
-  constexpr int S = kStreamStages;
+  constexpr int S = stream_stages<kW8>();
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_split;
@@ -528,9 +533,18 @@ cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const void* B, int
   const int threads = kStream ? kStreamThreads : kMmaThreads;
   const size_t smem = kStream ? stream_smem_bytes<MT, kW8>(pl.rows_per_split) : mma_smem_bytes<kW8>(pl.rows_per_split);
   {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
+    // opt in once per device, to the most any plan of this kernel asks for
+    static std::atomic<uint64_t> configured{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    const uint64_t bit = 1ull << dev;
+    if (!(configured.load(std::memory_order_acquire) & bit)) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemvMaxSmem);
+      if (e != cudaSuccess) return e;
+      configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    if (smem > static_cast<size_t>(kGemvMaxSmem)) return cudaErrorInvalidConfiguration;
   }
   const dim3 grid(static_cast<unsigned>(pl.slices), static_cast<unsigned>(pl.splits));
   cudaError_t e;
