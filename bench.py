@@ -499,6 +499,40 @@ def measure_block(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, X
     return out
 
 
+def measure_down(R, workloads, bf16_tensor, dev, stream, flush, steps, timed):
+    """The MLP down projection H [4096 x 14336] . W [14336 x 4096] at rho = 0.5
+    (H = SiLU(G) * U formed in fp64 and rounded): the config where the
+    selection reads the widest activation.  The same step and protocol as the
+    headline (rmm_matmul, 256 MiB flush between steps), next to cuBLAS."""
+    import torch
+    inp = workloads.mlp_down()
+    Hd, Wd = bf16_tensor(inp.A, dev), bf16_tensor(inp.B, dev)
+    Md, dd, Nd = inp.M, inp.d, inp.N
+    k = R.rmm_k_from_rho(0.5, dd)
+    Y = torch.empty((Md, Nd), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, Md, dd, Nd, 0.5), dtype=torch.uint8, device=dev)
+
+    def rmm(ev):
+        ev[0].record(stream)
+        R.rmm_matmul(Hd, Wd, 0.5, out=Y, ws=ws)
+        ev[1].record(stream)
+
+    def dense(ev):
+        ev[0].record(stream)
+        torch.matmul(Hd, Wd, out=Y)
+        ev[1].record(stream)
+    for _ in range(3):
+        rmm([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        dense([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    ms = statistics.mean(p[0] for p in timed(rmm, steps, 2))
+    dms = statistics.mean(p[0] for p in timed(dense, steps, 2))
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the down-projection runs")
+    return {"workload": f"MLP down projection H[{Md}x{dd}] . W[{dd}x{Nd}] bf16, rho=0.5, 256 MiB flush between steps",
+            "step_us": ms * 1e3, "dense_us": dms * 1e3, "speedup_vs_dense": dms / ms,
+            "effective_tflops": 2.0 * Md * Nd * k / (ms * 1e-3) / 1e12}
+
+
 DEC_ATTN = {"seed": 5, "Hq": 32, "Hkv": 8, "L": 32768, "D": 128, "rho_d": 0.5, "rho_t": 0.5}
 
 
@@ -721,6 +755,7 @@ def run_rmm(args):
     dec_attn = measure_decode_attention(R, workloads, bf16_tensor, dev, stream, min(args.steps, 30), timed,
                                         peaks["hbm_gbs"])
     block = measure_block(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 30), timed, X)
+    down = measure_down(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed)
     gemm_ms = stage_ms["gemm"]
     achieved = flops_step / (gemm_ms * 1e-3) / 1e12
     # the GEMM is timed inside a loop of seconds: when the power cap acted
@@ -777,6 +812,7 @@ def run_rmm(args):
             "int8_weight": w8,
             "decode_attention": dec_attn,
             "block_driver": block,
+            "mlp_down": down,
             "clocks": clk.summary(), "clock_remeasured": remeasured,
         }
         if world == 1 and not args.no_cpu_baseline:
