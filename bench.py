@@ -4,8 +4,9 @@
 One step = the whole path on one batch of the MLP up/gate projection
 workload (X [4096 x 4096] bf16 activation with per-channel lognormal scale
 and 1% outlier channels, W [4096 x 14336] bf16 ~ N(0, 0.02^2), rho = 0.5):
-column scores -> top-k -> compaction of X -> row gather of W -> tcgen05
-reduced GEMM, every stage a librmm kernel called through the C ABI.
+column scores -> top-k -> compaction of X -> tcgen05 reduced GEMM whose
+spare warps gather the kept rows of W while it multiplies, every stage a
+librmm kernel called through the C ABI.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl rmm|reference]
 
@@ -53,10 +54,10 @@ def parse_args():
     ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["bench", "attention", "decode", "w8", "decode_attention", "block"],
+    ap.add_argument("--case", choices=["bench", "matmul", "attention", "decode", "w8", "decode_attention", "block"],
                     default="bench",
-                    help="attention / decode / w8 / decode_attention / block: run only that workload a few times and exit "
-                         "(a short program for profiler captures; prints no JSON line)")
+                    help="matmul / attention / decode / w8 / decode_attention / block: run only that workload a few "
+                         "times and exit (a short program for profiler captures; prints no JSON line)")
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -617,13 +618,27 @@ def run_rmm(args):
     sws = torch.empty(max(sws_n, 256), dtype=torch.uint8, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches_per_step = 4  # score (one cluster launch for aligned bf16), top-k, compaction + gather, GEMM
+    gws = torch.empty(R.rmm_gemm_workspace_size(R.RMM_BF16, N, k), dtype=torch.uint8, device=dev)
+    # rmm_matmul: score (one cluster launch for aligned bf16), top-k, one
+    # launch compacting A and copying the first column blocks of the kept
+    # rows of B (zeroing the copy counters), the tensor-core product whose
+    # spare warps copy the rest of B's kept rows while it multiplies
+    launches_per_step = 4
     kernel_calls = {
         "score": lambda: R.rmm_score(X, out=ss, ws=sws),
         "topk": lambda: R.rmm_topk(ss, k, out=idx),
-        "compact_gather": lambda: R.rmm_compact_gather(X, Wt, idx, out_a=AI, out_b=BI),
-        "gemm": lambda: R.rmm_gemm_compacted(AI, BI, out=Y),
+        "compact": lambda: R.rmm_compact(X, idx, out=AI),
+        "gemm": lambda: R.rmm_gemm(AI, Wt, idx, out=Y, ws=gws),
     }
+    # the timed step: the whole path as one call
+    mws_step = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, M, D, N, RHO), dtype=torch.uint8, device=dev)
+    whole_path_call = lambda: R.rmm_matmul(X, Wt, RHO, out=Y, idx_out=idx, ws=mws_step)
+    # the earlier form: both operands in one launch, then the product on them
+    two_launch_calls = [
+        kernel_calls["score"], kernel_calls["topk"],
+        lambda: R.rmm_compact_gather(X, Wt, idx, out_a=AI, out_b=BI),
+        lambda: R.rmm_gemm_compacted(AI, BI, out=Y),
+    ]
 
     def step(ev=None):
         # Kernels are launched with programmatic dependent launch: each one's
@@ -634,7 +649,7 @@ def run_rmm(args):
             ev[0].record(stream)
         kernel_calls["score"]()
         kernel_calls["topk"]()
-        kernel_calls["compact_gather"]()
+        kernel_calls["compact"]()
         if ev is not None:
             ev[1].record(stream)
         kernel_calls["gemm"]()
@@ -663,27 +678,51 @@ def run_rmm(args):
         barrier()
         return [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(nev - 1)] for i in range(steps)]
 
+    def whole_path_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        whole_path_call()
+        if ev is not None:
+            ev[1].record(stream)
+
+    def two_launch_step(ev):
+        ev[0].record(stream)
+        for fn in two_launch_calls:
+            fn()
+        ev[1].record(stream)
+
     for _ in range(args.warmup):
+        flush.zero_()
+        whole_path_step()
         flush.zero_()
         step()
     torch.cuda.synchronize(dev)
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during warm-up")
 
+    # The timed steps are rmm_matmul calls (no event inside a step, so every
+    # kernel's launch overlaps its predecessor).  The GEMM's own duration for
+    # the roofline comes from the same path split into its public calls with
+    # an event before rmm_gemm, timed right after under the same clock record.
     remeasured = False
     for attempt in range(2):
         with ClockSampler(torch.cuda.get_device_properties(dev)) as clk:
-            per = timed(step, args.steps, 3)
+            per = timed(whole_path_step, args.steps, 2)
+            split = timed(step, min(args.steps, 100), 3)
         if not clk.rejected():
             break
         remeasured = True
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the timed steps")
-    step_ms = [sum(p) for p in per]
-    stage_ms = {"select_and_compact": statistics.mean(p[0] for p in per),
-                "gemm": statistics.mean(p[1] for p in per)}
+    step_ms = [p[0] for p in per]
+    stage_ms = {"select_and_compact": statistics.mean(p[0] for p in split),
+                "gemm": statistics.mean(p[1] for p in split)}
+    split_ms = statistics.mean(sum(p) for p in split)
     ser = timed(step_serialised, min(args.steps, 50), len(kernel_calls) + 1)
     serial_ms = {name: statistics.mean(p[j] for p in ser) for j, name in enumerate(kernel_calls)}
+    for _ in range(3):
+        two_launch_step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    two_launch_ms = statistics.mean(p[0] for p in timed(two_launch_step, min(args.steps, 50), 2))
     local_ms = sum(step_ms)
     flops_step = 2.0 * M * N * k
     tot_ms, tot_flops = aggregate(local_ms, flops_step * args.steps, world)
@@ -767,12 +806,12 @@ def run_rmm(args):
     traffic = traffic_per_launch()
     hbm = peaks["hbm_gbs"]
     # algorithmic bytes per launch: score reads A; top-k reads the d scores and
-    # writes k indices; compaction + gather read A (at half density every
-    # 32-byte sector holds a kept column) and the k kept rows of B, and write
-    # A_I and B_I
-    kbytes = {"score": 2.0 * M * D, "topk": 4.0 * D + 4.0 * k,
-              "compact_gather": 2.0 * M * D + 2.0 * M * k + 4.0 * k * N}
-    kernels = {"timed_step_us": {name: v * 1e3 for name, v in stage_ms.items()}}
+    # writes k indices; compaction reads A (at half density every 32-byte
+    # sector holds a kept column) and writes A_I
+    kbytes = {"score": 2.0 * M * D, "topk": 4.0 * D + 4.0 * k, "compact": 2.0 * M * D + 2.0 * M * k}
+    kernels = {"split_step_us": {name: v * 1e3 for name, v in stage_ms.items()},
+               "split_step_total_us": split_ms * 1e3,
+               "two_launch_gather_step_us": two_launch_ms * 1e3}
     for name, v in serial_ms.items():
         us = v * 1e3
         if name == "gemm":
@@ -797,7 +836,8 @@ def run_rmm(args):
             "dense_tflops": 2.0 * M * N * D / (dense_ms * 1e-3) / 1e12,
             "dense_equivalent_tflops": 2.0 * M * N * D / (path_ms * 1e-3) / 1e12,
             "path_roofline_frac": path_roof_ms / path_ms,
-            "roofline": {"kernel": "gemm_bf16_tc_pair_kernel", "bound": "tensor", "achieved": achieved,
+            "roofline": {"kernel": "rmm_gemm: first-wave row copy + gemm_bf16_tc_pair_kernel<true> (copies the rest)",
+                         "bound": "tensor", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "peak_source": peak_label, "frac_of_burst": achieved / peaks["bf16_tflops"],
                          "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]},
@@ -824,16 +864,28 @@ def run_rmm(args):
 
 
 def run_case(case):
-    """Short runs for profiler captures: the reduced-attention workload called
-    three times, or the decode products (1 and 16 rows on the MLP up/gate
-    weight) called twelve times each with a 256 MiB write in between."""
+    """Short runs for profiler captures: the timed matmul step four times, the
+    reduced-attention workload three times, the decode products (1 and 16
+    rows on the MLP up/gate weight) twelve times each with a 256 MiB write in
+    between, and so on for the other workloads."""
     import numpy as np
     import torch
     import input_adaptive_reduced_score_b200 as R
     import workloads
     from tests.helpers import bf16_tensor
     dev = torch.device("cuda", 0)
-    if case == "attention":
+    if case == "matmul":
+        # the timed step: rmm_matmul on the MLP up/gate workload, four calls
+        # with a 256 MiB write before each
+        X = bf16_tensor(workloads.llm_activation_bf16(1, M, D), dev)
+        Wt = bf16_tensor(workloads.weight_bf16(1, D, N), dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, M, D, N, RHO), dtype=torch.uint8, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(4):
+            flush.zero_()
+            R.rmm_matmul(X, Wt, RHO, out=Y, ws=ws)
+    elif case == "attention":
         a = ATTN
         inp = workloads.attention(a["seed"], a["B"], a["Hq"], a["Hkv"], a["S"], a["D"], a["rho_d"], a["rho_t"])
         Q, K, V = (bf16_tensor(x, dev) for x in (inp.Q, inp.K, inp.V))

@@ -164,9 +164,12 @@ RMM_API rmm_status rmm_compact_gather(const void* A, int64_t lda, const void* B,
  * compacted [M x k] activation (ld_ai), B the full [d x N] row-major operand
  * (ldb >= N) whose rows idx[0..k) are the kept contraction indices, and Y is
  * [M x N] (ldy >= N) written as out_dtype (RMM_BF16 or RMM_F32).
- *  - dtype RMM_BF16, M > 16: B's kept rows are first copied into workspace
- *    (a streaming row gather), then a persistent tcgen05 tensor-core kernel
- *    computes the product with fp32 accumulation in tensor memory.
+ *  - dtype RMM_BF16, M > 16: B's kept rows are copied into workspace (B_I),
+ *    and a persistent tcgen05 tensor-core kernel computes A_I · B_I with fp32
+ *    accumulation in tensor memory.  From M = 256 on, with N a multiple of 8,
+ *    the copy runs inside the product's kernel: spare warps copy blocks of
+ *    kept rows while the tensor cores work on blocks already copied.  Below
+ *    that, one streaming gather launch precedes the product.
  *  - dtype RMM_BF16, M <= 16 (decode): the kept rows of B are read in place,
  *    once each, by a row-streaming kernel with fp32 accumulation; the
  *    workspace holds fp32 partial sums over ranges of kept rows, added in a
@@ -174,7 +177,8 @@ RMM_API rmm_status rmm_compact_gather(const void* A, int64_t lda, const void* B,
  *    Both bf16 forms require 16-byte aligned A_I, B, Y, and ld_ai, ldb
  *    multiples of 8 (RMM_ERR_UNSUPPORTED otherwise).  B must be finite.
  *  - dtype RMM_F32: fp32 FMA kernel (A_I, B fp32; Y fp32 only); no workspace.
- * Workspace: rmm_gemm_workspace_size(dtype, N, k) bytes, 256-byte aligned.
+ * Workspace: rmm_gemm_workspace_size(dtype, N, k) bytes, 256-byte aligned
+ * (B_I, then the fused copy's counters, which the call zeroes itself).
  * Out-of-range indices contribute zero and are flagged.  k >= 1. */
 RMM_API size_t rmm_gemm_workspace_size(int dtype, int64_t N, int64_t k);
 RMM_API rmm_status rmm_gemm(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb,

@@ -111,6 +111,35 @@ int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 extern "C" size_t rmm_gemm_workspace_size(int dtype, int64_t N, int64_t k);
 namespace {
 
+// Workspace of the bf16 product: B_I [k x round_up(N, 8)], then the counters
+// of the fused row gather.
+size_t gemm_bi_bytes(int64_t N, int64_t k) {
+  return align_up(static_cast<size_t>(k) * static_cast<size_t>(round_up(N, 8)) * 2, kWsAlign);
+}
+uint32_t* gemm_counters(void* ws, int64_t N, int64_t k) {
+  return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + gemm_bi_bytes(N, k));
+}
+
+// The bf16 tensor-core product with B_I = B[idx, :] filled in two parts: one
+// launch copies the columns the product's first wave of tiles reads (and,
+// given A, compacts A_I = A[:, idx] in the same grid) and zeroes the
+// counters; then the product kernel, whose spare warps copy the remaining
+// columns while the first wave multiplies.  A_I is [M x k] (ld_ai); B_I
+// [k x N] (pitch round_up(N, 8)) at bi; ctr holds n_ctr zeroed words.
+cudaError_t launch_fused_product(const void* A, int64_t lda, int64_t d, const void* B, int64_t ldb, bool b_int8,
+                                 const int32_t* idx, int64_t k, void* ai, int64_t ld_ai, void* bi, uint32_t* ctr,
+                                 int64_t n_ctr, int64_t M, int64_t N, void* Y, int out_dtype, int64_t ldy,
+                                 const float* col_scale, unsigned* err, cudaStream_t s) {
+  const int64_t ld_bi = round_up(N, 8);
+  const int64_t n0 = fused_gather_first_cols(M, N);
+  cudaError_t e = launch_compact_and_gather(A, A ? M : 0, d, A ? lda : d, B, n0, ldb, idx, k, ai, ld_ai, bi, ld_bi,
+                                            err, s, b_int8, ctr, n_ctr);
+  if (e != cudaSuccess) return e;
+  const FusedGather fg{B, ldb, idx, d, ctr, b_int8, n0};
+  return launch_gemm_bf16_tc(ai, ld_ai, bi, ld_bi, M, N, k, Y, out_dtype, ldy, err, s, col_scale, &fg);
+}
+
+
 struct MatmulWs {
   size_t ss, idx, score, ai, bi, total;
   int64_t k, ld_ai;
@@ -253,7 +282,7 @@ rmm_status rmm_compact(const void* A, int dtype, int64_t M, int64_t d, int64_t l
 
 size_t rmm_gemm_workspace_size(int dtype, int64_t N, int64_t k) {
   if (dtype != RMM_BF16 || N < 1 || k < 1) return 0;
-  return align_up(static_cast<size_t>(k) * static_cast<size_t>(round_up(N, 8)) * 2, kWsAlign);
+  return gemm_bi_bytes(N, k) + align_up(static_cast<size_t>(fused_gather_counter_words(N)) * 4, kWsAlign);
 }
 
 rmm_status rmm_gather_rows(const void* B, int dtype, int64_t d, int64_t N, int64_t ldb, const int32_t* idx, int64_t k,
@@ -331,7 +360,15 @@ rmm_status rmm_gemm(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, 
     return from_cuda(e, "rmm_gemm(bf16, few rows): launch");
   }
   const int64_t ld_bi = round_up(N, 8);
-  cudaError_t e = launch_gather_rows(B, d, N * 2, ldb * 2, idx, k, ws, ld_bi * 2, err, s);
+  cudaError_t e;
+  if (fused_gather_supported(M, N, k, B, ldb, false)) {
+    e = launch_fused_product(nullptr, 0, d, B, ldb, false, idx, k, const_cast<void*>(A_I), ld_ai, ws,
+                             gemm_counters(ws, N, k), fused_gather_counter_words(N), M, N, Y, out_dtype, ldy, nullptr,
+                             err, s);
+    if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+    return from_cuda(e, "rmm_gemm(bf16): launch");
+  }
+  e = launch_gather_rows(B, d, N * 2, ldb * 2, idx, k, ws, ld_bi * 2, err, s);
   if (e != cudaSuccess) return from_cuda(e, "rmm_gemm: row gather launch");
   e = launch_gemm_bf16_tc(A_I, ld_ai, ws, ld_bi, M, N, k, Y, out_dtype, ldy, err, s);
   if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
@@ -395,6 +432,21 @@ rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t ldb, in
   if (st != RMM_OK) return st;
   st = rmm_topk(ss, 1, d, d, k, idx, k, stream);
   if (st != RMM_OK) return st;
+  if (dtype == RMM_BF16 && fused_gather_supported(M, N, k, B, ldb, false)) {
+    // A_I and the first columns of B_I in one launch, then the product, whose
+    // spare warps copy the rest of B's kept rows while it multiplies
+    if (!aligned16(Y)) return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul: needs a 16-byte aligned Y");
+    if (((M + 127) / 128) * ((N + 255) / 256) > kIntMax) return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul: too many tiles");
+    unsigned* err = device_error_word();
+    if (!err) return RMM_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void* bi = base + w.bi;
+    const cudaError_t e = launch_fused_product(A, lda, d, B, ldb, false, idx, k, ai, w.ld_ai, bi,
+                                               gemm_counters(bi, N, k), fused_gather_counter_words(N), M, N, Y,
+                                               out_dtype, ldy, nullptr, err, s);
+    if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+    return from_cuda(e, "rmm_matmul: launch");
+  }
   if (dtype == RMM_BF16 && M > kGemvMaxM && N > 0 && aligned16(B) && ldb % 8 == 0) {
     // both reduced operands in one launch, then the dense product on them
     const int64_t ld_bi = round_up(N, 8);
@@ -440,7 +492,15 @@ rmm_status rmm_gemm_w8(const void* A_I, int64_t ld_ai, const int8_t* Bq, int64_t
                      "rmm_gemm_w8(few rows): launch");
   }
   const int64_t ld_bi = round_up(N, 8);
-  cudaError_t e = launch_gather_rows_i8(Bq, d, N, ldb, idx, k, ws, ld_bi, err, s);
+  cudaError_t e;
+  if (fused_gather_supported(M, N, k, Bq, ldb, true)) {
+    e = launch_fused_product(nullptr, 0, d, Bq, ldb, true, idx, k, const_cast<void*>(A_I), ld_ai, ws,
+                             gemm_counters(ws, N, k), fused_gather_counter_words(N), M, N, Y, out_dtype, ldy, b_scale,
+                             err, s);
+    if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+    return from_cuda(e, "rmm_gemm_w8: launch");
+  }
+  e = launch_gather_rows_i8(Bq, d, N, ldb, idx, k, ws, ld_bi, err, s);
   if (e != cudaSuccess) return from_cuda(e, "rmm_gemm_w8: row gather launch");
   e = launch_gemm_bf16_tc(A_I, ld_ai, ws, ld_bi, M, N, k, Y, out_dtype, ldy, err, s, b_scale);
   if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
@@ -493,7 +553,16 @@ rmm_status rmm_matmul_w8(const void* A, int64_t lda, const int8_t* Bq, int64_t l
     if (!aligned16(Y)) return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_w8: needs a 16-byte aligned Y");
     unsigned* err = device_error_word();
     if (!err) return RMM_ERR_CUDA;
-    cudaError_t e = launch_compact_and_gather(A, M, d, lda, Bq, N, ldb, idx, k, ai, w.ld_ai, bi, ld_bi, err, s, true);
+    cudaError_t e;
+    if (fused_gather_supported(M, N, k, Bq, ldb, true)) {
+      // A_I and the first columns of B_I in one launch, then the product
+      // with the rest of the int8 rows widened by its spare warps
+      e = launch_fused_product(A, lda, d, Bq, ldb, true, idx, k, ai, w.ld_ai, bi, gemm_counters(bi, N, k),
+                               fused_gather_counter_words(N), M, N, Y, out_dtype, ldy, b_scale, err, s);
+      if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+      return from_cuda(e, "rmm_matmul_w8: launch");
+    }
+    e = launch_compact_and_gather(A, M, d, lda, Bq, N, ldb, idx, k, ai, w.ld_ai, bi, ld_bi, err, s, true);
     if (e != cudaSuccess) return from_cuda(e, "rmm_matmul_w8: compaction launch");
     e = launch_gemm_bf16_tc(ai, w.ld_ai, bi, ld_bi, M, N, k, Y, out_dtype, ldy, err, s, b_scale);
     if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
@@ -586,6 +655,20 @@ rmm_status rmm_matmul_multi(const void* A, int64_t lda, int64_t M, int64_t d, do
       }
       st = rmm_gemm(ai, w.ld_ai, B[i], ldb[i], idx, d, M, N[i], k, RMM_BF16, Y[i], out_dtype, ldy[i], bi, bi_bytes,
                     stream);
+    } else if (fused_gather_supported(M, N[i], k, B[i], ldb[i], false)) {
+      if (((M + 127) / 128) * ((N[i] + 255) / 256) > kIntMax)
+        return fail(RMM_ERR_UNSUPPORTED, "rmm_matmul_multi: too many tiles");
+      unsigned* err = device_error_word();
+      if (!err) return RMM_ERR_CUDA;
+      // A_I (first product only) and the first columns of this product's
+      // B_I in one launch, then the product copying the rest
+      const cudaError_t e = launch_fused_product(compacted ? nullptr : A, lda, d, B[i], ldb[i], false, idx, k, ai,
+                                                 w.ld_ai, bi, gemm_counters(bi, nmax, k),
+                                                 fused_gather_counter_words(nmax), M, N[i], Y[i], out_dtype, ldy[i],
+                                                 nullptr, err, s);
+      compacted = true;
+      if (e == cudaErrorInvalidValue && !g_last_error.empty()) return RMM_ERR_CUDA;
+      if (e != cudaSuccess) return from_cuda(e, "rmm_matmul_multi: product launch");
     } else {
       const int64_t ld_bi = round_up(N[i], 8);
       if (!compacted) {

@@ -298,11 +298,13 @@ __global__ void __launch_bounds__(kGatherThreads) compact_gather_kernel(
     const uint4* __restrict__ B, int64_t d, int64_t vecs, int64_t tail_elems, int64_t ldb_vec,
     uint4* __restrict__ BI, int64_t ldbi_vec, const uint16_t* __restrict__ A, int64_t M, int64_t lda,
     uint16_t* __restrict__ AI, int64_t ld_ai, int64_t chunks, int R, bool vec_ok, const int32_t* __restrict__ idx,
-    int64_t k, unsigned* err) {
+    int64_t k, unsigned* err, uint32_t* zero, int64_t n_zero) {
   extern __shared__ __align__(128) uint8_t stage[];
   pdl_wait();
   pdl_trigger();
   const int64_t blk = blockIdx.x;
+  if (blk == 0)
+    for (int64_t i = threadIdx.x; i < n_zero; i += kGatherThreads) zero[i] = 0u;
   if (blk < k) {
     if constexpr (kW8)
       gather_row_block_i8(blk, B, d, vecs, tail_elems, ldb_vec, idx, k, BI, ldbi_vec, err);
@@ -381,8 +383,10 @@ cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64
 
 cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64_t lda, const void* B, int64_t N,
                                       int64_t ldb, const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai,
-                                      void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream, bool b_int8) {
-  const int R = staged_rows(A, d, lda);
+                                      void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream, bool b_int8,
+                                      uint32_t* zero, int64_t n_zero) {
+  if (!zero) n_zero = 0;
+  const int R = M > 0 ? staged_rows(A, d, lda) : 0;
   const int64_t chunks = (k + kColsPerCta - 1) / kColsPerCta;
   const int64_t cblocks = M <= 0 ? 0 : (R > 0 ? (M + R - 1) / R : ((M + kRowsPerCta - 1) / kRowsPerCta) * chunks);
   const int64_t blocks = k + cblocks;
@@ -399,7 +403,7 @@ cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64
   uint16_t* ai = static_cast<uint16_t*>(A_I);
   auto go = [&](auto kernel, size_t smem, int r) {
     return launch_pdl(kernel, grid, block, smem, stream, b, d, vecs, tail, ldb_vec, bi, ldbi_vec, a, M, lda, ai, ld_ai,
-                      chunks, r, vec_ok, idx, k, err);
+                      chunks, r, vec_ok, idx, k, err, zero, n_zero);
   };
   if (R > 0) {
     const size_t smem = static_cast<size_t>(R) * 2 * d;

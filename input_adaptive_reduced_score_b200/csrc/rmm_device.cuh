@@ -187,6 +187,48 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same between generic-proxy global accesses and async-proxy (TMA) ones.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ------------------------------------------------------------------ flags between CTAs of one grid
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Wait until *p >= target, where *p is raised by other CTAs of the same grid
+// with red_release_gpu_add; then order this thread's later TMA reads after
+// the data those CTAs wrote before raising it.  Bounded like mbar_wait: on
+// expiry the site is recorded, the CTA's abort flag raised and false returned.
+__device__ __forceinline__ bool flag_wait_geq(const uint32_t* p, uint32_t target, volatile int* abort_flag,
+                                              unsigned* err, unsigned site) {
+  if (ld_acquire_gpu(p) < target) {
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+      __nanosleep(64);
+      if (ld_acquire_gpu(p) >= target) break;
+      if ((it & 15u) == 0u) {
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          record_error(err, kDevErrTimeoutBase + site);
+          return false;
+        }
+      }
+    }
+  }
+  fence_proxy_async_global();
+  return true;
+}
+
 // ------------------------------------------------------------------ tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {

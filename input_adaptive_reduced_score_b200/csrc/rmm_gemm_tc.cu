@@ -334,6 +334,15 @@ struct PairBars {
 };
 static_assert(sizeof(PairBars) <= BAR_BYTES, "barrier block");
 
+// Fused row gather: warps [2 + EPI_WARPS, 2 + EPI_WARPS + GATHER_WARPS)
+// copy units of GATHER_ROWS kept rows x BN columns of B into B_I.  Measured
+// on the MLP up-projection: 16-row units beat 32-row ones (the copy of a unit
+// is one round of loads), and 4 warps beat 2 or 8.
+constexpr int GATHER_WARPS = 4;
+constexpr int GATHER_ROWS = 16;
+static_assert(GATHER_ROWS % 16 == 0 && GATHER_ROWS <= 32, "a lane holds one kept row; rows are loaded 16 at a time");
+constexpr int THREADS_FUSED = THREADS + GATHER_WARPS * 32;
+
 struct Item {
   int m_blk, n0, width;  // tile rows m_blk*256.., columns n0 .. n0+width-1
 };
@@ -343,12 +352,95 @@ __device__ __forceinline__ Item item_of(int i, int split_from, int num_m) {
   const int tile = split_from + (j >> 1);
   return Item{tile % num_m, (tile / num_m) * BN + (j & 1) * (BN / 2), BN / 2};
 }
+// Device view of the fused gather.  ctr[0]: unit tickets; ctr[1]: unused;
+// ctr[2 + b]: finished units of 256-column block b.
+struct GatherArgs {
+  const uint8_t* B;
+  int64_t ldb_bytes;
+  const int32_t* idx;
+  int64_t d;
+  uint8_t* BI;
+  int64_t ldbi_bytes;
+  uint32_t* ctr;
+  int b_int8;
+  int nb_first;  // column blocks [0, nb_first) of B_I were copied before the launch
+};
+
+// One gather warp: take units until none is left.  Unit u covers column
+// block nb_first + u / chunks (BN columns; lane l copies columns 8l .. 8l+7
+// of it) and kept rows [16 (u % chunks), +16) (lane l < 16 holds the source
+// row of kept row l).  All sixteen rows are loaded before any is stored.  An
+// out-of-range index gives a zero row and is flagged.  When a unit's stores
+// are done the warp fences them (generic and async proxy) and adds one to its
+// block's counter with release semantics, which the TMA producer acquires.
+__device__ __forceinline__ void gather_units(const GatherArgs& g, int N, int K, unsigned* err) {
+  const int lane = threadIdx.x & 31;
+  const int num_n = (N + BN - 1) / BN;
+  const int chunks = (K + GATHER_ROWS - 1) / GATHER_ROWS;
+  const uint32_t units = static_cast<uint32_t>(num_n - g.nb_first) * static_cast<uint32_t>(chunks);
+  for (;;) {
+    uint32_t u = 0;
+    if (lane == 0) u = atomicAdd(g.ctr, 1u);
+    u = __shfl_sync(0xFFFFFFFFu, u, 0);
+    if (u >= units) break;
+    const int nb = g.nb_first + static_cast<int>(u / chunks), r0 = static_cast<int>(u % chunks) * GATHER_ROWS;
+    const int nr = min(GATHER_ROWS, K - r0);
+    const int col = nb * BN + lane * 8;
+    const bool cok = col < N;  // N is a multiple of 8
+    int j = lane < nr ? __ldg(g.idx + r0 + lane) : 0;
+    if (lane < nr && (j < 0 || static_cast<int64_t>(j) >= g.d)) {
+      record_error(err, kDevErrBadIndex);
+      j = -1;
+    }
+    uint8_t* dst = g.BI + static_cast<int64_t>(r0) * g.ldbi_bytes + static_cast<int64_t>(col) * 2;
+#pragma unroll 1
+    for (int h = 0; h < GATHER_ROWS; h += 16) {
+      uint4 v[16];
+      if (!g.b_int8) {
+        const uint8_t* src = g.B + static_cast<int64_t>(col) * 2;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int jr = __shfl_sync(0xFFFFFFFFu, j, h + q);
+          v[q] = (h + q < nr && cok && jr >= 0)
+                     ? __ldcs(reinterpret_cast<const uint4*>(src + static_cast<int64_t>(jr) * g.ldb_bytes))
+                     : make_uint4(0u, 0u, 0u, 0u);
+        }
+      } else {
+        const uint8_t* src = g.B + col;
+        uint2 w[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const int jr = __shfl_sync(0xFFFFFFFFu, j, h + q);
+          w[q] = (h + q < nr && cok && jr >= 0)
+                     ? __ldcs(reinterpret_cast<const uint2*>(src + static_cast<int64_t>(jr) * g.ldb_bytes))
+                     : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float lo[4], hi[4];
+          i8x4_to_f32(w[q].x, lo);
+          i8x4_to_f32(w[q].y, hi);
+          v[q] = make_uint4(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]), pack_bf16x2(hi[0], hi[1]),
+                            pack_bf16x2(hi[2], hi[3]));
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (h + q < nr && cok) *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(h + q) * g.ldbi_bytes) = v[q];
+    }
+    fence_proxy_async_global();
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) red_release_gpu_add(g.ctr + 2 + nb, 1u);
+  }
+}
 }  // namespace pairk
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
+template <bool kFused>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kFused ? pairk::THREADS_FUSED : pairk::THREADS, 1)
     gemm_bf16_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                              int M, int N, int K, int split_from, void* __restrict__ Y, int out_f32, int64_t ldy,
-                             int y_vec_ok, const float* __restrict__ col_scale, unsigned* err) {
+                             int y_vec_ok, const float* __restrict__ col_scale, unsigned* err, pairk::GatherArgs g) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
@@ -404,6 +496,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
       for (int i = cid; ok && i < num_items; i += ncl) {
         const pairk::Item t = pairk::item_of(i, split_from, num_m);
         const bool whole = t.width == pairk::BN;
+        if (kFused && t.n0 / pairk::BN >= g.nb_first) {
+          // every unit of this tile's column block of B_I has been written
+          const uint32_t chunks = static_cast<uint32_t>((K + pairk::GATHER_ROWS - 1) / pairk::GATHER_ROWS);
+          if (!flag_wait_geq(g.ctr + 2 + t.n0 / pairk::BN, chunks, abort_flag, err, 45)) {
+            ok = false;
+            break;
+          }
+        }
         const int a_row = t.m_blk * pairk::BM + static_cast<int>(rank) * 128;
         const int b_col = t.n0 + static_cast<int>(rank) * (t.width / 2);
         for (int kb = 0; kb < nk; ++kb) {
@@ -485,6 +585,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pairk::THREADS, 1)
       }
       __syncwarp();
     }
+  } else if (warp >= 2 + pairk::EPI_WARPS) {
+    // ------------------------------------------------------------ fused row gather (both CTAs)
+    if constexpr (kFused) pairk::gather_units(g, N, K, err);
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int qtr = warp & 3;
@@ -549,7 +652,9 @@ bool configure_kernel_once() {
   if (!done[dev]) {
     if (cudaFuncSetAttribute(gemm_bf16_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(gemm_bf16_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(gemm_bf16_tc_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             pairk::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_bf16_tc_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              pairk::SMEM_BYTES) != cudaSuccess)
       return false;
     done[dev] = true;
@@ -581,10 +686,46 @@ bool encode_2d(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, in
 
 }  // namespace
 
+int64_t fused_gather_counter_words(int64_t N) { return 2 + (N + pairk::BN - 1) / pairk::BN; }
+
+// Work items of the CTA-pair kernel and how many run in its first wave.
+namespace {
+struct PairPlan {
+  int64_t split_from, items, clusters;
+};
+PairPlan pair_plan(int64_t M, int64_t N) {
+  const int64_t tiles = ((M + pairk::BM - 1) / pairk::BM) * ((N + pairk::BN - 1) / pairk::BN);
+  const int64_t pairs = device_sm_count() / 2;
+  // split the tiles of a last partial wave into halves when those fit in one wave
+  const int64_t rem = tiles % pairs;
+  const int64_t split_from = (rem > 0 && 2 * rem <= pairs) ? tiles - rem : tiles;
+  const int64_t items = split_from + 2 * (tiles - split_from);
+  return PairPlan{split_from, items, items < pairs ? items : pairs};
+}
+}  // namespace
+
+int64_t fused_gather_first_cols(int64_t M, int64_t N) {
+  const PairPlan p = pair_plan(M, N);
+  const int64_t num_m = (M + pairk::BM - 1) / pairk::BM;
+  // items 0 .. clusters-1 run first; item i of a whole tile is column block i / num_m
+  const int64_t first_item = p.clusters - 1;
+  const int64_t nb = first_item < p.split_from ? first_item / num_m : (p.split_from + (first_item - p.split_from) / 2) / num_m;
+  const int64_t cols = (nb + 1) * pairk::BN;
+  return cols < N ? cols : N;
+}
+
+bool fused_gather_supported(int64_t M, int64_t N, int64_t k, const void* B, int64_t ldb, bool b_int8) {
+  const int64_t belt = b_int8 ? 1 : 2;
+  const int64_t units = ((N + pairk::BN - 1) / pairk::BN) * ((k + pairk::GATHER_ROWS - 1) / pairk::GATHER_ROWS);
+  return M >= pairk::BM && N > 0 && N % 8 == 0 && k >= 1 && B != nullptr &&
+         reinterpret_cast<uintptr_t>(B) % 16 == 0 && (ldb * belt) % 16 == 0 && units <= 0x7FFFFFFFLL;
+}
+
 cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I, int64_t ld_bi, int64_t M, int64_t N,
                                 int64_t k, void* Y, int out_dtype, int64_t ldy, unsigned* err, cudaStream_t stream,
-                                const float* col_scale) {
+                                const float* col_scale, const FusedGather* fg) {
   if (M == 0 || N == 0) return cudaSuccess;
+  if (fg && !fused_gather_supported(M, N, k, fg->B, fg->ldb, fg->b_int8)) return cudaErrorInvalidValue;
   CUtensorMap tmap_a, tmap_b;
   if (!encode_2d(&tmap_a, A_I, k, M, ld_ai, BK, BM, "A_I")) return cudaErrorInvalidValue;
   if (!encode_2d(&tmap_b, B_I, N, k, ld_bi, 64, BK, "B_I")) return cudaErrorInvalidValue;
@@ -598,17 +739,23 @@ cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I,
   const int y_vec_ok = (reinterpret_cast<uintptr_t>(Y) % 16 == 0) && ((ldy * oelt) % 16 == 0);
   if (M >= pairk::BM) {
     // 256 x 256 tiles on SM pairs: one 2-CTA cluster per pair of SMs
-    const int64_t tiles = ((M + pairk::BM - 1) / pairk::BM) * ((N + pairk::BN - 1) / pairk::BN);
-    const int64_t pairs = sms / 2;
-    // split the tiles of a last partial wave into halves when those fit in one wave
-    const int64_t rem = tiles % pairs;
-    const int64_t split_from = (rem > 0 && 2 * rem <= pairs) ? tiles - rem : tiles;
-    const int64_t items = split_from + 2 * (tiles - split_from);
-    if (items > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-    const int clusters = static_cast<int>(items < pairs ? items : pairs);
-    return launch_pdl(gemm_bf16_tc_pair_kernel, dim3(2 * clusters), dim3(pairk::THREADS), pairk::SMEM_BYTES,
+    const PairPlan p = pair_plan(M, N);
+    if (p.items > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+    const int64_t split_from = p.split_from;
+    const int clusters = static_cast<int>(p.clusters);
+    if (fg && fg->n_ready < N) {
+      const int64_t belt = fg->b_int8 ? 1 : 2;
+      const pairk::GatherArgs g{static_cast<const uint8_t*>(fg->B), fg->ldb * belt, fg->idx, fg->d,
+                                static_cast<uint8_t*>(const_cast<void*>(B_I)), ld_bi * 2, fg->ctr,
+                                fg->b_int8 ? 1 : 0, static_cast<int>(fg->n_ready / pairk::BN)};
+      return launch_pdl(gemm_bf16_tc_pair_kernel<true>, dim3(2 * clusters), dim3(pairk::THREADS_FUSED),
+                        pairk::SMEM_BYTES, stream, tmap_a, tmap_b, static_cast<int>(M), static_cast<int>(N),
+                        static_cast<int>(k), static_cast<int>(split_from), Y, out_f32, ldy, y_vec_ok, col_scale, err,
+                        g);
+    }
+    return launch_pdl(gemm_bf16_tc_pair_kernel<false>, dim3(2 * clusters), dim3(pairk::THREADS), pairk::SMEM_BYTES,
                       stream, tmap_a, tmap_b, static_cast<int>(M), static_cast<int>(N), static_cast<int>(k),
-                      static_cast<int>(split_from), Y, out_f32, ldy, y_vec_ok, col_scale, err);
+                      static_cast<int>(split_from), Y, out_f32, ldy, y_vec_ok, col_scale, err, pairk::GatherArgs{});
   }
   const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);

@@ -67,10 +67,13 @@ cudaError_t launch_gather_rows(const void* B, int64_t d, int64_t row_bytes, int6
 // Both reduced operands in one launch (bf16 A): A_I = A[:, idx] and
 // B_I = B[idx, :]; B, B_I bases and pitches 16-byte aligned.  b_int8: B is
 // int8 [d x N] (ldb in bytes, a multiple of 16) and B_I is written as bf16.
+// With M = 0 it is the row gather alone.  zero / n_zero (optional): words the
+// launch sets to zero after waiting for its predecessor (the counters of a
+// fused row gather).
 cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64_t lda, const void* B, int64_t N,
                                       int64_t ldb, const int32_t* idx, int64_t k, void* A_I, int64_t ld_ai,
                                       void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream,
-                                      bool b_int8 = false);
+                                      bool b_int8 = false, uint32_t* zero = nullptr, int64_t n_zero = 0);
 
 // Row gather of an int8 B [d x N] (ldb bytes, multiple of 16; 16-byte aligned)
 // into bf16 B_I [k x N] (ld_bi elements, multiple of 8; 16-byte aligned).
@@ -83,9 +86,34 @@ cudaError_t launch_gather_rows_i8(const void* Bq, int64_t d, int64_t N, int64_t 
 // Dense tcgen05 GEMM on the compacted operands: Y = A_I [M x k] · B_I [k x N].
 // col_scale (may be null): fp32 [N], multiplies column n of the product
 // before it is stored (the per-column scales of an int8 weight).
+//
+// Fused row gather (CTA-pair kernel, M >= 256): with `fg` the kernel itself
+// fills columns [n_ready, N) of B_I = B[idx, :] (bf16, or int8 widened to
+// exact bf16) while it multiplies: extra warps copy 16-row x 256-column units
+// taken from a ticket counter and count finished units per 256-column block;
+// a tile's loads of B_I wait for its block.  Columns [0, n_ready) must be in
+// place before the launch: fused_gather_first_cols(M, N) is what the first
+// wave of tiles reads, so that wave never waits.  fg->ctr holds
+// fused_gather_counter_words(N) words that must be zero when the kernel
+// starts.  With n_ready >= N the plain kernel runs.
+struct FusedGather {
+  const void* B;        // [d x N], row pitch ldb elements, rows 16-byte aligned
+  int64_t ldb;
+  const int32_t* idx;   // the k kept rows
+  int64_t d;
+  uint32_t* ctr;
+  bool b_int8;
+  int64_t n_ready;      // a multiple of 256, or N
+};
+int64_t fused_gather_counter_words(int64_t N);
+int64_t fused_gather_first_cols(int64_t M, int64_t N);
+// The fused gather applies: M >= 256, N a multiple of 8, B 16-byte aligned
+// with a 16-byte multiple row pitch, and the unit count fits 31 bits.
+bool fused_gather_supported(int64_t M, int64_t N, int64_t k, const void* B, int64_t ldb, bool b_int8);
 cudaError_t launch_gemm_bf16_tc(const void* A_I, int64_t ld_ai, const void* B_I, int64_t ld_bi, int64_t M,
                                 int64_t N, int64_t k, void* Y, int out_dtype, int64_t ldy, unsigned* err,
-                                cudaStream_t stream, const float* col_scale = nullptr);
+                                cudaStream_t stream, const float* col_scale = nullptr,
+                                const FusedGather* fg = nullptr);
 cudaError_t launch_gemm_f32_simt(const float* A_I, int64_t ld_ai, const float* B, int64_t ldb,
                                  const int32_t* idx, int64_t d, int64_t M, int64_t N, int64_t k,
                                  float* Y, int64_t ldy, unsigned* err, cudaStream_t stream);

@@ -89,6 +89,8 @@ def test_workspace_sizes():
     w = R.rmm_matmul_workspace_size(1, 4096, 4096, 14336, 0.5)
     # at least the compacted operands (M x k and k x N bf16) plus scores and indices
     assert w >= 4096 * 2048 * 2 + 2048 * 14336 * 2 + 4096 * 4 + 2048 * 4
-    assert R.rmm_gemm_workspace_size(1, 14336, 2048) == 2048 * 14336 * 2
+    # B_I, then 2 + ceil(N / 256) counter words of the fused row copy (256-byte aligned)
+    assert R.rmm_gemm_workspace_size(1, 14336, 2048) == 2048 * 14336 * 2 + 256
+    assert R.rmm_gemm_workspace_size(1, 256 * 70, 64) == 64 * 256 * 70 * 2 + 512
     assert R.rmm_gemm_workspace_size(0, 128, 64) == 0
     assert R.rmm_matmul_workspace_size(1, 4096, 4096, 14336, 1.5) == 0

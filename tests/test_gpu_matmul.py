@@ -243,6 +243,58 @@ def test_gemm_bf16_parity(M, d, N, k, out_dtype):
     no_device_error()
 
 
+FUSED_SHAPES = [  # M, d, N, k with M >= 256 and N a multiple of 8: the product copies B's kept rows itself
+    (256, 600, 264, 33),      # one pair tile; a 256-column block plus 8; a last row unit of one row
+    (512, 1500, 776, 1),      # one kept row
+    (768, 2048, 3000, 1000),  # ragged units (1000 = 31 x 32 + 8) and column blocks
+    (2048, 4096, 4104, 4096), # every row kept; 17 column blocks, the last 8 wide
+]
+
+
+@pytest.mark.parametrize("M,d,N,k", FUSED_SHAPES)
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_gemm_fused_gather_parity(M, d, N, k, out_dtype):
+    """The product kernel that fills B_I with its own warps: the same bounds as
+    the two-launch form, on a workspace filled with 0xFF bytes (the call must
+    zero its counters), called twice on that workspace with different index
+    sets (the kernel must leave its counters zero)."""
+    inp = W.scaled_matmul_bf16(23 + M, M, d, N)
+    A = oracle.decode(inp.A, "bf16")
+    Bm = oracle.decode(inp.B, "bf16")
+    At = bf16_tensor(inp.A)
+    Bt = bf16_tensor(inp.B)
+    ws = torch.full((R.rmm_gemm_workspace_size(R.RMM_BF16, N, k),), 0xFF, dtype=torch.uint8, device="cuda")
+    for trial in range(2):
+        rng = np.random.default_rng(k + 17 * trial)
+        idx = np.sort(rng.choice(d, k, replace=False)).astype(np.int32)
+        it = torch.from_numpy(idx).cuda()
+        Y = R.rmm_gemm(R.rmm_compact(At, it), Bt, it, out_dtype=out_dtype, ws=ws)
+        ref = oracle.reduced_matmul(A, Bm, idx)
+        if out_dtype == torch.bfloat16:
+            check_bf16_output(to_f64(Y), ref, oracle.reduced_matmul(np.abs(A), np.abs(Bm), idx), k)
+        else:
+            assert rel_fro(to_f64(Y), ref) <= 1e-5
+        no_device_error()
+
+
+def test_gemm_fused_gather_bad_index_flagged():
+    """An out-of-range kept row in the fused copy: a zero row of B_I, the
+    error word set, the rest of the product exact to the usual bound."""
+    M, d, N, k = 300, 256, 512, 64
+    inp = W.scaled_matmul_bf16(29, M, d, N)
+    idx = np.arange(k, dtype=np.int32) * 3
+    idx[40] = d + 5
+    it = torch.from_numpy(idx).cuda()
+    AI = R.rmm_compact(bf16_tensor(inp.A), it)
+    assert R.rmm_device_error(clear=True) == 1
+    Y = R.rmm_gemm(AI, bf16_tensor(inp.B), it, out_dtype=torch.float32)
+    assert R.rmm_device_error(clear=True) == 1
+    good = np.delete(np.arange(k), 40)
+    ref = to_f64(AI)[:, good] @ oracle.decode(inp.B, "bf16")[idx[good]]
+    assert rel_fro(to_f64(Y), ref) <= 1e-5
+    no_device_error()
+
+
 DECODE_SHAPES = [  # M, d, N, k: a few activation rows (decode); kept rows of B read in place
     (1, 4096, 4096, 2048),
     (2, 1000, 700, 333),       # ragged N and k
@@ -562,7 +614,7 @@ def test_path_w8_mlp_up_full():
     no_device_error()
 
 
-@pytest.mark.parametrize("M", [2, 200])
+@pytest.mark.parametrize("M", [2, 200, 300])  # in-place rows, gather launch, gather inside the product
 def test_gemm_w8_bad_index_flagged(M):
     d, N, k = 256, 128, 64
     A_bits = W.llm_activation_bf16(81, M, d)
