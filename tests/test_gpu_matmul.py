@@ -243,22 +243,39 @@ def test_gemm_bf16_parity(M, d, N, k, out_dtype):
     no_device_error()
 
 
-FUSED_SHAPES = [  # M, d, N, k with M >= 256 and N a multiple of 8: the product copies B's kept rows itself
-    (256, 600, 264, 33),      # one pair tile; a 256-column block plus 8; a last row unit of one row
-    (512, 1500, 776, 1),      # one kept row
-    (768, 2048, 3000, 1000),  # ragged units (1000 = 31 x 32 + 8) and column blocks
-    (2048, 4096, 4104, 4096), # every row kept; 17 column blocks, the last 8 wide
+def _fused_first_cols(M, N):
+    """Columns of B_I copied before the CTA-pair product starts, as the library
+    plans it (the column blocks its first wave of tiles reads); the product's
+    own warps copy the rest.  Mirrors the host rule so that each case below is
+    known to exercise the copy inside the product."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    pairs = sms // 2
+    num_m, num_n = (M + 255) // 256, (N + 255) // 256
+    tiles = num_m * num_n
+    rem = tiles % pairs
+    split_from = tiles - rem if (rem > 0 and 2 * rem <= pairs) else tiles
+    items = split_from + 2 * (tiles - split_from)
+    first = min(items, pairs) - 1
+    tile = first if first < split_from else split_from + (first - split_from) // 2
+    return min((tile // num_m + 1) * 256, N)
+
+
+FUSED_SHAPES = [  # M, d, N, k: M >= 256, N a multiple of 8, more tiles than one wave
+    (20480, 256, 512, 33),     # one column block copied inside; 3 row units, the last of one row
+    (16384, 600, 776, 257),    # two blocks inside, the last 8 columns wide; ragged units
+    (2048, 4096, 4104, 4096),  # every row kept; 7 of 17 blocks inside
 ]
 
 
 @pytest.mark.parametrize("M,d,N,k", FUSED_SHAPES)
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_gemm_fused_gather_parity(M, d, N, k, out_dtype):
-    """The product kernel that fills B_I with its own warps: the same bounds as
-    the two-launch form, on a workspace filled with 0xFF bytes (the call must
-    zero its counters), called twice on that workspace with different index
-    sets (the kernel must leave its counters zero)."""
-    inp = W.scaled_matmul_bf16(23 + M, M, d, N)
+    """The product kernel that fills part of B_I with its own warps: the same
+    bounds as the two-launch form, on a workspace filled with 0xFF bytes (the
+    call must zero its counters), called twice on that workspace with
+    different index sets."""
+    assert _fused_first_cols(M, N) < N
+    inp = W.scaled_matmul_bf16(23 + M % 1000, M, d, N)
     A = oracle.decode(inp.A, "bf16")
     Bm = oracle.decode(inp.B, "bf16")
     At = bf16_tensor(inp.A)
@@ -278,18 +295,20 @@ def test_gemm_fused_gather_parity(M, d, N, k, out_dtype):
 
 
 def test_gemm_fused_gather_bad_index_flagged():
-    """An out-of-range kept row in the fused copy: a zero row of B_I, the
-    error word set, the rest of the product exact to the usual bound."""
-    M, d, N, k = 300, 256, 512, 64
+    """An out-of-range kept row: zero in both parts of B_I (the column block
+    copied ahead and the one the product copies), the error word set, the
+    rest of the product exact to the usual bound."""
+    M, d, N, k, bad = 20480, 256, 512, 64, 40
+    assert _fused_first_cols(M, N) < N
     inp = W.scaled_matmul_bf16(29, M, d, N)
     idx = np.arange(k, dtype=np.int32) * 3
-    idx[40] = d + 5
+    idx[bad] = d + 5
     it = torch.from_numpy(idx).cuda()
     AI = R.rmm_compact(bf16_tensor(inp.A), it)
     assert R.rmm_device_error(clear=True) == 1
     Y = R.rmm_gemm(AI, bf16_tensor(inp.B), it, out_dtype=torch.float32)
     assert R.rmm_device_error(clear=True) == 1
-    good = np.delete(np.arange(k), 40)
+    good = np.delete(np.arange(k), bad)
     ref = to_f64(AI)[:, good] @ oracle.decode(inp.B, "bf16")[idx[good]]
     assert rel_fro(to_f64(Y), ref) <= 1e-5
     no_device_error()
@@ -614,9 +633,11 @@ def test_path_w8_mlp_up_full():
     no_device_error()
 
 
-@pytest.mark.parametrize("M", [2, 200, 300])  # in-place rows, gather launch, gather inside the product
+@pytest.mark.parametrize("M", [2, 200, 20480])  # in-place rows, gather launch, copy inside the product
 def test_gemm_w8_bad_index_flagged(M):
-    d, N, k = 256, 128, 64
+    d, N, k = 256, 512, 64
+    if M >= 256:
+        assert _fused_first_cols(M, N) < N
     A_bits = W.llm_activation_bf16(81, M, d)
     q, s = W.weight_int8(82, d, N)
     idx = np.arange(k, dtype=np.int32)
@@ -649,11 +670,14 @@ def test_gemm_w8_rejects_bad_layouts():
 
 # ------------------------------------------------------------------ block driver
 
-@pytest.mark.parametrize("M", [5, 300, 1024])
+@pytest.mark.parametrize("M", [5, 300, 1024, 20480])
 def test_matmul_multi_shared_selection(M):
     """q/k/v-style products on one activation: one index set, every product
-    against the oracle."""
+    against the oracle.  At 20480 rows the first and third products copy
+    part of their B_I inside the product kernel and the second does not."""
     d, Ns, rho = 1024, (512, 128, 264), 0.5
+    if M == 20480:
+        assert [_fused_first_cols(M, n) < n for n in Ns] == [True, False, True]
     A_bits = W.llm_activation_bf16(101 + M, M, d)
     k = oracle.k_from_rho(rho, d)
     cond, _ = widen_topk_gaps(A_bits, "bf16", [k])
