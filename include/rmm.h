@@ -218,9 +218,10 @@ RMM_API rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t
  * The selection is unchanged: it reads the activation only.
  *  - M <= 16: the kept int8 rows are read in place (half the bytes of bf16),
  *    widened exactly to fp32, and each column's sum is scaled at the end.
- *  - M > 16: the kept rows are gathered into workspace as exact bf16
- *    integers, the tcgen05 product runs on them, and the epilogue scales
- *    each column before rounding to out_dtype.
+ *  - M > 16: the kept rows are copied into workspace as exact bf16
+ *    integers (from M = 256, with N a multiple of 8, mostly by the product
+ *    kernel's own spare warps, as in rmm_gemm), the tcgen05 product runs on
+ *    them, and the epilogue scales each column before rounding to out_dtype.
  * A_I bf16 [M x k] (ld_ai, a multiple of 8), Bq (ldb a multiple of 16), Y
  * (ldy) 16-byte aligned, else RMM_ERR_UNSUPPORTED.  b_scale [N] fp32,
  * finite.  Workspace: rmm_gemm_w8_workspace_size(N, k) bytes, 256-byte
@@ -252,8 +253,9 @@ RMM_API rmm_status rmm_matmul_w8(const void* A, int64_t lda, const int8_t* Bq, i
  * I = topk(ss(A), k), k = rmm_k_from_rho(rho, d): one score pass (or none:
  * ss_in, the d column scores of A, may be given, e.g. by
  * rmm_silu_mul_score), one top-k, one compaction of A, then per product the
- * row gather of B[i] and the product (M > 16: tcgen05 GEMM; M <= 16: kept rows
- * read in place).  A bf16 [M x d] (lda); B[i] bf16 [d x N[i]] (ldb[i] a
+ * row gather of B[i] and the product (M > 16: tcgen05 GEMM, which from
+ * M = 256 copies most of B[i]'s kept rows itself as in rmm_gemm; M <= 16:
+ * kept rows read in place).  A bf16 [M x d] (lda); B[i] bf16 [d x N[i]] (ldb[i] a
  * multiple of 8, 16-byte aligned); Y[i] [M x N[i]] (ldy[i], 16-byte aligned)
  * in out_dtype.  idx_out (k, may be NULL) gets I; ss_out (d, may be NULL)
  * the computed scores (not written when ss_in is given).  Workspace:

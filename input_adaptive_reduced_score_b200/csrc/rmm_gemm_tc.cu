@@ -27,11 +27,14 @@
 // so cuts the operand bytes each SM pulls from L2 per MMA by a third; the
 // single-CTA kernel serves smaller M.
 //
-// Why B_I is gathered beforehand rather than inside this kernel: gathering
-// the k rows of B per k-block with tile::gather4 (64 four-row TMA gathers per
+// Why B_I is a copy rather than a gather in the operand path: gathering the
+// k rows of B per k-block with tile::gather4 (64 four-row TMA gathers per
 // stage) or with 16-byte cp.async was measured on B200 at about 2.2 TB/s of
 // operand delivery, an order of magnitude short of what the tensor cores
-// consume; the streaming row copy plus large-box TMA tiles is faster overall.
+// consume; a streaming row copy plus large-box TMA tiles is faster overall.
+// The pair kernel can run that copy itself (kFused): the launch before it
+// copies the column blocks its first wave of tiles reads, and four more warps
+// per CTA copy the rest while the first wave multiplies (see pairk below).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -305,7 +308,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 //     on the empty / accumulator-full barriers of both CTAs (multicast);
 //   - both CTAs' epilogue warps arrive on the leader's accumulator-empty
 //     barrier;
-//   - cluster barriers after set-up and before tensor memory is released.
+//   - cluster barriers after set-up and before tensor memory is released;
+//   - kFused: warps 10-13 of both CTAs copy B_I's column blocks from
+//     nb_first on, 16 kept rows x 256 columns per unit, in column-block order,
+//     and count finished units per block; the producer acquires an item's
+//     block count before its first B load (bounded wait, site 45).  The
+//     copy warps never wait, and units are handed out by a ticket counter, so
+//     the copy progresses whichever CTAs are resident.
 // Work items: tiles below `split_from` are whole 256 x 256 tiles; each tile
 // from `split_from` on is done as two 256 x 128 halves (MMA N = 128, each
 // CTA holding one 64-column chunk of B).  The host splits the tiles of a last
