@@ -346,6 +346,23 @@ RMM_API rmm_status rmm_decode_attention(const void* q, const void* K, const void
                                         float scale, void* O, int out_dtype, int32_t* idx_d, int32_t* idx_t,
                                         float* lse, float* logits, void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------ self-test
+ * Makes one of the library's bounded waits run out on purpose and returns
+ * (asynchronously, on `stream`); no fault, trap or endless loop is involved.
+ * Every wait in librmm's kernels gives up after 2 s, records
+ * RMM_DEVERR_TIMEOUT_BASE + site in the device error word, and lets its
+ * kernel return.  Read the code with rmm_device_error() afterwards; the
+ * context stays usable.
+ *   which 0: an mbarrier that nothing arrives on (site 62);
+ *   which 1: a global flag that nothing raises (site 63);
+ *   which 2: the CTA-pair product whose spare warps copy B_I, with its copy
+ *            counters preset so that nothing is copied.  Its producer, MMA
+ *            and epilogue waits give up, and the kernel unwinds through its
+ *            abort path (site 43, 44 or 45: whichever wait runs out first).
+ * Allocates and frees about 0.25 MB on the stream (cudaMallocAsync).
+ * Takes about 2 s of GPU time. */
+RMM_API rmm_status rmm_selftest_timeout(int which, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

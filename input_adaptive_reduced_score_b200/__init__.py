@@ -26,7 +26,7 @@ __all__ = [
     "rmm_matmul_w8_workspace_size", "rmm_attention", "rmm_attention_workspace_size", "rmm_decode_attention",
     "rmm_decode_attention_workspace_size", "rmm_matmul_multi", "rmm_matmul_multi_workspace_size",
     "rmm_silu_mul_score", "rmm_silu_mul_score_workspace_size", "rmm_mlp_block", "rmm_mlp_block_workspace_size",
-    "exported_symbols", "declared_symbols",
+    "rmm_selftest_timeout", "exported_symbols", "declared_symbols",
 ]
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -35,7 +35,7 @@ LIB_PATH = os.path.join(PKG_DIR, "librmm.so")
 HEADER_PATH = os.path.join(ROOT_DIR, "include", "rmm.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"librmm.so not built ({LIB_PATH}); run: python -m input_adaptive_reduced_score_b200.build")
+    raise ImportError(f"librmm.so not built ({LIB_PATH}); run: python input_adaptive_reduced_score_b200/build.py")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -48,7 +48,11 @@ c_i64, c_int, c_sz, c_dbl, c_flt, c_vp = (ctypes.c_int64, ctypes.c_int, ctypes.c
 
 
 def _sig(name, res, *args):
-    f = getattr(lib, name)
+    try:
+        f = getattr(lib, name)
+    except AttributeError:
+        raise ImportError(f"{LIB_PATH} does not export {name} (built from older sources?); "
+                          "run: python input_adaptive_reduced_score_b200/build.py") from None
     f.restype = res
     f.argtypes = list(args)
     return f
@@ -93,6 +97,7 @@ _sig("rmm_mlp_block", c_int, c_vp, c_i64, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp
 _sig("rmm_attention_workspace_size", c_sz, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl)
 _sig("rmm_attention", c_int, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i64, c_i64, c_dbl, c_dbl, c_flt, c_vp, c_int,
      c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp)
+_sig("rmm_selftest_timeout", c_int, c_int, c_vp)
 
 
 class RMMError(RuntimeError):
@@ -170,6 +175,15 @@ def rmm_device_error(stream=None, clear: bool = True) -> int:
     if st not in (0, 5):
         _check(st, "rmm_device_error")
     return code.value
+
+
+def rmm_selftest_timeout(which: int, stream=None) -> int:
+    """Make one of the library's bounded waits run out on purpose (0: an
+    mbarrier nothing arrives on; 1: a flag nothing raises; 2: the CTA-pair
+    product whose row copy never runs) and return the device error word it
+    left (RMM_DEVERR_TIMEOUT_BASE + site), clearing it.  Takes about 2 s."""
+    _check(lib.rmm_selftest_timeout(int(which), _stream_ptr(stream)), "rmm_selftest_timeout")
+    return rmm_device_error(stream, clear=True)
 
 
 def rmm_score_workspace_size(dtype: int, batch: int, M: int, d: int) -> int:

@@ -1,6 +1,6 @@
 """Builds librmm.so in-tree for sm_100a with nvcc (no JIT, no torch extension).
 
-    python -m input_adaptive_reduced_score_b200.build [--force] [--verbose]
+    python input_adaptive_reduced_score_b200/build.py [--force] [--verbose]
 
 Each .cu under csrc/ compiles to an object in _build/, then one shared
 library is linked next to this file.  Objects are rebuilt when their source or
