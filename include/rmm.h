@@ -14,7 +14,8 @@
  *
  * Conventions shared by every entry point
  *  - Every data pointer is a caller-owned DEVICE pointer on the current CUDA
- *    device; the library never allocates, frees or retains memory.  Scratch
+ *    device; the library never allocates, frees or retains memory (except
+ *    the self-test rmm_selftest_timeout, which documents its own).  Scratch
  *    space ("workspace") is passed in by the caller; its size comes from the
  *    matching *_workspace_size query.  A NULL workspace with ws_bytes == 0 is
  *    allowed when the query returns 0.
