@@ -500,6 +500,36 @@ def measure_block(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, X
     return out
 
 
+def rho_sweep(R, A, B, rhos, dense_ms, steps, timed, stream, dev):
+    """The same step (rmm_matmul, same flush protocol) at other rho values of
+    one workload, next to its dense product.  A failure is reported in the
+    entry of its rho, so it cannot cost the rest of the line."""
+    import torch
+    M, d = A.shape
+    N = B.shape[1]
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    out = {}
+    for rho in rhos:
+        try:
+            k = R.rmm_k_from_rho(rho, d)
+            ws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, M, d, N, rho), dtype=torch.uint8, device=dev)
+
+            def step(ev, rho=rho, ws=ws):
+                ev[0].record(stream)
+                R.rmm_matmul(A, B, rho, out=Y, ws=ws)
+                ev[1].record(stream)
+            for _ in range(3):
+                step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+            ms = statistics.mean(p[0] for p in timed(step, steps, 2))
+            if R.rmm_device_error(stream) != 0:
+                raise RuntimeError("device error word set")
+            out[f"rho={rho}"] = {"k": k, "step_us": ms * 1e3, "effective_tflops": 2.0 * M * N * k / (ms * 1e-3) / 1e12,
+                                 "speedup_vs_dense": dense_ms / ms}
+        except Exception as e:  # noqa: BLE001 - reported in the line
+            out[f"rho={rho}"] = {"error": f"{type(e).__name__}: {e}"[:200]}
+    return out
+
+
 def measure_down(R, workloads, bf16_tensor, dev, stream, flush, steps, timed):
     """The MLP down projection H [4096 x 14336] . W [14336 x 4096] at rho = 0.5
     (H = SiLU(G) * U formed in fp64 and rounded): the config where the
@@ -529,9 +559,10 @@ def measure_down(R, workloads, bf16_tensor, dev, stream, flush, steps, timed):
     dms = statistics.mean(p[0] for p in timed(dense, steps, 2))
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the down-projection runs")
+    sweep = rho_sweep(R, Hd, Wd, (0.8, 1.0), dms, min(steps, 30), timed, stream, dev)
     return {"workload": f"MLP down projection H[{Md}x{dd}] . W[{dd}x{Nd}] bf16, rho=0.5, 256 MiB flush between steps",
             "step_us": ms * 1e3, "dense_us": dms * 1e3, "speedup_vs_dense": dms / ms,
-            "effective_tflops": 2.0 * Md * Nd * k / (ms * 1e-3) / 1e12}
+            "effective_tflops": 2.0 * Md * Nd * k / (ms * 1e-3) / 1e12, "other_rho": sweep}
 
 
 DEC_ATTN = {"seed": 5, "Hq": 32, "Hkv": 8, "L": 32768, "D": 128, "rho_d": 0.5, "rho_t": 0.5}
@@ -736,6 +767,8 @@ def run_rmm(args):
     for _ in range(3):
         torch.matmul(X, Wt, out=Y)
     dense_ms = statistics.mean(p[0] for p in timed(dense, min(args.steps, 100), 2))
+    # the same workload at the other rho values of the up-projection config
+    other_rho = rho_sweep(R, X, Wt, (0.7, 0.8, 1.0), dense_ms, min(args.steps, 30), timed, stream, dev)
 
     # end to end through the public API, every step moving its X in from
     # pinned host memory and its Y out to pinned host memory.  Steps are
@@ -832,7 +865,7 @@ def run_rmm(args):
             "config": {"workload": WORKLOAD, "M": M, "d": D, "N": N, "rho": RHO, "k": k,
                        "l2": "256 MiB buffer written between steps, outside the timed intervals",
                        "parallelism": f"independent batch per GPU x{world}"},
-            "speedup_vs_dense": dense_ms / path_ms, "dense_ms": dense_ms,
+            "speedup_vs_dense": dense_ms / path_ms, "dense_ms": dense_ms, "other_rho": other_rho,
             "dense_tflops": 2.0 * M * N * D / (dense_ms * 1e-3) / 1e12,
             "dense_equivalent_tflops": 2.0 * M * N * D / (path_ms * 1e-3) / 1e12,
             "path_roofline_frac": path_roof_ms / path_ms,
