@@ -507,8 +507,11 @@ def rho_sweep(R, A, B, rhos, dense_ms, steps, timed, stream, dev):
     import torch
     M, d = A.shape
     N = B.shape[1]
-    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     out = {}
+    try:
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    except Exception as e:  # noqa: BLE001 - reported in the line
+        return {"error": f"{type(e).__name__}: {e}"[:200]}
     for rho in rhos:
         try:
             k = R.rmm_k_from_rho(rho, d)
