@@ -72,7 +72,69 @@ def test_validation_rejects_before_launch():
     assert _raw("rmm_attention", vp(16), vp(16), vp(16), 1, 4, 4, 16, 96, ctypes.c_double(0.5),
                 ctypes.c_double(0.5), ctypes.c_float(0), vp(16), 1, vp(0), vp(0), vp(0), vp(0), vp(16), 1 << 30,
                 s) == 2  # head_dim
-    assert b"ld_idx" in R.lib.rmm_last_error() or True
+    assert b"head_dim 96" in R.lib.rmm_last_error()
+
+
+def test_validation_of_the_block_int8_decode_and_selftest_entry_points():
+    """Each later entry point refuses bad arguments on the host, with the
+    documented status, before any CUDA call (this runs without a GPU)."""
+    vp, i64, dbl, flt = ctypes.c_void_p, ctypes.c_int64, ctypes.c_double, ctypes.c_float
+    s, ws, big = vp(0), vp(1 << 20), 1 << 20
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+    # rmm_gemm_w8(A_I, ld_ai, Bq, ldb, b_scale, idx, d, M, N, k, Y, out_dtype, ldy, ws, ws_bytes, stream)
+    assert _raw("rmm_gemm_w8", vp(16), 8, vp(16), 16, vp(16), vp(16), 8, 20, 8, 0, vp(16), 1, 8, ws, big, s) == INVALID
+    assert _raw("rmm_gemm_w8", vp(16), 8, vp(16), 16, vp(16), vp(16), 8, 20, 8, 4, vp(16), 5, 8, ws, big, s) == UNSUPPORTED
+    assert _raw("rmm_gemm_w8", vp(16), 8, vp(16), 16, vp(0), vp(16), 8, 20, 8, 4, vp(16), 1, 8, ws, big, s) == INVALID
+    assert _raw("rmm_gemm_w8", vp(16), 8, vp(16), 24, vp(16), vp(16), 8, 20, 8, 4, vp(16), 1, 8, ws, big, s) == UNSUPPORTED
+    assert _raw("rmm_gemm_w8", vp(16), 8, vp(16), 16, vp(16), vp(16), 8, 20, 8, 4, vp(16), 1, 8, vp(0), 0, s) == WORKSPACE
+    # rmm_matmul_w8(A, lda, Bq, ldb, b_scale, M, d, N, rho, Y, out_dtype, ldy, idx_out, ss_out, ws, ws_bytes, stream)
+    assert _raw("rmm_matmul_w8", vp(16), 8, vp(16), 16, vp(16), 20, 8, 8, dbl(1.5), vp(16), 1, 8, vp(0), vp(0), ws,
+                big, s) == INVALID
+    assert _raw("rmm_matmul_w8", vp(16), 8, vp(16), 24, vp(16), 20, 8, 8, dbl(0.5), vp(16), 1, 8, vp(0), vp(0), ws,
+                big, s) == UNSUPPORTED
+    assert _raw("rmm_matmul_w8", vp(16), 8, vp(16), 16, vp(16), 20, 8, 8, dbl(0.5), vp(16), 1, 8, vp(0), vp(0), vp(0),
+                0, s) == WORKSPACE
+    # rmm_matmul_multi(A, lda, M, d, rho, nprod, B[], ldb[], N[], Y[], ldy[], out_dtype, ss_in, idx_out, ss_out,
+    #                  ws, ws_bytes, stream)
+    Bs, Ys = (vp * 1)(16), (vp * 1)(16)
+    Ns, ldys = (i64 * 1)(8), (i64 * 1)(8)
+    ldb_ok, ldb_bad = (i64 * 1)(8), (i64 * 1)(12)
+    args = lambda nprod, ldbs, w, wb: ("rmm_matmul_multi", vp(16), 8, 20, 8, dbl(0.5), nprod, Bs, ldbs, Ns, Ys, ldys,
+                                       1, vp(0), vp(0), vp(0), w, wb, s)
+    assert _raw(*args(0, ldb_ok, ws, big)) == INVALID
+    assert _raw(*args(1, ldb_bad, ws, big)) == UNSUPPORTED
+    assert _raw(*args(1, ldb_ok, vp(0), 0)) == WORKSPACE
+    assert b"rmm_matmul_multi" in R.lib.rmm_last_error()
+    # rmm_silu_mul_score(G, ldg, U, ldu, M, N, H, ldh, ss_out, ws, ws_bytes, stream)
+    assert _raw("rmm_silu_mul_score", vp(16), 8, vp(16), 8, 4, 0, vp(16), 8, vp(16), ws, big, s) == INVALID
+    assert _raw("rmm_silu_mul_score", vp(0), 8, vp(16), 8, 4, 8, vp(16), 8, vp(16), ws, big, s) == INVALID
+    assert _raw("rmm_silu_mul_score", vp(16), 8, vp(20), 8, 4, 8, vp(16), 8, vp(16), ws, big, s) == UNSUPPORTED
+    assert R.rmm_silu_mul_score_workspace_size(4096, 1024) > 0
+    assert _raw("rmm_silu_mul_score", vp(16), 1024, vp(16), 1024, 4096, 1024, vp(16), 1024, vp(16), vp(0), 0,
+                s) == WORKSPACE
+    # rmm_mlp_block(X, ldx, M, d_model, d_ff, W_up, ld_up, W_gate, ld_gate, W_down, ld_down, rho_up, rho_down, Y,
+    #               out_dtype, ldy, idx_up, idx_down, ws, ws_bytes, stream)
+    mlp = lambda M, ru, w, wb: ("rmm_mlp_block", vp(16), 64, M, 64, 128, vp(16), 128, vp(16), 128, vp(16), 64,
+                                dbl(ru), dbl(0.5), vp(16), 1, 64, vp(0), vp(0), w, wb, s)
+    assert _raw(*mlp(0, 0.5, ws, big)) == INVALID
+    assert _raw(*mlp(32, 0.0, ws, big)) == INVALID
+    assert _raw(*mlp(32, 0.5, vp(0), 0)) == WORKSPACE
+    # rmm_decode_attention(q, K, V, B, Hq, Hkv, L, Lmax, D, rho_d, rho_t, scale, O, out_dtype, idx_d, idx_t, lse,
+    #                      logits, ws, ws_bytes, stream)
+    dec = lambda Hq, Hkv, D, rt, q, out, w, wb: ("rmm_decode_attention", vp(q), vp(16), vp(16), 1, Hq, Hkv, 300, 300,
+                                                 D, dbl(0.5), dbl(rt), flt(0), vp(16), out, vp(0), vp(0), vp(0),
+                                                 vp(0), w, wb, s)
+    assert _raw(*dec(8, 2, 128, 0.5, 16, 7, ws, big)) == UNSUPPORTED   # out dtype
+    assert _raw(*dec(8, 3, 128, 0.5, 16, 1, ws, big)) == INVALID       # Hq % Hkv
+    assert _raw(*dec(8, 2, 96, 0.5, 16, 1, ws, big)) == UNSUPPORTED    # head_dim
+    assert _raw(*dec(6, 2, 128, 0.5, 16, 1, ws, big)) == UNSUPPORTED   # 3 q-heads per kv-head
+    assert _raw(*dec(8, 2, 128, 0.0, 16, 1, ws, big)) == INVALID       # rho_t
+    assert _raw(*dec(8, 2, 128, 0.5, 0, 1, ws, big)) == INVALID        # null q
+    assert _raw(*dec(8, 2, 128, 0.5, 24, 1, ws, big)) == UNSUPPORTED   # misaligned q
+    assert _raw(*dec(8, 2, 128, 0.5, 16, 1, vp(0), 0)) == WORKSPACE
+    # rmm_selftest_timeout(which, stream)
+    assert _raw("rmm_selftest_timeout", 3, s) == INVALID
+    assert b"case 3" in R.lib.rmm_last_error()
 
 
 def test_error_message_is_set():
