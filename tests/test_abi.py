@@ -156,3 +156,37 @@ def test_workspace_sizes():
     assert R.rmm_gemm_workspace_size(1, 256 * 70, 64) == 64 * 256 * 70 * 2 + 512
     assert R.rmm_gemm_workspace_size(0, 128, 64) == 0
     assert R.rmm_matmul_workspace_size(1, 4096, 4096, 14336, 1.5) == 0
+
+
+def test_workspace_sizes_of_the_later_entry_points():
+    """Sizes cover the buffers each call carves from the workspace, are
+    256-byte multiples, and are 0 for arguments the call would refuse."""
+    M, d, N, rho = 4096, 4096, 14336, 0.5
+    k = R.rmm_k_from_rho(rho, d)
+    bi = k * N * 2
+    # int8 weight: B_I is widened to bf16, so the same bytes as the bf16 product
+    assert R.rmm_gemm_w8_workspace_size(N, k) == R.rmm_gemm_workspace_size(R.RMM_BF16, N, k)
+    assert R.rmm_matmul_w8_workspace_size(M, d, N, rho) == R.rmm_matmul_workspace_size(R.RMM_BF16, M, d, N, rho)
+    # shared selection: A_I plus the widest product's B_I (one product at a time)
+    w = R.rmm_matmul_multi_workspace_size(M, d, N, rho)
+    assert w >= M * k * 2 + bi and w % 256 == 0
+    assert w == R.rmm_matmul_workspace_size(R.RMM_BF16, M, d, N, rho)
+    assert R.rmm_matmul_multi_workspace_size(M, d, N, 0.0) == 0
+    # gated MLP block: U, G and H (bf16 [M x d_ff]) and H's scores, plus the inner products' workspace
+    dff = 14336
+    wb = R.rmm_mlp_block_workspace_size(M, d, dff, 0.8, 0.5)
+    inner = max(R.rmm_matmul_multi_workspace_size(M, d, dff, 0.8), R.rmm_matmul_multi_workspace_size(M, dff, d, 0.5))
+    assert wb >= 3 * M * dff * 2 + dff * 4 + inner and wb % 256 == 0
+    assert R.rmm_mlp_block_workspace_size(0, d, dff, 0.8, 0.5) == 0
+    assert R.rmm_mlp_block_workspace_size(M, d, dff, 1.2, 0.5) == 0
+    # SiLU * U with scores: partial sums only when rows are split
+    assert R.rmm_silu_mul_score_workspace_size(4096, 1024) % 256 == 0
+    assert R.rmm_silu_mul_score_workspace_size(4, 0) == 0
+    # decode attention: the logits [B*Hq, L] and token indices [B*Hq, k_t] live in
+    # the workspace unless the caller passes them
+    B, Hq, L, D, rt = 2, 32, 32768, 128, 0.5
+    kt = R.rmm_k_from_rho(rt, L)
+    own = R.rmm_decode_attention_workspace_size(B, Hq, L, D, rt, False, False)
+    given = R.rmm_decode_attention_workspace_size(B, Hq, L, D, rt, True, True)
+    assert own >= given + B * Hq * L * 4 + B * Hq * kt * 4
+    assert own % 256 == 0 and given % 256 == 0
