@@ -41,13 +41,11 @@ def kv_head_of(h: int, Hq: int, Hkv: int) -> int:
 
 
 def attention_head(Q, K, V, rho_d: float, rho_t: float, causal: bool = True, scale=None,
-                   token_idx=None, return_p: bool = False):
+                   return_p: bool = False):
     """One (batch, head): Q [S x D], K [S x D], V [S x D] in fp64.
 
     Returns dict(O [S x D], idx_d [k_d], idx_t [k_t], lse [S], t [S], ssq [D])
-    (plus P [S x S] when return_p).  `token_idx`, when given, replaces the
-    token selection (a test hook for cases where several sets are top-k
-    within floating-point error); everything else is unchanged.
+    (plus P [S x S] when return_p).
     Steps follow the method's order: score Q's columns, keep the top head_dim
     indices, form the reduced logits, the causal softmax, score P's columns,
     keep the top tokens, form the reduced PV product.
@@ -74,7 +72,7 @@ def attention_head(Q, K, V, rho_d: float, rho_t: float, causal: bool = True, sca
     P = e / z
     # token selection on A = P (R4)
     t = np.einsum("ij,ij->j", P, P)
-    idx_t = topk_indices(t, k_from_rho(rho_t, S)) if token_idx is None else np.asarray(token_idx, np.int64)
+    idx_t = topk_indices(t, k_from_rho(rho_t, S))
     # reduced PV (R5)
     O = P[:, idx_t] @ V[idx_t, :]
     out = dict(O=O, idx_d=idx_d, idx_t=idx_t, lse=lse, t=t, ssq=ssq)
@@ -125,31 +123,48 @@ def head_dim_selection(Q, rho_d: float):
     return topk_indices(column_sq_norms(Q), k_from_rho(rho_d, Q.shape[1]))
 
 
-def lse_rows(Q, K, idx_d, rows, scale=None):
-    """lse_i = logsumexp_{j<=i} scale * Q[i, I_d] . K[j, I_d] for i in rows (R2, R3)."""
+def lse_rows(Q, K, idx_d, rows, scale=None, chunk: int = 256):
+    """lse_i = logsumexp_{j<=i} scale * Q[i, I_d] . K[j, I_d] for i in rows (R2, R3).
+    Rows are evaluated `chunk` at a time: one library matmul gives their
+    logits against every key up to the chunk's last row, keys past a row's
+    position are masked out, and each row's log-sum-exp is then taken alone."""
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
     scale = 1.0 / math.sqrt(Q.shape[1]) if scale is None else scale
+    rows = np.asarray(rows, dtype=np.int64)
+    Qd, Kd = Q[:, idx_d], K[:, idx_d]
     out = np.empty(len(rows))
-    Kd = K[:, idx_d]
-    for n, i in enumerate(rows):
-        logits = scale * (Kd[: i + 1] @ Q[i, idx_d])
-        mx = logits.max()
-        out[n] = mx + np.log(np.sum(np.exp(logits - mx)))
+    for a in range(0, len(rows), chunk):
+        r = rows[a:a + chunk]
+        hi = int(r.max()) + 1
+        logits = scale * (Qd[r] @ Kd[:hi].T)                       # [rows, keys 0..hi)
+        logits[np.arange(hi)[None, :] > r[:, None]] = -np.inf      # causal: j <= i
+        mx = logits.max(axis=1)
+        out[a:a + len(r)] = mx + np.log(np.sum(np.exp(logits - mx[:, None]), axis=1))
     return out
 
 
-def token_scores(Q, K, idx_d, lse, cols, scale=None):
+def token_scores(Q, K, idx_d, lse, cols, scale=None, chunk: int = 256):
     """t_j = sum_{i>=j} P_ij^2 = sum_{i>=j} exp(2 (S_ij - lse_i)) for j in cols (R4),
-    given lse for every row."""
+    given lse for every row.  Columns are evaluated `chunk` at a time: one
+    library matmul gives their logits against every query from the chunk's
+    first column on, queries before a column's position are masked out, and
+    each column's sum is then taken alone."""
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
+    lse = np.asarray(lse, dtype=np.float64)
     scale = 1.0 / math.sqrt(Q.shape[1]) if scale is None else scale
-    Qd = Q[:, idx_d]
+    cols = np.asarray(cols, dtype=np.int64)
+    S = Q.shape[0]
+    Qd, Kd = Q[:, idx_d], K[:, idx_d]
     out = np.empty(len(cols))
-    for n, j in enumerate(cols):
-        logits = scale * (Qd[j:] @ K[j, idx_d])
-        out[n] = np.sum(np.exp(2.0 * (logits - lse[j:])))
+    for a in range(0, len(cols), chunk):
+        c = cols[a:a + chunk]
+        lo = int(c.min())
+        logits = scale * (Qd[lo:] @ Kd[c].T)                       # [queries lo..S, cols]
+        e = np.exp(2.0 * (logits - lse[lo:, None]))
+        e[np.arange(lo, S)[:, None] < c[None, :]] = 0.0            # causal: i >= j
+        out[a:a + len(c)] = e.sum(axis=0)
     return out
 
 
