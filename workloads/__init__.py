@@ -28,11 +28,18 @@ import numpy as np
 def f32_to_bf16_bits(x) -> np.ndarray:
     """Round finite fp32 (or wider) values to bf16, nearest-even; return uint16 bits."""
     f = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
-    if not np.all(np.isfinite(f)):
+    if not np.isfinite(f).all():
         raise ValueError("bf16 encoding: non-finite input")
-    u = f.view(np.uint32).astype(np.uint64)
-    bias = ((u >> 16) & 1) + 0x7FFF
-    return ((u + bias) >> 16).astype(np.uint16)
+    # (u + 0x7FFF + lsb) >> 16 on the fp32 bit pattern u, where lsb is bit 16
+    # (ties to even).  Finite patterns are at most 0xFF7FFFFF, so the sum
+    # stays below 2^32 and uint32 arithmetic is exact.
+    u = f.view(np.uint32)
+    r = u >> 16
+    r &= 1
+    r += 0x7FFF
+    r += u
+    r >>= 16
+    return r.astype(np.uint16)
 
 
 def bf16_bits_to_f64(bits) -> np.ndarray:
