@@ -61,6 +61,8 @@ typedef enum rmm_dtype { RMM_F32 = 0, RMM_BF16 = 1 } rmm_dtype;
 
 /* Device-side error codes stored in the error word (0 = none). */
 #define RMM_DEVERR_BAD_INDEX 1u        /* an index outside [0, d) was read; its row/column was zero-filled */
+#define RMM_DEVERR_FP16_RANGE 2u       /* rmm_attention: a kept value of V beyond fp16's range (|v| > 65504 or NaN)
+                                          was saturated for the reduced P V product */
 #define RMM_DEVERR_TIMEOUT_BASE 0x100u /* + site: a bounded wait ran out and the kernel returned early */
 
 /* ABI version of this header (incremented on any incompatible change). */
@@ -91,7 +93,10 @@ RMM_API rmm_status rmm_device_error(void* stream, int clear, unsigned* code);
  * square root can merge distinct scores, so rmm_topk should be given ss).
  * Layout: lda >= d; for the vectorised path A and lda*elt must be 16-byte
  * aligned (otherwise a scalar path runs).  Workspace: rmm_score_workspace_size
- * bytes (fp32 partial sums of the row splits; 0 when one split suffices).
+ * bytes (fp32 partial sums of the row splits; 0 when one split suffices), an
+ * upper bound that depends on the shape only.  Calls that take the one-launch
+ * path (bf16 with A, lda*2 and, for batch > 1, batch_stride*2 all multiples
+ * of 16 bytes) write no partial sums and accept ws = NULL, ws_bytes = 0.
  * M == 0 gives all-zero scores. */
 RMM_API size_t rmm_score_workspace_size(int dtype, int64_t batch, int64_t M, int64_t d);
 RMM_API rmm_status rmm_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t d,
@@ -103,17 +108,22 @@ RMM_API rmm_status rmm_score(const void* A, int dtype, int64_t batch, int64_t M,
  * device memory is all reserved up front by an external pool (where an extra
  * cudaMalloc fails, and synchronises the device even when it succeeds).  The
  * paper has no counterpart; this is a library-side convenience.
- * Same arguments and result as rmm_score, minus the workspace: the row-split
- * partial sums live in a fixed array of RMM_SCORE_NOALLOC_MAX_BYTES inside the
- * library, which every GPU that loads the library holds until exit.  Shapes
- * whose partial sums need more (rmm_score_workspace_size above the limit) are
- * rejected with RMM_ERR_INVALID_ARG and a message.  The first call on each
- * device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current); make that first call before any stream capture.  No
- * call allocates or frees memory.  All calls share the array and each call
- * overwrites it in full before reading it, so nothing has to be cleared
- * between calls; calls that overlap on the GPU race on it and must be
- * serialised by the caller. */
+ * Same arguments and result as rmm_score, minus the workspace, and bit-equal
+ * to it (same kernels, same summation order).  Inputs that rmm_score serves
+ * with its one-launch kernel (bf16 with 16-byte aligned base, row pitch and
+ * batch stride) need no scratch.  The others (fp32 activations, bf16 with an
+ * unaligned base, pitch or batch stride) keep their row-split partial sums in
+ * a fixed array of RMM_SCORE_NOALLOC_MAX_BYTES inside the library, which every
+ * GPU that loads the library holds until exit; such a call whose partial sums
+ * need more (rmm_score_workspace_size above the limit) is rejected with
+ * RMM_ERR_INVALID_ARG and a message, before any device work.  The first call
+ * in each CUDA context of a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current), so make that first call
+ * before any stream capture, and again after a device reset (the new context
+ * repeats the look-up).  No call allocates or frees memory.  All calls share
+ * the array and each call overwrites the part it reads before reading it, so
+ * nothing has to be cleared between calls; calls that overlap on the GPU
+ * race on it and must be serialised by the caller. */
 #define RMM_SCORE_NOALLOC_MAX_BYTES ((size_t)16 << 20)
 RMM_API rmm_status rmm_score_noalloc(const void* A, int dtype, int64_t batch, int64_t M, int64_t d,
                                      int64_t lda, int64_t batch_stride, float* ss, int64_t ld_ss,
@@ -306,6 +316,11 @@ RMM_API rmm_status rmm_mlp_block(const void* X, int64_t ldx, int64_t M, int64_t 
  *      I_t = top k_t = ceil(rho_t*S) tokens;
  *   4. O_i = sum_{j in I_t, j<=i} P_ij V[j,:]  (P not renormalised; a query
  *      with no kept token in its window gets a zero row).
+ * Arithmetic: logits are exact bf16 products summed in fp32; softmax and token
+ * scores in fp32; the P V product takes P' = 2^15 P and the kept rows of V in
+ * fp16 (11 significant bits; V's bf16 values are exact there for magnitudes
+ * in [2^-14, 65504]) with fp32 accumulation, scaled back by 2^-15.  A kept
+ * value beyond 65504 is saturated and sets RMM_DEVERR_FP16_RANGE.
  * O is [B, Hq, S, D] written as out_dtype.  Optional outputs (may be NULL):
  * idx_d [B*Hq, k_d], idx_t [B*Hq, k_t], lse [B*Hq, S], tscore [B*Hq, S].
  * Requires D in {64, 128}, 1 <= S <= 65535 * 128 and B * Hq <= 65535 (the

@@ -240,7 +240,7 @@ rmm_status rmm_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t
   if (batch > 1 && batch_stride < M * lda)
     return fail(RMM_ERR_INVALID_ARG, "rmm_score: batch_stride smaller than one matrix");
   if (!ss || (M > 0 && !A)) return fail(RMM_ERR_INVALID_ARG, "rmm_score: null pointer");
-  const size_t need = score_workspace_bytes(dtype, batch, M, d);
+  const size_t need = score_workspace_used(A, dtype, batch, M, d, lda, batch_stride);
   if (need && (!ws || ws_bytes < need))
     return fail(RMM_ERR_WORKSPACE, "rmm_score: workspace %zu < %zu bytes", ws_bytes, need);
   if (M == 0) {

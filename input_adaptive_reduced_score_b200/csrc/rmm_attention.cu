@@ -19,21 +19,21 @@
 //   7. pass C: O_i = sum_{r: pos_r <= i} exp(S_ir - lse_i) V_T[r]  (attn_out_kernel)
 // with S_ij = scale * Q_I[i] . K_I[j].  Passes A-C are tcgen05 kernels with
 // a TMA warp, an MMA warp and two softmax groups of four warps that take
-// alternate 128 x 128 logit tiles from tensor memory.  Pass C writes P as
-// bf16 back into tensor memory over the logits it has read and accumulates
-// O += P V_T in tensor memory.  Exponentials use the hardware ex2; the
+// alternate 128 x 128 logit tiles from tensor memory.  Pass C rounds
+// P' = 2^15 P to fp16 (11 significant bits; the power-of-two scale keeps the
+// small weights of long rows out of fp16's subnormal range), multiplies it
+// with V_T gathered as fp16 (exact for bf16 values of magnitude <= 65504) and
+// scales the fp32 accumulator back by 2^-15, an exact step.  Exponentials use the hardware ex2; the
 // scale is folded into packed (f32x2) FMAs; only tiles on the causal
 // diagonal or past the sequence end are masked.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
-#include <chrono>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <mutex>
-#include <thread>
 
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
@@ -47,6 +47,11 @@ constexpr int ATT_THREADS = 320;          // warp 0 TMA, warp 1 MMA, warps 2-9 s
 constexpr int SOFTMAX_THREADS = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// Pass C multiplies P by 2^kPScaleLog2 before rounding it to fp16: P <= 1, so
+// P' <= 32768 stays below fp16's largest finite value (65504), and every
+// weight above 2^-29 is an fp16 normal with 11 significant bits.
+constexpr float kPScaleLog2 = 15.f;
+constexpr float kPScaleInv = 1.f / 32768.f;
 
 struct AttnParams {
   int S;            // tokens
@@ -96,6 +101,38 @@ __global__ void __launch_bounds__(256) gather_heads_kernel(const uint4* __restri
   const uint4* s = src + ((static_cast<int64_t>(b) * Hsrc + g) * S + j) * src_ld_vec;
   uint4* d = dst + (static_cast<int64_t>(bh) * kt + r) * dst_ld_vec;
   for (int v = lane; v < row_vecs; v += 32) d[v] = __ldg(s + v);
+}
+
+// The same row gather for V, widened from bf16 to fp16 for pass C's product:
+// exact for magnitudes in [2^-14, 65504] (bf16 keeps 8 significant bits, fp16
+// 11); smaller ones round to fp16 subnormals (absolute error <= 2^-25).
+// Values beyond 65504 (or NaN) are saturated and flagged in the error word.
+__global__ void __launch_bounds__(256) gather_v_f16_kernel(const uint4* __restrict__ src, int Hq, int Hsrc, int S,
+                                                           int src_ld_vec, const int32_t* __restrict__ idx, int kt,
+                                                           int row_vecs, uint4* __restrict__ dst, int dst_ld_vec,
+                                                           unsigned* err) {
+  const int bh = blockIdx.y, b = bh / Hq, h = bh % Hq, g = (h * Hsrc) / Hq;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= kt) return;
+  const int j = __ldg(idx + static_cast<int64_t>(bh) * kt + r);
+  const uint4* s = src + ((static_cast<int64_t>(b) * Hsrc + g) * S + j) * src_ld_vec;
+  uint4* d = dst + (static_cast<int64_t>(bh) * kt + r) * dst_ld_vec;
+  bool bad = false;
+  for (int v = lane; v < row_vecs; v += 32) {
+    const uint4 x = __ldg(s + v);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xFFFF0000u);
+      bad |= !(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f);
+      lo = fminf(fmaxf(lo, -65504.f), 65504.f);
+      hi = fminf(fmaxf(hi, -65504.f), 65504.f);
+      o[e] = pack_f16x2(lo, hi);
+    }
+    d[v] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (bad) record_error(err, kDevErrFp16Range);
 }
 
 // nvalid[bh][qb] = number of kept positions <= the block's last query
@@ -408,11 +445,11 @@ __device__ __forceinline__ void drain_ring(const uint64_t* full, int issued, int
 
 // CTA = one query block.  Kept tokens are processed 128 at a time (only the
 // blocks that hold a kept position <= the block's last query): S = Q_I K_T^T
-// into tensor memory; the softmax warps turn row i into P_ir = exp(S_ir -
-// lse_i) for kept positions <= i (else 0) and write it as bf16 back into the
+// into tensor memory; the softmax warps turn row i into P'_ir = 2^15 exp(S_ir -
+// lse_i) for kept positions <= i (else 0) and write it as fp16 back into the
 // same tensor-memory buffer (two per column, over the logits already read);
-// the MMA lane accumulates O += P V_T with P read from tensor memory and V_T
-// (MN-major) from shared memory.
+// the MMA lane accumulates O += P' V_T with P' read from tensor memory and
+// V_T (fp16, MN-major) from shared memory; the epilogue scales O by 2^-15.
 //   Tensor memory (512 columns): three logit / P buffers of 128 columns and O.
 //   - kept block j uses buffer j % 3; the MMA lane issues PV(j) as soon as
 //     softmax(j) is done and then S(j+3) into the same buffer: tcgen05 MMAs
@@ -519,7 +556,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(TILE, TILE, false, false);
-      const uint32_t idesc_o = idesc_bf16_f32(TILE, p.D, false, true);
+      const uint32_t idesc_o = idesc_f16_f32(TILE, p.D, false, true);
       bool ok = nrb == 0 || mbar_wait(smem_u32(&bars->qfull), 0, abort_flag, err, 22);
       // S(t) = Q_I K_T(t)^T into buffer t % 3
       auto issue_s = [&](int t) -> bool {
@@ -570,7 +607,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const int r = qtr * 32 + lane;
     const int i = qb * TILE + r;
     const uint32_t lane_off = static_cast<uint32_t>(qtr * 32) << 16;
-    const float L2 = i < p.S ? lse[static_cast<int64_t>(bh) * p.S + i] * kLog2e : 0.f;
+    // exponent of P' = 2^15 P
+    const float L2 = i < p.S ? lse[static_cast<int64_t>(bh) * p.S + i] * kLog2e - kPScaleLog2 : 0.f;
     const int32_t* pos_bh = pos + static_cast<int64_t>(bh) * p.kt;
     const uint64_t slp = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(-L2, -L2);
     int* psh = bars->pos[warp - 2];
@@ -609,7 +647,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             if (psh[cc * 32 + 2 * e] > i) p0 = 0.f;
             if (psh[cc * 32 + 2 * e + 1] > i) p1 = 0.f;
           }
-          w[e] = pack_bf16x2(p0, p1);
+          w[e] = pack_f16x2(p0, p1);
         }
       };
       uint32_t va[32], vb[32], w[16];
@@ -655,20 +693,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       if (i >= p.S) continue;
       const int64_t off = (static_cast<int64_t>(bh) * p.S + i) * p.D + cc * 32;
+      float o[32];  // undo the 2^15 of P' (exact)
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(v[e]) * kPScaleInv;
       if (p.out_f32) {
         float4* y = reinterpret_cast<float4*>(static_cast<float*>(O) + off);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          y[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
-                             __uint_as_float(v[4 * q + 3]));
+        for (int q = 0; q < 8; ++q) y[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
       } else {
         uint4* y = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(O) + off);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          y[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+          y[q] = make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                            pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
       }
     }
     tc_fence_before();
@@ -693,7 +730,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 //   - S = Q_I K_T^T: each CTA's A is its own 128 query rows, its B the 64
 //     keys [j*128 + rank*64, +64) of kept block j; each CTA's tensor memory
 //     gets its 128 rows x 128 keys;
-//   - P (bf16) goes to each CTA's shared memory; O += P V_T: each CTA's B is
+//   - P' (fp16) goes to each CTA's shared memory; O += P V_T: each CTA's B is
 //     its 64 of V's 128 columns, each CTA's tensor memory gets its rows of O;
 //   - every load signals the leader's barriers; the leader's MMA lane waits
 //     on them, and its commits reach both CTAs (multicast); the softmax
@@ -824,7 +861,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   } else if (warp == 1) {
     if (leader && lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(2 * TILE, TILE, false, false);
-      const uint32_t idesc_o = idesc_bf16_f32(2 * TILE, p.D, false, true);
+      const uint32_t idesc_o = idesc_f16_f32(2 * TILE, p.D, false, true);
       bool ok = nrb == 0 || mbar_wait(smem_u32(&bars->qfull), 0, abort_flag, err, 33);
       auto issue_s = [&](int t) -> bool {
         const int st = t % ks;
@@ -873,7 +910,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     const int i = qb * TILE + r;    // this thread's query (negative for the spare CTA of an odd count)
     const bool row_ok = i >= 0 && i < p.S;
     const uint32_t lane_off = static_cast<uint32_t>(qtr * 32) << 16;
-    const float L2 = row_ok ? lse[static_cast<int64_t>(bh) * p.S + i] * kLog2e : 0.f;
+    // exponent of P' = 2^15 P
+    const float L2 = row_ok ? lse[static_cast<int64_t>(bh) * p.S + i] * kLog2e - kPScaleLog2 : 0.f;
     const int32_t* pos_bh = pos + static_cast<int64_t>(bh) * p.kt;
     const uint64_t slp = f2_pack(p.scale_log2, p.scale_log2), nl2 = f2_pack(-L2, -L2);
     int* psh = bars->pos[warp - 2];
@@ -910,7 +948,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
             if (psh[cc * 32 + 2 * e] > i) p0 = 0.f;
             if (psh[cc * 32 + 2 * e + 1] > i) p1 = 0.f;
           }
-          w[e] = pack_bf16x2(p0, p1);
+          w[e] = pack_f16x2(p0, p1);
         }
         uint8_t* crow = prow + (cc >> 1) * CHUNK_BYTES;
 #pragma unroll
@@ -957,20 +995,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
       }
       if (!row_ok) continue;
       const int64_t off = (static_cast<int64_t>(bh) * p.S + i) * p.D + cc * 32;
+      float o[32];  // undo the 2^15 of P' (exact)
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(v[e]) * kPScaleInv;
       if (p.out_f32) {
         float4* y = reinterpret_cast<float4*>(static_cast<float*>(O) + off);
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          y[q] = make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]), __uint_as_float(v[4 * q + 2]),
-                             __uint_as_float(v[4 * q + 3]));
+        for (int q = 0; q < 8; ++q) y[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
       } else {
         uint4* y = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(O) + off);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          y[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+          y[q] = make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                            pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
       }
     }
     tc_fence_before();
@@ -1001,10 +1038,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3-D bf16 map over [heads][rows][pitch] with logical row length `cols`;
-// boxes of 64 columns x box_rows rows x 1 head, 128-byte swizzle.
+// 3-D map of 16-bit elements (bf16, or fp16 for V_T) over
+// [heads][rows][pitch] with logical row length `cols`; boxes of 64 columns x
+// box_rows rows x 1 head, 128-byte swizzle.
 bool encode_heads(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows, int64_t heads, int64_t pitch,
-                  int box_rows = TILE) {
+                  int box_rows = TILE, CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn encode = encode_fn();
   if (!encode) {
     set_error("rmm_attention: cuTensorMapEncodeTiled entry point unavailable");
@@ -1015,7 +1053,7 @@ bool encode_heads(CUtensorMap* map, const void* ptr, int64_t cols, int64_t rows,
   const cuuint64_t gstride[2] = {static_cast<cuuint64_t>(pitch) * 2, static_cast<cuuint64_t>(pitch * rows) * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estride[3] = {1, 1, 1};
-  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), gdim, gstride, box,
+  const CUresult r = encode(map, dt, 3, const_cast<void*>(ptr), gdim, gstride, box,
                             estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -1060,37 +1098,6 @@ bool set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
-// With RMM_DEBUG_SYNC set in the environment, every step of the attention
-// pipeline is followed by a bounded wait (20 s) for the stream, and a step
-// that does not finish is reported by name on stderr; the process then exits
-// so the context (and any stuck kernel) is torn down.
-bool debug_sync_enabled() {
-  static const bool on = std::getenv("RMM_DEBUG_SYNC") != nullptr;
-  return on;
-}
-
-cudaError_t debug_step(cudaStream_t stream, const char* what) {
-  if (!debug_sync_enabled()) return cudaSuccess;
-  const auto t0 = std::chrono::steady_clock::now();
-  for (;;) {
-    const cudaError_t e = cudaStreamQuery(stream);
-    if (e == cudaSuccess) {
-      std::fprintf(stderr, "rmm_attention: %s done\n", what);
-      return cudaSuccess;
-    }
-    if (e != cudaErrorNotReady) {
-      std::fprintf(stderr, "rmm_attention: %s failed: %s\n", what, cudaGetErrorString(e));
-      return e;
-    }
-    if (std::chrono::steady_clock::now() - t0 > std::chrono::seconds(20)) {
-      std::fprintf(stderr, "rmm_attention: %s did not finish within 20 s; exiting\n", what);
-      std::fflush(stderr);
-      std::_Exit(3);
-    }
-    std::this_thread::sleep_for(std::chrono::milliseconds(1));
-  }
-}
-
 }  // namespace
 
 size_t attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D, int64_t kd, int64_t kt) {
@@ -1114,7 +1121,7 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
   int32_t* idx_t = idx_t_out ? idx_t_out : reinterpret_cast<int32_t*>(base + w.idx_t);
   int* nvalid = reinterpret_cast<int*>(base + w.nvalid);
   __nv_bfloat16* kt_rows = reinterpret_cast<__nv_bfloat16*>(base + w.kt_rows);
-  __nv_bfloat16* vt_rows = reinterpret_cast<__nv_bfloat16*>(base + w.vt_rows);
+  __half* vt_rows = reinterpret_cast<__half*>(base + w.vt_rows);  // fp16 rows of V
   const int nqb = static_cast<int>((S + TILE - 1) / TILE);
   const int kc = static_cast<int>((kd + 63) / 64);
 
@@ -1122,7 +1129,7 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
   cudaError_t e = launch_score(Q, 1, BH, S, D, D, S * D, ss, D, 0, base + w.score, stream);
   if (e != cudaSuccess) return e;
   e = launch_topk(ss, BH, D, D, kd, idx_d, kd, stream);
-  if (e != cudaSuccess || (e = debug_step(stream, "head_dim scores and top-k")) != cudaSuccess) return e;
+  if (e != cudaSuccess) return e;
   // 2. compacted Q_I and K_I per q-head
   {
     const int64_t items = S * ((kd + 7) / 8);
@@ -1134,11 +1141,12 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
                                                    static_cast<int>(Hkv), static_cast<int>(S), static_cast<int>(D),
                                                    idx_d, static_cast<int>(kd), ki, static_cast<int>(w.ldk));
     e = cudaGetLastError();
-    if (e != cudaSuccess || (e = debug_step(stream, "compaction of Q and K")) != cudaSuccess) return e;
+    if (e != cudaSuccess) return e;
   }
   CUtensorMap tm_q, tm_k, tm_kt, tm_vt;
   if (!encode_heads(&tm_q, qi, kd, S, BH, w.ldk) || !encode_heads(&tm_k, ki, kd, S, BH, w.ldk) ||
-      !encode_heads(&tm_kt, kt_rows, kd, kt, BH, w.ldk) || !encode_heads(&tm_vt, vt_rows, D, kt, BH, D))
+      !encode_heads(&tm_kt, kt_rows, kd, kt, BH, w.ldk) ||
+      !encode_heads(&tm_vt, vt_rows, D, kt, BH, D, TILE, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
     return cudaErrorInvalidValue;
   AttnParams prm{};
   prm.S = static_cast<int>(S);
@@ -1164,17 +1172,15 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
   if (nqb > 65535) return cudaErrorInvalidConfiguration;
   const dim3 grid_qk(static_cast<unsigned>(BH), static_cast<unsigned>(nqb));
   attn_qk_kernel<kLse><<<grid_qk, ATT_THREADS, qk_smem, stream>>>(tm_q, tm_k, lse, tsc, prm, err);
-  if ((e = cudaGetLastError()) != cudaSuccess || (e = debug_step(stream, "pass A (lse)")) != cudaSuccess) return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   attn_qk_kernel<kColScore><<<grid_qk, ATT_THREADS, qk_smem, stream>>>(tm_q, tm_k, lse, tsc, prm, err);
-  if ((e = cudaGetLastError()) != cudaSuccess || (e = debug_step(stream, "pass B (token scores)")) != cudaSuccess)
-    return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 5. token selection and causal prefixes
   e = launch_topk(tsc, BH, S, S, kt, idx_t, kt, stream);
   if (e != cudaSuccess) return e;
   attn_prefix_kernel<<<static_cast<unsigned>((BH * nqb + 255) / 256), 256, 0, stream>>>(
       idx_t, static_cast<int>(BH), static_cast<int>(kt), static_cast<int>(S), nqb, nvalid);
-  if ((e = cudaGetLastError()) != cudaSuccess || (e = debug_step(stream, "token top-k and prefixes")) != cudaSuccess)
-    return e;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // 6. kept rows of K_I and V
   {
     const dim3 grid(static_cast<unsigned>((kt + 7) / 8), static_cast<unsigned>(BH));
@@ -1183,13 +1189,13 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
                                                   static_cast<int>(w.ldk / 8), idx_t, static_cast<int>(kt),
                                                   static_cast<int>(w.ldk / 8), reinterpret_cast<uint4*>(kt_rows),
                                                   static_cast<int>(w.ldk / 8));
-    gather_heads_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(V), static_cast<int>(Hq),
+    gather_v_f16_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4*>(V), static_cast<int>(Hq),
                                                   static_cast<int>(Hkv), static_cast<int>(S),
                                                   static_cast<int>(D / 8), idx_t, static_cast<int>(kt),
                                                   static_cast<int>(D / 8), reinterpret_cast<uint4*>(vt_rows),
-                                                  static_cast<int>(D / 8));
+                                                  static_cast<int>(D / 8), err);
     e = cudaGetLastError();
-    if (e != cudaSuccess || (e = debug_step(stream, "row gathers")) != cudaSuccess) return e;
+    if (e != cudaSuccess) return e;
   }
   // 7. pass C: on SM pairs when D = 128 (a pair's CTA takes 64 of V's columns)
   int dev = 0, max_smem = 0;
@@ -1216,8 +1222,7 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
     const dim3 grid_pair(static_cast<unsigned>(2 * BH), static_cast<unsigned>((nqb + 1) / 2));
     attn_out_pair_kernel<<<grid_pair, ATT_THREADS, pair_smem, stream>>>(tm_q, tm_kh, tm_vt, lse, idx_t, nvalid, O,
                                                                          prm, err);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    return debug_step(stream, "pass C (output, SM pairs)");
+    return cudaGetLastError();
   }
   auto out_smem_for = [&](int ks, int vs) {
     return kc * CHUNK_BYTES + ks * kc * CHUNK_BYTES + vs * static_cast<int>(D / 64) * CHUNK_BYTES +
@@ -1243,8 +1248,7 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
     }
   }
   attn_out_kernel<<<grid_qk, ATT_THREADS, out_smem, stream>>>(tm_q, tm_kt, tm_vt, lse, idx_t, nvalid, O, prm, err);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  return debug_step(stream, "pass C (output)");
+  return cudaGetLastError();
 }
 
 }  // namespace rmm

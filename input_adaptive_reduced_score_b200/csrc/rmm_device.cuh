@@ -11,10 +11,12 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace rmm {
 
 constexpr unsigned kDevErrBadIndex = 1u;
+constexpr unsigned kDevErrFp16Range = 2u;
 constexpr unsigned kDevErrTimeoutBase = 0x100u;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
@@ -150,18 +152,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// TMA row gather: four rows (r0..r3) of a 2-D tensor, one box of columns
-// starting at x, written to consecutive row slots at dst (the tensor map's box
-// is one row high).  Completion is signalled on `bar` as transaction bytes.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, uint32_t bar, int x, int r0, int r1, int r2,
-                                            int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(tmap), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-      : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
@@ -331,6 +321,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// Instruction descriptor, kind::f16 with fp16 inputs (A and B both fp16;
+// formats may not be mixed) and fp32 accumulation.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                     // D format fp32
+         | (0u << 7)                                   // A format fp16
+         | (0u << 10)                                  // B format fp16
+         | ((a_mn_major ? 1u : 0u) << 15)              // A major
+         | ((b_mn_major ? 1u : 0u) << 16)              // B major
+         | (static_cast<uint32_t>(n >> 3) << 17)       // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24);      // M / 16
+}
+
 // Instruction descriptor, kind::f16 with bf16 inputs and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                     // D format fp32
@@ -486,6 +488,12 @@ __device__ __forceinline__ float max_of32(const uint32_t (&v)[32]) {
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two fp32 values rounded to fp16 (nearest even), lo in the low half.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 

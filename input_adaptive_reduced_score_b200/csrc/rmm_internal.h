@@ -34,6 +34,11 @@ struct ScorePlan {
 };
 ScorePlan score_plan(int dtype, int64_t batch, int64_t M, int64_t d);
 size_t score_workspace_bytes(int dtype, int64_t batch, int64_t M, int64_t d);
+// Bytes of partial sums launch_score will actually write for this call: 0 when
+// the one-launch kernel serves it (bf16 with 16-byte aligned base, pitch and
+// batch stride) or M == 0, else score_workspace_bytes.
+size_t score_workspace_used(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
+                            int64_t batch_stride);
 cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
                          int64_t batch_stride, float* ss, int64_t ld_ss, int sqrt_out, void* ws,
                          cudaStream_t stream);

@@ -13,11 +13,13 @@
 //
 // For bf16 with 16-byte aligned rows, score_cluster_kernel does it in one
 // launch: at most 8 row splits of a column strip run as one thread-block
-// cluster and are added in split order through distributed shared memory;
-// column strips are narrowed until there are about two CTAs per SM, and
-// every thread keeps 16 loads in flight.  (The two-kernel form spent a third
-// of its partial pass ramping and draining one wave, and its finalize pass
-// was a launch of pure latency.)
+// cluster and are added in split order through distributed shared memory.
+// The grid is sized to one wave of resident CTAs (two per SM), and every
+// thread keeps 8-16 loads in flight as a ring that is refilled as it drains,
+// so each SM streams from its first cycle to its last.  (The two-kernel form
+// spent a third of its partial pass ramping and draining one wave, and its
+// finalize pass was a launch of pure latency; a grid of 1.5-1.7 waves of
+// one-shot CTAs left SMs idle behind the partial second wave.)
 //
 // silu_mul_score_kernel fuses the score of the MLP down projection into the
 // producer of its activation: H = SiLU(G) * U (G, U the gate and up outputs,
@@ -149,12 +151,17 @@ __global__ void __launch_bounds__(kScoreThreads) score_partial_kernel(
   }
 }
 
-// Grid: x = column strip, y = row split (the cluster), z = batch.
-__global__ void __launch_bounds__(kScoreThreads) score_cluster_kernel(
+// Grid: x = column strip, y = row split (the cluster), z = batch.  Two CTAs
+// per SM are resident (the ring below takes about 110 registers per thread),
+// and the host sizes the grid to one resident wave.
+__global__ void __launch_bounds__(kScoreThreads, 2) score_cluster_kernel(
     const __nv_bfloat16* __restrict__ A, int64_t M, int64_t d, int64_t lda, int64_t batch_stride, int col_threads,
     int64_t rows_per_split, float* __restrict__ ss, int64_t ld_ss, int sqrt_out) {
   constexpr int V = 8;
-  constexpr int U = 16;  // loads in flight per thread
+  // ring slots per thread: the compiler issues a round's refills ahead of its
+  // consumption, so 8 slots keep 8-16 loads in flight (111 registers, two CTAs
+  // per SM: 64-128 KB in flight per SM); 16 slots would spill
+  constexpr int U = 8;
   __shared__ float red[kScoreThreads * V];
   pdl_wait();
   pdl_trigger();
@@ -168,23 +175,51 @@ __global__ void __launch_bounds__(kScoreThreads) score_cluster_kernel(
   float acc[V];
 #pragma unroll
   for (int e = 0; e < V; ++e) acc[e] = 0.f;
+  auto add = [&](const uint4 raw) {
+    float x[V];
+    Lanes<__nv_bfloat16>::unpack(raw, x);
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = fmaf(x[e], x[e], acc[e]);
+  };
   if (col0 < d) {
     if (col0 + V <= d) {
-      for (int64_t rb = r0 + ty; rb < r1; rb += static_cast<int64_t>(U) * row_groups) {
-        uint4 raw[U];
+      // this thread's rows r0 + ty + i * row_groups, i < n, summed in order;
+      // slot u of the ring holds row i + u while rows i.. are consumed, and is
+      // refilled with row i + u + U as soon as it has been read
+      const int64_t first = r0 + ty;
+      const int64_t n = first < r1 ? (r1 - first + row_groups - 1) / row_groups : 0;
+      const uint4* p = reinterpret_cast<const uint4*>(Ab + first * lda + col0);  // next row to load
+      const int64_t step = static_cast<int64_t>(row_groups) * lda / V;          // uint4 per row step
+      uint4 ring[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        ring[u] = u < n ? __ldg(p) : make_uint4(0, 0, 0, 0);
+        p += step;
+      }
+      int64_t i = 0;
+#pragma unroll 1
+      for (; i + 2 * U <= n; i += U) {  // every refill is a row of this thread
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-          const int64_t r = rb + static_cast<int64_t>(u) * row_groups;
-          raw[u] = r < r1 ? __ldg(reinterpret_cast<const uint4*>(Ab + r * lda + col0)) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          float x[V];
-          Lanes<__nv_bfloat16>::unpack(raw[u], x);
-#pragma unroll
-          for (int e = 0; e < V; ++e) acc[e] = fmaf(x[e], x[e], acc[e]);
+          const uint4 x = ring[u];
+          ring[u] = __ldg(p);
+          p += step;
+          add(x);
         }
       }
+      if (i + U < n) {  // the last, partial refill
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const uint4 x = ring[u];
+          ring[u] = i + U + u < n ? __ldg(p) : make_uint4(0, 0, 0, 0);
+          p += step;
+          add(x);
+        }
+        i += U;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (i + u < n) add(ring[u]);
     } else {
       for (int64_t r = r0 + ty; r < r1; r += row_groups) {
 #pragma unroll
@@ -376,42 +411,76 @@ size_t score_workspace_bytes(int dtype, int64_t batch, int64_t M, int64_t d) {
 
 namespace {
 
-// One-launch plan for bf16: the widest column strip (col_threads) that still
-// gives about two CTAs per SM, and up to 8 row splits (one cluster).
+// One-launch plan for bf16.  The grid is one wave of resident CTAs (two per
+// SM): each (column strip, row split, batch) CTA streams its rows through the
+// ring above from start to end, so no SM idles behind a partial second wave.
+// Among column-strip widths (col_threads 64 down to 4 vectors) the plan takes
+// the one whose strips x splits x batch fills the most of that wave, the
+// widest on ties (longer contiguous row segments); splits are at most 8 (one
+// cluster) and at least 16 rows per thread.  Shapes with more strips than the
+// wave holds take several waves of single-split CTAs.
 struct ClusterScorePlan {
   int col_threads;
   int64_t strips, splits, rows_per_split;
 };
 
 ClusterScorePlan cluster_score_plan(int64_t batch, int64_t M, int64_t d) {
-  const int sms = std::max(device_sm_count(), 1);
+  const int64_t slots = 2 * static_cast<int64_t>(std::max(device_sm_count(), 1));
   const int64_t vecs = (d + 7) / 8;
   int ct0 = 4;
   while (ct0 < 64 && ct0 < vecs) ct0 <<= 1;  // no wider than the row
   ClusterScorePlan best{};
+  int64_t best_fill = -1;
   for (int ct = ct0; ct >= 4; ct >>= 1) {
     const int rg = kScoreThreads / ct;
-    int64_t splits = (M + 16 * rg - 1) / (16 * rg);
-    splits = std::min<int64_t>(std::max<int64_t>(splits, 1), 8);
     const int64_t strips = (vecs + ct - 1) / ct;
-    best = {ct, strips, splits, (M + splits - 1) / splits};
-    if (strips * splits * batch >= 2 * sms) break;
+    const int64_t max_splits = std::min<int64_t>(std::max<int64_t>((M + 16 * rg - 1) / (16 * rg), 1), 8);
+    const int64_t per_split = strips * batch;
+    const int64_t splits = std::max<int64_t>(std::min<int64_t>(max_splits, slots / std::max<int64_t>(per_split, 1)), 1);
+    const int64_t ctas = per_split * splits;
+    const int64_t fill = std::min(ctas, slots);
+    if (fill > best_fill) {
+      best_fill = fill;
+      best = {ct, strips, splits, (M + splits - 1) / splits};
+    }
   }
   return best;
 }
 
 }  // namespace
 
+namespace {
+
+// 16-byte vector loads are possible: aligned base, row pitch and batch stride.
+bool score_vec_ok(const void* A, int dtype, int64_t batch, int64_t lda, int64_t batch_stride) {
+  const size_t elt = dtype == 1 ? 2 : 4;
+  return (reinterpret_cast<uintptr_t>(A) % 16 == 0) && ((lda * elt) % 16 == 0) &&
+         (batch == 1 || (batch_stride * elt) % 16 == 0);
+}
+
+// The one-launch cluster kernel serves this call (it writes no partial sums).
+bool score_cluster_path(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
+                        int64_t batch_stride) {
+  return dtype == 1 && score_vec_ok(A, dtype, batch, lda, batch_stride) && M > 0 && batch <= 65535 &&
+         cluster_score_plan(batch, M, d).strips <= 0x7FFFFFFFLL;
+}
+
+}  // namespace
+
+size_t score_workspace_used(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
+                            int64_t batch_stride) {
+  if (M == 0 || score_cluster_path(A, dtype, batch, M, d, lda, batch_stride)) return 0;
+  return score_workspace_bytes(dtype, batch, M, d);
+}
+
 cudaError_t launch_score(const void* A, int dtype, int64_t batch, int64_t M, int64_t d, int64_t lda,
                          int64_t batch_stride, float* ss, int64_t ld_ss, int sqrt_out, void* ws,
                          cudaStream_t stream) {
   const ScorePlan p = score_plan(dtype, batch, M, d);
-  const size_t elt = dtype == 1 ? 2 : 4;
-  const bool vec_ok = (reinterpret_cast<uintptr_t>(A) % 16 == 0) && ((lda * elt) % 16 == 0) &&
-                      (batch == 1 || (batch_stride * elt) % 16 == 0);
-  if (dtype == 1 && vec_ok && M > 0 && batch <= 65535) {
+  const bool vec_ok = score_vec_ok(A, dtype, batch, lda, batch_stride);
+  if (score_cluster_path(A, dtype, batch, M, d, lda, batch_stride)) {
     const ClusterScorePlan c = cluster_score_plan(batch, M, d);
-    if (c.strips <= 0x7FFFFFFFLL) {
+    {
       cudaLaunchConfig_t cfg{};
       cfg.gridDim = dim3(static_cast<unsigned>(c.strips), static_cast<unsigned>(c.splits),
                          static_cast<unsigned>(batch));
