@@ -397,10 +397,12 @@ __global__ void __launch_bounds__(1024, 1)
   const uint32_t k = static_cast<uint32_t>(k64);
   select_staged<1024>(keys, d, k, kmin, kmax, idx);
   __syncthreads();  // this block's index writes are visible to all its threads
+  // idx was written by this kernel: read it with coherent loads, not through
+  // the read-only path
   for (int64_t e = tid; e < static_cast<int64_t>(M) * k; e += 1024) {
     const int m = static_cast<int>(e / k);
     const int64_t r = e % k;
-    AI[m * ld_ai + r] = A[static_cast<int64_t>(m) * lda + __ldg(idx + r)];
+    AI[m * ld_ai + r] = A[static_cast<int64_t>(m) * lda + idx[r]];
   }
 }
 

@@ -4,17 +4,21 @@ Inputs are the seeded attention workload; kv-groups are redrawn (the
 generator's `attempt`) until every q-head's head_dim boundary has a relative
 score gap >= 2e-5 and its token boundary a relative gap >= 1e-3, so the fp32
 GPU ranking and the fp64 oracle ranking must agree and index sets are compared
-bit-exactly.  At full size, where such margins cannot be drawn in reasonable
-time, the token set is checked for validity instead (every kept score at
-least, every dropped score at most, the k-th largest oracle score within
-1e-4) and O is compared against the oracle evaluated on the GPU's set.
+bit-exactly.  At full size the search for such draws takes tens of minutes of
+CPU time, so it is done once by tests/golden/make_attention_attempts.py (gaps
+>= 2e-5 and >= 1e-4) and the test reads the stored attempts; the sets of the
+checked heads are again compared bit-exactly.
 
 Tolerances, from the arithmetic: logits are exact bf16 products summed in
 fp32; lse to 2e-5 absolute; token scores to 1e-4 relative; O elementwise
-within 2^-8 * sum_j P_ij |V_j| (P is rounded to bf16 before the PV product)
-plus the fp32 summation bound and, for bf16 output, one bf16 ulp; relative
-Frobenius of O <= 5e-3."""
+within 2^-11 * sum_j P_ij |V_j| (P is scaled by 2^15 and rounded to fp16,
+11 significant bits, before the PV product; V is widened exactly to fp16)
+plus the fp32 summation bound, the fp16 subnormal floors (2^-25 per unit of
+P, 2^-40 per unit of |V|) and, for bf16 output, one bf16 ulp; relative
+Frobenius of O <= 2e-3."""
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -24,10 +28,14 @@ import oracle
 import workloads as W
 from oracle import attention as OA
 from oracle.conditioning import boundary_gaps
+from tests import oracle_pool
 from tests.helpers import bf16_tensor, bf16_ulp, rel_fro, to_f64
 
 pytestmark = pytest.mark.gpu
 R = None
+# full-size lse and token-score tolerances (fp32 sums over up to 32768 terms)
+LSE_ATOL_FULL = 2e-5
+T_RTOL_FULL = 5e-5
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -84,7 +92,8 @@ def run_gpu(inp, out_dtype=torch.float32):
 
 
 def check_o(got, ref, P, V, idx_t, kt, bf16_out):
-    _bound_check(got, ref, np.abs(P[:, idx_t]) @ np.abs(V[idx_t]), kt, bf16_out)
+    Pk, Vk = P[:, idx_t], V[idx_t]
+    _bound_check(got, ref, np.abs(Pk) @ np.abs(Vk), Pk.sum(axis=1), np.abs(Vk).sum(axis=0), kt, bf16_out)
 
 
 CASES = [  # B, Hq, Hkv, S, D, rho_d, rho_t
@@ -116,7 +125,7 @@ def test_attention_parity(case, out_dtype):
             np.testing.assert_array_equal(idx_t[b, h], r["idx_t"])
             check_o(O[b, h], r["O"], r["P"], V[b, g], r["idx_t"], kt, out_dtype == torch.bfloat16)
             errs.append(rel_fro(O[b, h], r["O"]))
-    assert max(errs) <= 5e-3, errs
+    assert max(errs) <= 2e-3, errs
 
 
 def test_attention_rows_without_kept_tokens_are_zero():
@@ -141,50 +150,87 @@ def test_attention_rows_without_kept_tokens_are_zero():
     check_o(O[0, 0], r["O"], r["P"], V, r["idx_t"], 2, False)
 
 
-def _bound_check(got, ref, absterm, kt, bf16_out):
-    bound = (2.0 ** -8 + 2e-5 + kt * 2.0 ** -24) * absterm + 1e-30
+def test_attention_flags_v_beyond_fp16():
+    """A kept value of V beyond fp16's range (the P V product's operand type)
+    is saturated and reported in the device error word; nothing faults."""
+    S, D = 256, 64
+    rng = np.random.default_rng(21)
+    c = np.linspace(0.5, 1.5, D)
+    Qf = c[None, :] + 0.05 * rng.standard_normal((S, D))
+    Kf = 0.05 * rng.standard_normal((S, D))
+    Kf[[5, 9]] = 0.9 * c[None, :]
+    Vf = rng.standard_normal((S, D))
+    Vf[5, 3] = 1.0e5
+    enc = lambda x: W.f32_to_bf16_bits(x).reshape(1, 1, S, D)
+    Qt, Kt, Vt = (bf16_tensor(enc(x)) for x in (Qf, Kf, Vf))
+    R.rmm_device_error(clear=True)
+    R.rmm_attention(Qt, Kt, Vt, 1.0, 2.0 / S, out_dtype=torch.float32)
+    assert R.rmm_device_error(clear=True) == 2  # RMM_DEVERR_FP16_RANGE
+    Vf[5, 3] = 6.0e4                             # inside the range: no flag
+    R.rmm_attention(Qt, Kt, bf16_tensor(enc(Vf)), 1.0, 2.0 / S, out_dtype=torch.float32)
+    assert R.rmm_device_error(clear=True) == 0
+
+
+def _bound_check(got, ref, absterm, psum, vabs, kt, bf16_out):
+    """|O - O_ref| <= (2^-11 + 2e-5 + k_t 2^-24) sum_j P_j |V_j|
+                      + 2^-25 sum_j P_j + 2^-40 sum_j |V_j|  (+ a bf16 ulp)."""
+    bound = ((2.0 ** -11 + 2e-5 + kt * 2.0 ** -24) * absterm + 2.0 ** -25 * np.asarray(psum)[:, None]
+             + 2.0 ** -40 * np.asarray(vabs)[None, :] + 1e-30)
     if bf16_out:
         bound = bound + bf16_ulp(np.maximum(np.abs(got), np.abs(ref)))
     bad = np.abs(got - ref) > bound
     assert not bad.any(), f"{bad.sum()} of {bad.size} outside the bound"
 
 
+ATTEMPTS_FILE = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "attention_full_attempts.json")
+
+
 @pytest.mark.slow
-@pytest.mark.parametrize("S,Hq,Hkv,seed,heads", [(8192, 32, 32, 3, [0, 31]), (32768, 32, 8, 4, [13])])
-def test_attention_full_size_sampled_heads(S, Hq, Hkv, seed, heads):
-    """Full-size workloads (32 heads at 8192 tokens; GQA 32/8 at 32768 tokens),
-    bf16 output: every head runs on the GPU; sampled heads are checked with the
-    oracle's row/column-restricted forms: the head_dim set (bit-exact where its
-    margin is clear), lse of every row, token scores of every column, validity
-    of the kept token set, and O on 256 sampled rows given that set."""
-    inp = W.attention(seed, 1, Hq, Hkv, S, 128, 0.5, 0.5)
+@pytest.mark.parametrize("name", ["attn_32h_8192", "attn_gqa32x8_32768"])
+def test_attention_full_size_exact(name):
+    """Full-size workloads (32 heads at 8192 tokens; GQA 32/8 at 32768 tokens,
+    head_dim 128, rho_d = rho_t = 0.5), bf16 output.  The checked kv-groups
+    are drawn at the attempts stored by tests/golden/make_attention_attempts.py
+    (the oracle's boundary gaps are >= 2e-5 for head_dim and >= 1e-4 for
+    tokens, re-verified here), the other groups at attempt 0; every head runs
+    on the GPU.  Each checked head: the head_dim and token index sets equal
+    the oracle's bit for bit, lse of every row and the token score of every
+    column agree with the oracle's row/column-restricted forms, and O on 256
+    sampled rows (first, last and block edges included) is within the
+    elementwise bound, with relative Frobenius error <= 2e-3."""
+    with open(ATTEMPTS_FILE) as f:
+        man = json.load(f)
+    c = man["configs"][name]
+    S, Hq, Hkv, seed = c["S"], c["Hq"], c["Hkv"], c["seed"]
+    G = Hq // Hkv
+    attempts = [int(c["attempts"].get(str(g), 0)) for g in range(Hkv)]
+    groups = sorted(int(g) for g in c["attempts"])
+    heads = [h for g in groups for h in range(g * G, (g + 1) * G)]
+    inp = W.attention(seed, 1, Hq, Hkv, S, 128, 0.5, 0.5, attempts)
     O, idx_d, idx_t, lse, tsc = run_gpu(inp, torch.bfloat16)
     kd, kt = 64, oracle.k_from_rho(0.5, S)
-    rng = np.random.default_rng(S)
-    rows = np.unique(np.concatenate([[0, 1, 127, 128, S - 1], rng.integers(0, S, 251)]))
+    ref = {}
     for h in heads:
         g = OA.kv_head_of(h, Hq, Hkv)
         Q, K, V = (oracle.decode(x, "bf16") for x in (inp.Q[0, h], inp.K[0, g], inp.V[0, g]))
-        ssq = oracle.column_sq_norms(Q)
-        gd, _ = boundary_gaps(ssq, [kd])
-        if gd[kd] >= 2e-5:
-            np.testing.assert_array_equal(idx_d[0, h], OA.head_dim_selection(Q, 0.5))
-        else:  # a valid top-k within fp32 scoring error
-            T = np.sort(ssq)[::-1][kd - 1]
-            m = np.zeros(128, bool)
-            m[idx_d[0, h]] = True
-            assert ssq[m].min() >= T * (1 - 1e-5) and ssq[~m].max() <= T * (1 + 1e-5)
-        sel = idx_d[0, h]
-        L = OA.lse_rows(Q, K, sel, np.arange(S))
-        np.testing.assert_allclose(lse[0, h], L, rtol=0, atol=5e-5)
-        t = OA.token_scores(Q, K, sel, L, np.arange(S))
-        np.testing.assert_allclose(tsc[0, h], t, rtol=2e-4, atol=0)
-        T = np.sort(t)[::-1][kt - 1]
-        kept = np.zeros(S, bool)
-        kept[idx_t[0, h]] = True
-        assert kept.sum() == kt and np.all(np.diff(idx_t[0, h]) > 0)
-        assert t[kept].min() >= T * (1 - 2e-4) and t[~kept].max() <= T * (1 + 2e-4)
-        ref = OA.out_rows(Q, K, V, sel, L[rows], idx_t[0, h], rows)
+        ref[h] = (Q, K, V, OA.head_dim_selection(Q, 0.5))
+    pool = oracle_pool.spawn_pool(min(len(heads), 4))
+    try:
+        outs = pool.map(oracle_pool.head_lse_and_token_scores, [(ref[h][0], ref[h][1], ref[h][3]) for h in heads])
+    finally:
+        pool.close()
+    rng = np.random.default_rng(S)
+    rows = np.unique(np.concatenate([[0, 1, 127, 128, S - 1], rng.integers(0, S, 251)]))
+    for h, (L, t) in zip(heads, outs):
+        Q, K, V, sel = ref[h]
+        assert boundary_gaps(oracle.column_sq_norms(Q), [kd])[0][kd] >= man["gap_head_dim"]
+        assert boundary_gaps(t, [kt])[0][kt] >= man["gap_tokens"]
+        np.testing.assert_array_equal(idx_d[0, h], sel)
+        np.testing.assert_allclose(lse[0, h], L, rtol=0, atol=LSE_ATOL_FULL)
+        np.testing.assert_allclose(tsc[0, h], t, rtol=T_RTOL_FULL, atol=0)
+        np.testing.assert_array_equal(idx_t[0, h], oracle.topk_indices(t, kt))
+        ref_o = OA.out_rows(Q, K, V, sel, L[rows], idx_t[0, h], rows)
         absterm = OA.out_rows(Q, K, np.abs(V), sel, L[rows], idx_t[0, h], rows)
-        _bound_check(O[0, h][rows], ref, absterm, kt, True)
-        assert rel_fro(O[0, h][rows], ref) <= 5e-3
+        psum = OA.out_rows(Q, K, np.ones_like(V[:, :1]), sel, L[rows], idx_t[0, h], rows)[:, 0]
+        _bound_check(O[0, h][rows], ref_o, absterm, psum, np.abs(V[idx_t[0, h]]).sum(axis=0), kt, True)
+        assert rel_fro(O[0, h][rows], ref_o) <= 2e-3
