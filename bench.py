@@ -54,9 +54,11 @@ def parse_args():
     ap.add_argument("--impl", choices=["rmm", "reference"], default="rmm")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["bench", "matmul", "attention", "decode", "w8", "decode_attention", "block"],
+    ap.add_argument("--case", choices=["bench", "matmul", "attention", "attention_gqa", "layer70b", "decode", "w8",
+                                       "decode_attention", "block", "down"],
                     default="bench",
-                    help="matmul / attention / decode / w8 / decode_attention / block: run only that workload a few "
+                    help="matmul / attention / attention_gqa / layer70b / decode / w8 / decode_attention / block / "
+                         "down: run only that workload a few "
                          "times and exit (a short program for profiler captures; prints no JSON line)")
     a = ap.parse_args()
     if a.warmup < 3:
@@ -172,6 +174,13 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ CPU oracle timing
 
+def bench_config(world):
+    """The workload's config, identical in both arms' JSON lines."""
+    return {"workload": WORKLOAD, "M": M, "d": D, "N": N, "rho": RHO, "k": k_of(RHO, D),
+            "l2": "256 MiB buffer written between steps, outside the timed intervals",
+            "parallelism": f"independent batch per GPU x{world}"}
+
+
 def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -238,11 +247,12 @@ def run_reference(args):
     t = time.perf_counter() - t0
     value = 2.0 * rows_n * N * k * args.steps / t / 1e12
     cores = cpu_threads()
-    sample = f"each step: fp64 oracle on {rows_n} of {M} rows (scores, top-k, reduced product)"
+    sample = (f"each step: fp64 oracle on {rows_n} of {M} rows (scores, top-k, reduced product), on the host "
+              "cores; no GPU and so no L2 flush; value scaled to the FLOPs of the rows processed")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD, "M": M, "d": D, "N": N, "rho": RHO, "k": k},
+            "data": "synthetic", "config": bench_config(args.gpus),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -266,44 +276,174 @@ def aggregate(local_ms, local_flops, world):
 
 
 ATTN = dict(B=1, Hq=32, Hkv=32, S=8192, D=128, rho_d=0.5, rho_t=0.5, seed=3)
+ATTN_GQA = dict(B=1, Hq=32, Hkv=8, S=32768, D=128, rho_d=0.5, rho_t=0.5, seed=4)
+EX2_PER_CLK_SM = 16  # exp unit (MUFU ex2) results per clock per SM, measured with a throughput probe
 
 
-def measure_attention(R, workloads, bf16_tensor, dev, stream, flush, steps, timed):
-    """Reduced attention on the 32-head, 8192-token workload (same flush and
-    event protocol as the GEMM path), next to torch's causal SDPA."""
+def measure_attention(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, peaks, a=ATTN):
+    """Reduced attention (same flush and event protocol as the GEMM path), next
+    to torch's causal SDPA (flash/cuDNN; for GQA the kv heads are repeated
+    once, outside the timed region).  Rooflines of the whole pipeline: the
+    tensor-core work (logits of passes A and B over the causal pairs at k_d,
+    logits and P V of pass C over the kept causal pairs) at the measured bf16
+    peak, and the exponentials (one per causal pair in each of passes A and
+    B, one per kept causal pair in pass C) at 16 per clock per SM at the SM
+    clock sampled during the timed calls."""
+    import numpy as np
     import torch
-    a = ATTN
     inp = workloads.attention(a["seed"], a["B"], a["Hq"], a["Hkv"], a["S"], a["D"], a["rho_d"], a["rho_t"])
     Q, K, V = (bf16_tensor(x, dev) for x in (inp.Q, inp.K, inp.V))
+    del inp
     O = torch.empty_like(Q)
-    ws = torch.empty(R.rmm_attention_workspace_size(a["B"], a["Hq"], a["Hkv"], a["S"], a["D"], a["rho_d"],
-                                                    a["rho_t"]), dtype=torch.uint8, device=dev)
+    B, Hq, Hkv, S, D = a["B"], a["Hq"], a["Hkv"], a["S"], a["D"]
+    kd, kt = R.rmm_k_from_rho(a["rho_d"], D), R.rmm_k_from_rho(a["rho_t"], S)
+    idx_t = torch.empty((B * Hq, kt), dtype=torch.int32, device=dev)
+    ws = torch.empty(R.rmm_attention_workspace_size(B, Hq, Hkv, S, D, a["rho_d"], a["rho_t"]), dtype=torch.uint8,
+                     device=dev)
+    Kr = K if Hkv == Hq else K.repeat_interleave(Hq // Hkv, 1)
+    Vr = V if Hkv == Hq else V.repeat_interleave(Hq // Hkv, 1)
 
     def rmm(ev):
         ev[0].record(stream)
-        R.rmm_attention(Q, K, V, a["rho_d"], a["rho_t"], out=O, ws=ws)
+        R.rmm_attention(Q, K, V, a["rho_d"], a["rho_t"], out=O, idx_t=idx_t, ws=ws)
         ev[1].record(stream)
 
     def sdpa(ev):
         ev[0].record(stream)
-        torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=True)
+        torch.nn.functional.scaled_dot_product_attention(Q, Kr, Vr, is_causal=True)
         ev[1].record(stream)
 
     for fn in (rmm, sdpa):
         for _ in range(3):
             fn([torch.cuda.Event(enable_timing=True) for _ in range(2)])
-    rmm_ms = statistics.mean(p[0] for p in timed(rmm, steps, 2))
+    with ClockSampler(torch.cuda.get_device_properties(dev)) as clk:
+        rmm_ms = statistics.mean(p[0] for p in timed(rmm, steps, 2))
     sdpa_ms = statistics.mean(p[0] for p in timed(sdpa, steps, 2))
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the attention runs")
-    S, D, H = a["S"], a["D"], a["B"] * a["Hq"]
+    H = B * Hq
+    pairs = H * S * (S + 1) / 2.0
+    pos = idx_t.cpu().numpy().astype(np.int64)
+    kept_pairs = float(np.sum(S - pos))           # queries i >= pos_r, summed over kept tokens and heads
+    flops = 2.0 * kd * pairs * 2 + 2.0 * (kd + D) * kept_pairs
+    exps = 2.0 * pairs + kept_pairs
+    ck = clk.summary()
+    mhz = ck["sm_mhz"] or 1965.0
+    tensor_floor_ms = flops / (peaks["bf16_tflops"] * 1e12) * 1e3
+    exp_floor_ms = exps / (EX2_PER_CLK_SM * 148 * mhz * 1e6) * 1e3
     dense_flops = 4.0 * (S * (S + 1) / 2) * D * H
-    return {"workload": f"causal attention B{a['B']} H{a['Hq']} S{S} D{D}, rho_d={a['rho_d']} rho_t={a['rho_t']}, "
+    return {"workload": f"causal attention B{B} Hq{Hq} Hkv{Hkv} S{S} D{D}, rho_d={a['rho_d']} rho_t={a['rho_t']}, "
                         "Q/K/V N(0,1) x per-dim lognormal(0,0.5)",
             "ms": rmm_ms, "sdpa_ms": sdpa_ms, "speedup_vs_sdpa": sdpa_ms / rmm_ms,
             "dense_equivalent_tflops": dense_flops / (rmm_ms * 1e-3) / 1e12,
             "sdpa_tflops": dense_flops / (sdpa_ms * 1e-3) / 1e12,
-            "gpu_launches_per_call": 12, "calls": steps}
+            "kept_pair_frac": kept_pairs / pairs,
+            "roofline": {"tensor": {"flops": flops, "floor_ms": tensor_floor_ms, "frac": tensor_floor_ms / rmm_ms,
+                                    "peak_tflops": peaks["bf16_tflops"]},
+                         "exp_unit": {"exps": exps, "floor_ms": exp_floor_ms, "frac": exp_floor_ms / rmm_ms,
+                                      "ex2_per_clk_sm": EX2_PER_CLK_SM, "sm_mhz": mhz},
+                         "bound": "exp_unit" if exp_floor_ms > tensor_floor_ms else "tensor"},
+            "clocks": ck, "gpu_launches_per_call": 12, "calls": steps}
+
+
+def measure_layer70b(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, peaks):
+    """The 70B-shaped layer (2048 tokens, hidden 8192, MLP 28672; q/k/v/o at
+    rho = 0.5, up/gate/down at rho = 0.8), each projection on its own drawn
+    activation: the rmm_matmul step, the selection alone (score + top-k, one
+    event interval), the product alone (rmm_gemm on the compacted activation,
+    an event before and after it) and cuBLAS on the same shape, all with a
+    256 MiB write between calls.  q, k and v also run as one rmm_matmul_multi
+    call on q's activation (one selection for the three weights)."""
+    import torch
+    out = {}
+    qkv = {}
+    for name, Mg, dg, Ng, rho in workloads.layer70b_gemms():
+        inp = workloads.layer70b_inputs(name)
+        X, Wt = bf16_tensor(inp.A, dev), bf16_tensor(inp.B, dev)
+        del inp
+        k = R.rmm_k_from_rho(rho, dg)
+        Y = torch.empty((Mg, Ng), dtype=torch.bfloat16, device=dev)
+        ss = torch.empty(dg, dtype=torch.float32, device=dev)
+        idx = torch.empty(k, dtype=torch.int32, device=dev)
+        AI = torch.empty((Mg, (k + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)[:, :k]
+        mws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, Mg, dg, Ng, rho), dtype=torch.uint8, device=dev)
+        gws = torch.empty(R.rmm_gemm_workspace_size(R.RMM_BF16, Ng, k), dtype=torch.uint8, device=dev)
+        sws = torch.empty(max(R.rmm_score_workspace_size(R.RMM_BF16, 1, Mg, dg), 256), dtype=torch.uint8, device=dev)
+
+        def step(ev):
+            ev[0].record(stream)
+            R.rmm_matmul(X, Wt, rho, out=Y, ws=mws)
+            ev[1].record(stream)
+
+        def split(ev):
+            ev[0].record(stream)
+            R.rmm_score(X, out=ss, ws=sws)
+            R.rmm_topk(ss, k, out=idx)
+            ev[1].record(stream)
+            R.rmm_compact(X, idx, out=AI)
+            ev[2].record(stream)
+            R.rmm_gemm(AI, Wt, idx, out=Y, ws=gws)
+            ev[3].record(stream)
+
+        def dense(ev):
+            ev[0].record(stream)
+            torch.matmul(X, Wt, out=Y)
+            ev[1].record(stream)
+        for _ in range(3):
+            step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+            split([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+            dense([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        ms = statistics.mean(p[0] for p in timed(step, steps, 2))
+        sp = timed(split, steps, 4)
+        sel_ms = statistics.mean(p[0] for p in sp)
+        gemm_ms = statistics.mean(p[2] for p in sp)
+        dms = statistics.mean(p[0] for p in timed(dense, steps, 2))
+        if R.rmm_device_error(stream) != 0:
+            raise SystemExit(f"device error during the 70B-layer {name} runs")
+        fl = 2.0 * Mg * Ng * k
+        out[name] = {"M": Mg, "d": dg, "N": Ng, "rho": rho, "k": k, "step_us": ms * 1e3,
+                     "effective_tflops": fl / (ms * 1e-3) / 1e12, "dense_us": dms * 1e3,
+                     "speedup_vs_dense": dms / ms, "select_us": sel_ms * 1e3,
+                     "select_frac_of_dense": sel_ms / dms, "gemm_us": gemm_ms * 1e3,
+                     "gemm_roofline_frac": fl / (gemm_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]}
+        if name == "q_proj":
+            qkv["X"], qkv["q"] = X, Wt
+        elif name in ("k_proj", "v_proj"):
+            qkv[name[0]] = Wt
+        del Y, AI, mws, gws
+    # q, k, v on one activation: one selection, three products
+    X, Ws = qkv["X"], [qkv["q"], qkv["k"], qkv["v"]]
+    Ys = [torch.empty((X.shape[0], w.shape[1]), dtype=torch.bfloat16, device=dev) for w in Ws]
+    ws = torch.empty(R.rmm_matmul_multi_workspace_size(X.shape[0], X.shape[1], max(w.shape[1] for w in Ws), 0.5),
+                     dtype=torch.uint8, device=dev)
+
+    def multi(ev):
+        ev[0].record(stream)
+        R.rmm_matmul_multi(X, Ws, 0.5, outs=Ys, ws=ws)
+        ev[1].record(stream)
+
+    def dense3(ev):
+        ev[0].record(stream)
+        for w, y in zip(Ws, Ys):
+            torch.matmul(X, w, out=y)
+        ev[1].record(stream)
+    for _ in range(3):
+        multi([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        dense3([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    ms = statistics.mean(p[0] for p in timed(multi, steps, 2))
+    dms = statistics.mean(p[0] for p in timed(dense3, steps, 2))
+    if R.rmm_device_error(stream) != 0:
+        raise SystemExit("device error during the 70B-layer q/k/v runs")
+    k = R.rmm_k_from_rho(0.5, X.shape[1])
+    fl = sum(2.0 * X.shape[0] * w.shape[1] * k for w in Ws)
+    out["qkv_shared_selection"] = {"step_us": ms * 1e3, "dense_us": dms * 1e3, "speedup_vs_dense": dms / ms,
+                                   "effective_tflops": fl / (ms * 1e-3) / 1e12}
+    tot = sum(v["step_us"] for n, v in out.items() if n.endswith("_proj"))
+    tot_dense = sum(v["dense_us"] for n, v in out.items() if n.endswith("_proj"))
+    out["layer_total"] = {"step_us": tot, "dense_us": tot_dense, "speedup_vs_dense": tot_dense / tot}
+    out["workload"] = ("70B-shaped layer: 2048 tokens, hidden 8192, MLP 28672; activations as the MLP up "
+                       "projection's (lognormal channel scale, 1% outliers x20), weights N(0, 0.02^2)")
+    return out
 
 
 def measure_decode(R, workloads, bf16_tensor, dev, stream, flush, steps, timed, Wt, hbm_gbs):
@@ -545,10 +685,19 @@ def measure_down(R, workloads, bf16_tensor, dev, stream, flush, steps, timed):
     k = R.rmm_k_from_rho(0.5, dd)
     Y = torch.empty((Md, Nd), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(R.rmm_matmul_workspace_size(R.RMM_BF16, Md, dd, Nd, 0.5), dtype=torch.uint8, device=dev)
+    ss = torch.empty(dd, dtype=torch.float32, device=dev)
+    idx = torch.empty(k, dtype=torch.int32, device=dev)
+    sws = torch.empty(max(R.rmm_score_workspace_size(R.RMM_BF16, 1, Md, dd), 256), dtype=torch.uint8, device=dev)
 
     def rmm(ev):
         ev[0].record(stream)
         R.rmm_matmul(Hd, Wd, 0.5, out=Y, ws=ws)
+        ev[1].record(stream)
+
+    def select(ev):
+        ev[0].record(stream)
+        R.rmm_score(Hd, out=ss, ws=sws)
+        R.rmm_topk(ss, k, out=idx)
         ev[1].record(stream)
 
     def dense(ev):
@@ -558,14 +707,18 @@ def measure_down(R, workloads, bf16_tensor, dev, stream, flush, steps, timed):
     for _ in range(3):
         rmm([torch.cuda.Event(enable_timing=True) for _ in range(2)])
         dense([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+        select([torch.cuda.Event(enable_timing=True) for _ in range(2)])
     ms = statistics.mean(p[0] for p in timed(rmm, steps, 2))
     dms = statistics.mean(p[0] for p in timed(dense, steps, 2))
+    sel_ms = statistics.mean(p[0] for p in timed(select, steps, 2))
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the down-projection runs")
     sweep = rho_sweep(R, Hd, Wd, (0.8, 1.0), dms, min(steps, 30), timed, stream, dev)
     return {"workload": f"MLP down projection H[{Md}x{dd}] . W[{dd}x{Nd}] bf16, rho=0.5, 256 MiB flush between steps",
             "step_us": ms * 1e3, "dense_us": dms * 1e3, "speedup_vs_dense": dms / ms,
-            "effective_tflops": 2.0 * Md * Nd * k / (ms * 1e-3) / 1e12, "other_rho": sweep}
+            "effective_tflops": 2.0 * Md * Nd * k / (ms * 1e-3) / 1e12, "other_rho": sweep,
+            "select_overhead": {"score_topk_us": sel_ms * 1e3, "dense_us": dms * 1e3, "frac_of_dense": sel_ms / dms,
+                                "target": 0.10}}
 
 
 DEC_ATTN = {"seed": 5, "Hq": 32, "Hkv": 8, "L": 32768, "D": 128, "rho_d": 0.5, "rho_t": 0.5}
@@ -725,6 +878,13 @@ def run_rmm(args):
             fn()
         ev[1].record(stream)
 
+    def select_step(ev):
+        # the selection alone: column scores and top-k, one event interval
+        ev[0].record(stream)
+        kernel_calls["score"]()
+        kernel_calls["topk"]()
+        ev[1].record(stream)
+
     for _ in range(args.warmup):
         flush.zero_()
         whole_path_step()
@@ -770,6 +930,9 @@ def run_rmm(args):
     for _ in range(3):
         torch.matmul(X, Wt, out=Y)
     dense_ms = statistics.mean(p[0] for p in timed(dense, min(args.steps, 100), 2))
+    for _ in range(3):
+        select_step([torch.cuda.Event(enable_timing=True) for _ in range(2)])
+    select_ms = statistics.mean(p[0] for p in timed(select_step, min(args.steps, 100), 2))
     # the same workload at the other rho values of the up-projection config
     other_rho = rho_sweep(R, X, Wt, (0.7, 0.8, 1.0), dense_ms, min(args.steps, 30), timed, stream, dev)
 
@@ -821,9 +984,11 @@ def run_rmm(args):
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the dense / end-to-end runs")
 
-    attention = measure_attention(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 20), timed)
-
     peaks, peak_src = load_peaks()
+    attention = measure_attention(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 20), timed, peaks)
+    attention_gqa = measure_attention(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 10), timed,
+                                      peaks, ATTN_GQA)
+    layer70b = measure_layer70b(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 20), timed, peaks)
     decode = measure_decode(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed, Wt,
                             peaks["hbm_gbs"])
     w8 = measure_w8(R, workloads, bf16_tensor, dev, stream, flush, min(args.steps, 50), timed, X, peaks["hbm_gbs"])
@@ -865,10 +1030,12 @@ def run_rmm(args):
             "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded Philox inputs of the workload's shape and distribution)",
-            "config": {"workload": WORKLOAD, "M": M, "d": D, "N": N, "rho": RHO, "k": k,
-                       "l2": "256 MiB buffer written between steps, outside the timed intervals",
-                       "parallelism": f"independent batch per GPU x{world}"},
+            "config": bench_config(world),
             "speedup_vs_dense": dense_ms / path_ms, "dense_ms": dense_ms, "other_rho": other_rho,
+            "select_overhead_frac_of_dense": select_ms / dense_ms,
+            "select_overhead": {"score_topk_us": select_ms * 1e3, "dense_us": dense_ms * 1e3,
+                                "frac_of_dense": select_ms / dense_ms, "target": 0.10,
+                                "mlp_down": down["select_overhead"]},
             "dense_tflops": 2.0 * M * N * D / (dense_ms * 1e-3) / 1e12,
             "dense_equivalent_tflops": 2.0 * M * N * D / (path_ms * 1e-3) / 1e12,
             "path_roofline_frac": path_roof_ms / path_ms,
@@ -884,6 +1051,8 @@ def run_rmm(args):
                     "schedule": "steps pipelined over copy-in, compute and copy-out streams (double buffers)"},
             "gpu_launches": launches_per_step * args.steps,
             "attention": attention,
+            "attention_gqa32k": attention_gqa,
+            "layer70b": layer70b,
             "decode": decode,
             "int8_weight": w8,
             "decode_attention": dec_attn,
@@ -921,8 +1090,27 @@ def run_case(case):
         for _ in range(4):
             flush.zero_()
             R.rmm_matmul(X, Wt, RHO, out=Y, ws=ws)
-    elif case == "attention":
-        a = ATTN
+    elif case == "layer70b":
+        # every projection of the 70B-shaped layer, rmm_matmul twice each
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for name, Mg, dg, Ng, rho in workloads.layer70b_gemms():
+            inp = workloads.layer70b_inputs(name)
+            X, Wt = bf16_tensor(inp.A, dev), bf16_tensor(inp.B, dev)
+            Y = torch.empty((Mg, Ng), dtype=torch.bfloat16, device=dev)
+            for _ in range(2):
+                flush.zero_()
+                R.rmm_matmul(X, Wt, rho, out=Y)
+            del X, Wt, Y
+    elif case == "down":
+        inp = workloads.mlp_down()
+        Hd, Wd = bf16_tensor(inp.A, dev), bf16_tensor(inp.B, dev)
+        Y = torch.empty((inp.M, inp.N), dtype=torch.bfloat16, device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for _ in range(4):
+            flush.zero_()
+            R.rmm_matmul(Hd, Wd, 0.5, out=Y)
+    elif case in ("attention", "attention_gqa"):
+        a = ATTN if case == "attention" else ATTN_GQA
         inp = workloads.attention(a["seed"], a["B"], a["Hq"], a["Hkv"], a["S"], a["D"], a["rho_d"], a["rho_t"])
         Q, K, V = (bf16_tensor(x, dev) for x in (inp.Q, inp.K, inp.V))
         O = torch.empty_like(Q)
