@@ -420,6 +420,18 @@ rmm_status rmm_matmul(const void* A, int64_t lda, const void* B, int64_t ldb, in
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
   void* score_ws = base + w.score;
   void* ai = base + w.ai;
+  if (dtype == RMM_BF16 && M > 0 && N > 0 && aligned16(B) && ldb % 8 == 0 && gemv_select_supported(A, M, d, lda, false)) {
+    // up to 4 rows (decode): one launch whose CTAs each select the kept rows
+    // and stream their share of them
+    const GemvPlan pl = gemv_plan(M, N, k, device_sm_count());
+    if (pl.partial_bytes <= w.total - w.bi) {
+      unsigned* err = device_error_word();
+      if (!err) return RMM_ERR_CUDA;
+      return from_cuda(launch_gemv_select(A, lda, M, d, B, ldb, nullptr, N, k, pl, reinterpret_cast<float*>(base + w.bi),
+                                          Y, out_dtype, ldy, idx, ss, err, static_cast<cudaStream_t>(stream)),
+                       "rmm_matmul: fused decode launch");
+    }
+  }
   if (dtype == RMM_BF16 && M > 0 && N > 0 && select_rows_supported(M, d) && aligned16(B) && ldb % 8 == 0) {
     // a few rows (decode): scores, selection and A_I in one launch, then the
     // product that reads only the kept rows of B
@@ -531,6 +543,17 @@ rmm_status rmm_matmul_w8(const void* A, int64_t lda, const int8_t* Bq, int64_t l
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(base + w.idx);
   void* ai = base + w.ai;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M > 0 && N > 0 && aligned16(Bq) && ldb % 16 == 0 && b_scale && gemv_select_supported(A, M, d, lda, true)) {
+    // up to 4 rows (decode): selection and product in one launch
+    const GemvPlan pl = gemv_plan(M, N, k, device_sm_count());
+    if (pl.partial_bytes <= w.total - w.bi) {
+      unsigned* err = device_error_word();
+      if (!err) return RMM_ERR_CUDA;
+      return from_cuda(launch_gemv_select(A, lda, M, d, Bq, ldb, b_scale, N, k, pl,
+                                          reinterpret_cast<float*>(base + w.bi), Y, out_dtype, ldy, idx, ss, err, s),
+                       "rmm_matmul_w8: fused decode launch");
+    }
+  }
   if (M > 0 && N > 0 && select_rows_supported(M, d)) {
     const cudaError_t e = launch_select_rows(A, M, d, lda, k, idx, ss, ai, w.ld_ai, s);
     if (e != cudaSuccess) return from_cuda(e, "rmm_matmul_w8: row selection launch");

@@ -180,90 +180,94 @@ __global__ void __launch_bounds__(kCompactThreads) compact_staged_kernel(const u
   compact_rows_block(blockIdx.x, A, M, d, lda, idx, k, AI, ld_ai, R, err, stage);
 }
 
-// One CTA per kept row: the row I_r of B is copied whole with 16-byte loads and
-// stores, four in flight per thread (rows are contiguous, so this is a pure
-// streaming copy); a row length that is not a multiple of 16 bytes ends with
-// 2-byte copies.  Out-of-range indices produce a zero row and are flagged.
+// Kept rows of B, several per CTA when the copied slice of a row is short: CTA
+// `blk` copies kept rows [blk * rpb, +rpb).  Their source rows are read once
+// into shared memory; the (row, 16-byte vector) pairs are numbered row-major
+// and thread t copies pairs t, t + 256, ... with four loads in flight, so a
+// CTA moves at least ~16 KB however short the slice is (one CTA per row of a
+// few KB left the copy bound by block turnover).  A slice length that is not
+// a multiple of 16 bytes ends with 2-byte copies.  Out-of-range indices give
+// zero rows and are flagged.  kW8: B is int8 (vectors of 16 values, widened
+// to exact bf16: two 16-byte stores each; tail_elems trailing bytes); the
+// per-column scales are applied later, in the product's epilogue.
 constexpr int kGatherThreads = 256;
+constexpr int kGatherMaxRows = 32;                // kept rows per CTA at most
+constexpr int64_t kGatherTargetVecs = 1024;       // 16-byte source vectors per CTA (16 KB)
 static_assert(kGatherThreads == kCompactThreads, "the fused kernel runs compaction blocks at the gather block size");
 
-__device__ __forceinline__ void gather_row_block(int64_t r, const uint4* __restrict__ B, int64_t d, int64_t vecs,
-                                                 int64_t tail_halves, int64_t ldb_vec,
-                                                 const int32_t* __restrict__ idx, int64_t k,
-                                                 uint4* __restrict__ BI, int64_t ldbi_vec, unsigned* err) {
-  if (r >= k) return;
-  const int32_t j = __ldg(idx + r);
-  uint4* dst = BI + r * ldbi_vec;
-  if (j < 0 || j >= d) {
-    if (threadIdx.x == 0) record_error(err, kDevErrBadIndex);
-    for (int64_t v = threadIdx.x; v < vecs; v += kGatherThreads) dst[v] = make_uint4(0, 0, 0, 0);
-    if (threadIdx.x < tail_halves) reinterpret_cast<uint16_t*>(dst + vecs)[threadIdx.x] = 0;
-    return;
-  }
-  const uint4* src = B + static_cast<int64_t>(j) * ldb_vec;
-  if (threadIdx.x < tail_halves)  // bytes past the last whole 16-byte vector of the row
-    reinterpret_cast<uint16_t*>(dst + vecs)[threadIdx.x] = reinterpret_cast<const uint16_t*>(src + vecs)[threadIdx.x];
-  int64_t v = threadIdx.x;
-  for (; v + 3 * kGatherThreads < vecs; v += 4 * kGatherThreads) {
-    const uint4 a0 = __ldcs(src + v);
-    const uint4 a1 = __ldcs(src + v + kGatherThreads);
-    const uint4 a2 = __ldcs(src + v + 2 * kGatherThreads);
-    const uint4 a3 = __ldcs(src + v + 3 * kGatherThreads);
-    dst[v] = a0;
-    dst[v + kGatherThreads] = a1;
-    dst[v + 2 * kGatherThreads] = a2;
-    dst[v + 3 * kGatherThreads] = a3;
-  }
-  for (; v < vecs; v += kGatherThreads) dst[v] = __ldcs(src + v);
+// Kept rows per gather CTA for rows of `vecs` 16-byte source vectors.
+__host__ __device__ inline int gather_rows_per_block(int64_t vecs) {
+  if (vecs >= kGatherTargetVecs) return 1;
+  const int64_t r = kGatherTargetVecs / (vecs > 0 ? vecs : 1);
+  return static_cast<int>(r < kGatherMaxRows ? r : kGatherMaxRows);
 }
 
-// The int8 form (weight-only quantised B): row I_r of the int8 matrix is read
-// with 16-byte loads (16 values) and written as 16 exact bf16 values (two
-// 16-byte stores); the per-column scale is applied later, in the product's
-// epilogue.  A row length that is not a multiple of 16 ends with byte loads.
-__device__ __forceinline__ void gather_row_block_i8(int64_t r, const uint4* __restrict__ Bq, int64_t d, int64_t vecs,
-                                                    int64_t tail_bytes, int64_t ldb_vec,
-                                                    const int32_t* __restrict__ idx, int64_t k,
-                                                    uint4* __restrict__ BI, int64_t ldbi_vec, unsigned* err) {
-  if (r >= k) return;
-  const int32_t j = __ldg(idx + r);
-  uint4* dst = BI + r * ldbi_vec;
-  __nv_bfloat16* dst_tail = reinterpret_cast<__nv_bfloat16*>(dst + 2 * vecs);
-  if (j < 0 || j >= d) {
-    if (threadIdx.x == 0) record_error(err, kDevErrBadIndex);
-    for (int64_t v = threadIdx.x; v < 2 * vecs; v += kGatherThreads) dst[v] = make_uint4(0, 0, 0, 0);
-    if (threadIdx.x < tail_bytes) dst_tail[threadIdx.x] = __float2bfloat16_rn(0.f);
-    return;
+template <bool kW8>
+__device__ __forceinline__ void gather_rows_block(int64_t blk, int rpb, const uint4* __restrict__ B, int64_t d,
+                                                  int64_t vecs, int64_t tail_elems, int64_t ldb_vec,
+                                                  const int32_t* __restrict__ idx, int64_t k,
+                                                  uint4* __restrict__ BI, int64_t ldbi_vec, unsigned* err) {
+  __shared__ int32_t src_row[kGatherMaxRows];
+  const int64_t r0 = blk * rpb;
+  if (r0 >= k) return;  // block-uniform
+  const int nr = static_cast<int>(k - r0 < rpb ? k - r0 : rpb);
+  if (threadIdx.x < nr) {
+    const int32_t j = __ldg(idx + r0 + threadIdx.x);
+    const bool ok = j >= 0 && j < d;
+    if (!ok) record_error(err, kDevErrBadIndex);
+    src_row[threadIdx.x] = ok ? j : -1;
   }
-  const uint4* src = Bq + static_cast<int64_t>(j) * ldb_vec;
-  if (threadIdx.x < tail_bytes)
-    dst_tail[threadIdx.x] =
-        __float2bfloat16_rn(static_cast<float>(reinterpret_cast<const int8_t*>(src + vecs)[threadIdx.x]));
-  auto put = [&](int64_t v, const uint4& q) {
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    uint32_t o[8];
+  __syncthreads();
+  constexpr int OUT = kW8 ? 2 : 1;  // 16-byte output vectors per source vector
+  auto put = [&](int64_t r, int64_t v, const uint4& q) {
+    uint4* dst = BI + (r0 + r) * ldbi_vec + OUT * v;
+    if constexpr (kW8) {
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      uint32_t o[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float f[4];
-      i8x4_to_f32(w[e], f);
-      o[2 * e] = pack_bf16x2(f[0], f[1]);
-      o[2 * e + 1] = pack_bf16x2(f[2], f[3]);
+      for (int e = 0; e < 4; ++e) {
+        float f[4];
+        i8x4_to_f32(w[e], f);
+        o[2 * e] = pack_bf16x2(f[0], f[1]);
+        o[2 * e + 1] = pack_bf16x2(f[2], f[3]);
+      }
+      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    } else {
+      dst[0] = q;
     }
-    dst[2 * v] = make_uint4(o[0], o[1], o[2], o[3]);
-    dst[2 * v + 1] = make_uint4(o[4], o[5], o[6], o[7]);
   };
-  int64_t v = threadIdx.x;
-  for (; v + 3 * kGatherThreads < vecs; v += 4 * kGatherThreads) {
-    const uint4 a0 = __ldcs(src + v);
-    const uint4 a1 = __ldcs(src + v + kGatherThreads);
-    const uint4 a2 = __ldcs(src + v + 2 * kGatherThreads);
-    const uint4 a3 = __ldcs(src + v + 3 * kGatherThreads);
-    put(v, a0);
-    put(v + kGatherThreads, a1);
-    put(v + 2 * kGatherThreads, a2);
-    put(v + 3 * kGatherThreads, a3);
+  const int64_t items = static_cast<int64_t>(nr) * vecs;
+  for (int64_t it = threadIdx.x; it < items; it += 4 * kGatherThreads) {
+    uint4 a[4];
+    int64_t rr[4], vv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = it + u * kGatherThreads;
+      rr[u] = i / vecs;
+      vv[u] = i - rr[u] * vecs;
+      const int32_t j = i < items ? src_row[rr[u]] : -1;
+      a[u] = j >= 0 ? __ldcs(B + static_cast<int64_t>(j) * ldb_vec + vv[u]) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (it + u * kGatherThreads < items) put(rr[u], vv[u], a[u]);
   }
-  for (; v < vecs; v += kGatherThreads) put(v, __ldcs(src + v));
+  // elements past the last whole 16-byte vector of each row
+  for (int e = threadIdx.x; e < nr * tail_elems; e += kGatherThreads) {
+    const int r = static_cast<int>(e / tail_elems), t = static_cast<int>(e % tail_elems);
+    const int32_t j = src_row[r];
+    if constexpr (kW8) {
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(BI + (r0 + r) * ldbi_vec + 2 * vecs);
+      dst[t] = __float2bfloat16_rn(
+          j >= 0 ? static_cast<float>(reinterpret_cast<const int8_t*>(B + static_cast<int64_t>(j) * ldb_vec + vecs)[t])
+                 : 0.f);
+    } else {
+      uint16_t* dst = reinterpret_cast<uint16_t*>(BI + (r0 + r) * ldbi_vec + vecs);
+      dst[t] = j >= 0 ? reinterpret_cast<const uint16_t*>(B + static_cast<int64_t>(j) * ldb_vec + vecs)[t]
+                      : static_cast<uint16_t>(0);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_i8_kernel(const uint4* __restrict__ Bq, int64_t d,
@@ -271,26 +275,26 @@ __global__ void __launch_bounds__(kGatherThreads) gather_rows_i8_kernel(const ui
                                                                           int64_t ldb_vec,
                                                                           const int32_t* __restrict__ idx, int64_t k,
                                                                           uint4* __restrict__ BI, int64_t ldbi_vec,
-                                                                          unsigned* err) {
+                                                                          int rpb, unsigned* err) {
   pdl_wait();
   pdl_trigger();
-  gather_row_block_i8(blockIdx.x, Bq, d, vecs, tail_bytes, ldb_vec, idx, k, BI, ldbi_vec, err);
+  gather_rows_block<true>(blockIdx.x, rpb, Bq, d, vecs, tail_bytes, ldb_vec, idx, k, BI, ldbi_vec, err);
 }
 
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(const uint4* __restrict__ B, int64_t d,
                                                                        int64_t vecs, int64_t tail_halves,
                                                                        int64_t ldb_vec, const int32_t* __restrict__ idx,
                                                                        int64_t k, uint4* __restrict__ BI,
-                                                                       int64_t ldbi_vec, unsigned* err) {
+                                                                       int64_t ldbi_vec, int rpb, unsigned* err) {
   pdl_wait();
   pdl_trigger();
-  gather_row_block(blockIdx.x, B, d, vecs, tail_halves, ldb_vec, idx, k, BI, ldbi_vec, err);
+  gather_rows_block<false>(blockIdx.x, rpb, B, d, vecs, tail_halves, ldb_vec, idx, k, BI, ldbi_vec, err);
 }
 
-// Both reduced operands in one grid: blocks [0, k) gather the kept rows of B,
-// the remaining blocks compact the kept columns of A (bf16; staged R rows per
-// block, or the direct gather of 8 rows x 2048 columns), so the two HBM
-// streams overlap.
+// Both reduced operands in one grid: blocks [0, kb) gather the kept rows of B
+// (rpb rows each), the remaining blocks compact the kept columns of A (bf16;
+// staged R rows per block, or the direct gather of 8 rows x 2048 columns), so
+// the two HBM streams overlap.
 // kW8: B is int8 (vecs counts 16-value vectors, tail_elems trailing bytes)
 // and B_I is written as bf16; otherwise B is bf16 (tail_elems trailing halves).
 template <bool kStagedA, bool kW8>
@@ -298,22 +302,19 @@ __global__ void __launch_bounds__(kGatherThreads) compact_gather_kernel(
     const uint4* __restrict__ B, int64_t d, int64_t vecs, int64_t tail_elems, int64_t ldb_vec,
     uint4* __restrict__ BI, int64_t ldbi_vec, const uint16_t* __restrict__ A, int64_t M, int64_t lda,
     uint16_t* __restrict__ AI, int64_t ld_ai, int64_t chunks, int R, bool vec_ok, const int32_t* __restrict__ idx,
-    int64_t k, unsigned* err, uint32_t* zero, int64_t n_zero) {
+    int64_t k, int rpb, int64_t kb, unsigned* err, uint32_t* zero, int64_t n_zero) {
   extern __shared__ __align__(128) uint8_t stage[];
   pdl_wait();
   pdl_trigger();
   const int64_t blk = blockIdx.x;
   if (blk == 0)
     for (int64_t i = threadIdx.x; i < n_zero; i += kGatherThreads) zero[i] = 0u;
-  if (blk < k) {
-    if constexpr (kW8)
-      gather_row_block_i8(blk, B, d, vecs, tail_elems, ldb_vec, idx, k, BI, ldbi_vec, err);
-    else
-      gather_row_block(blk, B, d, vecs, tail_elems, ldb_vec, idx, k, BI, ldbi_vec, err);
+  if (blk < kb) {
+    gather_rows_block<kW8>(blk, rpb, B, d, vecs, tail_elems, ldb_vec, idx, k, BI, ldbi_vec, err);
   } else if constexpr (kStagedA) {
-    compact_rows_block(blk - k, A, M, d, lda, idx, k, AI, ld_ai, R, err, stage);
+    compact_rows_block(blk - kb, A, M, d, lda, idx, k, AI, ld_ai, R, err, stage);
   } else {
-    compact_block<__nv_bfloat16>(blk - k, reinterpret_cast<const __nv_bfloat16*>(A), M, d, lda, idx, k,
+    compact_block<__nv_bfloat16>(blk - kb, reinterpret_cast<const __nv_bfloat16*>(A), M, d, lda, idx, k,
                                  reinterpret_cast<__nv_bfloat16*>(AI), ld_ai, chunks, vec_ok, err);
   }
 }
@@ -324,7 +325,11 @@ __global__ void __launch_bounds__(kGatherThreads) compact_gather_kernel(
 int staged_rows(const void* A, int64_t d, int64_t lda) {
   if (reinterpret_cast<uintptr_t>(A) % 16 || lda % 8 || d % 8) return 0;
   const int64_t row_bytes = 2 * d;
-  if (row_bytes > kMaxStagedRowBytes) return 0;
+  // rows wider than the staging target (one row per block, an index round
+  // trip exposed per 2048-column chunk) measured slower than the direct
+  // gather: 172 vs 133 us for 2048 x 28672 at rho = 0.8; up to 32 KB (one
+  // row of 14336 columns) staging was the faster, 50 vs 57 us
+  if (row_bytes > kMaxStagedRowBytes || row_bytes > kStageTargetBytes) return 0;
   const int64_t r = kStageTargetBytes / row_bytes;
   return static_cast<int>(r < 1 ? 1 : (r > 8 ? 8 : r));
 }
@@ -349,10 +354,12 @@ bool allow_staged_smem() {
 cudaError_t launch_gather_rows(const void* B, int64_t d, int64_t row_bytes, int64_t ldb_bytes, const int32_t* idx,
                                int64_t k, void* B_I, int64_t ldbi_bytes, unsigned* err, cudaStream_t stream) {
   if (k == 0 || row_bytes == 0) return cudaSuccess;
-  if (k > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  return launch_pdl(gather_rows_kernel, dim3(static_cast<unsigned>(k)), dim3(kGatherThreads), 0, stream,
+  const int rpb = gather_rows_per_block(row_bytes / 16);
+  const int64_t blocks = (k + rpb - 1) / rpb;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  return launch_pdl(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kGatherThreads), 0, stream,
                     static_cast<const uint4*>(B), d, row_bytes / 16, (row_bytes % 16) / 2, ldb_bytes / 16, idx, k,
-                    static_cast<uint4*>(B_I), ldbi_bytes / 16, err);
+                    static_cast<uint4*>(B_I), ldbi_bytes / 16, rpb, err);
 }
 
 cudaError_t launch_compact(const void* A, int dtype, int64_t M, int64_t d, int64_t lda, const int32_t* idx,
@@ -389,12 +396,14 @@ cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64
   const int R = M > 0 ? staged_rows(A, d, lda) : 0;
   const int64_t chunks = (k + kColsPerCta - 1) / kColsPerCta;
   const int64_t cblocks = M <= 0 ? 0 : (R > 0 ? (M + R - 1) / R : ((M + kRowsPerCta - 1) / kRowsPerCta) * chunks);
-  const int64_t blocks = k + cblocks;
-  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  const bool vec_ok = reinterpret_cast<uintptr_t>(A_I) % 16 == 0 && (ld_ai * 2) % 16 == 0;
   const int64_t belt = b_int8 ? 1 : 2;
   const int64_t row_bytes = N * belt;
   const int64_t vecs = row_bytes / 16, tail = (row_bytes % 16) / belt;
+  const int rpb = gather_rows_per_block(vecs);
+  const int64_t kb = (k + rpb - 1) / rpb;
+  const int64_t blocks = kb + cblocks;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  const bool vec_ok = reinterpret_cast<uintptr_t>(A_I) % 16 == 0 && (ld_ai * 2) % 16 == 0;
   const int64_t ldb_vec = ldb * belt / 16, ldbi_vec = ld_bi * 2 / 16;
   const dim3 grid(static_cast<unsigned>(blocks)), block(kGatherThreads);
   const uint4* b = static_cast<const uint4*>(B);
@@ -403,7 +412,7 @@ cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64
   uint16_t* ai = static_cast<uint16_t*>(A_I);
   auto go = [&](auto kernel, size_t smem, int r) {
     return launch_pdl(kernel, grid, block, smem, stream, b, d, vecs, tail, ldb_vec, bi, ldbi_vec, a, M, lda, ai, ld_ai,
-                      chunks, r, vec_ok, idx, k, err, zero, n_zero);
+                      chunks, r, vec_ok, idx, k, rpb, kb, err, zero, n_zero);
   };
   if (R > 0) {
     const size_t smem = static_cast<size_t>(R) * 2 * d;
@@ -421,10 +430,12 @@ cudaError_t launch_compact_and_gather(const void* A, int64_t M, int64_t d, int64
 cudaError_t launch_gather_rows_i8(const void* Bq, int64_t d, int64_t N, int64_t ldb, const int32_t* idx, int64_t k,
                                   void* B_I, int64_t ld_bi, unsigned* err, cudaStream_t stream) {
   if (k == 0 || N == 0) return cudaSuccess;
-  if (k > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
-  return launch_pdl(gather_rows_i8_kernel, dim3(static_cast<unsigned>(k)), dim3(kGatherThreads), 0, stream,
+  const int rpb = gather_rows_per_block(N / 16);
+  const int64_t blocks = (k + rpb - 1) / rpb;
+  if (blocks > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  return launch_pdl(gather_rows_i8_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kGatherThreads), 0, stream,
                     static_cast<const uint4*>(Bq), d, N / 16, N % 16, ldb / 16, idx, k, static_cast<uint4*>(B_I),
-                    ld_bi * 2 / 16, err);
+                    ld_bi * 2 / 16, rpb, err);
 }
 
 }  // namespace rmm

@@ -37,6 +37,7 @@
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
 #include "rmm_launch.cuh"
+#include "rmm_select.cuh"
 
 namespace rmm {
 namespace {
@@ -78,16 +79,41 @@ size_t stream_smem_bytes(int rows_per_split) {
   return std::max(stream_ring_bytes<kW8>() + stage_ai, red);
 }
 
+// The selection done inside the product (kSel): the activation rows X
+// [M x d] bf16 (base and rows 16-byte aligned, d a multiple of 8), and the
+// outputs CTA (0, 0) writes for the caller.
+struct GemvSelect {
+  const uint16_t* X;
+  int64_t ldx;
+  int32_t* idx_out;  // the k kept indices, ascending
+  float* ss_out;     // the d column scores (may be null)
+};
+
+// Largest d the fused selection stages: its keys and bins use the ring.
+template <bool kW8>
+constexpr int64_t stream_select_max_d() {
+  return static_cast<int64_t>(stream_ring_bytes<kW8>()) / 4 - kSelectBins;
+}
+
 // grid: x = column slice of 256, y = row split.  Warp w takes the split's
 // kept rows w, w + 8, w + 16, ..., four per stage, and keeps six stages of
 // 16-byte asynchronous copies in flight (no registers held, no copy engine
 // requests); a row whose index is out of range is copied as zeros.
-template <int MT, bool kW8>
+//
+// kSel: no selection launch before this one.  Every CTA computes the column
+// scores of X (fp32 sums of the rows' exact squares, in row order: the same
+// arithmetic as the selection kernel) into keys staged where its ring will
+// be, runs the exact top-k search on them, and keeps the kept indices of its
+// own rank range [r0, r0 + rows) straight in shared memory; CTA (0, 0) also
+// writes the whole ascending index list and the scores.  A_I is read from X.
+// The redundant selections run concurrently on every SM, so the product
+// streams after a few microseconds instead of after a separate launch.
+template <int MT, bool kW8, bool kSel>
 __global__ void __launch_bounds__(kStreamThreads, 2)
     gemv_stream_kernel(const uint16_t* __restrict__ AI, int64_t ld_ai, const void* __restrict__ Bv, int64_t ldb,
                        const float* __restrict__ b_scale, const int32_t* __restrict__ idx, int M, int64_t d,
                        int64_t N, int64_t k, int rows_per_split, float* __restrict__ partial, void* __restrict__ Y,
-                       int out_f32, int64_t ldy, int clustered, unsigned* err) {
+                       int out_f32, int64_t ldy, int clustered, unsigned* err, GemvSelect sel) {
   constexpr int ELT = kW8 ? 1 : 2;
   constexpr int ROWB = stream_row_bytes<kW8>();
   constexpr int CPL = kStreamCols / 32;  // 8 columns per lane
@@ -102,22 +128,6 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
   const int ncols = static_cast<int>(N - c0 < COLS ? N - c0 : COLS);
   float* sa = reinterpret_cast<float*>(smem + stream_ring_bytes<kW8>());  // A_I [row][MT]
   int32_t* sidx = reinterpret_cast<int32_t*>(sa + static_cast<size_t>(rows_per_split) * MT);
-  pdl_wait();
-  pdl_trigger();
-  for (int m = 0; m < MT; ++m)
-    for (int rr = threadIdx.x; rr < nrows; rr += kStreamThreads)
-      sa[rr * MT + m] =
-          m < M ? __uint_as_float(static_cast<uint32_t>(AI[static_cast<int64_t>(m) * ld_ai + r0 + rr]) << 16) : 0.f;
-  bool bad = false;
-  for (int rr = threadIdx.x; rr < nrows; rr += kStreamThreads) {
-    const int32_t j = __ldg(idx + r0 + rr);
-    const bool ok = j >= 0 && j < d;
-    bad |= !ok;
-    sidx[rr] = ok ? j : -1;
-  }
-  if (bad) record_error(err, kDevErrBadIndex);
-  __syncthreads();
-
   // this lane's 16-byte piece of a row slice: bf16, piece = lane (its own 8
   // columns); int8, 16 lanes per row, two rows per instruction
   const char* B8 = static_cast<const char*>(Bv);
@@ -156,14 +166,78 @@ __global__ void __launch_bounds__(kStreamThreads, 2)
     cp_async_commit();  // one group per stage, empty past the end, so the wait count stays fixed
   };
 
+  pdl_wait();
+  pdl_trigger();
+  if constexpr (kSel) {
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem);                       // d words, in the ring
+    uint32_t* hist = keys + (static_cast<int>(d) + 3) / 4 * 4;                 // kSelectBins words
+    const bool first = blockIdx.x == 0 && blockIdx.y == 0;
+    const int dv = static_cast<int>(d / 8);
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int v = threadIdx.x; v < dv; v += kStreamThreads) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int m = 0; m < M; ++m) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(sel.X + static_cast<int64_t>(m) * sel.ldx) + v);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float lo = bf16_lo(w[t]), hi = bf16_hi(w[t]);
+          acc[2 * t] = fmaf(lo, lo, acc[2 * t]);
+          acc[2 * t + 1] = fmaf(hi, hi, acc[2 * t + 1]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t key = score_key(acc[e]);
+        keys[8 * v + e] = key;
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+        if (first && sel.ss_out) sel.ss_out[8 * v + e] = acc[e];
+      }
+    }
+    const uint32_t lo_rank = static_cast<uint32_t>(r0), hi_rank = static_cast<uint32_t>(r0 + nrows);
+    select_staged_keys<kStreamThreads>(keys, static_cast<int>(d), static_cast<uint32_t>(k), kmin, kmax, hist,
+                                       [&](uint32_t pos, int j) {
+                                         if (pos >= lo_rank && pos < hi_rank) sidx[pos - lo_rank] = j;
+                                         if (first) sel.idx_out[pos] = j;
+                                       });
+    __syncthreads();  // sidx is complete and the ring's keys and bins are no longer read
+    // the first stages' copies go out before A_I is gathered from X, so the
+    // two latencies overlap
+#pragma unroll
+    for (int st = 0; st < S - 1; ++st) issue(st);
+    for (int m = 0; m < MT; ++m)
+      for (int rr = threadIdx.x; rr < nrows; rr += kStreamThreads)
+        sa[rr * MT + m] =
+            m < M ? __uint_as_float(static_cast<uint32_t>(sel.X[static_cast<int64_t>(m) * sel.ldx + sidx[rr]]) << 16)
+                  : 0.f;
+    __syncthreads();
+  } else {
+    for (int m = 0; m < MT; ++m)
+      for (int rr = threadIdx.x; rr < nrows; rr += kStreamThreads)
+        sa[rr * MT + m] =
+            m < M ? __uint_as_float(static_cast<uint32_t>(AI[static_cast<int64_t>(m) * ld_ai + r0 + rr]) << 16) : 0.f;
+    bool bad = false;
+    for (int rr = threadIdx.x; rr < nrows; rr += kStreamThreads) {
+      const int32_t j = __ldg(idx + r0 + rr);
+      const bool ok = j >= 0 && j < d;
+      bad |= !ok;
+      sidx[rr] = ok ? j : -1;
+    }
+    if (bad) record_error(err, kDevErrBadIndex);
+    __syncthreads();
+  }
+
   float acc[MT][CPL];
 #pragma unroll
   for (int m = 0; m < MT; ++m)
 #pragma unroll
     for (int c = 0; c < CPL; ++c) acc[m][c] = 0.f;
 
+  if constexpr (!kSel) {
 #pragma unroll
-  for (int st = 0; st < S - 1; ++st) issue(st);
+    for (int st = 0; st < S - 1; ++st) issue(st);
+  }
   for (int st = 0; st < nst; ++st) {
     issue(st + S - 1);
     cp_async_wait<S - 1>();  // stage st has landed (this lane's copies)
@@ -308,13 +382,20 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// grid: x = column slice of 256, y = row split; M <= 16 (rows past M are zero).
+// Largest d the fused selection of the tensor-core kernel stages (its ring).
 template <bool kW8>
+constexpr int64_t mma_select_max_d() {
+  return static_cast<int64_t>(mma_stages<kW8>()) * kMmaRowsPerStage * mma_stage_pitch<kW8>() / 4 - kSelectBins;
+}
+
+// grid: x = column slice of 256, y = row split; M <= 16 (rows past M are zero).
+// kSel: the selection inside the product, as in the streaming kernel.
+template <bool kW8, bool kSel>
 __global__ void __launch_bounds__(kMmaThreads, 2)
     gemv_mma_kernel(const uint16_t* __restrict__ AI, int64_t ld_ai, const void* __restrict__ Bv, int64_t ldb,
                     const float* __restrict__ b_scale, const int32_t* __restrict__ idx, int M, int64_t d, int64_t N,
                     int64_t k, int rows_per_split, float* __restrict__ partial, void* __restrict__ Y, int out_f32,
-                    int64_t ldy, int clustered, unsigned* err) {
+                    int64_t ldy, int clustered, unsigned* err, GemvSelect sel) {
   constexpr int ELT = kW8 ? 1 : 2;
   constexpr int PITCH = mma_stage_pitch<kW8>();
   constexpr int RPS = kMmaRowsPerStage;
@@ -334,31 +415,6 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
   uint8_t* wide = smem + ring_bytes;
   uint8_t* sai = smem + std::max(ring_bytes + wide_bytes, static_cast<size_t>(16) * COLS * 4);
   int32_t* sidx = reinterpret_cast<int32_t*>(sai + static_cast<size_t>(16) * ai_pitch);
-  pdl_wait();
-  pdl_trigger();
-
-  // A_I rows (zero past M and past the split's rows) and the kept indices
-  // (-1 for an index outside [0, d) and past the split's rows)
-  for (int e = threadIdx.x; e < 16 * rows16; e += kMmaThreads) {
-    const int m = e / rows16, r = e % rows16;
-    const uint16_t v = (m < M && r < nrows) ? AI[static_cast<int64_t>(m) * ld_ai + r0 + r] : uint16_t{0};
-    *reinterpret_cast<uint16_t*>(sai + m * ai_pitch + r * 2) = v;
-  }
-  bool bad = false;
-  for (int r = threadIdx.x; r < rows16; r += kMmaThreads) {
-    int32_t j = -1;
-    if (r < nrows) {
-      j = __ldg(idx + r0 + r);
-      if (j < 0 || j >= d) {
-        bad = true;
-        j = -1;
-      }
-    }
-    sidx[r] = j;
-  }
-  if (bad) record_error(err, kDevErrBadIndex);
-  __syncthreads();
-
   const char* B8 = static_cast<const char*>(Bv);
   const int nst = (nrows + RPS - 1) / RPS;
   const uint32_t ring = smem_u32(smem);
@@ -378,6 +434,78 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
     cp_async_commit();
   };
 
+  pdl_wait();
+  pdl_trigger();
+
+  if constexpr (kSel) {
+    // scores of X, the exact top-k, and this split's kept indices (ranks
+    // [r0, r0 + nrows)), with keys and bins where the ring will be
+    uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
+    uint32_t* hist = keys + (static_cast<int>(d) + 3) / 4 * 4;
+    const bool first = blockIdx.x == 0 && blockIdx.y == 0;
+    for (int r = nrows + threadIdx.x; r < rows16; r += kMmaThreads) sidx[r] = -1;
+    const int dv = static_cast<int>(d / 8);
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int v = threadIdx.x; v < dv; v += kMmaThreads) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int m = 0; m < M; ++m) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(sel.X + static_cast<int64_t>(m) * sel.ldx) + v);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float lo = bf16_lo(w[t]), hi = bf16_hi(w[t]);
+          acc[2 * t] = fmaf(lo, lo, acc[2 * t]);
+          acc[2 * t + 1] = fmaf(hi, hi, acc[2 * t + 1]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t key = score_key(acc[e]);
+        keys[8 * v + e] = key;
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+        if (first && sel.ss_out) sel.ss_out[8 * v + e] = acc[e];
+      }
+    }
+    const uint32_t lo_rank = static_cast<uint32_t>(r0), hi_rank = static_cast<uint32_t>(r0 + nrows);
+    select_staged_keys<kMmaThreads>(keys, static_cast<int>(d), static_cast<uint32_t>(k), kmin, kmax, hist,
+                                    [&](uint32_t pos, int j) {
+                                      if (pos >= lo_rank && pos < hi_rank) sidx[pos - lo_rank] = j;
+                                      if (first) sel.idx_out[pos] = j;
+                                    });
+    __syncthreads();  // sidx complete; keys and bins no longer read
+    // the first stages' copies go out before A_I is gathered from X
+#pragma unroll
+    for (int st = 0; st < S - 1; ++st) issue(st);
+    for (int e = threadIdx.x; e < 16 * rows16; e += kMmaThreads) {
+      const int m = e / rows16, r = e % rows16;
+      const uint16_t v = (m < M && r < nrows) ? sel.X[static_cast<int64_t>(m) * sel.ldx + sidx[r]] : uint16_t{0};
+      *reinterpret_cast<uint16_t*>(sai + m * ai_pitch + r * 2) = v;
+    }
+  } else {
+    // A_I rows (zero past M and past the split's rows) and the kept indices
+    // (-1 for an index outside [0, d) and past the split's rows)
+    for (int e = threadIdx.x; e < 16 * rows16; e += kMmaThreads) {
+      const int m = e / rows16, r = e % rows16;
+      const uint16_t v = (m < M && r < nrows) ? AI[static_cast<int64_t>(m) * ld_ai + r0 + r] : uint16_t{0};
+      *reinterpret_cast<uint16_t*>(sai + m * ai_pitch + r * 2) = v;
+    }
+    bool bad = false;
+    for (int r = threadIdx.x; r < rows16; r += kMmaThreads) {
+      int32_t j = -1;
+      if (r < nrows) {
+        j = __ldg(idx + r0 + r);
+        if (j < 0 || j >= d) {
+          bad = true;
+          j = -1;
+        }
+      }
+      sidx[r] = j;
+    }
+    if (bad) record_error(err, kDevErrBadIndex);
+  }
+  __syncthreads();
+
   float acc[4][4];
 #pragma unroll
   for (int t = 0; t < 4; ++t)
@@ -385,8 +513,10 @@ __global__ void __launch_bounds__(kMmaThreads, 2)
     for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
   const uint32_t ai_base = smem_u32(sai);
   const uint32_t wide_base = smem_u32(wide);
+  if constexpr (!kSel) {
 #pragma unroll
-  for (int st = 0; st < S - 1; ++st) issue(st);
+    for (int st = 0; st < S - 1; ++st) issue(st);
+  }
   for (int st = 0; st < nst; ++st) {
     issue(st + S - 1);
     cp_async_wait<S - 1>();
@@ -519,16 +649,17 @@ GemvPlan plan_mt(int64_t M, int64_t N, int64_t k, int sms) {
   return p;
 }
 
-template <int MT, bool kW8>
+template <int MT, bool kW8, bool kSel = false>
 cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const void* B, int64_t ldb, const float* b_scale,
                            const int32_t* idx, int M, int64_t d, int64_t N, int64_t k, const GemvPlan& pl,
-                           float* partial, void* Y, int out_f32, int64_t ldy, unsigned* err, cudaStream_t stream) {
+                           float* partial, void* Y, int out_f32, int64_t ldy, unsigned* err, cudaStream_t stream,
+                           GemvSelect sel = GemvSelect{}) {
   constexpr bool kStream = MT <= 4;
   auto kernel = [] {
     if constexpr (kStream)
-      return gemv_stream_kernel<MT, kW8>;
+      return gemv_stream_kernel<MT, kW8, kSel>;
     else
-      return gemv_mma_kernel<kW8>;
+      return gemv_mma_kernel<kW8, kSel>;
   }();
   const int threads = kStream ? kStreamThreads : kMmaThreads;
   const size_t smem = kStream ? stream_smem_bytes<MT, kW8>(pl.rows_per_split) : mma_smem_bytes<kW8>(pl.rows_per_split);
@@ -564,11 +695,11 @@ cudaError_t launch_gemv_mt(const uint16_t* AI, int64_t ld_ai, const void* B, int
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kernel, AI, ld_ai, B, ldb, b_scale, idx, M, d, N, k, pl.rows_per_split, partial, Y,
-                           out_f32, ldy, 1, err);
+                           out_f32, ldy, 1, err, sel);
     return e;
   }
   e = launch_pdl(kernel, grid, dim3(threads), smem, stream, AI, ld_ai, B, ldb, b_scale, idx, M, d, N, k,
-                 pl.rows_per_split, partial, Y, out_f32, ldy, 0, err);
+                 pl.rows_per_split, partial, Y, out_f32, ldy, 0, err, sel);
   if (e != cudaSuccess || pl.splits == 1) return e;
   const int64_t outs = static_cast<int64_t>(M) * N;
   return launch_pdl(gemv_reduce_kernel, dim3(static_cast<unsigned>((outs + 255) / 256)), dim3(256), 0, stream,
@@ -599,6 +730,36 @@ cudaError_t launch_gemv(const void* A_I, int64_t ld_ai, const void* B, int64_t l
                                       stream);
     return launch_gemv_mt<MT, false>(ai, ld_ai, B, ldb, nullptr, idx, m, d, N, k, pl, partial, Y, out_f32, ldy, err,
                                      stream);
+  };
+  if (M <= 1) return go(std::integral_constant<int, 1>{});
+  if (M <= 2) return go(std::integral_constant<int, 2>{});
+  if (M <= 4) return go(std::integral_constant<int, 4>{});
+  if (M <= 8) return go(std::integral_constant<int, 8>{});
+  return go(std::integral_constant<int, 16>{});
+}
+
+bool gemv_select_supported(const void* X, int64_t M, int64_t d, int64_t ldx, bool b_int8) {
+  const int64_t max_d = M <= 4 ? (b_int8 ? stream_select_max_d<true>() : stream_select_max_d<false>())
+                               : (b_int8 ? mma_select_max_d<true>() : mma_select_max_d<false>());
+  return M >= 1 && M <= 16 && d >= 8 && d % 8 == 0 && d <= max_d && ldx % 8 == 0 &&
+         reinterpret_cast<uintptr_t>(X) % 16 == 0;
+}
+
+cudaError_t launch_gemv_select(const void* X, int64_t ldx, int64_t M, int64_t d, const void* B, int64_t ldb,
+                               const float* b_scale, int64_t N, int64_t k, const GemvPlan& pl, float* partial,
+                               void* Y, int out_dtype, int64_t ldy, int32_t* idx_out, float* ss_out, unsigned* err,
+                               cudaStream_t stream) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  const GemvSelect sel{static_cast<const uint16_t*>(X), ldx, idx_out, ss_out};
+  const int out_f32 = out_dtype == 0 ? 1 : 0;
+  const int m = static_cast<int>(M);
+  auto go = [&](auto mt) {
+    constexpr int MT = decltype(mt)::value;
+    if (b_scale)
+      return launch_gemv_mt<MT, true, true>(nullptr, 0, B, ldb, b_scale, nullptr, m, d, N, k, pl, partial, Y, out_f32,
+                                            ldy, err, stream, sel);
+    return launch_gemv_mt<MT, false, true>(nullptr, 0, B, ldb, nullptr, nullptr, m, d, N, k, pl, partial, Y, out_f32,
+                                           ldy, err, stream, sel);
   };
   if (M <= 1) return go(std::integral_constant<int, 1>{});
   if (M <= 2) return go(std::integral_constant<int, 2>{});

@@ -139,6 +139,15 @@ GemvPlan gemv_plan(int64_t M, int64_t N, int64_t k, int sms);
 cudaError_t launch_gemv(const void* A_I, int64_t ld_ai, const void* B, int64_t ldb, const int32_t* idx, int64_t M,
                         int64_t d, int64_t N, int64_t k, const GemvPlan& plan, float* partial, void* Y, int out_dtype,
                         int64_t ldy, unsigned* err, cudaStream_t stream, const float* b_scale = nullptr);
+// The same product with the selection inside it (M <= 16): every CTA scores
+// X [M x d] bf16 (16-byte aligned rows, d a multiple of 8), selects the k
+// kept indices and streams its share of their rows of B; idx_out receives the
+// ascending index list and ss_out (may be null) the scores.
+bool gemv_select_supported(const void* X, int64_t M, int64_t d, int64_t ldx, bool b_int8);
+cudaError_t launch_gemv_select(const void* X, int64_t ldx, int64_t M, int64_t d, const void* B, int64_t ldb,
+                               const float* b_scale, int64_t N, int64_t k, const GemvPlan& plan, float* partial,
+                               void* Y, int out_dtype, int64_t ldy, int32_t* idx_out, float* ss_out, unsigned* err,
+                               cudaStream_t stream);
 
 // ---- reduced attention (rmm_attention.cu)
 size_t attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t S, int64_t D, int64_t kd,

@@ -383,6 +383,42 @@ def test_path_decode_rows(M):
     no_device_error()
 
 
+@pytest.mark.parametrize("M,d,N,rho,ties", [(2, 1000, 777, 0.37, False), (3, 22528, 512, 0.9, False),
+                                             (1, 64, 8, 1.0, False), (4, 4096, 1000, 0.5, True),
+                                             (1, 2048, 4104, 0.25, True), (8, 4096, 2048, 0.5, False),
+                                             (13, 1024, 296, 0.6, True), (16, 19072, 512, 0.5, False)])
+def test_path_decode_fused_selection(M, d, N, rho, ties):
+    """Up to 16 rows with d a multiple of 8 run the product whose CTAs each make
+    the selection themselves: the index list, the scores and Y against the
+    oracle, including heavy ties (groups of equal columns: lowest index wins),
+    rho = 1 and ragged N."""
+    bits = W.llm_activation_bf16(300 + M + d, M, d)
+    if ties:
+        bits = bits.copy()
+        bits[:, 1::4] = bits[:, 0::4][:, : bits[:, 1::4].shape[1]]  # every 4th pair of columns equal
+        bits[:, 2::4] = bits[:, 0::4][:, : bits[:, 2::4].shape[1]]
+    k = oracle.k_from_rho(rho, d)
+    if not ties:
+        bits, _ = widen_topk_gaps(bits, "bf16", [k])
+    A = oracle.decode(bits, "bf16")
+    Wb = W.weight_bf16(6, d, N)
+    Bm = oracle.decode(Wb, "bf16")
+    idx_out = torch.full((k,), -1, dtype=torch.int32, device="cuda")
+    ss_out = torch.empty(d, dtype=torch.float32, device="cuda")
+    Y = R.rmm_matmul(bf16_tensor(bits), _pitched(bf16_tensor(Wb)), rho, idx_out=idx_out, ss_out=ss_out,
+                     out_dtype=torch.float32)
+    np.testing.assert_allclose(to_f64(ss_out), oracle.column_sq_norms(A), rtol=1e-5)
+    # with ties the set is defined on the scores as computed (equal columns
+    # give equal fp32 sums): the oracle's top-k of the GPU's own scores; else
+    # the oracle's scores, whose boundary gap was widened
+    idx = oracle.topk_indices(to_f64(ss_out) if ties else oracle.column_sq_norms(A), k)
+    np.testing.assert_array_equal(idx_out.cpu().numpy(), idx)
+    ref = A[:, idx] @ Bm[idx, :]
+    bound = k * 2.0 ** -24 * (np.abs(A[:, idx]) @ np.abs(Bm[idx, :])) + 1e-30
+    assert np.all(np.abs(to_f64(Y) - ref) <= bound)
+    no_device_error()
+
+
 def test_path_decode_unaligned_rows():
     """Few rows with a row pitch that is not a multiple of 8 (the fused
     selection's scalar path) and d not a multiple of 8."""
