@@ -45,6 +45,10 @@ constexpr int TILE = 128;                 // rows of every tile (queries or keys
 constexpr int CHUNK_BYTES = TILE * 128;   // one [128 x 64] bf16 tile, 128-byte rows: 16 KB
 constexpr int ATT_THREADS = 320;          // warp 0 TMA, warp 1 MMA, warps 2-9 softmax (two groups of four)
 constexpr int SOFTMAX_THREADS = 256;
+// pass C on SM pairs: warp 0 TMA, warp 1 issues the logit MMAs, warps 2-9
+// softmax (two groups of four), warp 10 issues the P V MMAs
+constexpr int PAIR_THREADS = 352;
+constexpr int PAIR_PV_WARP = 10;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // Pass C multiplies P by 2^kPScaleLog2 before rounding it to fp16: P <= 1, so
@@ -62,7 +66,6 @@ struct AttnParams {
   int out_f32;      // O written as fp32 (else bf16)
   int c_ks;         // pass C key ring depth (as shared memory allows)
   int c_vs;         // pass C value ring depth (as shared memory allows)
-  int c_ps;         // pass C on SM pairs: P buffers in shared memory (2 or 3)
   float scale_log2; // logit scale times log2(e)
 };
 
@@ -730,36 +733,50 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 //   - S = Q_I K_T^T: each CTA's A is its own 128 query rows, its B the 64
 //     keys [j*128 + rank*64, +64) of kept block j; each CTA's tensor memory
 //     gets its 128 rows x 128 keys;
-//   - P' (fp16) goes to each CTA's shared memory; O += P V_T: each CTA's B is
-//     its 64 of V's 128 columns, each CTA's tensor memory gets its rows of O;
+//   - P' (fp16) goes back into each CTA's tensor memory over the logits it
+//     came from (two per column); O += P V_T takes A = P' from both CTAs'
+//     tensor memory and B = each CTA's 64 of V's 128 columns, each CTA's
+//     tensor memory gets its rows of O.  (With P' in shared memory each
+//     CTA moved ~128 KB per kept block through shared memory, and back-to-back
+//     pair MMAs were accepted every ~147 cycles against ~68 alone: the P
+//     write and the P operand read were half of that traffic);
 //   - every load signals the leader's barriers; the leader's MMA lane waits
 //     on them, and its commits reach both CTAs (multicast); the softmax
 //     groups of both CTAs arrive on the leader's P barrier;
-//   - three logit buffers: after softmax(j) (both CTAs) the leader issues
-//     S(j+3) into buffer j % 3 (softmax(j) has read it) and then PV(j);
-//   - key stage j % 3 is free when S(j) is done and value stage j % c_ps
-//     when PV(j) is done, so the producers wait on the logit and P barriers
-//     (one commit each per kept block instead of two).
+//   - two issuing lanes in the leader: warp 1 issues the logit MMAs, warp 10
+//     the P V MMAs (one issuing thread spent ~120-150 cycles per M256 N128 K16
+//     pair MMA, about twice the tensor pipe's time for it, so a single issuer
+//     left the pipe idle two thirds of the time);
+//   - three logit / P' buffers: once both CTAs have written P'(j) the P V
+//     issuer issues PV(j); once PV(j) is done the logit issuer puts S(j+3)
+//     into buffer j % 3;
+//   - key stage j % 3 is free when S(j) is done and value stage j % 3 when
+//     PV(j) is done, so the producers wait on the logit and P V commits
+//     (one commit each per kept block).
 // Every wait is bounded; every path reaches the final cluster barrier.
 constexpr int CP_KS = C_SBUF;  // key ring depth = logit buffers (a key stage is freed with its logits)
-constexpr int CP_MAX_PS = 3;   // P buffers = value ring depth (a value stage is freed with its P)
+constexpr int CP_VS = C_SBUF;  // value ring depth = logit/P buffers (a value stage is freed with its P V)
 constexpr int CP_HALF_ROWS = TILE / 2;                 // keys of a kept block per CTA
 constexpr int CP_KCHUNK_BYTES = CP_HALF_ROWS * 128;    // [64 x 64] bf16, 128-byte rows: 8 KB
+// one CTA per SM: each holds all 512 tensor-memory columns, so a second one
+// would wait in tcgen05.alloc while its cluster partner holds another SM's
+constexpr int CP_MIN_SMEM = 116 * 1024;
 
 struct PairOutBars {
   uint64_t kfull[CP_KS];
-  uint64_t vfull[CP_MAX_PS];
+  uint64_t vfull[CP_VS];
   uint64_t qfull;
-  uint64_t sfull[C_SBUF];
-  uint64_t pfull[CP_MAX_PS], pempty[CP_MAX_PS];
+  uint64_t sfull[C_SBUF];   // multicast commit: S(t) is in buffer t % 3
+  uint64_t pfull[C_SBUF];   // leader: both CTAs' softmax groups wrote P'(t) over buffer t % 3
+  uint64_t pvdone[C_SBUF];  // multicast commit: PV(t) is done, so buffer t % 3 and value stage t % 3 are free
   uint64_t ofull;
-  uint64_t drain;
+  uint64_t drain, drain_pv;
   uint32_t tmem_slot;
   int abort_flag;
   int pos[8][TILE];
 };
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
     attn_out_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
                          const __grid_constant__ CUtensorMap tm_vt, const float* __restrict__ lse,
                          const int32_t* __restrict__ pos, const int* __restrict__ nvalid, void* __restrict__ O,
@@ -768,24 +785,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
   const uint32_t raw_s = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_s & 1023u)) & 1023u);
   const uint32_t base = smem_u32(smem);
-  constexpr int ks = CP_KS;
-  const int ps = p.c_ps, vs = ps;
+  constexpr int ks = CP_KS, vs = CP_VS;
   const int q_bytes = p.kc * CHUNK_BYTES;
   const int k_bytes = p.kc * CP_KCHUNK_BYTES;  // this CTA's half of a key block
   const int v_bytes = CHUNK_BYTES;             // this CTA's 64 columns of a value block
   const uint32_t q_tile = base;
   auto kst = [&](int s) { return base + q_bytes + s * k_bytes; };
   auto vst = [&](int s) { return base + q_bytes + ks * k_bytes + s * v_bytes; };
-  const uint32_t p_base = base + q_bytes + ks * k_bytes + vs * v_bytes;  // P buffers of 2 chunks
-  auto pbuf = [&](int b) { return p_base + b * 2 * CHUNK_BYTES; };
-  PairOutBars* bars =
-      reinterpret_cast<PairOutBars*>(smem + q_bytes + ks * k_bytes + vs * v_bytes + ps * 2 * CHUNK_BYTES);
+  PairOutBars* bars = reinterpret_cast<PairOutBars*>(smem + q_bytes + ks * k_bytes + vs * v_bytes);
   volatile int* abort_flag = &bars->abort_flag;
   auto kfull = [&](int s) { return smem_u32(&bars->kfull[s]); };
   auto vfull = [&](int s) { return smem_u32(&bars->vfull[s]); };
   auto sfull = [&](int b) { return smem_u32(&bars->sfull[b]); };
   auto pfull = [&](int b) { return smem_u32(&bars->pfull[b]); };
-  auto pempty = [&](int b) { return smem_u32(&bars->pempty[b]); };
+  auto pvdone = [&](int b) { return smem_u32(&bars->pvdone[b]); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -802,13 +815,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     for (int s = 0; s < ks; ++s) mbar_init(kfull(s), 1);  // leader: its producer's arrive + both CTAs' bytes
     for (int s = 0; s < vs; ++s) mbar_init(vfull(s), 1);
     mbar_init(smem_u32(&bars->qfull), 1);
-    for (int b = 0; b < C_SBUF; ++b) mbar_init(sfull(b), 1);  // multicast commit
-    for (int b = 0; b < ps; ++b) {
+    for (int b = 0; b < C_SBUF; ++b) {
+      mbar_init(sfull(b), 1);   // multicast commit
       mbar_init(pfull(b), 8);   // leader: four warps of a softmax group in each CTA
-      mbar_init(pempty(b), 1);  // multicast commit
+      mbar_init(pvdone(b), 1);  // multicast commit
     }
     mbar_init(smem_u32(&bars->ofull), 1);
     mbar_init(smem_u32(&bars->drain), 1);
+    mbar_init(smem_u32(&bars->drain_pv), 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -848,8 +862,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     } else if (lane == 1 && nrb > 0) {
       int n = 0;
       for (int t = 0; t < nrb; ++t) {
-        const int st = t % vs;  // freed by PV(t - c_ps): P buffer st
-        if (!mbar_wait(pempty(st), ((t / vs) & 1) ^ 1u, abort_flag, err, 32)) break;
+        const int st = t % vs;  // freed by PV(t - 3)
+        if (!mbar_wait(pvdone(st), ((t / vs) & 1) ^ 1u, abort_flag, err, 32)) break;
         const uint32_t vf = mapa_shared(vfull(st), 0);
         if (leader) mbar_arrive_expect_tx(vfull(st), 2 * v_bytes);
         tma_load_3d_pair(vst(st), &tm_vt, vf, static_cast<int>(rank) * 64, t * TILE, bh);
@@ -859,48 +873,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
+    // logit MMAs: S(t) into buffer t % 3 once PV(t - 3) has read P'(t - 3) there
     if (leader && lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(2 * TILE, TILE, false, false);
-      const uint32_t idesc_o = idesc_f16_f32(2 * TILE, p.D, false, true);
       bool ok = nrb == 0 || mbar_wait(smem_u32(&bars->qfull), 0, abort_flag, err, 33);
-      auto issue_s = [&](int t) -> bool {
-        const int st = t % ks;
-        if (!mbar_wait(kfull(st), (t / ks) & 1, abort_flag, err, 34)) return false;
+      for (int t = 0; ok && t < nrb; ++t) {
+        const int st = t % ks, b = t % C_SBUF;
+        if (t >= C_SBUF) ok = mbar_wait(pvdone(b), ((t - C_SBUF) / C_SBUF) & 1, abort_flag, err, 40);
+        ok = ok && mbar_wait(kfull(st), (t / ks) & 1, abort_flag, err, 34);
+        if (!ok) break;
         tc_fence_after();
         for (int c = 0; c < p.kc; ++c) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = sdesc_sw128(q_tile + c * CHUNK_BYTES + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(kst(st) + c * CP_KCHUNK_BYTES + kk * 32, 16, 1024);
-            mma_f16_ss_pair(buf_tmem(t % C_SBUF), ad, bd, idesc_s, (c | kk) != 0 ? 1u : 0u);
+            mma_f16_ss_pair(buf_tmem(b), ad, bd, idesc_s, (c | kk) != 0 ? 1u : 0u);
           }
         }
-        mma_commit_pair_multicast(sfull(t % C_SBUF), 0x3);
-        return true;
-      };
-      auto issue_pv = [&](int t) -> bool {
-        const int st = t % vs, pb = t % ps;
-        if (!mbar_wait(vfull(st), (t / vs) & 1, abort_flag, err, 35)) return false;
+        mma_commit_pair_multicast(sfull(b), 0x3);
+      }
+      mma_commit_pair_multicast(smem_u32(&bars->drain), 0x1);
+      wait_drain(smem_u32(&bars->drain), 0);
+    }
+    __syncwarp();
+  } else if (warp == PAIR_PV_WARP) {
+    // P V MMAs: PV(j) with P'(j) read from both CTAs' tensor memory (buffer
+    // j % 3) once both have written it and V(j) has landed
+    if (leader && lane == 0) {
+      const uint32_t idesc_o = idesc_f16_f32(2 * TILE, p.D, false, true);
+      bool ok = true;
+      for (int j = 0; ok && j < nrb; ++j) {
+        const int b = j % C_SBUF, st = j % vs;
+        ok = mbar_wait(pfull(b), (j / C_SBUF) & 1, abort_flag, err, 36) &&
+             mbar_wait(vfull(st), (j / vs) & 1, abort_flag, err, 35);
+        if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < TILE / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(pbuf(pb) + (kk / 4) * CHUNK_BYTES + (kk % 4) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(vst(st) + kk * 16 * 128, CHUNK_BYTES, 1024);
-          mma_f16_ss_pair(o_tmem, ad, bd, idesc_o, (t | kk) != 0 ? 1u : 0u);
+          mma_f16_ts_pair(o_tmem, buf_tmem(b) + kk * 8, bd, idesc_o, (j | kk) != 0 ? 1u : 0u);
         }
-        mma_commit_pair_multicast(pempty(pb), 0x3);
-        return true;
-      };
-      for (int t = 0; ok && t < C_SBUF && t < nrb; ++t) ok = issue_s(t);
-      for (int j = 0; ok && j < nrb; ++j) {
-        ok = mbar_wait(pfull(j % ps), (j / ps) & 1, abort_flag, err, 36);
-        if (ok) tc_fence_after();
-        if (ok && j + C_SBUF < nrb) ok = issue_s(j + C_SBUF);
-        ok = ok && issue_pv(j);
+        mma_commit_pair_multicast(pvdone(b), 0x3);
       }
       if (ok && nrb > 0) mma_commit_pair_multicast(smem_u32(&bars->ofull), 0x3);
-      mma_commit_pair_multicast(smem_u32(&bars->drain), 0x1);
-      wait_drain(smem_u32(&bars->drain), 0);
+      mma_commit_pair_multicast(smem_u32(&bars->drain_pv), 0x1);
+      wait_drain(smem_u32(&bars->drain_pv), 0);
     }
     __syncwarp();
   } else {
@@ -917,8 +935,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
     int* psh = bars->pos[warp - 2];
     bool ok = true;
     for (int rb = g; ok && rb < nrb; rb += 2) {
-      const int b = rb % C_SBUF, pb = rb % ps;
-      const uint32_t sph = (rb / C_SBUF) & 1, pph = (rb / ps) & 1;
+      const int b = rb % C_SBUF;
+      const uint32_t sph = (rb / C_SBUF) & 1;
       const bool masked = rb * TILE + TILE > nbefore;
       if (masked) {
         __syncwarp();
@@ -929,16 +947,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
         }
         __syncwarp();
       }
-      if (!mbar_wait_warp(sfull(b), sph, abort_flag, err, 37) ||
-          !mbar_wait_warp(pempty(pb), pph ^ 1u, abort_flag, err, 38)) {
+      if (!mbar_wait_warp(sfull(b), sph, abort_flag, err, 37)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      // P' goes over the logits of the same buffer, two fp16 per column: chunk
+      // cc's P' (16 columns from 16 cc) only covers logits already loaded
       const uint32_t s_addr = buf_tmem(b) + lane_off;
-      uint8_t* prow = smem + (pbuf(pb) - base) + r * 128;
-      auto emit = [&](int cc, const uint32_t (&v)[32]) {
-        uint32_t w[16];
+      const uint32_t p_addr = s_addr;
+      auto exps = [&](int cc, const uint32_t (&v)[32], uint32_t (&w)[16]) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           float x0, x1;
@@ -950,34 +968,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(ATT_THREADS, 1)
           }
           w[e] = pack_f16x2(p0, p1);
         }
-        uint8_t* crow = prow + (cc >> 1) * CHUNK_BYTES;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int piece = (cc & 1) * 4 + q;
-          *reinterpret_cast<uint4*>(crow + ((piece ^ (r & 7)) << 4)) =
-              make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-        }
       };
-      uint32_t va[32], vb[32];
-      __syncwarp();  // tensor-memory loads are warp-synchronous: reconverge first
+      uint32_t va[32], vb[32], w[16];
+      __syncwarp();  // tensor-memory accesses are warp-synchronous: reconverge first
       tmem_ld32(s_addr, va);
       tmem_wait_ld_into(va);
       tmem_ld32(s_addr + 32, vb);
-      emit(0, va);
+      exps(0, va, w);
+      tmem_st16(p_addr, w);
       tmem_wait_ld_into(vb);
       __syncwarp();
       tmem_ld32(s_addr + 64, va);
-      emit(1, vb);
+      exps(1, vb, w);
+      tmem_st16(p_addr + 16, w);
       tmem_wait_ld_into(va);
       __syncwarp();
       tmem_ld32(s_addr + 96, vb);
-      emit(2, va);
+      exps(2, va, w);
+      tmem_st16(p_addr + 32, w);
       tmem_wait_ld_into(vb);
-      emit(3, vb);
+      exps(3, vb, w);
+      tmem_st16(p_addr + 48, w);
+      tmem_wait_st();
       tc_fence_before();
-      fence_proxy_async_smem();  // P is read by the tensor core (async proxy)
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(mapa_shared(pfull(pb), 0));
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(pfull(b), 0));
     }
     // epilogue: O row i, columns [g D/2, (g+1) D/2)
     const bool have = ok && nrb > 0 && mbar_wait_warp(smem_u32(&bars->ofull), 0, abort_flag, err, 39);
@@ -1203,13 +1218,12 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
       (e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
     return e;
   if (D == 128) {
-    // key ring of 3 (one per logit buffer); value ring = P buffers, 3 when they fit
-    auto pair_smem_for = [&](int ps) {
-      return kc * CHUNK_BYTES + CP_KS * kc * CP_KCHUNK_BYTES + ps * CHUNK_BYTES + ps * 2 * CHUNK_BYTES +
-             static_cast<int>(sizeof(PairOutBars)) + 1024;
-    };
-    prm.c_ps = pair_smem_for(3) <= max_smem ? 3 : 2;
-    const int pair_smem = pair_smem_for(prm.c_ps);
+    // key and value rings of 3 (one stage per logit / P' buffer); at least
+    // CP_MIN_SMEM so a second CTA cannot share the SM's tensor memory
+    const int pair_smem = std::max(kc * CHUNK_BYTES + CP_KS * kc * CP_KCHUNK_BYTES + CP_VS * CHUNK_BYTES +
+                                       static_cast<int>(sizeof(PairOutBars)) + 1024,
+                                   CP_MIN_SMEM);
+    if (pair_smem > max_smem) return cudaErrorInvalidValue;
     CUtensorMap tm_kh;
     if (!encode_heads(&tm_kh, kt_rows, kd, kt, BH, w.ldk, CP_HALF_ROWS)) return cudaErrorInvalidValue;
     {
@@ -1220,7 +1234,7 @@ cudaError_t launch_attention(const void* Q, const void* K, const void* V, int64_
       }
     }
     const dim3 grid_pair(static_cast<unsigned>(2 * BH), static_cast<unsigned>((nqb + 1) / 2));
-    attn_out_pair_kernel<<<grid_pair, ATT_THREADS, pair_smem, stream>>>(tm_q, tm_kh, tm_vt, lse, idx_t, nvalid, O,
+    attn_out_pair_kernel<<<grid_pair, PAIR_THREADS, pair_smem, stream>>>(tm_q, tm_kh, tm_vt, lse, idx_t, nvalid, O,
                                                                          prm, err);
     return cudaGetLastError();
   }

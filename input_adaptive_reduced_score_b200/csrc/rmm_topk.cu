@@ -136,7 +136,7 @@ constexpr int64_t kMaxStagedKeys = 51200;  // 200 KB of keys + 8 KB of bins per 
 // The staged search with this file's static bins, writing the k selected
 // indices, ascending, to out.
 template <int NT>
-__device__ __forceinline__ void select_staged(const uint32_t* keys, int d, uint32_t k, uint32_t kmin, uint32_t kmax,
+__device__ __forceinline__ void select_staged(uint32_t* keys, int d, uint32_t k, uint32_t kmin, uint32_t kmax,
                                               int32_t* __restrict__ out) {
   __shared__ __align__(16) uint32_t hist[kSelectBins];
   select_staged_keys<NT>(keys, d, k, kmin, kmax, hist, [&](uint32_t pos, int j) { out[pos] = j; });
