@@ -69,17 +69,21 @@ __device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32
     const uint64_t range = hi - lo;
     const int nbits = 64 - __clzll(static_cast<long long>(range - 1u));  // ceil(log2(range))
     const int shift = nbits > 11 ? nbits - 11 : 0;
+    // key - lo < range, in 32 bits: range - 1 fits (the range is at most 2^32)
+    const uint32_t lo32 = static_cast<uint32_t>(lo), span = static_cast<uint32_t>(range - 1u);
     const int dv = d >> 2;
     for (int v = tid; v < dv; v += NT) {
       const uint4 q = reinterpret_cast<const uint4*>(keys)[v];
       const uint32_t kq[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (kq[e] >= lo && kq[e] < hi) atomicAdd(&hist[static_cast<uint32_t>((kq[e] - lo) >> shift)], 1u);
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t off = kq[e] - lo32;  // wraps for keys below lo
+        if (off <= span) atomicAdd(&hist[off >> shift], 1u);
+      }
     }
     for (int j = 4 * dv + tid; j < d; j += NT) {
-      const uint32_t key = keys[j];
-      if (key >= lo && key < hi) atomicAdd(&hist[static_cast<uint32_t>((key - lo) >> shift)], 1u);
+      const uint32_t off = keys[j] - lo32;
+      if (off <= span) atomicAdd(&hist[off >> shift], 1u);
     }
     __syncthreads();
     // this thread's bins [tid*BPT, tid*BPT + BPT), read and cleared for the next round
@@ -145,27 +149,37 @@ __device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32
   const uint32_t need = k - above;
   // this thread's run [j0, j0 + R): bit masks of its keys at or above hi and
   // of its keys in [lo, hi)
+  // (word and bit positions are compile-time: a runtime index would put the
+  // masks in local memory)
   constexpr int kWords = 4;  // up to 128 keys per thread
   const int R = (((d + NT - 1) / NT) + 3) & ~3;
   const int j0 = tid * R;
+  const bool hi_in = hi <= 0xFFFFFFFFull;  // hi = 2^32: no key lies at or above it
+  const uint32_t lo32 = static_cast<uint32_t>(lo), hi32 = static_cast<uint32_t>(hi);
   uint32_t gtm[kWords] = {0u, 0u, 0u, 0u}, eqm[kWords] = {0u, 0u, 0u, 0u};
-  for (int q = 0; q < R; q += 4) {
-    const int j = j0 + q;
-    if (j >= d) break;
-    uint32_t kq[4];
-    if (j + 4 <= d) {
-      const uint4 v = reinterpret_cast<const uint4*>(keys)[j >> 2];
-      kq[0] = v.x; kq[1] = v.y; kq[2] = v.z; kq[3] = v.w;
-    } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) kq[e] = j + e < d ? keys[j + e] : 0u;
-    }
+  for (int w = 0; w < kWords; ++w) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int bit = q + e;
-      const bool valid = j + e < d;
-      if (valid && kq[e] >= hi) gtm[bit >> 5] |= 1u << (bit & 31);
-      if (valid && kq[e] >= lo && kq[e] < hi) eqm[bit >> 5] |= 1u << (bit & 31);
+    for (int u = 0; u < 8; ++u) {
+      const int q = 32 * w + 4 * u;  // this vector's first key in the run
+      const int j = j0 + q;
+      if (q < R && j < d) {
+        uint32_t kq[4];
+        if (j + 4 <= d) {
+          const uint4 v = reinterpret_cast<const uint4*>(keys)[j >> 2];
+          kq[0] = v.x; kq[1] = v.y; kq[2] = v.z; kq[3] = v.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) kq[e] = j + e < d ? keys[j + e] : 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool valid = j + e < d;
+          const bool ge_hi = hi_in && kq[e] >= hi32;
+          gtm[w] |= static_cast<uint32_t>(valid && ge_hi) << (4 * u + e);
+          eqm[w] |= static_cast<uint32_t>(valid && kq[e] >= lo32 && !ge_hi) << (4 * u + e);
+        }
+      }
     }
   }
   uint32_t ngt = 0u, neq = 0u;
