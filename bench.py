@@ -765,7 +765,7 @@ def measure_decode_attention(R, workloads, bf16_tensor, dev, stream, steps, time
         gbs = alg / (rmm_us * 1e-6) / 1e9
         out[f"B{B}"] = {"rmm_us": rmm_us, "sdpa_us": sdpa_us, "speedup_vs_sdpa": sdpa_us / rmm_us,
                         "algorithmic_MB": alg / 1e6, "GB/s": gbs, "frac_hbm": gbs / hbm_gbs,
-                        "kept_value_rows_union_frac": union / (B * a["Hkv"] * a["L"]), "gpu_launches_per_call": 6}
+                        "kept_value_rows_union_frac": union / (B * a["Hkv"] * a["L"]), "gpu_launches_per_call": 3}
     if R.rmm_device_error(stream) != 0:
         raise SystemExit("device error during the decode-attention runs")
     out["workload"] = (f"decode step: q[B x {a['Hq']} x {a['D']}] over K/V caches [B x {a['Hkv']} x {a['L']} x "

@@ -136,8 +136,9 @@ RMM_API rmm_status rmm_score_noalloc(const void* A, int dtype, int64_t batch, in
  * de Selección keeps the top-k; the tie rule and the order are this library's
  * reading).  Scores must be finite; -0.0 ranks equal to +0.0.  The selection
  * is exact on the fp32 bit patterns (a histogram search over the key range,
- * or a radix select for rows longer than 51200), so the index set is the
- * unique one defined by that rule.  1 <= k <= d, ld_idx >= k, ld_s >= d.  */
+ * by one CTA or a cluster of up to eight per row, or a radix select for rows
+ * longer than 409600), so the index set is the unique one defined by that
+ * rule.  1 <= k <= d, ld_idx >= k, ld_s >= d.  */
 RMM_API rmm_status rmm_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k,
                     int32_t* idx, int64_t ld_idx, void* stream);
 

@@ -786,11 +786,9 @@ rmm_status rmm_decode_attention(const void* q, const void* K, const void* V, int
   if (!ws || ws_bytes < need || reinterpret_cast<uintptr_t>(ws) % kWsAlign)
     return fail(RMM_ERR_WORKSPACE, "rmm_decode_attention: workspace %zu < %zu bytes or not 256-byte aligned",
                 ws_bytes, need);
-  unsigned* err = device_error_word();
-  if (!err) return RMM_ERR_CUDA;
   const float sc = scale > 0.f ? scale : static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   const cudaError_t e = launch_decode_attention(q, K, V, B, Hq, Hkv, L, Lmax, D, kd, kt, sc, O, out_dtype, idx_d,
-                                                idx_t, lse, logits, ws, err, static_cast<cudaStream_t>(stream));
+                                                idx_t, lse, logits, ws, static_cast<cudaStream_t>(stream));
   return from_cuda(e, "rmm_decode_attention: launch");
 }
 

@@ -10,32 +10,37 @@
 //   lse = logsumexp_j s_j;  P_j = exp(s_j - lse);
 //   I_t = top ceil(rho_t L) of t_j = P_j^2;  O = sum_{j in I_t} P_j V[g, j, :].
 //
-// Six launches on one stream (programmatic dependent launch between them):
-//  1. dec_select_kernel, one warp per (b, h): the head_dim set from the query
-//     row; the query is kept as fp32 with the dropped entries zeroed.
-//  2. dec_logits_kernel, grid (token chunks of 128, B * Hkv): the chunk's key
+// Three launches on one stream (programmatic dependent launch between them):
+//  1. dec_logits_kernel, grid (token chunks of 128, B * Hkv): the chunk's key
 //     rows are copied into shared memory with coalesced 16-byte asynchronous
 //     copies (rows padded by 16 bytes, so 8x8 matrix loads hit no bank
-//     twice); then each warp forms the logits of 32 tokens for every q-head
-//     of the group as a tensor-core product (mma m16n8k16, bf16 operands,
-//     fp32 accumulation): keys [tokens x head_dim] times the masked queries
-//     [head_dim x heads].  The dropped entries add exact zeros, so each sum
-//     is the reduced dot product.  Logits go to a [B*Hq, L] buffer; each CTA
-//     also leaves its chunk's maximum and sum of exponentials per head.  A
-//     plain FMA form of this contraction was bound by shared-memory traffic
-//     and issue (about 800 instructions per key row) at half the HBM rate.
-//  3. the histogram top-k over each head's L logits.  t_j = exp(2(s_j - lse))
-//     is increasing in s_j, so ranking the logits ranks the token scores
-//     (without the rounding of the exponential merging close values).
-//  4. dec_prefix_kernel: for each head, where each 512-token chunk starts in
-//     its ascending kept list.
-//  5. dec_out_kernel, grid (token chunks of 512, B * Hkv): the weights
+//     twice); while they arrive, each warp finds the head_dim set of a q-head
+//     of the group (a bitwise search for the k_d-th largest |q_c| with warp
+//     ballots) and leaves the masked query in shared memory.  Then each warp
+//     forms the logits of 32 tokens for every q-head of the group as a
+//     tensor-core product (mma m16n8k16, bf16 operands, fp32 accumulation):
+//     keys [tokens x head_dim] times the masked queries [head_dim x heads].
+//     The dropped entries add exact zeros, so each sum is the reduced dot
+//     product.  Logits go to a [B*Hq, L] buffer; each CTA also leaves its
+//     chunk's maximum and sum of exponentials per head.  (A plain FMA form of
+//     this contraction was bound by shared-memory traffic and issue, about
+//     800 instructions per key row, at half the HBM rate.)
+//  2. dec_topk_kernel, the histogram top-k of rmm_select.cuh over each head's
+//     L logits, on one CTA or a thread-block cluster of 2, 4 or 8 CTAs per
+//     head (so that a few sequences still fill the SMs).  t_j = exp(2(s_j -
+//     lse)) is increasing in s_j, so ranking the logits ranks the token
+//     scores (without the rounding of the exponential merging close values).
+//     It also writes where each 512-token output chunk starts in the kept
+//     list, the heads' lse, and clears the output kernel's arrival counters.
+//     (Rows too long for eight CTAs take the radix pass of rmm_topk.cu and
+//     dec_prefix_kernel instead.)
+//  3. dec_out_kernel, grid (token chunks of 512, B * Hkv): the weights
 //     P_j = exp(s_j - lse) of every q-head of the group are scattered into a
 //     table over the chunk's positions; the value rows kept by any of the
 //     group's heads are read once each (16-byte asynchronous copies, six
 //     stages of four rows per warp) and added into every head that keeps
-//     them; per-chunk sums go to global memory.
-//  6. dec_reduce_kernel: O = the chunk sums added in chunk order.
+//     them; per-chunk sums go to global memory, and the group's last CTA to
+//     finish adds them in chunk order into O.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -44,6 +49,7 @@
 #include "rmm_device.cuh"
 #include "rmm_internal.h"
 #include "rmm_launch.cuh"
+#include "rmm_select.cuh"
 
 namespace rmm {
 namespace {
@@ -55,11 +61,26 @@ constexpr int kDecChunk = kLogitThreads;        // tokens per logits CTA, one pe
 constexpr int kDecOutChunk = 512;               // token positions per output CTA
 constexpr int kDecStages = 6;
 constexpr int kDecRowsPerStage = 4;
+constexpr int kDecMaxSliceKeys = 51200;         // logits one top-k CTA stages (200 KB)
+constexpr int kDecWarpTokens = kDecOutChunk / kDecWarps;  // token positions per output warp (64)
+static_assert(kDecWarpTokens == 64, "an output warp covers two bitmap words");
 
 struct DecParams {
-  int B, Hq, Hkv, G, L, Lmax, kd, kt, chunks, out_chunks;
+  int B, Hq, Hkv, G, L, Lmax, kd, kt, chunks, out_chunks, nwords;
   float scale;
 };
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -70,46 +91,55 @@ constexpr int key_pitch() { return D * 2 + 16; }  // bytes per staged key row
 template <int D>
 constexpr size_t dec_logits_smem() { return static_cast<size_t>(kDecChunk) * key_pitch<D>(); }
 
-// The head_dim set of one (b, h), one warp: rank of q_c^2 (exact in fp32 for
-// bf16 q) counting larger values and equal ones at lower indices.  Writes
-// the query as fp32 with the dropped entries zeroed, and the ascending set.
+// The head_dim set of query row qh (D bf16 values), one warp: the kd entries
+// of largest q_c^2, lowest index first among equals.  q_c^2 is ordered as
+// |q_c|, whose bf16 bits without the sign are an order-preserving 15-bit
+// key; the kd-th largest key T is found bit by bit (the largest t with at
+// least kd keys >= t), then the keys above T and the first equal ones are
+// kept.  Lane l holds entries l*PER .. l*PER + PER - 1.  Writes the masked
+// row (dropped entries +0) as bf16 pairs to sqm, and, if idx_d is given, the
+// ascending set.
 template <int D>
-__global__ void __launch_bounds__(32) dec_select_kernel(const uint16_t* __restrict__ q, DecParams p,
-                                                        float* __restrict__ qm, int32_t* __restrict__ idx_d) {
+__device__ __forceinline__ void head_dim_select(const uint16_t* __restrict__ qh, int kd, uint32_t* sqm,
+                                                int32_t* __restrict__ idx_d) {
   constexpr int PER = D / 32;
-  __shared__ float sq[D];
-  const int lane = threadIdx.x;
-  const int64_t bh = blockIdx.x;
-  pdl_wait();
-  pdl_trigger();
-  float v[PER];
+  const int lane = threadIdx.x & 31;
+  uint32_t bits[PER], key[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) {
-    v[e] = __uint_as_float(static_cast<uint32_t>(q[bh * D + lane * PER + e]) << 16);
-    sq[lane * PER + e] = v[e] * v[e];
+    bits[e] = __ldg(qh + lane * PER + e);
+    key[e] = bits[e] & 0x7FFFu;
   }
-  __syncwarp();
-  int rank[PER];
+  uint32_t T = 0u;
+#pragma unroll 1
+  for (int bit = 14; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    int n = 0;
 #pragma unroll
-  for (int e = 0; e < PER; ++e) rank[e] = 0;
-#pragma unroll 16
-  for (int c = 0; c < D; ++c) {
-    const float sx = sq[c];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      const float se = sq[lane * PER + e];
-      rank[e] += (sx > se || (sx == se && c < lane * PER + e)) ? 1 : 0;
-    }
+    for (int e = 0; e < PER; ++e) n += __popc(__ballot_sync(0xFFFFFFFFu, key[e] >= cand));
+    if (n >= kd) T = cand;
   }
+  int gt = 0, eq_before = 0;
+  const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    gt += __popc(__ballot_sync(0xFFFFFFFFu, key[e] > T));
+    eq_before += __popc(__ballot_sync(0xFFFFFFFFu, key[e] == T) & below);
+  }
+  const int need = kd - gt;  // equal keys kept, lowest index first
   int nkept = 0;
+  bool kept[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) {
-    const bool kept = rank[e] < p.kd;
-    qm[bh * D + lane * PER + e] = kept ? v[e] : 0.f;
-    nkept += kept ? 1 : 0;
+    const bool eq = key[e] == T;
+    kept[e] = key[e] > T || (eq && eq_before < need);
+    eq_before += eq ? 1 : 0;
+    nkept += kept[e] ? 1 : 0;
   }
+#pragma unroll
+  for (int i = 0; i < PER / 2; ++i)
+    sqm[lane * (PER / 2) + i] = (kept[2 * i] ? bits[2 * i] : 0u) | ((kept[2 * i + 1] ? bits[2 * i + 1] : 0u) << 16);
   if (idx_d) {
-    // ascending position of each kept entry: kept entries at lower lanes, then lower e
     int before = nkept;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -119,7 +149,7 @@ __global__ void __launch_bounds__(32) dec_select_kernel(const uint16_t* __restri
     before -= nkept;
 #pragma unroll
     for (int e = 0; e < PER; ++e)
-      if (rank[e] < p.kd) idx_d[bh * p.kd + before++] = lane * PER + e;
+      if (kept[e]) idx_d[before++] = lane * PER + e;
   }
 }
 
@@ -140,14 +170,16 @@ __device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4],
 
 template <int D, int G>
 __global__ void __launch_bounds__(kLogitThreads)
-    dec_logits_kernel(const float* __restrict__ qmask, const uint16_t* __restrict__ K, DecParams p,
-                      float* __restrict__ logits, float2* __restrict__ part) {
+    dec_logits_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ K, DecParams p,
+                      float* __restrict__ logits, float2* __restrict__ part, int32_t* __restrict__ idx_d) {
   extern __shared__ __align__(128) uint8_t kt_smem[];  // [kDecChunk][key_pitch]
   constexpr int NW = kLogitThreads / 32;
   constexpr int NT = (G + 7) / 8;   // 8-head column tiles
   constexpr int KS = D / 16;        // 16-deep head_dim steps
+  constexpr int QP = D / 2 + 4;     // words per masked query row (padded: the 8 heads of a fragment hit 8 banks)
   __shared__ float wred[NW][NT * 8];
   __shared__ float hmax[NT * 8];
+  __shared__ uint32_t sqm[G][QP];   // the group's masked queries, bf16 pairs
   constexpr int PITCH = key_pitch<D>();
   constexpr int PIECES = D * 2 / 16;  // 16-byte pieces per key row
   const int chunk = blockIdx.x;
@@ -173,24 +205,23 @@ __global__ void __launch_bounds__(kLogitThreads)
     }
     cp_async_commit();
   }
+  // while the keys arrive: the head_dim set of each q-head of the group,
+  // warp w taking heads w, w + NW, ...; the first chunk's CTA writes idx_d
+  for (int hh = warp; hh < G; hh += NW) {
+    const int64_t bh = static_cast<int64_t>(b) * p.Hq + g * G + hh;
+    head_dim_select<D>(q + bh * D, p.kd, sqm[hh], (idx_d && chunk == 0) ? idx_d + bh * p.kd : nullptr);
+  }
+  __syncthreads();
   // B fragments: masked query of head (8 t + gq), head_dim 16 s + 2 cq (+1)
-  // and 16 s + 2 cq + 8 (+1), as bf16 pairs (exact: the values are bf16)
+  // and 16 s + 2 cq + 8 (+1), as bf16 pairs
   uint32_t bq[NT][KS][2];
-  const float* qg = qmask + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
     const int hh = t * 8 + gq;
 #pragma unroll
     for (int s = 0; s < KS; ++s) {
-      if (hh < G) {
-        const float2 lo = __ldg(reinterpret_cast<const float2*>(qg + hh * D + 16 * s + 2 * cq));
-        const float2 hi = __ldg(reinterpret_cast<const float2*>(qg + hh * D + 16 * s + 2 * cq + 8));
-        bq[t][s][0] = pack_bf16x2(lo.x, lo.y);
-        bq[t][s][1] = pack_bf16x2(hi.x, hi.y);
-      } else {
-        bq[t][s][0] = 0u;
-        bq[t][s][1] = 0u;
-      }
+      bq[t][s][0] = hh < G ? sqm[hh][8 * s + cq] : 0u;
+      bq[t][s][1] = hh < G ? sqm[hh][8 * s + cq + 4] : 0u;
     }
   }
   cp_async_wait<0>();
@@ -290,150 +321,174 @@ __global__ void __launch_bounds__(kLogitThreads)
   }
 }
 
-// start[bh][c] = index in head bh's ascending kept list of its first token at
-// or past position c * kDecOutChunk (c = 0 .. out_chunks; the last is k_t).
-// One thread per list index r in [0, k_t]: it writes the chunks its step
-// from entry r-1 to entry r crosses.
-__global__ void __launch_bounds__(kDecThreads) dec_prefix_kernel(const int32_t* __restrict__ idx_t, DecParams p,
-                                                                 int32_t* __restrict__ start) {
+// lse of head bh from the logits kernel's chunk partials (max, sum of
+// exponentials), one warp; also zeroes the output kernel's arrival counter
+// of the head's kv-group (from its first q-head).
+__device__ __forceinline__ void head_lse(const float2* __restrict__ part, const DecParams& p, int64_t bh,
+                                         float* __restrict__ lse_ws, float* __restrict__ lse_out,
+                                         unsigned* __restrict__ arrivals) {
+  const int lane = threadIdx.x & 31;
+  const float2* pp = part + bh * p.chunks;
+  float m = -INFINITY;
+  for (int c = lane; c < p.chunks; c += 32) m = fmaxf(m, pp[c].x);
+  m = warp_max(m);
+  float z = 0.f;
+  for (int c = lane; c < p.chunks; c += 32) z += pp[c].y * __expf(pp[c].x - m);
+  z = warp_sum(z);
+  if (lane == 0) {
+    const float l = m + __logf(z);
+    lse_ws[bh] = l;
+    if (lse_out) lse_out[bh] = l;
+    if (bh % p.G == 0) arrivals[bh / p.G] = 0u;
+  }
+}
+
+// The token top-k of each head (grid x = the C CTAs of a cluster, y = head):
+// CTA r stages the logits of tokens [r * slice, (r + 1) * slice) (slice a
+// multiple of 32), takes its part of the exact selection (rmm_select.cuh;
+// ranking the logits ranks t_j = exp(2 (s_j - lse))), and writes its kept
+// tokens to idx_t and as bits of the head's kept-token bitmap (bit t % 32 of
+// word t / 32).  Rank 0 also forms the head's lse.
+template <int NT, int C>
+__global__ void __launch_bounds__(NT, 1)
+    dec_topk_kernel(const float* __restrict__ logits, const float2* __restrict__ part, DecParams p, int slice,
+                    int32_t* __restrict__ idx_t, uint32_t* __restrict__ kept, float* __restrict__ lse_ws,
+                    float* __restrict__ lse_out, unsigned* __restrict__ arrivals) {
+  extern __shared__ __align__(16) uint32_t keys[];
+  __shared__ __align__(16) uint32_t hist[(C > 1 ? 2 : 1) * kSelectBins];
+  const int rank = C > 1 ? static_cast<int>(blockIdx.x) : 0;
+  const int64_t bh = blockIdx.y;
+  const int j0 = rank * slice;
+  const int dl = max(0, min(slice, p.L - j0));
+  pdl_wait();
+  pdl_trigger();
+  if (rank == 0 && threadIdx.x < 32) head_lse(part, p, bh, lse_ws, lse_out, arrivals);
+  uint32_t kmin, kmax;
+  stage_score_keys<NT>(logits + bh * p.L + j0, dl, keys, kmin, kmax);
+  const StagedSelection sel = select_staged_compact<NT, C>(keys, dl, static_cast<uint32_t>(p.kt), kmin, kmax, hist);
+  int32_t* out = idx_t + bh * p.kt;
+  for (int q = threadIdx.x; q < static_cast<int>(sel.count); q += NT) out[sel.base + q] = j0 + static_cast<int32_t>(keys[q]);
+  // the bitmap of the slice's words, built in the bins (no CTA reads them
+  // any more: the search's last remote reads came before its count exchange)
+  const int nw = (dl + 31) / 32;
+  for (int w = threadIdx.x; w < nw; w += NT) hist[w] = 0u;
+  __syncthreads();
+  for (int q = threadIdx.x; q < static_cast<int>(sel.count); q += NT) atomicOr(&hist[keys[q] >> 5], 1u << (keys[q] & 31u));
+  __syncthreads();
+  uint32_t* kw = kept + bh * p.nwords + j0 / 32;
+  for (int w = threadIdx.x; w < nw; w += NT) kw[w] = hist[w];
+  if constexpr (C > 1) cluster_wait();  // no CTA leaves while another may still read its shared memory
+}
+
+// Rows too long for a cluster to stage (their top-k is the radix pass of
+// rmm_topk.cu): the kept-token bitmap from the finished ascending list, one
+// thread per word (the word's first entry found by bisection), and the lse.
+__global__ void __launch_bounds__(kDecThreads) dec_mark_kernel(const int32_t* __restrict__ idx_t,
+                                                               const float2* __restrict__ part, DecParams p,
+                                                               uint32_t* __restrict__ kept,
+                                                               float* __restrict__ lse_ws,
+                                                               float* __restrict__ lse_out,
+                                                               unsigned* __restrict__ arrivals) {
   pdl_wait();
   pdl_trigger();
   const int64_t bh = blockIdx.y;
-  const int r = blockIdx.x * kDecThreads + threadIdx.x;
-  if (r > p.kt) return;
+  if (blockIdx.x == 0 && threadIdx.x < 32) head_lse(part, p, bh, lse_ws, lse_out, arrivals);
+  const int w = blockIdx.x * kDecThreads + threadIdx.x;
+  if (w >= p.nwords) return;
   const int32_t* it = idx_t + bh * p.kt;
-  int32_t* st = start + bh * (p.out_chunks + 1);
-  auto chunk_of = [&](int i) {
-    const int32_t j = __ldg(it + i);
-    const int c = j < 0 ? 0 : j / kDecOutChunk;
-    return c < p.out_chunks ? c : p.out_chunks - 1;
-  };
-  const int prev = r == 0 ? -1 : chunk_of(r - 1);
-  const int cur = r == p.kt ? p.out_chunks : chunk_of(r);
-  for (int c = prev + 1; c <= cur; ++c) st[c] = r;
+  int lo = 0, hi = p.kt;  // first entry >= 32 w
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (it[mid] < 32 * w) lo = mid + 1;
+    else hi = mid;
+  }
+  uint32_t bits = 0u;
+  for (int i = lo; i < p.kt && it[i] < 32 * w + 32; ++i) bits |= 1u << (it[i] - 32 * w);
+  kept[bh * p.nwords + w] = bits;
 }
 
 template <int D, int G>
 constexpr size_t dec_out_smem() {
   return static_cast<size_t>(kDecWarps) * kDecStages * kDecRowsPerStage * D * 2 +  // value rings
-         static_cast<size_t>(G) * kDecOutChunk * 4 * 2 +                            // weights by position, by union row
-         static_cast<size_t>(kDecOutChunk) * 4 * 2;                                 // kept flags, union list
+         static_cast<size_t>(kDecWarps) * kDecWarpTokens * 4 * (G + 1);             // weights, union list
 }
 
 template <int D, int G>
 __global__ void __launch_bounds__(kDecThreads, 2)
     dec_out_kernel(const uint16_t* __restrict__ V, DecParams p, const float* __restrict__ logits,
-                   const float2* __restrict__ part, const int32_t* __restrict__ idx_t,
-                   const int32_t* __restrict__ start, float* __restrict__ opart, float* __restrict__ lse_out,
-                   unsigned* err) {
+                   const float* __restrict__ lse_ws, const uint32_t* __restrict__ kept, float* __restrict__ opart,
+                   void* __restrict__ O, int out_f32, unsigned* __restrict__ arrivals) {
   constexpr int ROWB = D * 2;                 // bytes of a value row
   constexpr int PIECES = ROWB / 16;           // 16-byte pieces per row
   constexpr int ROWS_PER_COPY = 32 / PIECES;  // rows one warp-wide copy instruction covers
   constexpr int DPL = D / 32;                 // dims per lane
   constexpr int RPS = kDecRowsPerStage;
   constexpr int S = kDecStages;
+  constexpr int WT = kDecWarpTokens;          // token positions per warp (two bitmap words)
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[kDecWarps][D];
-  __shared__ float s_lse[G];
-  __shared__ int s_cnt[kDecWarps];
-  __shared__ int s_a[G], s_n[G];
-  float* wtab = reinterpret_cast<float*>(smem + static_cast<size_t>(kDecWarps) * S * RPS * ROWB);  // [G][chunk]
-  float* wrow = wtab + G * kDecOutChunk;  // [G][chunk]: the weights in union-row order, zero past the union
-  int32_t* flag = reinterpret_cast<int32_t*>(wrow + G * kDecOutChunk);
-  int32_t* list = flag + kDecOutChunk;
+  __shared__ unsigned s_last;
   const int chunk = blockIdx.x;
   const int b = blockIdx.y / p.Hkv, g = blockIdx.y % p.Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p0 = chunk * kDecOutChunk;
   const int64_t bh0 = static_cast<int64_t>(b) * p.Hq + g * G;  // first q-head of the group
-  for (int e = threadIdx.x; e < 2 * G * kDecOutChunk; e += kDecThreads) wtab[e] = 0.f;
-  for (int e = threadIdx.x; e < kDecOutChunk; e += kDecThreads) flag[e] = 0;
+  const int pw = chunk * kDecOutChunk + warp * WT;              // this warp's first token position
+  int32_t* list = reinterpret_cast<int32_t*>(smem + static_cast<size_t>(kDecWarps) * S * RPS * ROWB) + warp * WT;
+  float* wl = reinterpret_cast<float*>(smem + static_cast<size_t>(kDecWarps) * S * RPS * ROWB +
+                                       static_cast<size_t>(kDecWarps) * WT * 4) + warp * G * WT;
   pdl_wait();
   pdl_trigger();
 
-  // lse of each q-head of the group from the logits kernel's chunk partials
-  for (int hh = warp; hh < G; hh += kDecWarps) {
-    const float2* pp = part + (bh0 + hh) * p.chunks;
-    float m = -INFINITY;
-    for (int c = lane; c < p.chunks; c += 32) m = fmaxf(m, pp[c].x);
+  // every head's kept bits, lse and logits over the warp's positions: one
+  // round of independent loads
+  const int w0 = pw >> 5;
+  uint32_t m0[G], m1[G];
+  float lg0[G], lg1[G], ls[G];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    float z = 0.f;
-    for (int c = lane; c < p.chunks; c += 32) z += pp[c].y * __expf(pp[c].x - m);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
-    if (lane == 0) {
-      s_lse[hh] = m + __logf(z);
-      if (lse_out && chunk == 0) lse_out[bh0 + hh] = s_lse[hh];
-    }
+  for (int hh = 0; hh < G; ++hh) {
+    const uint32_t* kb = kept + (bh0 + hh) * p.nwords;
+    const float* lr = logits + (bh0 + hh) * p.L;
+    m0[hh] = w0 < p.nwords ? kb[w0] : 0u;
+    m1[hh] = w0 + 1 < p.nwords ? kb[w0 + 1] : 0u;
+    ls[hh] = lse_ws[bh0 + hh];
+    lg0[hh] = pw + lane < p.L ? lr[pw + lane] : 0.f;
+    lg1[hh] = pw + 32 + lane < p.L ? lr[pw + 32 + lane] : 0.f;
   }
-  __syncthreads();
+  // the union of the group's kept rows in position order, with each head's
+  // weight P_j = exp(s_j - lse) (zero where the head does not keep j)
+  uint32_t u0 = 0u, u1 = 0u;
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    u0 |= m0[hh];
+    u1 |= m1[hh];
+  }
+  const int n0 = __popc(u0), n = n0 + __popc(u1);
+  const uint32_t below = (1u << lane) - 1u;
+  if ((u0 >> lane) & 1u) {
+    const int r = __popc(u0 & below);
+    list[r] = lane;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) wl[hh * WT + r] = ((m0[hh] >> lane) & 1u) ? __expf(lg0[hh] - ls[hh]) : 0.f;
+  }
+  if ((u1 >> lane) & 1u) {
+    const int r = n0 + __popc(u1 & below);
+    list[r] = 32 + lane;
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) wl[hh * WT + r] = ((m1[hh] >> lane) & 1u) ? __expf(lg1[hh] - ls[hh]) : 0.f;
+  }
+  // rows past the union in its last stage are copied as zeros with zero weight
+  const int npad = (n + RPS - 1) / RPS * RPS;
+  if (n + lane < npad) {
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) wl[hh * WT + n + lane] = 0.f;
+  }
+  __syncwarp();
 
-  // weights of the kept tokens in this chunk, every q-head at once: thread t
-  // takes entries t, t + 256, ... of the heads' ranges laid end to end
-  if (threadIdx.x < G) {
-    const int32_t* st = start + (bh0 + threadIdx.x) * (p.out_chunks + 1);
-    const int a = min(max(__ldg(st + chunk), 0), p.kt), e = min(max(__ldg(st + chunk + 1), a), p.kt);
-    s_a[threadIdx.x] = a;
-    s_n[threadIdx.x] = e - a;
-  }
-  __syncthreads();
-  int total = 0;
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) total += s_n[hh];
-  bool bad = false;
-  for (int f = threadIdx.x; f < total; f += kDecThreads) {
-    int hh = 0, r = f;
-    while (hh < G - 1 && r >= s_n[hh]) r -= s_n[hh++];
-    const int32_t j = __ldg(idx_t + (bh0 + hh) * p.kt + s_a[hh] + r);
-    if (j < p0 || j >= p0 + kDecOutChunk || j >= p.L) {
-      bad = true;
-      continue;
-    }
-    wtab[hh * kDecOutChunk + (j - p0)] = __expf(__ldg(logits + (bh0 + hh) * p.L + j) - s_lse[hh]);
-    flag[j - p0] = 1;
-  }
-  if (bad) record_error(err, kDevErrBadIndex);
-  __syncthreads();
-
-  // the union of the group's kept rows, in position order
-  constexpr int PT = kDecOutChunk / kDecThreads;  // positions per thread
-  int mine = 0;
-#pragma unroll
-  for (int e = 0; e < PT; ++e) mine += flag[threadIdx.x * PT + e];
-  int incl = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) s_cnt[warp] = incl;
-  __syncthreads();
-  int before = incl - mine, n = 0;
-  for (int w = 0; w < kDecWarps; ++w) {
-    if (w < warp) before += s_cnt[w];
-    n += s_cnt[w];
-  }
-#pragma unroll
-  for (int e = 0; e < PT; ++e) {
-    const int pos = threadIdx.x * PT + e;
-    if (flag[pos]) {
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) wrow[hh * kDecOutChunk + before] = wtab[hh * kDecOutChunk + pos];
-      list[before++] = pos;
-    }
-  }
-  __syncthreads();
-
-  // stream the union rows: warp w takes a contiguous run of them, four per
-  // stage; a stage's four weights of a head are one 16-byte load, rows past
-  // the run are copied as zeros with zero weight, so no row needs a test
+  // stream the union rows, four per stage; a stage's four weights of a head
+  // are one 16-byte load
   const char* Vg = reinterpret_cast<const char*>(V + (static_cast<int64_t>(b) * p.Hkv + g) * p.Lmax * D);
   const uint32_t ring = smem_u32(smem) + static_cast<uint32_t>(warp * S * RPS * ROWB);
-  const int per = ((n + kDecWarps - 1) / kDecWarps + RPS - 1) / RPS * RPS;
-  const int r0w = warp * per;
-  const int rend = min(n, r0w + per);
-  const int nst = rend > r0w ? (rend - r0w + RPS - 1) / RPS : 0;
+  const int nst = npad / RPS;
   constexpr int NP = DPL / 2;  // dim pairs per lane
   uint64_t acc[G][NP];
 #pragma unroll
@@ -446,9 +501,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 #pragma unroll
       for (int h2 = 0; h2 < RPS / ROWS_PER_COPY; ++h2) {
         const int u = h2 * ROWS_PER_COPY + lane / PIECES, piece = lane % PIECES;
-        const int row = r0w + stg * RPS + u;
-        const bool ok = row < rend;
-        const int j = ok ? p0 + list[row] : 0;
+        const int row = stg * RPS + u;
+        const bool ok = row < n;
+        const int j = ok ? pw + list[row] : 0;
         cp_async16(base + u * ROWB + piece * 16, Vg + static_cast<int64_t>(j) * ROWB + piece * 16, ok ? 16u : 0u);
       }
     }
@@ -463,8 +518,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     const uint8_t* base = smem + (warp * S + stg % S) * RPS * ROWB + lane * DPL * 2;
     float4 w4[G];
 #pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-      w4[hh] = *reinterpret_cast<const float4*>(wrow + hh * kDecOutChunk + r0w + stg * RPS);
+    for (int hh = 0; hh < G; ++hh) w4[hh] = *reinterpret_cast<const float4*>(wl + hh * WT + stg * RPS);
 #pragma unroll
     for (int u = 0; u < RPS; ++u) {
       uint64_t v[NP];
@@ -501,21 +555,27 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     }
     __syncthreads();
   }
-}
 
-// O[bh, :] = sum over token chunks, in chunk order, of the chunk sums.
-template <int D>
-__global__ void __launch_bounds__(D) dec_reduce_kernel(const float* __restrict__ opart, DecParams p,
-                                                       void* __restrict__ O, int out_f32) {
-  pdl_wait();
-  pdl_trigger();
-  const int64_t bh = blockIdx.x;
-  float v = 0.f;
-  for (int c = 0; c < p.out_chunks; ++c) v += __ldg(opart + (bh * p.out_chunks + c) * D + threadIdx.x);
-  if (out_f32)
-    static_cast<float*>(O)[bh * D + threadIdx.x] = v;
-  else
-    static_cast<__nv_bfloat16*>(O)[bh * D + threadIdx.x] = __float2bfloat16_rn(v);
+  // the group's last CTA to finish adds the chunk sums, in chunk order:
+  // O[bh, :] = sum_c opart[bh, c, :]
+  if (threadIdx.x == 0) {
+    __threadfence();  // this CTA's chunk sums are visible before its arrival
+    s_last = atomicAdd(arrivals + blockIdx.y, 1u) == static_cast<unsigned>(p.out_chunks) - 1u ? 1u : 0u;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < G * D; e += kDecThreads) {
+    const int hh = e / D, c0 = e % D;
+    const float* src = opart + (bh0 + hh) * p.out_chunks * D + c0;
+    float v = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < p.out_chunks; ++c) v += __ldcg(src + static_cast<int64_t>(c) * D);
+    if (out_f32)
+      static_cast<float*>(O)[(bh0 + hh) * D + c0] = v;
+    else
+      static_cast<__nv_bfloat16*>(O)[(bh0 + hh) * D + c0] = __float2bfloat16_rn(v);
+  }
 }
 
 // Opt a kernel into `bytes` of dynamic shared memory, once per device (also
@@ -536,14 +596,12 @@ bool allow_smem(size_t bytes) {
 
 struct DecLayout {
   int chunks, out_chunks;
-  size_t qm, logits, part, idx_t, start, opart, total;
+  size_t logits, part, idx_t, kept, opart, lse, arrivals, total;
 };
 
 DecLayout dec_layout(int64_t B, int64_t Hq, int64_t L, int64_t D, int64_t kt, bool own_logits, bool own_idx) {
   DecLayout w{};
   size_t off = 0;
-  w.qm = off;
-  off += align_up(static_cast<size_t>(B * Hq * D) * 4, kWsAlign);
   w.chunks = static_cast<int>((L + kDecChunk - 1) / kDecChunk);
   w.out_chunks = static_cast<int>((L + kDecOutChunk - 1) / kDecOutChunk);
   const size_t heads = static_cast<size_t>(B * Hq);
@@ -553,54 +611,96 @@ DecLayout dec_layout(int64_t B, int64_t Hq, int64_t L, int64_t D, int64_t kt, bo
   off += align_up(heads * w.chunks * 8, kWsAlign);
   w.idx_t = off;
   if (own_idx) off += align_up(heads * kt * 4, kWsAlign);
-  w.start = off;
-  off += align_up(heads * (w.out_chunks + 1) * 4, kWsAlign);
+  w.kept = off;
+  off += align_up(heads * ((L + 31) / 32) * 4, kWsAlign);
   w.opart = off;
   off += align_up(heads * w.out_chunks * D * 4, kWsAlign);
+  w.lse = off;
+  off += align_up(heads * 4, kWsAlign);
+  w.arrivals = off;
+  off += align_up(heads * 4, kWsAlign);  // one per kv-group (at most one per head)
   w.total = off;
   return w;
 }
 
+struct DecBuffers {
+  float* logits;
+  float2* part;
+  int32_t *idx_d, *idx_t;
+  uint32_t* kept;
+  float *opart, *lse_ws, *lse_out;
+  unsigned* arrivals;
+};
+
+// Token top-k with the kept-token bitmaps: a cluster of C CTAs per head, or
+// (rows longer than eight slices) the radix pass followed by dec_mark_kernel.
+template <int C>
+cudaError_t launch_dec_topk(const DecParams& p, const DecBuffers& b, cudaStream_t stream) {
+  constexpr int NT = C > 1 ? 512 : 1024;  // the thread counts of rmm_topk.cu's plan
+  const int slice = C > 1 ? (p.L + C - 1) / C : p.L;
+  const int slice_c = C > 1 ? (slice + 31) / 32 * 32 : slice;
+  if (!allow_smem<dec_topk_kernel<NT, C>>(static_cast<size_t>(kDecMaxSliceKeys) * 4)) return cudaErrorInvalidValue;
+  const size_t bytes = static_cast<size_t>(slice_c) * 4;
+  const dim3 grid(C, static_cast<unsigned>(p.B * p.Hq));
+  if (C > 1)
+    return launch_pdl_cluster(dec_topk_kernel<NT, C>, grid, dim3(NT), bytes, C, stream,
+                              static_cast<const float*>(b.logits), static_cast<const float2*>(b.part), p, slice_c,
+                              b.idx_t, b.kept, b.lse_ws, b.lse_out, b.arrivals);
+  return launch_pdl(dec_topk_kernel<NT, C>, grid, dim3(NT), bytes, stream, static_cast<const float*>(b.logits),
+                    static_cast<const float2*>(b.part), p, slice_c, b.idx_t, b.kept, b.lse_ws, b.lse_out,
+                    b.arrivals);
+}
+
+// CTAs per head of the token top-k (0: the radix pass).  A cluster's slices
+// are whole bitmap words, so a slice may hold up to 31 more keys than an
+// even split.
+int dec_topk_cluster(int64_t rows, int64_t L) {
+  const int c = topk_cluster_size(rows, L);
+  if (c <= 0) return 0;
+  const int64_t slice = (L + c - 1) / c;
+  const int64_t slice_c = c > 1 ? (slice + 31) / 32 * 32 : slice;
+  return slice_c <= kDecMaxSliceKeys ? c : 0;
+}
+
 template <int D, int G>
-cudaError_t launch_dec(const void* q, const void* K, const void* V, const DecParams& p, float* qm, float* logits,
-                       float2* part, int32_t* idx_d, int32_t* idx_t, int32_t* start, float* opart, void* O,
-                       int out_f32, float* lse, unsigned* err, cudaStream_t stream) {
-  cudaError_t e = launch_pdl(dec_select_kernel<D>, dim3(p.B * p.Hq), dim3(32), 0, stream,
-                             static_cast<const uint16_t*>(q), p, qm, idx_d);
-  if (e != cudaSuccess) return e;
+cudaError_t launch_dec(const void* q, const void* K, const void* V, const DecParams& p, const DecBuffers& b, void* O,
+                       int out_f32, cudaStream_t stream) {
   constexpr size_t lsm = dec_logits_smem<D>();
   if (!allow_smem<dec_logits_kernel<D, G>>(lsm)) return cudaErrorInvalidValue;
-  e = launch_pdl(dec_logits_kernel<D, G>, dim3(p.chunks, p.B * p.Hkv), dim3(kLogitThreads), lsm, stream,
-                 static_cast<const float*>(qm), static_cast<const uint16_t*>(K), p, logits, part);
+  cudaError_t e = launch_pdl(dec_logits_kernel<D, G>, dim3(p.chunks, p.B * p.Hkv), dim3(kLogitThreads), lsm, stream,
+                             static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(K), p, b.logits, b.part,
+                             b.idx_d);
   if (e != cudaSuccess) return e;
-  e = launch_topk(logits, static_cast<int64_t>(p.B) * p.Hq, p.L, p.L, p.kt, idx_t, p.kt, stream);
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(dec_prefix_kernel, dim3((p.kt + kDecThreads) / kDecThreads, p.B * p.Hq), dim3(kDecThreads), 0,
-                 stream, static_cast<const int32_t*>(idx_t), p, start);
+  switch (dec_topk_cluster(static_cast<int64_t>(p.B) * p.Hq, p.L)) {
+    case 1: e = launch_dec_topk<1>(p, b, stream); break;
+    case 2: e = launch_dec_topk<2>(p, b, stream); break;
+    case 4: e = launch_dec_topk<4>(p, b, stream); break;
+    case 8: e = launch_dec_topk<8>(p, b, stream); break;
+    default:
+      e = launch_topk(b.logits, static_cast<int64_t>(p.B) * p.Hq, p.L, p.L, p.kt, b.idx_t, p.kt, stream);
+      if (e == cudaSuccess)
+        e = launch_pdl(dec_mark_kernel, dim3((p.nwords + kDecThreads - 1) / kDecThreads, p.B * p.Hq),
+                       dim3(kDecThreads), 0, stream, static_cast<const int32_t*>(b.idx_t),
+                       static_cast<const float2*>(b.part), p, b.kept, b.lse_ws, b.lse_out, b.arrivals);
+  }
   if (e != cudaSuccess) return e;
   constexpr size_t osm = dec_out_smem<D, G>();
   if (!allow_smem<dec_out_kernel<D, G>>(osm)) return cudaErrorInvalidValue;
-  e = launch_pdl(dec_out_kernel<D, G>, dim3(p.out_chunks, p.B * p.Hkv), dim3(kDecThreads), osm, stream,
-                 static_cast<const uint16_t*>(V), p, static_cast<const float*>(logits),
-                 static_cast<const float2*>(part), static_cast<const int32_t*>(idx_t),
-                 static_cast<const int32_t*>(start), opart, lse, err);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(dec_reduce_kernel<D>, dim3(p.B * p.Hq), dim3(D), 0, stream, static_cast<const float*>(opart), p,
-                    O, out_f32);
+  return launch_pdl(dec_out_kernel<D, G>, dim3(p.out_chunks, p.B * p.Hkv), dim3(kDecThreads), osm, stream,
+                    static_cast<const uint16_t*>(V), p, static_cast<const float*>(b.logits),
+                    static_cast<const float*>(b.lse_ws), static_cast<const uint32_t*>(b.kept), b.opart, O, out_f32,
+                    b.arrivals);
 }
 
 template <int D>
-cudaError_t launch_dec_g(const void* q, const void* K, const void* V, const DecParams& p, float* qm, float* logits,
-                         float2* part,
-                         int32_t* idx_d, int32_t* idx_t, int32_t* start, float* opart, void* O, int out_f32,
-                         float* lse, unsigned* err, cudaStream_t stream) {
+cudaError_t launch_dec_g(const void* q, const void* K, const void* V, const DecParams& p, const DecBuffers& b, void* O,
+                         int out_f32, cudaStream_t stream) {
   switch (p.G) {
-    case 1: return launch_dec<D, 1>(q, K, V, p, qm, logits, part, idx_d, idx_t, start, opart, O, out_f32, lse, err, stream);
-    case 2: return launch_dec<D, 2>(q, K, V, p, qm, logits, part, idx_d, idx_t, start, opart, O, out_f32, lse, err, stream);
-    case 4: return launch_dec<D, 4>(q, K, V, p, qm, logits, part, idx_d, idx_t, start, opart, O, out_f32, lse, err, stream);
-    case 8: return launch_dec<D, 8>(q, K, V, p, qm, logits, part, idx_d, idx_t, start, opart, O, out_f32, lse, err, stream);
-    case 16:
-      return launch_dec<D, 16>(q, K, V, p, qm, logits, part, idx_d, idx_t, start, opart, O, out_f32, lse, err, stream);
+    case 1: return launch_dec<D, 1>(q, K, V, p, b, O, out_f32, stream);
+    case 2: return launch_dec<D, 2>(q, K, V, p, b, O, out_f32, stream);
+    case 4: return launch_dec<D, 4>(q, K, V, p, b, O, out_f32, stream);
+    case 8: return launch_dec<D, 8>(q, K, V, p, b, O, out_f32, stream);
+    case 16: return launch_dec<D, 16>(q, K, V, p, b, O, out_f32, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -617,15 +717,19 @@ size_t decode_attention_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int64_
 cudaError_t launch_decode_attention(const void* q, const void* K, const void* V, int64_t B, int64_t Hq, int64_t Hkv,
                                     int64_t L, int64_t Lmax, int64_t D, int64_t kd, int64_t kt, float scale, void* O,
                                     int out_dtype, int32_t* idx_d, int32_t* idx_t, float* lse, float* logits,
-                                    void* ws, unsigned* err, cudaStream_t stream) {
+                                    void* ws, cudaStream_t stream) {
   const DecLayout w = dec_layout(B, Hq, L, D, kt, logits == nullptr, idx_t == nullptr);
   char* base = static_cast<char*>(ws);
-  float* lg = logits ? logits : reinterpret_cast<float*>(base + w.logits);
-  float2* part = reinterpret_cast<float2*>(base + w.part);
-  int32_t* it = idx_t ? idx_t : reinterpret_cast<int32_t*>(base + w.idx_t);
-  int32_t* start = reinterpret_cast<int32_t*>(base + w.start);
-  float* opart = reinterpret_cast<float*>(base + w.opart);
-  float* qm = reinterpret_cast<float*>(base + w.qm);
+  DecBuffers b{};
+  b.logits = logits ? logits : reinterpret_cast<float*>(base + w.logits);
+  b.part = reinterpret_cast<float2*>(base + w.part);
+  b.idx_d = idx_d;
+  b.idx_t = idx_t ? idx_t : reinterpret_cast<int32_t*>(base + w.idx_t);
+  b.kept = reinterpret_cast<uint32_t*>(base + w.kept);
+  b.opart = reinterpret_cast<float*>(base + w.opart);
+  b.lse_ws = reinterpret_cast<float*>(base + w.lse);
+  b.lse_out = lse;
+  b.arrivals = reinterpret_cast<unsigned*>(base + w.arrivals);
   DecParams p{};
   p.B = static_cast<int>(B);
   p.Hq = static_cast<int>(Hq);
@@ -637,11 +741,11 @@ cudaError_t launch_decode_attention(const void* q, const void* K, const void* V,
   p.kt = static_cast<int>(kt);
   p.chunks = w.chunks;
   p.out_chunks = w.out_chunks;
+  p.nwords = static_cast<int>((L + 31) / 32);
   p.scale = scale;
   const int out_f32 = out_dtype == 0 ? 1 : 0;
-  if (D == 128)
-    return launch_dec_g<128>(q, K, V, p, qm, lg, part, idx_d, it, start, opart, O, out_f32, lse, err, stream);
-  return launch_dec_g<64>(q, K, V, p, qm, lg, part, idx_d, it, start, opart, O, out_f32, lse, err, stream);
+  if (D == 128) return launch_dec_g<128>(q, K, V, p, b, O, out_f32, stream);
+  return launch_dec_g<64>(q, K, V, p, b, O, out_f32, stream);
 }
 
 }  // namespace rmm

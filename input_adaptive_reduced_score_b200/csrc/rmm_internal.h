@@ -50,6 +50,10 @@ cudaError_t launch_silu_mul_score(const void* G, int64_t ldg, const void* U, int
                                   int64_t M, int64_t d, float* ss, void* ws, cudaStream_t stream);
 
 // ---- top-k (rmm_topk.cu)
+// CTAs per row of the top-k search (0: the row is too long to stage; it
+// takes the radix pass), and the keys each CTA of such a cluster stages.
+int topk_cluster_size(int64_t batch, int64_t d);
+int topk_cluster_slice(int64_t d, int c);
 cudaError_t launch_topk(const float* scores, int64_t batch, int64_t d, int64_t ld_s, int64_t k,
                         int32_t* idx, int64_t ld_idx, cudaStream_t stream);
 
@@ -166,6 +170,6 @@ size_t decode_attention_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int64_
 cudaError_t launch_decode_attention(const void* q, const void* K, const void* V, int64_t B, int64_t Hq, int64_t Hkv,
                                     int64_t L, int64_t Lmax, int64_t D, int64_t kd, int64_t kt, float scale, void* O,
                                     int out_dtype, int32_t* idx_d, int32_t* idx_t, float* lse, float* logits,
-                                    void* ws, unsigned* err, cudaStream_t stream);
+                                    void* ws, cudaStream_t stream);
 
 }  // namespace rmm

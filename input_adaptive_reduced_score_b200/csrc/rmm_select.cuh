@@ -18,9 +18,18 @@
 // (A ballot sweep over every index, twice, cost about 30 instructions per key
 // and took half of a 32768-key selection.)  Integer work only: the result is
 // the unique set defined by the rule.
+//
+// A row too long for one CTA to search quickly is split over a thread-block
+// cluster: CTA r of C stages the r-th consecutive slice, each round's
+// histogram is the sum of the C CTAs' bins read through distributed shared
+// memory (two bin buffers, so one cluster barrier per round suffices), every
+// CTA takes the same decision from the same sums, and one more exchange of
+// the CTAs' counts places each slice's selections in the row's list.
 #pragma once
 
 #include <cstdint>
+
+#include "rmm_device.cuh"
 
 namespace rmm {
 
@@ -32,25 +41,88 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // monotone in the float order
 }
 
+// Stage the keys of scores s[0 .. d) in shared memory and return this
+// thread's smallest and largest key.  16-byte loads when s is 16-byte
+// aligned, four in flight per thread (one memory round trip per batch).
+template <int NT>
+__device__ __forceinline__ void stage_score_keys(const float* __restrict__ s, int d, uint32_t* keys, uint32_t& kmin,
+                                                 uint32_t& kmax) {
+  const int tid = threadIdx.x;
+  kmin = 0xFFFFFFFFu;
+  kmax = 0u;
+  const int nv = (reinterpret_cast<uintptr_t>(s) & 15u) == 0 ? d >> 2 : 0;
+  const float4* s4 = reinterpret_cast<const float4*>(s);
+  for (int v0 = tid; v0 < nv; v0 += 4 * NT) {
+    float4 f[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + u * NT;
+      f[u] = v < nv ? __ldg(s4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = v0 + u * NT;
+      if (v < nv) {
+        const uint4 q = make_uint4(score_key(f[u].x), score_key(f[u].y), score_key(f[u].z), score_key(f[u].w));
+        reinterpret_cast<uint4*>(keys)[v] = q;
+        kmin = min(kmin, min(min(q.x, q.y), min(q.z, q.w)));
+        kmax = max(kmax, max(max(q.x, q.y), max(q.z, q.w)));
+      }
+    }
+  }
+  for (int j0 = 4 * nv + tid; j0 < d; j0 += 8 * NT) {
+    float f[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * NT;
+      f[u] = j < d ? __ldg(s + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u * NT;
+      if (j < d) {
+        const uint32_t key = score_key(f[u]);
+        keys[j] = key;
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+      }
+    }
+  }
+}
+
+// Where a CTA's selections go: its slice's selected indices (slice-local,
+// ascending) are in keys[0 .. count), and they take places base .. base +
+// count - 1 of the row's ascending list.
+struct StagedSelection {
+  uint32_t base, count;
+};
+
 // Histogram search on keys staged in shared memory.  Invariant of the
-// search: count(key >= hi) = `above` < k <= count(key >= lo).  The caller has
-// written keys[0..d) and passes each thread's minimum and maximum key and a
-// shared-memory array of kSelectBins words (`hist`, 16-byte aligned, any
-// contents); every thread of the block calls this once.  emit(pos, j) is
-// called once for each selected index j, with pos its place in the ascending
-// list (0 .. k-1), by thread pos % NT.  keys must be 16-byte aligned and
-// d <= 128 * NT; the keys are overwritten.
-template <int NT, typename Emit>
-__device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32_t k, uint32_t kmin,
-                                                   uint32_t kmax, uint32_t* hist, Emit&& emit) {
+// search: count(key >= hi) = `above` < k <= count(key >= lo), counted over
+// the whole row.  The caller has written this CTA's keys[0..d) and passes
+// each thread's minimum and maximum key; every thread of the block (of every
+// block of the cluster, C > 1) calls this once.  hist: kSelectBins words
+// (2 kSelectBins when C > 1) of shared memory, 16-byte aligned, any contents.
+// keys must be 16-byte aligned and d <= 128 * NT; 1 <= k <= the row's length.
+// With C > 1 the row is the concatenation of the slices of cluster ranks
+// 0 .. C-1 (launched as a cluster along x), and on return this thread has
+// arrived on the cluster barrier after its last access to another CTA's
+// shared memory: the caller must call cluster_wait() before it exits and
+// must not use the cluster barrier in between.
+template <int NT, int C>
+__device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys, int d, uint32_t k, uint32_t kmin,
+                                                                 uint32_t kmax, uint32_t* hist) {
   constexpr int NW = NT / 32;
   constexpr int BPT = kSelectBins / NT;  // bins per thread, contiguous
-  static_assert(BPT == 2 || BPT == 8, "bin vectors are 2 or 8 words");
+  static_assert(BPT == 2 || BPT == 4 || BPT == 8, "bin vectors are 2, 4 or 8 words");
+  static_assert(C == 1 || C == 2 || C == 4 || C == 8 || C == 16, "cluster of 1, 2, 4, 8 or 16 CTAs");
+  constexpr int NBUF = C > 1 ? 2 : 1;
   __shared__ uint32_t wred[NW][2];  // per-warp min/max, then per-warp bin totals
   __shared__ uint32_t wcnt[NW][2];  // per-warp (above, in-range) counts for the emission
   __shared__ uint32_t sh_bin, sh_above, sh_done;
+  __shared__ uint32_t xch[4];       // read by the cluster's CTAs: block min, max; block counts
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int b = tid; b < kSelectBins; b += NT) hist[b] = 0u;
+  for (int b = tid; b < NBUF * kSelectBins; b += NT) hist[b] = 0u;
   kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
   kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
   if (lane == 0) {
@@ -58,8 +130,27 @@ __device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32
     wred[warp][1] = kmax;
   }
   __syncthreads();
-  uint64_t lo = __reduce_min_sync(0xFFFFFFFFu, lane < NW ? wred[lane][0] : 0xFFFFFFFFu);
-  uint64_t hi = static_cast<uint64_t>(__reduce_max_sync(0xFFFFFFFFu, lane < NW ? wred[lane][1] : 0u)) + 1u;
+  kmin = __reduce_min_sync(0xFFFFFFFFu, lane < NW ? wred[lane][0] : 0xFFFFFFFFu);
+  kmax = __reduce_max_sync(0xFFFFFFFFu, lane < NW ? wred[lane][1] : 0u);
+  [[maybe_unused]] uint32_t rank = 0u;
+  if constexpr (C > 1) {
+    rank = cluster_ctarank();
+    if (tid == 0) {
+      xch[0] = kmin;
+      xch[1] = kmax;
+    }
+    cluster_sync();  // every CTA's extremes and cleared bins are in place
+    uint32_t m0 = 0xFFFFFFFFu, m1 = 0u;
+    if (lane < C) {
+      const uint32_t a = mapa_shared(smem_u32(xch), static_cast<uint32_t>(lane));
+      m0 = ld_dsmem_u32(a);
+      m1 = ld_dsmem_u32(a + 4u);
+    }
+    kmin = __reduce_min_sync(0xFFFFFFFFu, m0);
+    kmax = __reduce_max_sync(0xFFFFFFFFu, m1);
+  }
+  uint64_t lo = kmin;
+  uint64_t hi = static_cast<uint64_t>(kmax) + 1u;
   uint32_t above = 0u;
   bool done = false;
 
@@ -71,6 +162,7 @@ __device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32
     const int shift = nbits > 11 ? nbits - 11 : 0;
     // key - lo < range, in 32 bits: range - 1 fits (the range is at most 2^32)
     const uint32_t lo32 = static_cast<uint32_t>(lo), span = static_cast<uint32_t>(range - 1u);
+    uint32_t* h = hist + (NBUF > 1 ? (round & 1) * kSelectBins : 0);
     const int dv = d >> 2;
     for (int v = tid; v < dv; v += NT) {
       const uint4 q = reinterpret_cast<const uint4*>(keys)[v];
@@ -78,28 +170,61 @@ __device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t off = kq[e] - lo32;  // wraps for keys below lo
-        if (off <= span) atomicAdd(&hist[off >> shift], 1u);
+        if (off <= span) atomicAdd(&h[off >> shift], 1u);
       }
     }
     for (int j = 4 * dv + tid; j < d; j += NT) {
       const uint32_t off = keys[j] - lo32;
-      if (off <= span) atomicAdd(&hist[off >> shift], 1u);
+      if (off <= span) atomicAdd(&h[off >> shift], 1u);
     }
-    __syncthreads();
-    // this thread's bins [tid*BPT, tid*BPT + BPT), read and cleared for the next round
+    // this thread's bins [tid*BPT, tid*BPT + BPT), summed over the cluster
     uint32_t c[BPT];
-    if constexpr (BPT == 2) {
-      const uint2 v = reinterpret_cast<const uint2*>(hist)[tid];
-      c[0] = v.x;
-      c[1] = v.y;
-      reinterpret_cast<uint2*>(hist)[tid] = make_uint2(0u, 0u);
+    if constexpr (C == 1) {
+      __syncthreads();
+      // read and cleared for the next round
+      if constexpr (BPT == 2) {
+        const uint2 v = reinterpret_cast<const uint2*>(h)[tid];
+        c[0] = v.x;
+        c[1] = v.y;
+        reinterpret_cast<uint2*>(h)[tid] = make_uint2(0u, 0u);
+      } else if constexpr (BPT == 4) {
+        const uint4 v = reinterpret_cast<const uint4*>(h)[tid];
+        c[0] = v.x; c[1] = v.y; c[2] = v.z; c[3] = v.w;
+        reinterpret_cast<uint4*>(h)[tid] = make_uint4(0u, 0u, 0u, 0u);
+      } else {
+        const uint4 v0 = reinterpret_cast<const uint4*>(h)[2 * tid];
+        const uint4 v1 = reinterpret_cast<const uint4*>(h)[2 * tid + 1];
+        c[0] = v0.x; c[1] = v0.y; c[2] = v0.z; c[3] = v0.w;
+        c[4] = v1.x; c[5] = v1.y; c[6] = v1.z; c[7] = v1.w;
+        reinterpret_cast<uint4*>(h)[2 * tid] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4*>(h)[2 * tid + 1] = make_uint4(0u, 0u, 0u, 0u);
+      }
     } else {
-      const uint4 v0 = reinterpret_cast<const uint4*>(hist)[2 * tid];
-      const uint4 v1 = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
-      c[0] = v0.x; c[1] = v0.y; c[2] = v0.z; c[3] = v0.w;
-      c[4] = v1.x; c[5] = v1.y; c[6] = v1.z; c[7] = v1.w;
-      reinterpret_cast<uint4*>(hist)[2 * tid] = make_uint4(0u, 0u, 0u, 0u);
-      reinterpret_cast<uint4*>(hist)[2 * tid + 1] = make_uint4(0u, 0u, 0u, 0u);
+      cluster_sync();  // every CTA's bins of this round are complete
+#pragma unroll
+      for (int i = 0; i < BPT; ++i) c[i] = 0u;
+      const uint32_t mine = smem_u32(h) + static_cast<uint32_t>(tid * BPT * 4);
+#pragma unroll
+      for (int r = 0; r < C; ++r) {
+        const uint32_t a = mapa_shared(mine, static_cast<uint32_t>(r));
+        if constexpr (BPT == 2) {
+          const uint2 v = ld_dsmem_v2(a);
+          c[0] += v.x;
+          c[1] += v.y;
+        } else if constexpr (BPT == 4) {
+          const uint4 v = ld_dsmem_v4(a);
+          c[0] += v.x; c[1] += v.y; c[2] += v.z; c[3] += v.w;
+        } else {
+          const uint4 v0 = ld_dsmem_v4(a), v1 = ld_dsmem_v4(a + 16u);
+          c[0] += v0.x; c[1] += v0.y; c[2] += v0.z; c[3] += v0.w;
+          c[4] += v1.x; c[5] += v1.y; c[6] += v1.z; c[7] += v1.w;
+        }
+      }
+      // the other buffer was last read (by every CTA, last round) before
+      // this round's barrier: clear this thread's bins of it for next round
+      uint32_t* o = hist + ((round + 1) & 1) * kSelectBins + tid * BPT;
+#pragma unroll
+      for (int i = 0; i < BPT; ++i) o[i] = 0u;
     }
     uint32_t local = 0u;
 #pragma unroll
@@ -215,8 +340,29 @@ __device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32
       wei += en;
     }
   }
-  const uint32_t gt_before = __shfl_sync(0xFFFFFFFFu, wgi - wg, warp) + (gi - ngt);
-  const uint32_t eq_before = __shfl_sync(0xFFFFFFFFu, wei - we, warp) + (ei - neq);
+  uint32_t gt_before = __shfl_sync(0xFFFFFFFFu, wgi - wg, warp) + (gi - ngt);
+  uint32_t eq_before = __shfl_sync(0xFFFFFFFFu, wei - we, warp) + (ei - neq);
+  // this CTA's totals, and the totals of the cluster's lower ranks
+  const uint32_t cta_gt = __shfl_sync(0xFFFFFFFFu, wgi, 31), cta_eq = __shfl_sync(0xFFFFFFFFu, wei, 31);
+  uint32_t gt_pre = 0u, eq_pre = 0u;
+  if constexpr (C > 1) {
+    if (tid == 0) {
+      xch[2] = cta_gt;
+      xch[3] = cta_eq;
+    }
+    cluster_sync();
+    uint32_t g0 = 0u, e0 = 0u;
+    if (lane < static_cast<int>(rank)) {
+      const uint32_t a = mapa_shared(smem_u32(xch), static_cast<uint32_t>(lane));
+      g0 = ld_dsmem_u32(a + 8u);
+      e0 = ld_dsmem_u32(a + 12u);
+    }
+    gt_pre = __reduce_add_sync(0xFFFFFFFFu, g0);
+    eq_pre = __reduce_add_sync(0xFFFFFFFFu, e0);
+    cluster_arrive();  // no further access to another CTA's shared memory
+    gt_before += gt_pre;
+    eq_before += eq_pre;
+  }
   // of this thread's equal keys, the first `take` (lowest indices) are kept
   uint32_t take = eq_before < need ? min(neq, need - eq_before) : 0u;
 #pragma unroll
@@ -230,8 +376,11 @@ __device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32
     }
     gtm[w] |= keep;
   }
-  // compact the selected indices, ascending, over the keys
-  uint32_t pos = gt_before + min(eq_before, need);
+  // compact the selected indices, ascending, over the keys (slice-local
+  // places: minus this CTA's first place in the row's list)
+  const uint32_t base = gt_pre + min(eq_pre, need);
+  const uint32_t count = cta_gt + (eq_pre < need ? min(cta_eq, need - eq_pre) : 0u);
+  uint32_t pos = gt_before + min(eq_before, need) - base;
 #pragma unroll
   for (int w = 0; w < kWords; ++w) {
     uint32_t m = gtm[w];
@@ -242,7 +391,17 @@ __device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32
     }
   }
   __syncthreads();
-  for (int q = tid; q < static_cast<int>(k); q += NT) emit(static_cast<uint32_t>(q), static_cast<int>(keys[q]));
+  return StagedSelection{base, count};
+}
+
+// The one-CTA search (C = 1) followed by the emission: emit(pos, j) is called
+// once for each selected index j, with pos its place in the ascending list
+// (0 .. k-1), by thread pos % NT.
+template <int NT, typename Emit>
+__device__ __forceinline__ void select_staged_keys(uint32_t* keys, int d, uint32_t k, uint32_t kmin,
+                                                   uint32_t kmax, uint32_t* hist, Emit&& emit) {
+  select_staged_compact<NT, 1>(keys, d, k, kmin, kmax, hist);
+  for (int q = threadIdx.x; q < static_cast<int>(k); q += NT) emit(static_cast<uint32_t>(q), static_cast<int>(keys[q]));
 }
 
 }  // namespace rmm

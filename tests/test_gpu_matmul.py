@@ -102,9 +102,16 @@ def _topk_cases():
     cases += [("negative", (rng.standard_normal(3001) * 5).astype(np.float32), 1500)]
     s = np.concatenate([np.float32([3e38, 1e-38]), rng.random(5000).astype(np.float32)])
     cases += [("wide range", s, 2000)]
-    s = rng.random(51200).astype(np.float32)             # longest row staged in shared memory
+    s = rng.random(51200).astype(np.float32)             # longest row one CTA could stage
     cases += [("staged max", s, 25600)]
-    s = rng.random(51201).astype(np.float32)             # first row length re-read from global memory
+    # rows split over a cluster of CTAs: equal keys on every slice boundary,
+    # all keys equal (no histogram round), ragged last slices
+    s = rng.integers(0, 3, 40001).astype(np.float32)
+    cases += [("cluster ties", s, 13335), ("cluster ties k=1", s, 1)]
+    cases += [("cluster all equal", np.full(40000, -2.5, np.float32), 12345)]
+    s = rng.random(8 * 51200).astype(np.float32)         # longest row a cluster of eight stages
+    cases += [("cluster max", s, 204800)]
+    s = rng.random(8 * 51200 + 1).astype(np.float32)     # first row length re-read from global memory
     cases += [("global radix", s, 17)]
     return cases
 
@@ -119,19 +126,23 @@ def test_topk_bit_exact(case):
     no_device_error()
 
 
-def test_topk_batched_rows():
-    rng = np.random.default_rng(9)
-    S = rng.random((6, 5000)).astype(np.float32)
+@pytest.mark.parametrize("rows,d,k", [(6, 20000, 2500),     # clusters of 4, rows not 16-byte aligned
+                                      (40, 8192, 3000),     # clusters of 2
+                                      (20, 30001, 9999),    # clusters of 4, ragged last slices
+                                      (100, 3000, 1500)])   # one CTA per row
+def test_topk_batched_rows(rows, d, k):
+    rng = np.random.default_rng(9 + rows)
+    S = rng.random((rows, d)).astype(np.float32)
     S[2] = np.round(S[2] * 3)
-    pad = np.zeros((6, 5003), np.float32)
-    pad[:, :5000] = S
-    st = torch.from_numpy(pad).cuda()[:, :5000]
-    out = torch.full((6, 2600), -7, dtype=torch.int32, device="cuda")
-    R.rmm_topk(st, 2500, out=out[:, :2500])
+    pad = np.zeros((rows, d + 3), np.float32)
+    pad[:, :d] = S
+    st = torch.from_numpy(pad).cuda()[:, :d]
+    out = torch.full((rows, k + 100), -7, dtype=torch.int32, device="cuda")
+    R.rmm_topk(st, k, out=out[:, :k])
     got = out.cpu().numpy()
-    for b in range(6):
-        np.testing.assert_array_equal(got[b, :2500], oracle.topk_indices(S[b].astype(np.float64), 2500))
-    assert np.all(got[:, 2500:] == -7)   # nothing written past k
+    for b in range(rows):
+        np.testing.assert_array_equal(got[b, :k], oracle.topk_indices(S[b].astype(np.float64), k))
+    assert np.all(got[:, k:] == -7)   # nothing written past k
     no_device_error()
 
 
