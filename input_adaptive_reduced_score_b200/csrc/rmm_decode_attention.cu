@@ -37,7 +37,7 @@
 //  3. dec_out_kernel, grid (token chunks of 512, B * Hkv): the weights
 //     P_j = exp(s_j - lse) of every q-head of the group are scattered into a
 //     table over the chunk's positions; the value rows kept by any of the
-//     group's heads are read once each (16-byte asynchronous copies, six
+//     group's heads are read once each (16-byte asynchronous copies, five
 //     stages of four rows per warp) and added into every head that keeps
 //     them; per-chunk sums go to global memory, and the group's last CTA to
 //     finish adds them in chunk order into O.
@@ -59,7 +59,7 @@ constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kLogitThreads = 128;              // logits kernel
 constexpr int kDecChunk = kLogitThreads;        // tokens per logits CTA, one per thread
 constexpr int kDecOutChunk = 512;               // token positions per output CTA
-constexpr int kDecStages = 6;
+constexpr int kDecStages = 5;
 constexpr int kDecRowsPerStage = 4;
 constexpr int kDecMaxSliceKeys = 51200;         // logits one top-k CTA stages (200 KB)
 constexpr int kDecWarpTokens = kDecOutChunk / kDecWarps;  // token positions per output warp (64)
@@ -347,13 +347,14 @@ __device__ __forceinline__ void head_lse(const float2* __restrict__ part, const 
 // CTA r stages the logits of tokens [r * slice, (r + 1) * slice) (slice a
 // multiple of 32), takes its part of the exact selection (rmm_select.cuh;
 // ranking the logits ranks t_j = exp(2 (s_j - lse))), and writes its kept
-// tokens to idx_t and as bits of the head's kept-token bitmap (bit t % 32 of
-// word t / 32).  Rank 0 also forms the head's lse.
+// tokens as bits of the head's kept-token bitmap (bit t % 32 of word t / 32)
+// and, when the list is wanted or copies of the k_t-th largest logit are
+// split, as the ascending list idx_t.  Rank 0 also forms the head's lse.
 template <int NT, int C>
 __global__ void __launch_bounds__(NT, 1)
     dec_topk_kernel(const float* __restrict__ logits, const float2* __restrict__ part, DecParams p, int slice,
-                    int32_t* __restrict__ idx_t, uint32_t* __restrict__ kept, float* __restrict__ lse_ws,
-                    float* __restrict__ lse_out, unsigned* __restrict__ arrivals) {
+                    int32_t* __restrict__ idx_t, int write_list, uint32_t* __restrict__ kept,
+                    float* __restrict__ lse_ws, float* __restrict__ lse_out, unsigned* __restrict__ arrivals) {
   extern __shared__ __align__(16) uint32_t keys[];
   __shared__ __align__(16) uint32_t hist[(C > 1 ? 2 : 1) * kSelectBins];
   const int rank = C > 1 ? static_cast<int>(blockIdx.x) : 0;
@@ -365,17 +366,33 @@ __global__ void __launch_bounds__(NT, 1)
   if (rank == 0 && threadIdx.x < 32) head_lse(part, p, bh, lse_ws, lse_out, arrivals);
   uint32_t kmin, kmax;
   stage_score_keys<NT>(logits + bh * p.L + j0, dl, keys, kmin, kmax);
-  const StagedSelection sel = select_staged_compact<NT, C>(keys, dl, static_cast<uint32_t>(p.kt), kmin, kmax, hist);
+  const SelectThreshold thr = select_threshold<NT, C>(keys, dl, static_cast<uint32_t>(p.kt), kmin, kmax, hist);
+  const int nw = (dl + 31) / 32;
+  uint32_t* kw = kept + bh * p.nwords + j0 / 32;
+  if (!thr.split && !write_list) {
+    // every key >= lo is kept: the bitmap straight from the staged keys, a
+    // word per warp step (lane l tests key 32 w + l)
+    if constexpr (C > 1) cluster_arrive();  // released only after every CTA's last read of the bins
+    const uint32_t lo32 = static_cast<uint32_t>(thr.lo);
+    const int lane = threadIdx.x & 31;
+    for (int w = threadIdx.x >> 5; w < nw; w += NT / 32) {
+      const int j = 32 * w + lane;
+      const uint32_t bits = __ballot_sync(0xFFFFFFFFu, j < dl && keys[j] >= lo32);
+      if (lane == 0) kw[w] = bits;
+    }
+    if constexpr (C > 1) cluster_wait();  // no CTA leaves while another may still read its shared memory
+    return;
+  }
+  const StagedSelection sel = select_compact<NT, C>(keys, dl, thr);
   int32_t* out = idx_t + bh * p.kt;
   for (int q = threadIdx.x; q < static_cast<int>(sel.count); q += NT) out[sel.base + q] = j0 + static_cast<int32_t>(keys[q]);
   // the bitmap of the slice's words, built in the bins (no CTA reads them
-  // any more: the search's last remote reads came before its count exchange)
-  const int nw = (dl + 31) / 32;
+  // any more: the search's last remote reads came before the compaction's
+  // count exchange)
   for (int w = threadIdx.x; w < nw; w += NT) hist[w] = 0u;
   __syncthreads();
   for (int q = threadIdx.x; q < static_cast<int>(sel.count); q += NT) atomicOr(&hist[keys[q] >> 5], 1u << (keys[q] & 31u));
   __syncthreads();
-  uint32_t* kw = kept + bh * p.nwords + j0 / 32;
   for (int w = threadIdx.x; w < nw; w += NT) kw[w] = hist[w];
   if constexpr (C > 1) cluster_wait();  // no CTA leaves while another may still read its shared memory
 }
@@ -414,7 +431,7 @@ constexpr size_t dec_out_smem() {
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecThreads, 2)
+__global__ void __launch_bounds__(kDecThreads, G <= 4 ? 4 : 2)
     dec_out_kernel(const uint16_t* __restrict__ V, DecParams p, const float* __restrict__ logits,
                    const float* __restrict__ lse_ws, const uint32_t* __restrict__ kept, float* __restrict__ opart,
                    void* __restrict__ O, int out_f32, unsigned* __restrict__ arrivals) {
@@ -426,7 +443,6 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   constexpr int S = kDecStages;
   constexpr int WT = kDecWarpTokens;          // token positions per warp (two bitmap words)
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ float red[kDecWarps][D];
   __shared__ unsigned s_last;
   const int chunk = blockIdx.x;
   const int b = blockIdx.y / p.Hkv, g = blockIdx.y % p.Hkv;
@@ -542,16 +558,30 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   }
   cp_async_wait<0>();
 
-  // warps summed in a fixed order, one q-head at a time
-  for (int hh = 0; hh < G; ++hh) {
+  // warps summed in a fixed order, HP q-heads per pass, in the value rings'
+  // space (every warp has finished with its ring at the barrier)
+  constexpr int HP = (S * RPS * ROWB / (D * 4)) < G ? (S * RPS * ROWB / (D * 4)) : G;
+  float* scr = reinterpret_cast<float*>(smem);  // [kDecWarps][HP][D]
+  __syncthreads();
 #pragma unroll
-    for (int e = 0; e < NP; ++e) f2_unpack(acc[hh][e], red[warp][lane * DPL + 2 * e], red[warp][lane * DPL + 2 * e + 1]);
+  for (int h0 = 0; h0 < G; h0 += HP) {
+#pragma unroll
+    for (int hq = 0; hq < HP; ++hq) {
+      if (h0 + hq < G) {
+        float* dst = scr + (warp * HP + hq) * D + lane * DPL;
+#pragma unroll
+        for (int e = 0; e < NP; ++e) f2_unpack(acc[h0 + hq][e], dst[2 * e], dst[2 * e + 1]);
+      }
+    }
     __syncthreads();
-    if (threadIdx.x < D) {
-      float v = 0.f;
+    for (int o = threadIdx.x; o < HP * D; o += kDecThreads) {
+      const int hq = o / D, dd = o % D;
+      if (h0 + hq < G) {
+        float v = 0.f;
 #pragma unroll
-      for (int w = 0; w < kDecWarps; ++w) v += red[w][threadIdx.x];
-      opart[((bh0 + hh) * p.out_chunks + chunk) * D + threadIdx.x] = v;
+        for (int w = 0; w < kDecWarps; ++w) v += scr[(w * HP + hq) * D + dd];
+        opart[((bh0 + h0 + hq) * p.out_chunks + chunk) * D + dd] = v;
+      }
     }
     __syncthreads();
   }
@@ -565,16 +595,25 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int e = threadIdx.x; e < G * D; e += kDecThreads) {
-    const int hh = e / D, c0 = e % D;
-    const float* src = opart + (bh0 + hh) * p.out_chunks * D + c0;
-    float v = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < p.out_chunks; ++c) v += __ldcg(src + static_cast<int64_t>(c) * D);
+  // two outputs per thread at a time, their loads interleaved (64 in flight)
+  auto put = [&](int e, float v) {
     if (out_f32)
-      static_cast<float*>(O)[(bh0 + hh) * D + c0] = v;
+      static_cast<float*>(O)[bh0 * D + e] = v;
     else
-      static_cast<__nv_bfloat16*>(O)[(bh0 + hh) * D + c0] = __float2bfloat16_rn(v);
+      static_cast<__nv_bfloat16*>(O)[bh0 * D + e] = __float2bfloat16_rn(v);
+  };
+  for (int e = threadIdx.x; e < G * D; e += 2 * kDecThreads) {
+    const int e1 = e + kDecThreads < G * D ? e + kDecThreads : e;
+    const float* s0 = opart + (bh0 + e / D) * p.out_chunks * D + e % D;
+    const float* s1 = opart + (bh0 + e1 / D) * p.out_chunks * D + e1 % D;
+    float v0 = 0.f, v1 = 0.f;
+#pragma unroll 32
+    for (int c = 0; c < p.out_chunks; ++c) {
+      v0 += __ldcg(s0 + static_cast<int64_t>(c) * D);
+      v1 += __ldcg(s1 + static_cast<int64_t>(c) * D);
+    }
+    put(e, v0);
+    if (e1 != e) put(e1, v1);
   }
 }
 
@@ -627,6 +666,7 @@ struct DecBuffers {
   float* logits;
   float2* part;
   int32_t *idx_d, *idx_t;
+  int write_list;  // the caller asked for idx_t
   uint32_t* kept;
   float *opart, *lse_ws, *lse_out;
   unsigned* arrivals;
@@ -645,10 +685,10 @@ cudaError_t launch_dec_topk(const DecParams& p, const DecBuffers& b, cudaStream_
   if (C > 1)
     return launch_pdl_cluster(dec_topk_kernel<NT, C>, grid, dim3(NT), bytes, C, stream,
                               static_cast<const float*>(b.logits), static_cast<const float2*>(b.part), p, slice_c,
-                              b.idx_t, b.kept, b.lse_ws, b.lse_out, b.arrivals);
+                              b.idx_t, b.write_list, b.kept, b.lse_ws, b.lse_out, b.arrivals);
   return launch_pdl(dec_topk_kernel<NT, C>, grid, dim3(NT), bytes, stream, static_cast<const float*>(b.logits),
-                    static_cast<const float2*>(b.part), p, slice_c, b.idx_t, b.kept, b.lse_ws, b.lse_out,
-                    b.arrivals);
+                    static_cast<const float2*>(b.part), p, slice_c, b.idx_t, b.write_list, b.kept, b.lse_ws,
+                    b.lse_out, b.arrivals);
 }
 
 // CTAs per head of the token top-k (0: the radix pass).  A cluster's slices
@@ -725,6 +765,7 @@ cudaError_t launch_decode_attention(const void* q, const void* K, const void* V,
   b.part = reinterpret_cast<float2*>(base + w.part);
   b.idx_d = idx_d;
   b.idx_t = idx_t ? idx_t : reinterpret_cast<int32_t*>(base + w.idx_t);
+  b.write_list = idx_t ? 1 : 0;
   b.kept = reinterpret_cast<uint32_t*>(base + w.kept);
   b.opart = reinterpret_cast<float*>(base + w.opart);
   b.lse_ws = reinterpret_cast<float*>(base + w.lse);

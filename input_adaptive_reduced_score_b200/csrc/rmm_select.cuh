@@ -97,6 +97,17 @@ struct StagedSelection {
   uint32_t base, count;
 };
 
+// The outcome of the search, the same in every CTA of a cluster: the
+// selected keys are every key >= hi and, lowest index first, `need` of the
+// keys in [lo, hi).  `split` is false when those are all of the keys in
+// [lo, hi) (then the selection is simply key >= lo); when true, [lo, hi) is
+// the single key of the k-th largest score and some of its copies are left.
+struct SelectThreshold {
+  uint64_t lo, hi;
+  uint32_t need;
+  bool split;
+};
+
 // Histogram search on keys staged in shared memory.  Invariant of the
 // search: count(key >= hi) = `above` < k <= count(key >= lo), counted over
 // the whole row.  The caller has written this CTA's keys[0..d) and passes
@@ -105,22 +116,20 @@ struct StagedSelection {
 // (2 kSelectBins when C > 1) of shared memory, 16-byte aligned, any contents.
 // keys must be 16-byte aligned and d <= 128 * NT; 1 <= k <= the row's length.
 // With C > 1 the row is the concatenation of the slices of cluster ranks
-// 0 .. C-1 (launched as a cluster along x), and on return this thread has
-// arrived on the cluster barrier after its last access to another CTA's
-// shared memory: the caller must call cluster_wait() before it exits and
-// must not use the cluster barrier in between.
+// 0 .. C-1 (launched as a cluster along x), and the other CTAs may still
+// read this CTA's bins until all pass the next cluster barrier: the caller
+// must not write hist, nor exit, before one (select_compact has one).
 template <int NT, int C>
-__device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys, int d, uint32_t k, uint32_t kmin,
-                                                                 uint32_t kmax, uint32_t* hist) {
+__device__ __forceinline__ SelectThreshold select_threshold(const uint32_t* keys, int d, uint32_t k, uint32_t kmin,
+                                                            uint32_t kmax, uint32_t* hist) {
   constexpr int NW = NT / 32;
   constexpr int BPT = kSelectBins / NT;  // bins per thread, contiguous
   static_assert(BPT == 2 || BPT == 4 || BPT == 8, "bin vectors are 2, 4 or 8 words");
   static_assert(C == 1 || C == 2 || C == 4 || C == 8 || C == 16, "cluster of 1, 2, 4, 8 or 16 CTAs");
   constexpr int NBUF = C > 1 ? 2 : 1;
   __shared__ uint32_t wred[NW][2];  // per-warp min/max, then per-warp bin totals
-  __shared__ uint32_t wcnt[NW][2];  // per-warp (above, in-range) counts for the emission
-  __shared__ uint32_t sh_bin, sh_above, sh_done;
-  __shared__ uint32_t xch[4];       // read by the cluster's CTAs: block min, max; block counts
+  __shared__ uint32_t sh_bin, sh_above, sh_done, sh_count;
+  __shared__ uint32_t xch[2];       // read by the cluster's CTAs: block min, max
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int b = tid; b < NBUF * kSelectBins; b += NT) hist[b] = 0u;
   kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
@@ -132,9 +141,7 @@ __device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys,
   __syncthreads();
   kmin = __reduce_min_sync(0xFFFFFFFFu, lane < NW ? wred[lane][0] : 0xFFFFFFFFu);
   kmax = __reduce_max_sync(0xFFFFFFFFu, lane < NW ? wred[lane][1] : 0u);
-  [[maybe_unused]] uint32_t rank = 0u;
   if constexpr (C > 1) {
-    rank = cluster_ctarank();
     if (tid == 0) {
       xch[0] = kmin;
       xch[1] = kmax;
@@ -152,6 +159,7 @@ __device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys,
   uint64_t lo = kmin;
   uint64_t hi = static_cast<uint64_t>(kmax) + 1u;
   uint32_t above = 0u;
+  uint32_t in_range = 0xFFFFFFFFu;  // keys in [lo, hi) over the row (unknown before the first round)
   bool done = false;
 
   // each round shrinks the range at least 2048-fold (or to one key), so four
@@ -254,6 +262,7 @@ __device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys,
       if (higher < k && ge >= k) {
         sh_bin = static_cast<uint32_t>(tid * BPT + i);
         sh_above = higher;
+        sh_count = c[i];
         sh_done = ge == k ? 1u : 0u;
       }
       higher = ge;
@@ -264,14 +273,30 @@ __device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys,
     hi = nhi < hi ? nhi : hi;
     lo = nlo;
     above = sh_above;
+    in_range = sh_count;
     done = sh_done != 0u;
   }
-
-  // Selected: every key >= hi (`above` of them) and, lowest index first,
-  // need = k - above of the keys in [lo, hi).  When the search stopped with
-  // exactly k keys at or above lo, that is all of them; otherwise [lo, hi)
-  // is the single key T of the k-th largest score.
+  // When the search stopped with exactly k keys at or above lo, all keys in
+  // [lo, hi) are taken; otherwise [lo, hi) is the single key T of the k-th
+  // largest score, of which need = k - above copies are taken.
   const uint32_t need = k - above;
+  return SelectThreshold{lo, hi, need, need < in_range};
+}
+
+// The selected indices of this CTA's slice compacted, ascending, over its
+// keys (every thread of the block, of every block of the cluster, calls this
+// once, after select_threshold on the same keys).  With C > 1, on return this
+// thread has arrived on the cluster barrier after its last access to another
+// CTA's shared memory: the caller must call cluster_wait() before it exits
+// and must not use the cluster barrier in between.
+template <int NT, int C>
+__device__ __forceinline__ StagedSelection select_compact(uint32_t* keys, int d, const SelectThreshold& thr) {
+  constexpr int NW = NT / 32;
+  __shared__ uint32_t wcnt[NW][2];  // per-warp (above, in-range) counts
+  __shared__ uint32_t xch[2];       // read by the cluster's CTAs: block counts
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint64_t lo = thr.lo, hi = thr.hi;
+  const uint32_t need = thr.need;
   // this thread's run [j0, j0 + R): bit masks of its keys at or above hi and
   // of its keys in [lo, hi)
   // (word and bit positions are compile-time: a runtime index would put the
@@ -347,15 +372,16 @@ __device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys,
   uint32_t gt_pre = 0u, eq_pre = 0u;
   if constexpr (C > 1) {
     if (tid == 0) {
-      xch[2] = cta_gt;
-      xch[3] = cta_eq;
+      xch[0] = cta_gt;
+      xch[1] = cta_eq;
     }
     cluster_sync();
+    const int rank = static_cast<int>(cluster_ctarank());
     uint32_t g0 = 0u, e0 = 0u;
-    if (lane < static_cast<int>(rank)) {
+    if (lane < rank) {
       const uint32_t a = mapa_shared(smem_u32(xch), static_cast<uint32_t>(lane));
-      g0 = ld_dsmem_u32(a + 8u);
-      e0 = ld_dsmem_u32(a + 12u);
+      g0 = ld_dsmem_u32(a);
+      e0 = ld_dsmem_u32(a + 4u);
     }
     gt_pre = __reduce_add_sync(0xFFFFFFFFu, g0);
     eq_pre = __reduce_add_sync(0xFFFFFFFFu, e0);
@@ -392,6 +418,14 @@ __device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys,
   }
   __syncthreads();
   return StagedSelection{base, count};
+}
+
+// Search and compaction (the contract of select_compact).
+template <int NT, int C>
+__device__ __forceinline__ StagedSelection select_staged_compact(uint32_t* keys, int d, uint32_t k, uint32_t kmin,
+                                                                 uint32_t kmax, uint32_t* hist) {
+  const SelectThreshold thr = select_threshold<NT, C>(keys, d, k, kmin, kmax, hist);
+  return select_compact<NT, C>(keys, d, thr);
 }
 
 // The one-CTA search (C = 1) followed by the emission: emit(pos, j) is called

@@ -116,6 +116,11 @@ def test_decode_attention_parity(case, out_dtype):
             assert np.all(np.abs(got_o[b, h] - ref["O"][b, h]) <= bound), (b, h)
     np.testing.assert_allclose(lse.cpu().numpy().astype(np.float64).reshape(B, Hq), ref["lse"], rtol=0, atol=2e-5)
     assert rel_fro(got_o, ref["O"]) <= (2e-3 if out_dtype == torch.bfloat16 else 1e-5)
+    # without the optional outputs the token top-k writes only its bitmap:
+    # the same kept set, so the same bits of O
+    O2 = R.rmm_decode_attention(bf16_tensor(inp.q), bf16_tensor(inp.K), bf16_tensor(inp.V), L, rho_d, rho_t,
+                                out_dtype=out_dtype)
+    assert torch.equal(O2, O)
 
 
 def _check_own_selection(inp, B, Hq, Hkv, L, D, rho_d, rho_t, heads):
@@ -152,6 +157,35 @@ def _check_own_selection(inp, B, Hq, Hkv, L, D, rho_d, rho_t, heads):
         ref_o = oracle.reduced_matmul(P[None, :], V[b, g, :L], It)[0]
         bound = (kt * 2.0 ** -24 + 1e-5) * (P[It] @ np.abs(V[b, g, It])) + 1e-30
         assert np.all(np.abs(got_o[b, h] - ref_o) <= bound), (b, h)
+    # without the optional outputs (the top-k writes only its bitmap): the same O
+    O2 = R.rmm_decode_attention(bf16_tensor(inp.q), bf16_tensor(inp.K), bf16_tensor(inp.V), L, rho_d, rho_t,
+                                out_dtype=torch.float32)
+    assert torch.equal(O2, O)
+
+
+def test_decode_attention_tied_logits():
+    """Key rows repeating three patterns: each head's logits take three
+    values, and the k_t boundary falls inside a run of equal logits, so only
+    the lowest-index copies are kept (the top-k's compaction path, with and
+    without the list output; clusters of 4 CTAs per head)."""
+    B, Hq, Hkv, L, D = 1, 4, 1, 20000, 128
+    inp = W.decode_attention(11, B, Hq, Hkv, L, D, 0.5, 0.5)
+    inp.K[:, :, :L] = inp.K[:, :, np.arange(L) % 3]
+    q, K, V = (oracle.decode(x, "bf16") for x in (inp.q, inp.K, inp.V))
+    ref = OD.decode_attention(q, K, V, L, 0.5, 0.5)
+    kt = oracle.k_from_rho(0.5, L)
+    for h in range(Hq):   # the boundary splits a run of equal logits
+        s = np.sort(ref["logits"][0, h])[::-1]
+        assert s[kt - 1] == s[kt]
+    idx_t = torch.full((Hq, kt), -1, dtype=torch.int32, device="cuda")
+    O = R.rmm_decode_attention(bf16_tensor(inp.q), bf16_tensor(inp.K), bf16_tensor(inp.V), L, 0.5, 0.5,
+                               out_dtype=torch.float32, idx_t=idx_t)
+    np.testing.assert_array_equal(idx_t.cpu().numpy().reshape(B, Hq, kt), ref["idx_t"])
+    assert rel_fro(to_f64(O), ref["O"]) <= 1e-5
+    O2 = R.rmm_decode_attention(bf16_tensor(inp.q), bf16_tensor(inp.K), bf16_tensor(inp.V), L, 0.5, 0.5,
+                                out_dtype=torch.float32)
+    assert torch.equal(O2, O)
+    assert R.rmm_device_error(clear=True) == 0
 
 
 def test_decode_attention_full_size():
