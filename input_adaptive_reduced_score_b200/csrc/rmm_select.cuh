@@ -308,28 +308,24 @@ __device__ __forceinline__ StagedSelection select_compact(uint32_t* keys, int d,
   const uint32_t lo32 = static_cast<uint32_t>(lo), hi32 = static_cast<uint32_t>(hi);
   uint32_t gtm[kWords] = {0u, 0u, 0u, 0u}, eqm[kWords] = {0u, 0u, 0u, 0u};
 #pragma unroll
-  for (int w = 0; w < kWords; ++w) {
+  for (int v4 = 0; v4 < 8 * kWords; ++v4) {
+    const int q = 4 * v4;  // this vector's first key in the run
+    const int j = j0 + q;
+    if (q >= R || j >= d) break;  // runs are short for small rows: leave the unrolled sweep early
+    uint32_t kq[4];
+    if (j + 4 <= d) {
+      const uint4 v = reinterpret_cast<const uint4*>(keys)[j >> 2];
+      kq[0] = v.x; kq[1] = v.y; kq[2] = v.z; kq[3] = v.w;
+    } else {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int q = 32 * w + 4 * u;  // this vector's first key in the run
-      const int j = j0 + q;
-      if (q < R && j < d) {
-        uint32_t kq[4];
-        if (j + 4 <= d) {
-          const uint4 v = reinterpret_cast<const uint4*>(keys)[j >> 2];
-          kq[0] = v.x; kq[1] = v.y; kq[2] = v.z; kq[3] = v.w;
-        } else {
+      for (int e = 0; e < 4; ++e) kq[e] = j + e < d ? keys[j + e] : 0u;
+    }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) kq[e] = j + e < d ? keys[j + e] : 0u;
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool valid = j + e < d;
-          const bool ge_hi = hi_in && kq[e] >= hi32;
-          gtm[w] |= static_cast<uint32_t>(valid && ge_hi) << (4 * u + e);
-          eqm[w] |= static_cast<uint32_t>(valid && kq[e] >= lo32 && !ge_hi) << (4 * u + e);
-        }
-      }
+    for (int e = 0; e < 4; ++e) {
+      const bool valid = j + e < d;
+      const bool ge_hi = hi_in && kq[e] >= hi32;
+      gtm[v4 >> 3] |= static_cast<uint32_t>(valid && ge_hi) << (4 * (v4 & 7) + e);
+      eqm[v4 >> 3] |= static_cast<uint32_t>(valid && kq[e] >= lo32 && !ge_hi) << (4 * (v4 & 7) + e);
     }
   }
   uint32_t ngt = 0u, neq = 0u;
