@@ -275,6 +275,8 @@ cudaError_t launch_topk_cluster(const float* scores, int64_t batch, int64_t d, i
 }  // namespace
 
 int topk_cluster_size(int64_t batch, int64_t d) {
+  // a cluster launch puts the rows on grid y (at most 65535 of them)
+  if (batch > 65535) return d <= kMaxStagedKeys ? 1 : 0;
   const int64_t sms = std::max(device_sm_count(), 1);
   int c = 1;
   // split while the clusters still fit the SMs and each slice keeps at
