@@ -30,17 +30,20 @@
 //     head (so that a few sequences still fill the SMs).  t_j = exp(2(s_j -
 //     lse)) is increasing in s_j, so ranking the logits ranks the token
 //     scores (without the rounding of the exponential merging close values).
-//     It also writes where each 512-token output chunk starts in the kept
-//     list, the heads' lse, and clears the output kernel's arrival counters.
-//     (Rows too long for eight CTAs take the radix pass of rmm_topk.cu and
-//     dec_prefix_kernel instead.)
-//  3. dec_out_kernel, grid (token chunks of 512, B * Hkv): the weights
-//     P_j = exp(s_j - lse) of every q-head of the group are scattered into a
-//     table over the chunk's positions; the value rows kept by any of the
-//     group's heads are read once each (16-byte asynchronous copies, five
-//     stages of four rows per warp) and added into every head that keeps
-//     them; per-chunk sums go to global memory, and the group's last CTA to
-//     finish adds them in chunk order into O.
+//     It writes each head's kept tokens as a bitmap (and as the ascending
+//     list idx_t when that is asked for or copies of the k_t-th largest
+//     logit are split), the heads' lse, and clears the output kernel's
+//     arrival counters.  (Rows too long for eight CTAs take the radix pass
+//     of rmm_topk.cu, then dec_mark_kernel builds the bitmap.)
+//  3. dec_out_kernel, grid (token chunks of 512, B * Hkv), four CTAs per SM
+//     up to four q-heads per kv-head (two above): each warp takes 64 positions, i.e. two bitmap words per q-head of the
+//     group; the union of the group's kept rows and each head's weights
+//     P_j = exp(s_j - lse) (zero where the head drops j) come from one round
+//     of independent loads, with no block barrier.  The union rows are read
+//     once each (16-byte asynchronous copies, five stages of four rows per
+//     warp) and added into every head that keeps them; the warps' sums are
+//     added in a fixed order, per-chunk sums go to global memory, and the
+//     group's last CTA to finish adds them in chunk order into O.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -54,7 +57,7 @@
 namespace rmm {
 namespace {
 
-constexpr int kDecThreads = 256;                // output and prefix kernels
+constexpr int kDecThreads = 256;                // output and bitmap kernels
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kLogitThreads = 128;              // logits kernel
 constexpr int kDecChunk = kLogitThreads;        // tokens per logits CTA, one per thread
