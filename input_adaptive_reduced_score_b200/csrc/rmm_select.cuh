@@ -111,8 +111,8 @@ struct SelectThreshold {
 // Histogram search on keys staged in shared memory.  Invariant of the
 // search: count(key >= hi) = `above` < k <= count(key >= lo), counted over
 // the whole row.  The caller has written this CTA's keys[0..d) and passes
-// each thread's minimum and maximum key; every thread of the block (of every
-// block of the cluster, C > 1) calls this once.  hist: kSelectBins words
+// each thread's minimum and maximum key (unused when C > 1); every thread of
+// the block (of every block of the cluster, C > 1) calls this once.  hist: kSelectBins words
 // (2 kSelectBins when C > 1) of shared memory, 16-byte aligned, any contents.
 // keys must be 16-byte aligned and d <= 128 * NT; 1 <= k <= the row's length.
 // With C > 1 the row is the concatenation of the slices of cluster ranks
@@ -129,35 +129,27 @@ __device__ __forceinline__ SelectThreshold select_threshold(const uint32_t* keys
   constexpr int NBUF = C > 1 ? 2 : 1;
   __shared__ uint32_t wred[NW][2];  // per-warp min/max, then per-warp bin totals
   __shared__ uint32_t sh_bin, sh_above, sh_done, sh_count;
-  __shared__ uint32_t xch[2];       // read by the cluster's CTAs: block min, max
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int b = tid; b < NBUF * kSelectBins; b += NT) hist[b] = 0u;
-  kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
-  kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
-  if (lane == 0) {
-    wred[warp][0] = kmin;
-    wred[warp][1] = kmax;
-  }
-  __syncthreads();
-  kmin = __reduce_min_sync(0xFFFFFFFFu, lane < NW ? wred[lane][0] : 0xFFFFFFFFu);
-  kmax = __reduce_max_sync(0xFFFFFFFFu, lane < NW ? wred[lane][1] : 0u);
+  uint64_t lo, hi;
   if constexpr (C > 1) {
-    if (tid == 0) {
-      xch[0] = kmin;
-      xch[1] = kmax;
+    // a cluster starts from the whole key range: exchanging the CTAs'
+    // extremes costs a cluster barrier and a remote read, and saves a round
+    // only when every key of the row lies within 2^22 of the others
+    __syncthreads();  // the bins are cleared before any thread counts
+    lo = 0u;
+    hi = 1ull << 32;
+  } else {
+    kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+    kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+    if (lane == 0) {
+      wred[warp][0] = kmin;
+      wred[warp][1] = kmax;
     }
-    cluster_sync();  // every CTA's extremes and cleared bins are in place
-    uint32_t m0 = 0xFFFFFFFFu, m1 = 0u;
-    if (lane < C) {
-      const uint32_t a = mapa_shared(smem_u32(xch), static_cast<uint32_t>(lane));
-      m0 = ld_dsmem_u32(a);
-      m1 = ld_dsmem_u32(a + 4u);
-    }
-    kmin = __reduce_min_sync(0xFFFFFFFFu, m0);
-    kmax = __reduce_max_sync(0xFFFFFFFFu, m1);
+    __syncthreads();
+    lo = __reduce_min_sync(0xFFFFFFFFu, lane < NW ? wred[lane][0] : 0xFFFFFFFFu);
+    hi = static_cast<uint64_t>(__reduce_max_sync(0xFFFFFFFFu, lane < NW ? wred[lane][1] : 0u)) + 1u;
   }
-  uint64_t lo = kmin;
-  uint64_t hi = static_cast<uint64_t>(kmax) + 1u;
   uint32_t above = 0u;
   uint32_t in_range = 0xFFFFFFFFu;  // keys in [lo, hi) over the row (unknown before the first round)
   bool done = false;
