@@ -55,10 +55,10 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", choices=["bench", "matmul", "attention", "attention_gqa", "layer70b", "decode", "w8",
-                                       "decode_attention", "block", "down"],
+                                       "decode_attention", "block", "down", "topk"],
                     default="bench",
                     help="matmul / attention / attention_gqa / layer70b / decode / w8 / decode_attention / block / "
-                         "down: run only that workload a few "
+                         "down / topk: run only that workload a few "
                          "times and exit (a short program for profiler captures; prints no JSON line)")
     a = ap.parse_args()
     if a.warmup < 3:
@@ -1133,6 +1133,17 @@ def run_case(case):
             R.rmm_matmul_multi(X, Ws, 0.5)
             flush.zero_()
             R.rmm_mlp_block(X, Wu, Wg, Wd, 0.8, 0.5)
+    elif case == "topk":
+        # the top-k on its own, at the row counts and lengths the paths give
+        # it: one row of 4096 and of 14336 scores (the MLP up and down
+        # projections), 32 rows of 32768 (a decode step's token top-k, one
+        # sequence) and 256 such rows (eight sequences); k = d / 2
+        gen = torch.Generator(device=dev).manual_seed(3)
+        for rows, d in ((1, 4096), (1, 14336), (32, 32768), (256, 32768)):
+            sc = torch.randn(rows, d, device=dev, generator=gen)
+            out = torch.empty(rows, d // 2, dtype=torch.int32, device=dev)
+            for _ in range(3):
+                R.rmm_topk(sc, d // 2, out=out)
     elif case == "decode_attention":
         a = DEC_ATTN
         for B in (1, 8):
